@@ -1,0 +1,267 @@
+/*
+ * sf.h -- C ABI of the B200 Streaming Sortformer diarization engine (libsf.so).
+ *
+ * The engine computes the forward pass described on the "Streaming Sortformer
+ * Diarizer" page (Pipeline): 16 kHz audio -> 128-bin log-mel (25 ms window,
+ * 10 ms stride) -> ConvSubsampling 8x -> 17 FastConformer layers (d=512) ->
+ * Linear 512->192 -> 18 Transformer layers (d=192, 8 heads) ->
+ * Linear-ReLU-Linear-sigmoid head: per-80 ms activity of 4 speakers.  In
+ * streaming mode each step runs the encoder on [speaker cache | FIFO | chunk]
+ * (page section "Streaming Architecture"; NeMo Speaker Diarization API,
+ * forward_streaming_step).
+ *
+ * Conventions for every call:
+ *  - Pointers prefixed d_ are CUDA device memory, h_ are host memory; all
+ *    are owned by the caller, who keeps them valid until the call's GPU work
+ *    has finished on the given stream.
+ *  - Element types: audio, mel features and probabilities are float32.
+ *    Embeddings exchanged through sf_pre_encode / sf_encode / the state view
+ *    use the engine's precision: float32 in SF_FP32 mode, bfloat16 (raw
+ *    uint16 bit patterns) in SF_BF16 mode ("act" type below).
+ *  - All arrays are dense row-major with the shapes given.
+ *  - `cuda_stream` is a cudaStream_t (NULL = the legacy default stream).
+ *    Work is enqueued asynchronously unless a call says it synchronises.
+ *  - Return value: SF_OK, or an error code with a message retrievable by
+ *    sf_last_error().  Argument and shape checks happen on the host before
+ *    any work is enqueued; on such an error nothing is enqueued and no
+ *    output is written.  SF_ECUDA reports a launch or runtime error.
+ *    SF_ETIMEOUT reports that a bounded device-side wait gave up (the
+ *    engine's kernels never spin without a limit).
+ *  - An engine or stream object must not be used from two host threads at
+ *    once.
+ */
+#ifndef SF_H_
+#define SF_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SF_API __attribute__((visibility("default")))
+#else
+#define SF_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct sf_engine sf_engine;
+typedef struct sf_stream sf_stream;
+
+typedef enum {
+  SF_OK = 0,
+  SF_EINVAL = 1,    /* bad argument (null pointer, out-of-range value)      */
+  SF_ESHAPE = 2,    /* sizes beyond what the engine was created for         */
+  SF_ENOMEM = 3,    /* device or pinned-host allocation failed               */
+  SF_ECUDA = 4,     /* CUDA launch / runtime error                           */
+  SF_ESTATE = 5,    /* call not valid in the object's current state          */
+  SF_ETIMEOUT = 6,  /* a bounded device wait gave up                         */
+  SF_EDEVICE = 7,   /* no usable sm_100 device                               */
+  SF_EFORMAT = 8    /* weight blob malformed or missing a tensor             */
+} sf_status;
+
+typedef enum { SF_FP32 = 0, SF_BF16 = 1 } sf_precision;
+
+/* Model and capacity description ("Streaming Sortformer Diarizer", Model
+ * Parameters table; metadata of the exported program: sample_rate,
+ * window_stride, subsampling_factor, fc_d_model, tf_d_model,
+ * max_num_of_spks, spkcache_len).  Only n_conformer, n_transformer,
+ * precision, max_batch and max_samples may differ from sf_default_config();
+ * the other fields are checked. */
+typedef struct {
+  int sample_rate;     /* 16000 */
+  int n_mels;          /* 128 */
+  int n_fft;           /* 512 */
+  int win_length;      /* 400 samples (25 ms) */
+  int hop_length;      /* 160 samples (10 ms) */
+  int subsampling;     /* 8 */
+  int d_model;         /* 512  (fc_d_model) */
+  int tf_d_model;      /* 192 */
+  int n_conformer;     /* 17 */
+  int n_transformer;   /* 18 */
+  int n_heads;         /* 8 */
+  int ff_mult;         /* 4 (FFN 512 -> 2048) */
+  int tf_ff;           /* 768 */
+  int conv_kernel;     /* 9 */
+  int n_spk;           /* 4 (max_num_of_spks) */
+  int spkcache_len;    /* 188 */
+  int precision;       /* sf_precision */
+  int max_batch;       /* max clips per offline call and streams per sf_stream (<= 512) */
+  int64_t max_samples; /* max samples per clip (default 1,920,000 = 120 s) */
+} sf_config;
+
+/* Streaming preset, all lengths in 80 ms encoder frames ("Streaming
+ * Configurations" table: Very high 340/40/40/300/188, High 124/1/124/124/188,
+ * Low 6/7/188/144/188, Ultra low 3/1/188/144/188).  Input-buffer latency is
+ * (chunk_len + right_context) x 80 ms. */
+typedef struct {
+  int chunk_len;
+  int right_context;
+  int fifo_len;
+  int update_period;
+  int spkcache_len;    /* <= config spkcache_len, multiple of n_spk */
+} sf_preset;
+
+/* State of one stream (NeMo SortformerStreamingState fields spkcache,
+ * spkcache_lengths, spkcache_preds, fifo, fifo_lengths, fifo_preds; plus the
+ * engine's silence mean used for cache placeholders and the position of the
+ * next chunk).  Device buffers are caller-owned; capacities are
+ * spkcache_len rows for the cache and fifo_len + chunk_len rows for the
+ * FIFO. */
+typedef struct {
+  int n_cache;          /* rows in the speaker cache */
+  int n_fifo;           /* rows in the FIFO */
+  int64_t next_frame;   /* encoder frame index of the next chunk (c0) */
+  int finished;         /* 1 after the step that consumed the recording end */
+  int sil_count;        /* popped silent frames averaged into sil_mean */
+  void* d_cache_emb;    /* act [capacity_cache x d_model] pre-encode embeddings */
+  float* d_cache_preds; /* f32 [capacity_cache x n_spk] */
+  void* d_fifo_emb;     /* act [capacity_fifo x d_model] */
+  float* d_fifo_preds;  /* f32 [capacity_fifo x n_spk] */
+  float* d_sil_mean;    /* f32 [d_model] */
+} sf_state_view;
+
+/* ---------------------------------------------------------------- engine */
+
+/* Fill `cfg` with the full model (17 + 18 layers), bf16, max_batch 64,
+ * max_samples 1,920,000. */
+SF_API sf_status sf_default_config(sf_config* cfg);
+
+/* Create an engine on the current CUDA device from a weight blob in host
+ * memory (SFW1 container: magic "SFW1", u32 tensor count, u64 payload
+ * offset, then per tensor u16 name length, name, u8 ndim, u32 dims, u64
+ * payload offset; float32 payloads).  Weights are converted to the engine's
+ * precision, BatchNorm is folded into the depthwise conv, the relative
+ * position projections are precomputed for every distance up to the longest
+ * sequence the configuration allows, and the workspace is allocated.  The
+ * blob may be freed after the call.  Synchronises.  Errors: SF_EINVAL,
+ * SF_EFORMAT (missing/mis-shaped tensor), SF_EDEVICE, SF_ENOMEM. */
+SF_API sf_status sf_create(const void* h_blob, uint64_t nbytes, const sf_config* cfg, sf_engine** out);
+SF_API sf_status sf_create_from_file(const char* path, const sf_config* cfg, sf_engine** out);
+SF_API sf_status sf_destroy(sf_engine* e);
+SF_API sf_status sf_get_metadata(const sf_engine* e, sf_config* out);
+/* Message of the last error on this engine (never NULL; "" if none). */
+SF_API const char* sf_last_error(const sf_engine* e);
+SF_API const char* sf_status_str(sf_status s);
+
+/* ------------------------------------------------------------ front-end */
+
+/* Preprocessor ("Exported Methods / preprocessor": audio (N,) + length ->
+ * mel (1, 128, T) + mel_len), batched.
+ *   d_audio  f32 [B x n_max]  16 kHz mono, clip b valid for h_len[b] samples
+ *   h_len    i64 [B]          1600 <= h_len[b] <= min(n_max, max_samples)
+ *   d_mel    f32 [B x 128 x (1 + n_max/160)]  normalised log-mel; every
+ *            element is written, frames >= h_mel_len[b] are 0
+ *   h_mel_len i64 [B] (out)   h_len[b] / 160
+ * Preemphasis 0.97, centred STFT (n_fft 512, Hann 400, hop 160), power,
+ * 128 Slaney mel bins 0-8 kHz, log(x + 2^-24), per-bin mean/std
+ * normalisation over the valid frames. */
+SF_API sf_status sf_mel(sf_engine* e, const float* d_audio, const int64_t* h_len, int B, int64_t n_max,
+                 float* d_mel, int64_t* h_mel_len, void* cuda_stream);
+
+/* ------------------------------------------------- exported-method split */
+
+/* pre_encode ("Exported Methods / pre_encode": chunk (1, T, 128) -> embs
+ * (1, 1+(T-1)//8, 512)), batched over windows of normalised features.
+ *   d_feats  f32 [n_buf x 128 x t_buf]  channels-first features
+ *   h_buf    i32 [n]  which buffer row each window reads
+ *   h_start  i64 [n]  first column of the window in that row
+ *   h_frames i64 [n]  window length W_i (>= 1); columns outside
+ *                     [start, start + W_i) are treated as zero
+ *   d_embs   act [n x emb_stride x d_model] (out) window i's
+ *            1 + (W_i-1)//8 embeddings; emb_stride >= the largest count */
+SF_API sf_status sf_pre_encode(sf_engine* e, const float* d_feats, int n_buf, int64_t t_buf, const int* h_buf,
+                        const int64_t* h_start, const int64_t* h_frames, int n, void* d_embs,
+                        int64_t emb_stride, void* cuda_stream);
+
+/* encode ("Exported Methods / encode": embs (1, T_total, 512) -> preds
+ * (1, T_total, 4)), over n packed sequences.
+ *   d_embs   act [sum(h_seq_len) x d_model]  sequences back to back
+ *   h_seq_len i32 [n]  each >= 1, <= the longest sequence supported
+ *   d_preds  f32 [sum(h_seq_len) x n_spk] (out) sigmoid probabilities */
+SF_API sf_status sf_encode(sf_engine* e, const void* d_embs, const int* h_seq_len, int n, float* d_preds,
+                    void* cuda_stream);
+
+/* ----------------------------------------------------------------- offline */
+
+/* forward(audio, lengths) -> probs (NeMo Speaker Diarization API, forward).
+ *   d_audio, h_len, B, n_max as for sf_mel
+ *   d_probs   f32 [B x T'_max x 4] (out), T'_max = 1 + (n_max/160 - 1)/8;
+ *             rows >= h_out_len[b] are 0
+ *   h_out_len i64 [B] (out) = 1 + (h_len[b]/160 - 1)/8 */
+SF_API sf_status sf_forward_offline(sf_engine* e, const float* d_audio, const int64_t* h_len, int B, int64_t n_max,
+                             float* d_probs, int64_t* h_out_len, void* cuda_stream);
+
+/* Same, from and to HOST memory (pinned or pageable): the call copies the
+ * audio to the device, runs, copies the probabilities back and
+ * synchronises on `cuda_stream`. */
+SF_API sf_status sf_forward_offline_host(sf_engine* e, const float* h_audio, const int64_t* h_len, int B,
+                                  int64_t n_max, float* h_probs, int64_t* h_out_len, void* cuda_stream);
+
+/* ---------------------------------------------------------------- streaming */
+
+/* A batch of n_streams independent streams sharing one preset; all state
+ * (cache, FIFO, predictions, silence mean) lives on the device. */
+SF_API sf_status sf_stream_create(sf_engine* e, const sf_preset* p, int n_streams, sf_stream** out);
+SF_API sf_status sf_stream_destroy(sf_stream* s);
+
+/* Restore the empty state of the listed streams (h_ids NULL = all). */
+SF_API sf_status sf_stream_reset(sf_stream* s, const int* h_ids, int n);
+
+/* Mel-frame window [*h_start, *h_end) the next step of stream `id` reads
+ * for a recording of h_total valid mel frames: one encoder frame (8 mel
+ * frames) of left context when the stream is past its first chunk, then
+ * chunk_len + right_context encoder frames, clipped at the end. */
+SF_API sf_status sf_stream_window(const sf_stream* s, int id, int64_t h_total, int64_t* h_start, int64_t* h_end);
+
+/* One step of every unfinished stream (forward_streaming_step):
+ * pre_encode on the new window only, encoder on [cache | FIFO | chunk],
+ * chunk predictions out (look-ahead frames are attended to but not
+ * emitted), FIFO push/pop, cache compression.
+ *   d_feats      f32 [n_streams x 128 x t_buf] normalised features; column t
+ *                of stream i is mel frame h_feat_start[i] + t
+ *   h_feat_start i64 [n_streams]
+ *   h_feat_end   i64 [n_streams]  the recording has h_feat_end[i] mel
+ *                frames (a window reaching past it is clipped there; a
+ *                step whose window reaches it finishes the stream)
+ *   d_chunk_probs f32 [n_streams x chunk_len x 4] (out); rows >= h_n_out[i] are 0
+ *   h_n_out      i32 [n_streams] (out) frames emitted (0 for finished streams)
+ * The window columns the step needs must lie inside the buffer (SF_ESHAPE). */
+SF_API sf_status sf_stream_step(sf_stream* s, const float* d_feats, int64_t t_buf, const int64_t* h_feat_start,
+                         const int64_t* h_feat_end, float* d_chunk_probs, int* h_n_out, void* cuda_stream);
+
+/* Copy one stream's state out to / in from caller buffers (forward_for_export
+ * style state injection).  Synchronise on `cuda_stream`. */
+SF_API sf_status sf_stream_get_state(sf_stream* s, int id, sf_state_view* v, void* cuda_stream);
+SF_API sf_status sf_stream_set_state(sf_stream* s, int id, const sf_state_view* v, void* cuda_stream);
+
+/* State update alone (FIFO refresh/push/pop, silence mean, compression)
+ * given each stream's window predictions, for teacher-forced checks of the
+ * bookkeeping.  Stream i's window is [cache | FIFO | n_new[i] new frames].
+ *   d_preds    f32 [sum_i (n_cache_i + n_fifo_i + h_n_new[i]) x 4] packed
+ *   d_new_embs act [n_streams x new_stride x d_model] new frames' embeddings
+ *   h_n_new    i32 [n_streams] new frames (chunk + look-ahead), 0 = skip stream
+ *   d_scores   f32 [n_streams x (spkcache_len + fifo_len + chunk_len) x 4]
+ *              (out, may be NULL) compression scores, -inf = not a candidate
+ *   d_src      i32 [n_streams x spkcache_len] (out, may be NULL) source of each
+ *              new cache slot after a compression: candidate index, or
+ *              -1 - s for a placeholder of speaker s; untouched otherwise
+ *   d_scores_in f32, same shape as d_scores, or NULL: use these scores
+ *              instead of computing them */
+SF_API sf_status sf_stream_update(sf_stream* s, const float* d_preds, const void* d_new_embs, int64_t new_stride,
+                           const int* h_n_new, float* d_scores, int* d_src, const float* d_scores_in,
+                           void* cuda_stream);
+
+/* Per-speaker top-k selection alone (the compression's selection step).
+ *   d_scores f32 [n_sets x stride x n_spk], set i has h_n[i] candidates
+ *   d_src    i32 [n_sets x (k * n_spk)] (out) kept candidate indices in
+ *            ascending order, then -1 - s placeholders in speaker order
+ * Order: score descending, candidate index ascending; -inf never kept. */
+SF_API sf_status sf_select_topk(sf_engine* e, const float* d_scores, const int* h_n, int n_sets, int stride, int k,
+                         int* d_src, void* cuda_stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SF_H_ */

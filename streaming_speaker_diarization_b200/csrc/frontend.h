@@ -1,0 +1,29 @@
+// Log-mel front-end launchers and tables.
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace sf {
+
+constexpr int MEL_MAX_NK = 16;   // FFT bins per Slaney filter (widest is ~13 at 8 kHz)
+
+// Host-computed (double, then rounded) tables for the mel kernels.
+struct MelTables {
+  float2 tw256[128];             // exp(-2 pi i k / 256)
+  float2 tw512[257];             // exp(-2 pi i k / 512)
+  float win[512];                // symmetric 400-point Hann centred in 512
+  int mel_k0[128];               // first FFT bin of filter m
+  int mel_nk[128];               // number of FFT bins of filter m
+  float mel_w[128 * MEL_MAX_NK]; // filter weights (area-normalised)
+};
+
+struct MelArgs {
+  const int64_t* len;            // device [B] clip lengths in samples
+};
+
+cudaError_t launch_mel(const float* audio, int B, int64_t n_max, const MelArgs& args, const MelTables* tab,
+                       float* mel, float* part, cudaStream_t st);
+size_t mel_part_floats(int B, int64_t n_max);
+void build_mel_tables(MelTables* t);   // host
+
+}  // namespace sf

@@ -1,0 +1,186 @@
+// Row-wise and elementwise kernels: LayerNorm, the conformer conv module's
+// depthwise conv (BatchNorm folded) + swish, the head's output layer,
+// precision conversion and packed-row extraction.
+#include "common.cuh"
+#include "layers.h"
+
+namespace sf {
+
+// One warp per row; lane j holds elements j, j + 32, ... (coalesced).
+template <typename T, int D>
+__global__ void __launch_bounds__(256) layernorm_kernel(float* __restrict__ x, const float* __restrict__ g,
+                                                        const float* __restrict__ b, int M, bool write_x,
+                                                        T* __restrict__ h) {
+  constexpr int V = D / 32;
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= M) return;
+  float* xr = x + (int64_t)row * D;
+  float v[V];
+  float s = 0.f;
+#pragma unroll
+  for (int j = 0; j < V; ++j) { v[j] = xr[lane + 32 * j]; s += v[j]; }
+  const float mean = warp_sum(s) * (1.0f / D);
+  float q = 0.f;
+#pragma unroll
+  for (int j = 0; j < V; ++j) { const float d = v[j] - mean; q = fmaf(d, d, q); }
+  const float inv = 1.0f / sqrtf(warp_sum(q) * (1.0f / D) + 1e-5f);
+#pragma unroll
+  for (int j = 0; j < V; ++j) {
+    const int c = lane + 32 * j;
+    const float y = (v[j] - mean) * inv * g[c] + b[c];
+    if (write_x) xr[c] = y;
+    if (h) h[(int64_t)row * D + c] = from_f<T>(y);
+  }
+}
+
+template <typename T>
+cudaError_t launch_layernorm(float* x, const float* g, const float* b, int M, int D, bool write_x, T* h,
+                             cudaStream_t st) {
+  if (M <= 0) return cudaSuccess;
+  const int grid = (M + 7) / 8;
+  if (D == 512) layernorm_kernel<T, 512><<<grid, 256, 0, st>>>(x, g, b, M, write_x, h);
+  else if (D == 192) layernorm_kernel<T, 192><<<grid, 256, 0, st>>>(x, g, b, M, write_x, h);
+  else return cudaErrorInvalidValue;
+  return cudaGetLastError();
+}
+
+template <typename T> struct Vec2;
+template <> struct Vec2<float> {
+  typedef float2 type;
+  static __device__ __forceinline__ float2 load(const float* p) { return *reinterpret_cast<const float2*>(p); }
+  static __device__ __forceinline__ void store(float* p, float a, float b) { *reinterpret_cast<float2*>(p) = make_float2(a, b); }
+  static __device__ __forceinline__ float lo(float2 v) { return v.x; }
+  static __device__ __forceinline__ float hi(float2 v) { return v.y; }
+};
+template <> struct Vec2<bf16> {
+  typedef __nv_bfloat162 type;
+  static __device__ __forceinline__ __nv_bfloat162 load(const bf16* p) { return *reinterpret_cast<const __nv_bfloat162*>(p); }
+  static __device__ __forceinline__ void store(bf16* p, float a, float b) { *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(a, b); }
+  static __device__ __forceinline__ float lo(__nv_bfloat162 v) { return __low2float(v); }
+  static __device__ __forceinline__ float hi(__nv_bfloat162 v) { return __high2float(v); }
+};
+
+// Each thread: two channels over DW_ROWS rows; taps outside the row's
+// sequence read as zero.
+constexpr int DW_ROWS = 32;
+template <typename T>
+__global__ void __launch_bounds__(256) dwconv1d_kernel(const T* __restrict__ in, T* __restrict__ out,
+                                                       const float* __restrict__ w, const float* __restrict__ bias,
+                                                       int M, int D, int K, const SeqTable* __restrict__ seq) {
+  const int c = 2 * (blockIdx.y * 256 + threadIdx.x);
+  if (c >= D) return;
+  const int r0 = blockIdx.x * DW_ROWS;
+  const int pad = (K - 1) / 2;
+  float w0[16], w1[16];
+  for (int j = 0; j < K; ++j) { w0[j] = w[c * K + j]; w1[j] = w[(c + 1) * K + j]; }
+  const float b0 = bias[c], b1 = bias[c + 1];
+  int s = seq_of_row(seq, r0 < M ? r0 : M - 1);
+  for (int r = r0; r < min(r0 + DW_ROWS, M); ++r) {
+    while (r >= seq->off[s + 1]) ++s;
+    const int sb = seq->off[s], se = seq->off[s + 1];
+    float a0 = b0, a1 = b1;
+    for (int j = 0; j < K; ++j) {
+      const int ri = r + j - pad;
+      if (ri < sb || ri >= se) continue;
+      const auto v = Vec2<T>::load(in + (int64_t)ri * D + c);
+      a0 = fmaf(w0[j], Vec2<T>::lo(v), a0);
+      a1 = fmaf(w1[j], Vec2<T>::hi(v), a1);
+    }
+    a0 = a0 / (1.f + expf(-a0));
+    a1 = a1 / (1.f + expf(-a1));
+    Vec2<T>::store(out + (int64_t)r * D + c, a0, a1);
+  }
+}
+
+template <typename T>
+cudaError_t launch_dwconv1d(const T* in, T* out, const float* w, const float* b, int M, int D, int K,
+                            const SeqTable* seq, cudaStream_t st) {
+  if (M <= 0) return cudaSuccess;
+  if (K > 16 || (D % 2)) return cudaErrorInvalidValue;
+  dim3 grid((M + DW_ROWS - 1) / DW_ROWS, (D / 2 + 255) / 256);
+  dwconv1d_kernel<T><<<grid, 256, 0, st>>>(in, out, w, b, M, D, K, seq);
+  return cudaGetLastError();
+}
+
+// One warp per row: 4 dot products of length E, sigmoid.
+template <typename T>
+__global__ void __launch_bounds__(256) head_out_kernel(const T* __restrict__ h, const float* __restrict__ w,
+                                                       const float* __restrict__ b, float* __restrict__ probs,
+                                                       int M, int E) {
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= M) return;
+  float a[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int c = lane; c < E; c += 32) {
+    const float x = to_f<T>(h[(int64_t)row * E + c]);
+#pragma unroll
+    for (int s = 0; s < 4; ++s) a[s] = fmaf(x, w[s * E + c], a[s]);
+  }
+#pragma unroll
+  for (int s = 0; s < 4; ++s) a[s] = warp_sum(a[s]);
+  if (lane == 0) {
+    float4 o;
+    o.x = 1.f / (1.f + expf(-(a[0] + b[0])));
+    o.y = 1.f / (1.f + expf(-(a[1] + b[1])));
+    o.z = 1.f / (1.f + expf(-(a[2] + b[2])));
+    o.w = 1.f / (1.f + expf(-(a[3] + b[3])));
+    reinterpret_cast<float4*>(probs)[row] = o;
+  }
+}
+
+template <typename T>
+cudaError_t launch_head_out(const T* h, const float* w, const float* b, float* probs, int M, int E,
+                            cudaStream_t st) {
+  if (M <= 0) return cudaSuccess;
+  head_out_kernel<T><<<(M + 7) / 8, 256, 0, st>>>(h, w, b, probs, M, E);
+  return cudaGetLastError();
+}
+
+template <typename T>
+__global__ void to_f32_kernel(const T* __restrict__ in, float* __restrict__ out, int64_t n) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+    out[i] = to_f<T>(in[i]);
+}
+
+template <typename T>
+cudaError_t launch_to_f32(const T* in, float* out, int64_t n, cudaStream_t st) {
+  if (n <= 0) return cudaSuccess;
+  const int64_t want = (n + 255) / 256;
+  const int64_t blocks = want < 148 * 16 ? want : 148 * 16;
+  to_f32_kernel<T><<<(int)blocks, 256, 0, st>>>(in, out, n);
+  return cudaGetLastError();
+}
+
+__global__ void extract_rows_kernel(const float* __restrict__ packed, const SeqTable* __restrict__ seq,
+                                    const int* __restrict__ first, const int* __restrict__ count,
+                                    const int* __restrict__ dst, float* __restrict__ out, int t_max) {
+  const int s = blockIdx.y;
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= t_max) return;
+  const int len = seq->off[s + 1] - seq->off[s];
+  const int f = first ? first[s] : 0;
+  const int n = count ? count[s] : len;
+  float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (t < n && f + t < len) v = reinterpret_cast<const float4*>(packed)[seq->off[s] + f + t];
+  reinterpret_cast<float4*>(out)[(int64_t)(dst ? dst[s] : s) * t_max + t] = v;
+}
+
+cudaError_t launch_extract_rows(const float* packed, const SeqTable* seq, const int* d_first, const int* d_count,
+                                const int* d_dst, int n_seq, float* out, int t_max, cudaStream_t st) {
+  if (n_seq <= 0 || t_max <= 0) return cudaSuccess;
+  extract_rows_kernel<<<dim3((t_max + 127) / 128, n_seq), 128, 0, st>>>(packed, seq, d_first, d_count, d_dst, out,
+                                                                         t_max);
+  return cudaGetLastError();
+}
+
+template cudaError_t launch_layernorm<float>(float*, const float*, const float*, int, int, bool, float*, cudaStream_t);
+template cudaError_t launch_layernorm<bf16>(float*, const float*, const float*, int, int, bool, bf16*, cudaStream_t);
+template cudaError_t launch_dwconv1d<float>(const float*, float*, const float*, const float*, int, int, int, const SeqTable*, cudaStream_t);
+template cudaError_t launch_dwconv1d<bf16>(const bf16*, bf16*, const float*, const float*, int, int, int, const SeqTable*, cudaStream_t);
+template cudaError_t launch_head_out<float>(const float*, const float*, const float*, float*, int, int, cudaStream_t);
+template cudaError_t launch_head_out<bf16>(const bf16*, const float*, const float*, float*, int, int, cudaStream_t);
+template cudaError_t launch_to_f32<float>(const float*, float*, int64_t, cudaStream_t);
+template cudaError_t launch_to_f32<bf16>(const bf16*, float*, int64_t, cudaStream_t);
+
+}  // namespace sf

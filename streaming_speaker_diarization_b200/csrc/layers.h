@@ -1,0 +1,88 @@
+// Launchers of the engine's kernels (host-callable, stream-ordered).
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace sf {
+
+// ------------------------------------------------------------------ GEMM
+enum EpiKind : int {
+  EPI_BIAS = 0,        // out(act) = acc + b
+  EPI_BIAS_RELU = 1,   // out(act) = relu(acc + b)
+  EPI_BIAS_SWISH = 2,  // out(act) = swish(acc + b)
+  EPI_BIAS_GLU = 3,    // columns (2c, 2c+1) = (a_c, g_c): out(act)[c] = a_c * sigmoid(g_c)
+  EPI_RESID = 4,       // out(f32) += alpha * (acc + b)
+  EPI_F32 = 5,         // out(f32) = acc + b
+  EPI_F32_AND_T = 6,   // out(f32) = acc + b and out2(act) = acc + b
+};
+
+struct Epi {
+  int kind;
+  const float* bias;   // [N] or null
+  void* out;
+  int ldo;             // elements
+  float alpha;
+  void* out2;
+  int ldo2;
+  int rpg;             // row remap: 0 = identity, else row r -> (r / rpg) * gstride + r % rpg
+  int64_t gstride;
+};
+
+cudaError_t gemm_f32(const float* A, int lda, const float* W, int M, int N, int K, const Epi& e, cudaStream_t st);
+cudaError_t gemm_bf16_mma(const bf16* A, int lda, const bf16* W, int M, int N, int K, const Epi& e,
+                          cudaStream_t st);
+cudaError_t gemm_init_attributes();
+
+// --------------------------------------------------------- subsampling
+struct PreArgs {        // device arrays, one entry per window
+  const int* buf;       // feature buffer row
+  const int64_t* start; // first column
+  const int64_t* frames;// window length W (mel frames)
+};
+
+template <typename T>
+cudaError_t launch_conv1(const float* feats, int64_t t_buf, const PreArgs& a, int n_win, const float* w,
+                         const float* b, T* out, int T1max, cudaStream_t st);
+template <typename T>
+cudaError_t launch_dwconv3x3s2(const T* in, int Tin_max, int Fin, T* out, int Tout_max, int Fout, const PreArgs& a,
+                               int n_win, int stage, const float* w, const float* b, cudaStream_t st);
+
+// ------------------------------------------------------- norms / elementwise
+// x (f32, M x D) -> optional in-place LN(x) (f32) and/or h = act(LN(x)).
+template <typename T>
+cudaError_t launch_layernorm(float* x, const float* g, const float* b, int M, int D, bool write_x, T* h,
+                             cudaStream_t st);
+// Conformer depthwise conv (k=9, zero padding at sequence edges) with the
+// folded BatchNorm and swish: in/out act (M x D).
+template <typename T>
+cudaError_t launch_dwconv1d(const T* in, T* out, const float* w, const float* b, int M, int D, int K,
+                            const SeqTable* seq, cudaStream_t st);
+// Head output layer: probs[r][s] = sigmoid(h[r] . w[s] + b[s]), w f32 (4 x E).
+template <typename T>
+cudaError_t launch_head_out(const T* h, const float* w, const float* b, float* probs, int M, int E,
+                            cudaStream_t st);
+// Packed embeddings (act, M x D) -> f32 residual stream.
+template <typename T>
+cudaError_t launch_to_f32(const T* in, float* out, int64_t n, cudaStream_t st);
+// out[s][t][0..3] = t < count_s ? packed[off_s + first_s + t][0..3] : 0 for t < t_max
+// (d_first null = 0, d_count null = sequence length).
+// d_dst (null = identity) gives the output row block of each sequence.
+cudaError_t launch_extract_rows(const float* packed, const SeqTable* seq, const int* d_first, const int* d_count,
+                                const int* d_dst, int n_seq, float* out, int t_max, cudaStream_t st);
+void attention_set_max_seq(int s);
+
+// ------------------------------------------------------------- attention
+// Relative-position MHSA (d_model 512, 8 heads of 64) over packed sequences.
+//   qkv act [M x 3*512] (q | k | v), ptab act [(2R-1) x 512] projected
+//   sinusoid rows for r = -(R-1) .. R-1, u/v f32 [8 x 64]; ctx act [M x 512].
+template <typename T>
+cudaError_t launch_relpos_attention(const T* qkv, const T* ptab, int R, const float* u, const float* v, T* ctx,
+                                    const SeqTable* seq, int n_tiles, int M, cudaStream_t st);
+// Plain MHSA (d 192, 8 heads of 24), qkv act [M x 576] -> ctx act [M x 192].
+template <typename T>
+cudaError_t launch_mha(const T* qkv, T* ctx, const SeqTable* seq, int n_tiles, int M, cudaStream_t st);
+cudaError_t attention_init_attributes();
+
+}  // namespace sf
