@@ -1,0 +1,260 @@
+"""Benchmark of the Sortformer engine: audio-seconds per second (RTFx).
+
+Workload (one step): the offline forward of one 90 s, 16 kHz synthetic
+meeting clip (4 speakers, 15 % overlap; audio seed 1001) through the full
+model (ConvSubsampling, 17 FastConformer layers, 18 Transformer layers,
+head), bf16 weights/activations with fp32 accumulation, random weights
+N(0, 0.02) from seed 0: front-end -> probabilities, all in the engine's
+kernels.  Inputs are resident in HBM when the timed region starts; L2 is
+flushed (256 MiB write) between timed steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU (torchrun, one process per GPU): the path has no exchange step, so
+every rank runs its own replica of the workload ("replicas only"); value =
+audio processed by all ranks / max-over-ranks device time.
+
+--impl reference times the CPU oracle (test infrastructure, fp64 numpy) on
+this machine's host cores, each step a bounded sample of the same workload
+(the first 10 s of the clip).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "audio-sec/sec (RTFx) offline & streaming at 1 B200; % of bf16 tensor/HBM roofline"
+UNIT = "audio-s/s"
+CONFIG = {"workload": "offline forward, 1 clip x 90 s (16 kHz, 4 speakers, 15% overlap), full Sortformer "
+                      "(17 FastConformer + 18 Transformer layers), bf16, fp32 accumulation",
+          "audio_s": 90.0, "batch": 1, "mel_frames": 9000, "encoder_frames": 1125,
+          "l2": "flushed between timed steps (256 MiB write)"}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+class Clocks:
+    """nvidia-smi sampling during the timed region."""
+
+    def __init__(self, idx):
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{idx}.csv")
+        os.makedirs(os.path.dirname(self.path), exist_ok=True)
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.f = open(self.path, "w")
+            self.p = subprocess.Popen(["nvidia-smi", "-i", str(idx), f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                                       "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except Exception:
+            self.p.kill()
+        self.f.close()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def cpu_baseline(audio, seconds=30.0):
+    import oracle as O
+    from synth import FULL, make_weights
+    w = make_weights(FULL, seed=0)
+    n = int(seconds * 16000)
+    t0 = time.perf_counter()
+    O.forward_offline(audio[:, :n], np.array([n]), w)
+    dt = time.perf_counter() - t0
+    return {"value": seconds / dt, "unit": UNIT, "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
+            "sample": f"first {seconds:.0f} s of the 90 s workload clip, full model, fp64 numpy, one pass "
+                      f"({dt:.1f} s)"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    import oracle as O
+    from synth import FULL, clip_for_config, make_weights
+    w = make_weights(FULL, seed=0)
+    audio, _, _ = clip_for_config(1)
+    n = 10 * 16000
+    x = audio[:, :n]
+    for _ in range(args.warmup):
+        O.forward_offline(x, np.array([n]), w)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        O.forward_offline(x, np.array([n]), w)
+        times.append(time.perf_counter() - t0)
+    ms = 1000 * float(np.mean(times))
+    v = 10.0 / (ms / 1000)
+    cores = len(os.sched_getaffinity(0))
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": CONFIG,
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": "each step: first 10 s of the 90 s workload clip, full model, fp64 numpy"},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import torch
+    import torch.distributed as dist
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    from streaming_speaker_diarization_b200 import binding as b
+    from synth import FULL, clip_for_config, make_weights, weights_blob
+
+    audio_np, lens, _ = clip_for_config(1)
+    w = make_weights(FULL, seed=0)
+    eng = b.sf_create(weights_blob(w), b.default_config(max_batch=1))
+    st = torch.cuda.current_stream()
+    audio = torch.from_numpy(audio_np).cuda()
+    probs = torch.zeros((1, 1125, 4), device="cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        b.sf_forward_offline(eng, audio, lens, probs)
+    torch.cuda.synchronize()
+    b.sf_profile_read(eng, reset=True)
+
+    # timed region: per-step CUDA events on the launching stream, L2 flushed between steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier()
+    clk = Clocks(local)
+    for i in range(args.steps):
+        flush.zero_()
+        ev[i][0].record(st)
+        b.sf_forward_offline(eng, audio, lens, probs)
+        ev[i][1].record(st)
+    barrier()
+    clocks = clk.stop()
+    step_ms = [a.elapsed_time(c) for a, c in ev]
+    stats = b.sf_profile_read(eng, reset=True)
+    launches = int(sum(v[0] for v in stats.values()))
+    total_ms = float(sum(step_ms))
+    t = torch.tensor([total_ms], device="cuda", dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    max_ms = float(t.item())
+    audio_s = 90.0 * args.steps * world
+    value = audio_s / (max_ms / 1000.0)
+
+    # per-kernel attribution: the same K steps again with CUDA events around every launch
+    b.sf_profile_enable(eng, True)
+    for i in range(args.steps):
+        flush.zero_()
+        b.sf_forward_offline(eng, audio, lens, probs)
+    torch.cuda.synchronize()
+    prof = b.sf_profile_read(eng, reset=True)
+    b.sf_profile_enable(eng, False)
+
+    # end to end through the host-memory entry point (H2D + compute + D2H every step)
+    h_audio = torch.from_numpy(audio_np).pin_memory()
+    h_probs = torch.zeros((1, 1125, 4)).pin_memory()
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    b.sf_forward_offline_host(eng, h_audio.numpy(), lens, h_probs.numpy())
+    barrier()
+    for i in range(args.steps):
+        flush.zero_()
+        e2e_ev[i][0].record(st)
+        b.sf_forward_offline_host(eng, h_audio.numpy(), lens, h_probs.numpy())
+        e2e_ev[i][1].record(st)
+    barrier()
+    e2e_ms = float(sum(a.elapsed_time(c) for a, c in e2e_ev))
+    te = torch.tensor([e2e_ms], device="cuda", dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_value = audio_s / (float(te.item()) / 1000.0)
+
+    pk, pk_kind = peaks()
+    g = prof.get("gemm", (0, 0.0, 0.0, 0.0))
+    timed_s = max_ms / 1000.0
+    peak_tf = pk["bf16_tflops_sustained"] if timed_s > 1.0 else pk["bf16_tflops"]
+    achieved = (g[2] / (g[1] / 1000.0)) / 1e12 if g[1] > 0 else None
+    roof = {"bound": "tensor", "kernel": "gemm (all projection launches)", "achieved": achieved, "peak": peak_tf,
+            "unit": "TFLOP/s", "frac": (achieved / peak_tf) if achieved else None, "traffic": None,
+            "peak_kind": f"{pk_kind} bf16 {'sustained' if timed_s > 1.0 else 'burst'}",
+            "launches_per_step": g[0] / args.steps if args.steps else None,
+            "ms_per_step": g[1] / args.steps if args.steps else None}
+    kernels = {k: {"launches": int(v[0]), "ms": round(v[1], 4),
+                   "tflops": round(v[2] / (v[1] / 1000) / 1e12, 2) if v[1] > 0 and v[2] > 0 else None,
+                   "gbs": round(v[3] / (v[1] / 1000) / 1e9, 1) if v[1] > 0 and v[3] > 0 else None}
+               for k, v in sorted(prof.items(), key=lambda kv: -kv[1][1])}
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": dict(CONFIG, parallelism=f"replicas x{world}"),
+            "roofline": roof, "clocks": clocks, "gpu_launches": launches,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(audio_np.nbytes),
+                    "d2h_bytes_per_step": int(h_probs.numel() * 4)},
+            "step_ms_p50": float(np.median(step_ms)), "step_ms_p95": float(np.percentile(step_ms, 95)),
+            "kernels": kernels}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(audio_np)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    b.sf_destroy(eng)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -28,7 +28,9 @@
  *    SF_ETIMEOUT reports that a bounded device-side wait gave up (the
  *    engine's kernels never spin without a limit).
  *  - An engine or stream object must not be used from two host threads at
- *    once.
+ *    once, and calls on one engine must be ordered: issue them on one CUDA
+ *    stream (or order the streams yourself), because every call reuses the
+ *    engine's workspace and descriptor block.
  */
 #ifndef SF_H_
 #define SF_H_
@@ -260,6 +262,29 @@ SF_API sf_status sf_stream_update(sf_stream* s, const float* d_preds, const void
  * Order: score descending, candidate index ascending; -inf never kept. */
 SF_API sf_status sf_select_topk(sf_engine* e, const float* d_scores, const int* h_n, int n_sets, int stride, int k,
                          int* d_src, void* cuda_stream);
+
+/* ---------------------------------------------------------------- profiling */
+
+/* Per kernel class: launches, device time between CUDA events recorded on
+ * the launching stream around each launch, and the algorithmic work of those
+ * launches (flops of the contraction, or the bytes the operation must move
+ * through HBM at minimum). */
+typedef struct {
+  char name[32];
+  int64_t launches;
+  double ms;
+  double flops;
+  double bytes;
+} sf_kernel_stat;
+
+/* Launch counting is always on.  enable = 1 also brackets every launch with
+ * a pair of CUDA events (adds a few microseconds of event records per
+ * launch; use for attribution, not for end-to-end timing). */
+SF_API sf_status sf_profile_enable(sf_engine* e, int enable);
+/* Synchronise on the recorded events and report one entry per kernel class
+ * with at least one launch since the last reset (at most `max` entries,
+ * count in *n_out).  reset = 1 clears the counters afterwards. */
+SF_API sf_status sf_profile_read(sf_engine* e, sf_kernel_stat* out, int max, int* n_out, int reset);
 
 #ifdef __cplusplus
 }

@@ -188,11 +188,14 @@ def state_update(st, P, chunk_embs, n_chunk, preset, scores=None):
 def _decision_margin(P, sc, k):
     """Smallest distance of any float decision to its threshold: |p - 0.5|
     over the frames, the gap between the two largest probabilities of a
-    frame (the argmax), and the score gap at each speaker's top-k boundary."""
+    frame whose largest probability exceeds 0.5 (the argmax decides its
+    speaker), and the score gap at each speaker's top-k boundary."""
     m = float(np.min(np.abs(P - 0.5))) if P.size else np.inf
     if P.shape[1] > 1 and P.size:
         s = np.sort(P, axis=1)
-        m = min(m, float(np.min(s[:, -1] - s[:, -2])))
+        live = s[:, -1] > 0.5
+        if live.any():
+            m = min(m, float(np.min(s[live, -1] - s[live, -2])))
     if sc is not None:
         for s_ in range(sc.shape[1]):
             f = np.sort(sc[np.isfinite(sc[:, s_]), s_])[::-1]

@@ -40,11 +40,16 @@ class sf_state_view(ctypes.Structure):
                 ("d_fifo_emb", ctypes.c_void_p), ("d_fifo_preds", ctypes.c_void_p), ("d_sil_mean", ctypes.c_void_p)]
 
 
+class sf_kernel_stat(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 32), ("launches", ctypes.c_int64), ("ms", ctypes.c_double),
+                ("flops", ctypes.c_double), ("bytes", ctypes.c_double)]
+
+
 EXPORTED = ["sf_default_config", "sf_create", "sf_create_from_file", "sf_destroy", "sf_get_metadata",
             "sf_last_error", "sf_status_str", "sf_mel", "sf_pre_encode", "sf_encode", "sf_forward_offline",
             "sf_forward_offline_host", "sf_stream_create", "sf_stream_destroy", "sf_stream_reset",
             "sf_stream_window", "sf_stream_step", "sf_stream_get_state", "sf_stream_set_state",
-            "sf_stream_update", "sf_select_topk"]
+            "sf_stream_update", "sf_select_topk", "sf_profile_enable", "sf_profile_read"]
 
 
 class SFError(RuntimeError):
@@ -78,6 +83,8 @@ def _load():
         "sf_stream_set_state": ([VP, I, P(sf_state_view), VP], I),
         "sf_stream_update": ([VP, VP, VP, I64, VP, VP, VP, VP, VP], I),
         "sf_select_topk": ([VP, VP, VP, I, I, I, VP, VP], I),
+        "sf_profile_enable": ([VP, I], I),
+        "sf_profile_read": ([VP, P(sf_kernel_stat), I, P(I), I], I),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -236,3 +243,15 @@ def sf_select_topk(eng, scores, n, k, src, stream=None):
     n = np.ascontiguousarray(n, np.int32)
     n_sets, stride, _ = scores.shape
     _check(lib.sf_select_topk(eng, _ptr(scores), _ptr(n), n_sets, stride, k, _ptr(src), _stream(stream)), eng)
+
+
+def sf_profile_enable(eng, enable=True):
+    _check(lib.sf_profile_enable(eng, int(bool(enable))), eng)
+
+
+def sf_profile_read(eng, reset=True):
+    """Per kernel class: dict name -> (launches, ms, flops, bytes)."""
+    arr = (sf_kernel_stat * 32)()
+    n = ctypes.c_int()
+    _check(lib.sf_profile_read(eng, arr, 32, ctypes.byref(n), int(bool(reset))), eng)
+    return {arr[i].name.decode(): (arr[i].launches, arr[i].ms, arr[i].flops, arr[i].bytes) for i in range(n.value)}

@@ -118,6 +118,20 @@ struct Arena {
 
 }  // namespace
 
+namespace {
+enum KClass : int {
+  K_MEL = 0, K_CONV1, K_DW2D, K_GEMM, K_ATT_REL, K_ATT_MHA, K_LN, K_DW1D, K_HEAD, K_ASSEMBLE, K_EXTRACT,
+  K_UPDATE, K_TOF32, K_SELECT, K_COUNT
+};
+const char* const KNAMES[K_COUNT] = {"mel", "conv1", "dwconv3x3s2", "gemm", "attention_relpos", "attention_mha",
+                                     "layernorm", "dwconv1d", "head_out", "assemble", "extract", "state_update",
+                                     "to_f32", "select_topk"};
+struct ProfRec {
+  int cls;
+  cudaEvent_t a, b;
+};
+}  // namespace
+
 struct sf_engine {
   sf_config cfg{};
   int device = 0;
@@ -134,6 +148,15 @@ struct sf_engine {
   int* d_err = nullptr;
   Weights<float> wf;
   Weights<bf16> wb;
+  // profiling: launch/work counters always; event pairs when prof is set
+  bool prof = false;
+  int64_t launches[K_COUNT] = {};
+  double kflops[K_COUNT] = {};
+  double kbytes[K_COUNT] = {};
+  std::vector<ProfRec> recs;
+  std::vector<cudaEvent_t> pool;
+  size_t pool_used = 0;
+  double att_s2 = 0;      // sum of squared sequence lengths of the current call
   // workspace (grow-only)
   Buf mel, part, audio, sub1, sub2a, sub2b, sub3a, sub3b, emb, x, h, big, ctx, x2, h2, probs, out;
 };
@@ -158,6 +181,45 @@ sf_status cuda_fail(sf_engine* e, cudaError_t c, const char* where) {
   return fail(e, c == cudaErrorMemoryAllocation ? SF_ENOMEM : SF_ECUDA,
               std::string(where) + ": " + cudaGetErrorString(c));
 }
+
+cudaEvent_t pool_event(sf_engine* e) {
+  if (e->pool_used == e->pool.size()) {
+    cudaEvent_t ev;
+    if (cudaEventCreate(&ev) != cudaSuccess) return nullptr;
+    e->pool.push_back(ev);
+  }
+  return e->pool[e->pool_used++];
+}
+
+// Accounts one launch site: counters always, an event pair when profiling.
+struct Scope {
+  sf_engine* e;
+  cudaStream_t st;
+  cudaEvent_t b = nullptr;
+  Scope(sf_engine* e_, int cls, int n_kernels, double flops, double bytes, cudaStream_t st_) : e(e_), st(st_) {
+    e->launches[cls] += n_kernels;
+    e->kflops[cls] += flops;
+    e->kbytes[cls] += bytes;
+    if (e->prof) {
+      cudaEvent_t a = pool_event(e);
+      b = pool_event(e);
+      if (a && b) {
+        cudaEventRecord(a, st);
+        e->recs.push_back({cls, a, b});
+      } else {
+        b = nullptr;
+      }
+    }
+  }
+  ~Scope() {
+    if (b) cudaEventRecord(b, st);
+  }
+};
+#define RUN(cls, nk, flops, bytes, call)                 \
+  do {                                                   \
+    Scope _scope(e, cls, nk, (double)(flops), (double)(bytes), st); \
+    CK(call);                                            \
+  } while (0)
 
 cudaError_t ensure(Buf& b, size_t bytes) {
   if (bytes <= b.bytes) return cudaSuccess;
@@ -458,6 +520,16 @@ cudaError_t gemm<bf16>(const bf16* A, int lda, const bf16* W, int M, int N, int 
   return gemm_bf16_mma(A, lda, W, M, N, K, ep, st);
 }
 
+template <typename T>
+cudaError_t gemm_acc(sf_engine* e, const T* A, int lda, const T* W, int M, int N, int K, const Epi& ep,
+                     cudaStream_t st) {
+  const double a = sizeof(T);
+  const double out_b = (ep.kind == EPI_RESID) ? 8.0 : (ep.kind == EPI_F32 ? 4.0 : (ep.kind == EPI_F32_AND_T ? 4.0 + a : (ep.kind == EPI_BIAS_GLU ? a / 2 : a)));
+  RUN(K_GEMM, 1, 2.0 * M * N * K, ((double)M * K + (double)N * K) * a + (double)M * N * out_b,
+      gemm<T>(A, lda, W, M, N, K, ep, st));
+  return cudaSuccess;
+}
+
 Epi epi(int kind, const float* bias, void* out, int ldo, float alpha = 1.f) {
   Epi e{};
   e.kind = kind;
@@ -483,6 +555,11 @@ cudaError_t desc_upload(sf_engine* e, cudaStream_t st) {
   return cudaSuccess;
 }
 // Fill the sequence table from lengths; returns total rows and tile count.
+double sum_sq(const std::vector<int>& lens) {
+  double s2 = 0;
+  for (int v : lens) s2 += (double)v * v;
+  return s2;
+}
 void fill_seq(DescBlock* d, const std::vector<int>& lens, int& M, int& tiles) {
   d->seq.n_seq = (int)lens.size();
   M = 0;
@@ -518,15 +595,18 @@ cudaError_t run_pre_encode(sf_engine* e, const float* feats, int64_t t_buf, int 
   T* s2b = static_cast<T*>(e->sub2b.p);
   T* s3a = static_cast<T*>(e->sub3a.p);
   T* s3b = static_cast<T*>(e->sub3b.p);
-  CK(launch_conv1<T>(feats, t_buf, pa, n_win, W.c1_w, W.c1_b, s1, T1, st));
-  CK(launch_dwconv3x3s2<T>(s1, T1, 64, s2a, T2, 32, pa, n_win, 1, W.dw_w[0], W.dw_b[0], st));
-  CK(gemm<T>(s2a, 256, W.pw_w[0], n_win * T2 * 32, 256, 256, epi(EPI_BIAS_RELU, W.pw_b[0], s2b, 256), st));
-  CK(launch_dwconv3x3s2<T>(s2b, T2, 32, s3a, T3, 16, pa, n_win, 2, W.dw_w[1], W.dw_b[1], st));
-  CK(gemm<T>(s3a, 256, W.pw_w[1], n_win * T3 * 16, 256, 256, epi(EPI_BIAS_RELU, W.pw_b[1], s3b, 256), st));
+  RUN(K_CONV1, 1, 18.0 * 256 * 64 * T1 * n_win, (double)n_win * W_max * 128 * 4 + (double)n_win * T1 * 64 * 256 * sizeof(T),
+      launch_conv1<T>(feats, t_buf, pa, n_win, W.c1_w, W.c1_b, s1, T1, st));
+  RUN(K_DW2D, 1, 18.0 * 256 * 32 * T2 * n_win, (double)n_win * (T1 * 64 + T2 * 32) * 256 * sizeof(T),
+      launch_dwconv3x3s2<T>(s1, T1, 64, s2a, T2, 32, pa, n_win, 1, W.dw_w[0], W.dw_b[0], st));
+  CK(gemm_acc<T>(e, s2a, 256, W.pw_w[0], n_win * T2 * 32, 256, 256, epi(EPI_BIAS_RELU, W.pw_b[0], s2b, 256), st));
+  RUN(K_DW2D, 1, 18.0 * 256 * 16 * T3 * n_win, (double)n_win * (T2 * 32 + T3 * 16) * 256 * sizeof(T),
+      launch_dwconv3x3s2<T>(s2b, T2, 32, s3a, T3, 16, pa, n_win, 2, W.dw_w[1], W.dw_b[1], st));
+  CK(gemm_acc<T>(e, s3a, 256, W.pw_w[1], n_win * T3 * 16, 256, 256, epi(EPI_BIAS_RELU, W.pw_b[1], s3b, 256), st));
   Epi eo = epi(EPI_BIAS, W.out_b, out, D);
   eo.rpg = T3;
   eo.gstride = out_stride;
-  CK(gemm<T>(s3b, 16 * 256, W.out_w, n_win * T3, D, 16 * 256, eo, st));
+  CK(gemm_acc<T>(e, s3b, 16 * 256, W.out_w, n_win * T3, D, 16 * 256, eo, st));
   return cudaSuccess;
 }
 
@@ -544,21 +624,28 @@ cudaError_t run_encode(sf_engine* e, int M, int n_tiles, float* probs, cudaStrea
   T* ctx = static_cast<T*>(e->ctx.p);
   for (int l = 0; l < c.n_conformer; ++l) {
     const ConfW<T>& w = W.conf[l];
-    CK(launch_layernorm<T>(x, w.ff1_g, w.ff1_b, M, D, false, h, st));
-    CK(gemm<T>(h, D, w.ff1_w1, M, DFF, D, epi(EPI_BIAS_SWISH, w.ff1_b1, big, DFF), st));
-    CK(gemm<T>(big, DFF, w.ff1_w2, M, D, DFF, epi(EPI_RESID, w.ff1_b2, x, D, 0.5f), st));
-    CK(launch_layernorm<T>(x, w.att_g, w.att_b, M, D, false, h, st));
-    CK(gemm<T>(h, D, w.wqkv, M, 3 * D, D, epi(EPI_BIAS, w.bqkv, big, 3 * D), st));
-    CK(launch_relpos_attention<T>(big, w.ptab, e->R, w.pu, w.pv, ctx, seq, n_tiles, M, st));
-    CK(gemm<T>(ctx, D, w.wo, M, D, D, epi(EPI_RESID, w.bo, x, D, 1.f), st));
-    CK(launch_layernorm<T>(x, w.conv_g, w.conv_b, M, D, false, h, st));
-    CK(gemm<T>(h, D, w.pw1, M, 2 * D, D, epi(EPI_BIAS_GLU, w.pw1_b, ctx, D), st));
-    CK(launch_dwconv1d<T>(ctx, h, w.dw_w, w.dw_b, M, D, c.conv_kernel, seq, st));
-    CK(gemm<T>(h, D, w.pw2, M, D, D, epi(EPI_RESID, w.pw2_b, x, D, 1.f), st));
-    CK(launch_layernorm<T>(x, w.ff2_g, w.ff2_b, M, D, false, h, st));
-    CK(gemm<T>(h, D, w.ff2_w1, M, DFF, D, epi(EPI_BIAS_SWISH, w.ff2_b1, big, DFF), st));
-    CK(gemm<T>(big, DFF, w.ff2_w2, M, D, DFF, epi(EPI_RESID, w.ff2_b2, x, D, 0.5f), st));
-    CK(launch_layernorm<T>(x, w.out_g, w.out_b, M, D, true, h, st));
+    RUN(K_LN, 1, 0, (double)M * D * (4 + sizeof(T) + (false ? 4 : 0)),
+        launch_layernorm<T>(x, w.ff1_g, w.ff1_b, M, D, false, h, st));
+    CK(gemm_acc<T>(e, h, D, w.ff1_w1, M, DFF, D, epi(EPI_BIAS_SWISH, w.ff1_b1, big, DFF), st));
+    CK(gemm_acc<T>(e, big, DFF, w.ff1_w2, M, D, DFF, epi(EPI_RESID, w.ff1_b2, x, D, 0.5f), st));
+    RUN(K_LN, 1, 0, (double)M * D * (4 + sizeof(T) + (false ? 4 : 0)),
+        launch_layernorm<T>(x, w.att_g, w.att_b, M, D, false, h, st));
+    CK(gemm_acc<T>(e, h, D, w.wqkv, M, 3 * D, D, epi(EPI_BIAS, w.bqkv, big, 3 * D), st));
+    RUN(K_ATT_REL, 1, 6.0 * e->att_s2 * D, (double)M * 4 * D * sizeof(T),
+        launch_relpos_attention<T>(big, w.ptab, e->R, w.pu, w.pv, ctx, seq, n_tiles, M, st));
+    CK(gemm_acc<T>(e, ctx, D, w.wo, M, D, D, epi(EPI_RESID, w.bo, x, D, 1.f), st));
+    RUN(K_LN, 1, 0, (double)M * D * (4 + sizeof(T) + (false ? 4 : 0)),
+        launch_layernorm<T>(x, w.conv_g, w.conv_b, M, D, false, h, st));
+    CK(gemm_acc<T>(e, h, D, w.pw1, M, 2 * D, D, epi(EPI_BIAS_GLU, w.pw1_b, ctx, D), st));
+    RUN(K_DW1D, 1, 2.0 * M * D * c.conv_kernel, (double)M * D * 2 * sizeof(T),
+        launch_dwconv1d<T>(ctx, h, w.dw_w, w.dw_b, M, D, c.conv_kernel, seq, st));
+    CK(gemm_acc<T>(e, h, D, w.pw2, M, D, D, epi(EPI_RESID, w.pw2_b, x, D, 1.f), st));
+    RUN(K_LN, 1, 0, (double)M * D * (4 + sizeof(T) + (false ? 4 : 0)),
+        launch_layernorm<T>(x, w.ff2_g, w.ff2_b, M, D, false, h, st));
+    CK(gemm_acc<T>(e, h, D, w.ff2_w1, M, DFF, D, epi(EPI_BIAS_SWISH, w.ff2_b1, big, DFF), st));
+    CK(gemm_acc<T>(e, big, DFF, w.ff2_w2, M, D, DFF, epi(EPI_RESID, w.ff2_b2, x, D, 0.5f), st));
+    RUN(K_LN, 1, 0, (double)M * D * (4 + sizeof(T) + (true ? 4 : 0)),
+        launch_layernorm<T>(x, w.out_g, w.out_b, M, D, true, h, st));
   }
   float* x2 = static_cast<float*>(e->x2.p);
   T* h2 = static_cast<T*>(e->h2.p);
@@ -566,20 +653,22 @@ cudaError_t run_encode(sf_engine* e, int M, int n_tiles, float* probs, cudaStrea
     Epi ep = epi(EPI_F32_AND_T, W.proj_b, x2, E);
     ep.out2 = h2;
     ep.ldo2 = E;
-    CK(gemm<T>(h, D, W.proj_w, M, E, D, ep, st));
+    CK(gemm_acc<T>(e, h, D, W.proj_w, M, E, D, ep, st));
   }
   for (int l = 0; l < c.n_transformer; ++l) {
     const TfW<T>& w = W.tf[l];
-    CK(gemm<T>(h2, E, w.wqkv, M, 3 * E, E, epi(EPI_BIAS, w.bqkv, big, 3 * E), st));
-    CK(launch_mha<T>(big, ctx, seq, n_tiles, M, st));
-    CK(gemm<T>(ctx, E, w.wo, M, E, E, epi(EPI_RESID, w.bo, x2, E, 1.f), st));
-    CK(launch_layernorm<T>(x2, w.ln1_g, w.ln1_b, M, E, true, h2, st));
-    CK(gemm<T>(h2, E, w.w1, M, c.tf_ff, E, epi(EPI_BIAS_RELU, w.b1, big, c.tf_ff), st));
-    CK(gemm<T>(big, c.tf_ff, w.w2, M, E, c.tf_ff, epi(EPI_RESID, w.b2, x2, E, 1.f), st));
-    CK(launch_layernorm<T>(x2, w.ln2_g, w.ln2_b, M, E, true, h2, st));
+    CK(gemm_acc<T>(e, h2, E, w.wqkv, M, 3 * E, E, epi(EPI_BIAS, w.bqkv, big, 3 * E), st));
+    RUN(K_ATT_MHA, 1, 4.0 * e->att_s2 * E, (double)M * 4 * E * sizeof(T), launch_mha<T>(big, ctx, seq, n_tiles, M, st));
+    CK(gemm_acc<T>(e, ctx, E, w.wo, M, E, E, epi(EPI_RESID, w.bo, x2, E, 1.f), st));
+    RUN(K_LN, 1, 0, (double)M * E * (4 + sizeof(T) + (true ? 4 : 0)),
+        launch_layernorm<T>(x2, w.ln1_g, w.ln1_b, M, E, true, h2, st));
+    CK(gemm_acc<T>(e, h2, E, w.w1, M, c.tf_ff, E, epi(EPI_BIAS_RELU, w.b1, big, c.tf_ff), st));
+    CK(gemm_acc<T>(e, big, c.tf_ff, w.w2, M, E, c.tf_ff, epi(EPI_RESID, w.b2, x2, E, 1.f), st));
+    RUN(K_LN, 1, 0, (double)M * E * (4 + sizeof(T) + (true ? 4 : 0)),
+        launch_layernorm<T>(x2, w.ln2_g, w.ln2_b, M, E, true, h2, st));
   }
-  CK(gemm<T>(h2, E, W.head_w1, M, E, E, epi(EPI_BIAS_RELU, W.head_b1, ctx, E), st));
-  CK(launch_head_out<T>(ctx, W.head_w2, W.head_b2, probs, M, E, st));
+  CK(gemm_acc<T>(e, h2, E, W.head_w1, M, E, E, epi(EPI_BIAS_RELU, W.head_b1, ctx, E), st));
+  RUN(K_HEAD, 1, 2.0 * M * E * 4, (double)M * (E * sizeof(T) + 16), launch_head_out<T>(ctx, W.head_w2, W.head_b2, probs, M, E, st));
   return cudaSuccess;
 }
 
@@ -618,6 +707,7 @@ cudaError_t offline_impl(sf_engine* e, const float* d_audio, const std::vector<i
   }
   int M, tiles;
   fill_seq(d, tp, M, tiles);
+  e->att_s2 = sum_sq(tp);
   const int T3 = (int)enc_frames(L_max);
   const int Tp_max = (int)enc_frames(n_max / 160);
   CK(ensure(e->mel, (size_t)B * 128 * T_cols * 4));
@@ -626,15 +716,18 @@ cudaError_t offline_impl(sf_engine* e, const float* d_audio, const std::vector<i
   CK(ensure_encode_ws(e, M));
   CK(desc_upload(e, st));
   MelArgs ma{e->d_desc->len};
-  CK(launch_mel(d_audio, B, n_max, ma, e->d_mel_tab, static_cast<float*>(e->mel.p), static_cast<float*>(e->part.p), st));
+  RUN(K_MEL, 2, 0, (double)B * n_max * 4 + (double)B * 128 * T_cols * 4,
+      launch_mel(d_audio, B, n_max, ma, e->d_mel_tab, static_cast<float*>(e->mel.p), static_cast<float*>(e->part.p), st));
   CK(run_pre_encode<T>(e, static_cast<float*>(e->mel.p), T_cols, B, L_max, static_cast<T*>(e->emb.p), T3, st));
   StateBufs none{};
   none.D = e->cfg.d_model;
-  CK(launch_assemble<T>(static_cast<float*>(e->x.p), &e->d_desc->seq, &e->d_desc->step, none,
-                        static_cast<T*>(e->emb.p), T3, M, st));
+  RUN(K_ASSEMBLE, 1, 0, (double)M * e->cfg.d_model * (4 + sizeof(T)),
+      launch_assemble<T>(static_cast<float*>(e->x.p), &e->d_desc->seq, &e->d_desc->step, none,
+                         static_cast<T*>(e->emb.p), T3, M, st));
   CK(run_encode<T>(e, M, tiles, static_cast<float*>(e->probs.p), st));
-  CK(launch_extract_rows(static_cast<float*>(e->probs.p), &e->d_desc->seq, nullptr, nullptr, nullptr, B, d_probs,
-                         Tp_max, st));
+  RUN(K_EXTRACT, 1, 0, (double)M * 16 + (double)B * Tp_max * 16,
+      launch_extract_rows(static_cast<float*>(e->probs.p), &e->d_desc->seq, nullptr, nullptr, nullptr, B, d_probs,
+                          Tp_max, st));
   return cudaSuccess;
 }
 
@@ -781,6 +874,7 @@ sf_status sf_destroy(sf_engine* e) {
   if (e->d_desc) cudaFree(e->d_desc);
   if (e->h_desc) cudaFreeHost(e->h_desc);
   if (e->desc_ev) cudaEventDestroy(e->desc_ev);
+  for (cudaEvent_t ev : e->pool) cudaEventDestroy(ev);
   if (e->d_err) cudaFree(e->d_err);
   delete e;
   return SF_OK;
@@ -806,7 +900,10 @@ sf_status sf_mel(sf_engine* e, const float* d_audio, const int64_t* h_len, int B
   cudaError_t ce = ensure(e->part, mel_part_floats(B, n_max) * 4);
   if (ce == cudaSuccess) ce = desc_upload(e, st);
   MelArgs ma{e->d_desc->len};
-  if (ce == cudaSuccess) ce = launch_mel(d_audio, B, n_max, ma, e->d_mel_tab, d_mel, static_cast<float*>(e->part.p), st);
+  if (ce == cudaSuccess) {
+    Scope sc(e, K_MEL, 2, 0, (double)B * n_max * 4 + (double)B * 128 * (1 + n_max / 160) * 4, st);
+    ce = launch_mel(d_audio, B, n_max, ma, e->d_mel_tab, d_mel, static_cast<float*>(e->part.p), st);
+  }
   if (ce != cudaSuccess) return cuda_fail(e, ce, "sf_mel");
   if (h_mel_len)
     for (int b = 0; b < B; ++b) h_mel_len[b] = len[b] / 160;
@@ -889,16 +986,57 @@ sf_status sf_encode(sf_engine* e, const void* d_embs, const int* h_seq_len, int 
   DescBlock* d = desc_begin(e);
   int M, tiles;
   fill_seq(d, lens, M, tiles);
+  e->att_s2 = sum_sq(lens);
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
   cudaError_t ce = ensure_encode_ws(e, M);
   if (ce == cudaSuccess) ce = desc_upload(e, st);
   const int64_t nel = (int64_t)M * e->cfg.d_model;
-  if (ce == cudaSuccess)
+  if (ce == cudaSuccess) {
+    Scope sc(e, K_TOF32, 1, 0, (double)nel * (4 + act_size(e)), st);
     ce = e->cfg.precision == SF_BF16 ? launch_to_f32<bf16>(static_cast<const bf16*>(d_embs), static_cast<float*>(e->x.p), nel, st)
                                      : launch_to_f32<float>(static_cast<const float*>(d_embs), static_cast<float*>(e->x.p), nel, st);
+  }
   if (ce == cudaSuccess)
     ce = e->cfg.precision == SF_BF16 ? run_encode<bf16>(e, M, tiles, d_preds, st) : run_encode<float>(e, M, tiles, d_preds, st);
   if (ce != cudaSuccess) return cuda_fail(e, ce, "sf_encode");
+  return SF_OK;
+}
+
+sf_status sf_profile_enable(sf_engine* e, int enable) {
+  if (!e) return SF_EINVAL;
+  e->prof = enable != 0;
+  return SF_OK;
+}
+
+sf_status sf_profile_read(sf_engine* e, sf_kernel_stat* out, int max, int* n_out, int reset) {
+  if (!e || !n_out || (max > 0 && !out)) return SF_EINVAL;
+  double ms[K_COUNT] = {};
+  for (const ProfRec& r : e->recs) {
+    float t = 0.f;
+    if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess)
+      return fail(e, SF_ECUDA, "sf_profile_read: event query failed");
+    ms[r.cls] += t;
+  }
+  int n = 0;
+  for (int k = 0; k < K_COUNT; ++k) {
+    if (e->launches[k] == 0) continue;
+    if (n < max) {
+      sf_kernel_stat& o = out[n];
+      memset(&o, 0, sizeof(o));
+      strncpy(o.name, KNAMES[k], sizeof(o.name) - 1);
+      o.launches = e->launches[k];
+      o.ms = ms[k];
+      o.flops = e->kflops[k];
+      o.bytes = e->kbytes[k];
+    }
+    ++n;
+  }
+  *n_out = n;
+  if (reset) {
+    for (int k = 0; k < K_COUNT; ++k) e->launches[k] = 0, e->kflops[k] = e->kbytes[k] = 0;
+    e->recs.clear();
+    e->pool_used = 0;
+  }
   return SF_OK;
 }
 
@@ -915,7 +1053,10 @@ sf_status sf_select_topk(sf_engine* e, const float* d_scores, const int* h_n, in
   }
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
   cudaError_t ce = desc_upload(e, st);
-  if (ce == cudaSuccess) ce = launch_select_topk(d_scores, e->d_desc->n_cand, n_sets, stride, k, d_src, st);
+  if (ce == cudaSuccess) {
+    Scope sc(e, K_SELECT, 1, 0, 0, st);
+    ce = launch_select_topk(d_scores, e->d_desc->n_cand, n_sets, stride, k, d_src, st);
+  }
   if (ce != cudaSuccess) return cuda_fail(e, ce, "sf_select_topk");
   return SF_OK;
 }
@@ -956,6 +1097,7 @@ void fill_step(sf_stream* s, DescBlock* d, const StepPlan& pl, int& M, int& tile
     lens.push_back(s->n_c[id] + s->n_f[id] + pl.n_new[i]);
   }
   fill_seq(d, lens, M, tiles);
+  s->e->att_s2 = sum_sq(lens);
 }
 
 // Host bookkeeping after a state update (sizes are data-independent).
@@ -1001,13 +1143,16 @@ cudaError_t stream_step_impl(sf_stream* s, const float* d_feats, int64_t t_buf, 
   CK(desc_upload(e, st));
   if (n < s->n) CK(cudaMemsetAsync(d_chunk_probs, 0, (size_t)s->n * s->p.chunk_len * 4 * 4, st));
   CK(run_pre_encode<T>(e, d_feats, t_buf, n, W_max, static_cast<T*>(e->emb.p), T3, st));
-  CK(launch_assemble<T>(static_cast<float*>(e->x.p), &e->d_desc->seq, &e->d_desc->step, s->sb,
-                        static_cast<T*>(e->emb.p), T3, M, st));
+  RUN(K_ASSEMBLE, 1, 0, (double)M * e->cfg.d_model * (4 + sizeof(T)),
+      launch_assemble<T>(static_cast<float*>(e->x.p), &e->d_desc->seq, &e->d_desc->step, s->sb,
+                         static_cast<T*>(e->emb.p), T3, M, st));
   CK(run_encode<T>(e, M, tiles, static_cast<float*>(e->probs.p), st));
-  CK(launch_extract_rows(static_cast<float*>(e->probs.p), &e->d_desc->seq, e->d_desc->first, e->d_desc->count,
-                         e->d_desc->dst, n, d_chunk_probs, s->p.chunk_len, st));
-  CK(launch_state_update<T>(static_cast<float*>(e->probs.p), &e->d_desc->seq, &e->d_desc->step, s->sb,
-                            static_cast<T*>(e->emb.p), T3, n, nullptr, nullptr, nullptr, 0, st));
+  RUN(K_EXTRACT, 1, 0, (double)n * s->p.chunk_len * 32,
+      launch_extract_rows(static_cast<float*>(e->probs.p), &e->d_desc->seq, e->d_desc->first, e->d_desc->count,
+                          e->d_desc->dst, n, d_chunk_probs, s->p.chunk_len, st));
+  RUN(K_UPDATE, 1, 0, 0,
+      launch_state_update<T>(static_cast<float*>(e->probs.p), &e->d_desc->seq, &e->d_desc->step, s->sb,
+                             static_cast<T*>(e->emb.p), T3, n, nullptr, nullptr, nullptr, 0, st));
   return cudaSuccess;
 }
 
@@ -1184,6 +1329,7 @@ sf_status sf_stream_update(sf_stream* s, const float* d_preds, const void* d_new
                          (size_t)new_stride * D * a, cudaMemcpyDeviceToDevice, st);
   if (ce == cudaSuccess) ce = desc_upload(e, st);
   const int score_stride = s->p.spkcache_len + s->p.fifo_len + s->p.chunk_len;
+  Scope sc(e, K_UPDATE, ce == cudaSuccess ? 1 : 0, 0, 0, st);
   if (ce == cudaSuccess)
     ce = e->cfg.precision == SF_BF16
              ? launch_state_update<bf16>(d_preds, &e->d_desc->seq, &e->d_desc->step, s->sb, static_cast<bf16*>(e->emb.p),

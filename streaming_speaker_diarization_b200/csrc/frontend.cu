@@ -7,8 +7,8 @@
 // time: windowed samples packed as 256 complex points, radix-2 FFT in shared
 // memory, split into the 257 real-FFT bins, power, sparse Slaney filterbank,
 // log.  The 32 x 128 log-mel tile is written channels-first with coalesced
-// stores, and per-bin (count, mean, M2) of the tile's valid frames go to a
-// partial-statistics buffer.
+// stores, and per-bin (count, shift, shifted sum, M2) of the tile's valid
+// frames go to a partial-statistics buffer.
 // Kernel 2 (mel_normalize): one CTA per (clip, bin) merges the partials
 // (Chan's pairwise update, double) and normalises the row in place; frames
 // >= L are zeroed.
@@ -130,23 +130,25 @@ __global__ void __launch_bounds__(256) mel_frames_kernel(const float* __restrict
     int t = t0 + f;
     if (t < T_cols) mel[((int64_t)b * 128 + m) * T_cols + t] = tile[m][f];
   }
-  // per-bin statistics of the valid frames of this tile
+  // per-bin statistics of the valid frames of this tile, shifted by the
+  // tile's first value so that a constant bin gives an exact mean
   if (tid < 128) {
     const int nv = max(0, min(MEL_FB, L - t0));
-    float mean = 0.f, m2 = 0.f;
+    float c = 0.f, sh = 0.f, m2 = 0.f;
     if (nv > 0) {
-      float s = 0.f;
-      for (int f = 0; f < nv; ++f) s += tile[tid][f];
-      mean = s / nv;
+      c = tile[tid][0];
+      for (int f = 0; f < nv; ++f) sh += tile[tid][f] - c;
+      const float mean = c + sh / nv;
       for (int f = 0; f < nv; ++f) {
         float d = tile[tid][f] - mean;
         m2 = fmaf(d, d, m2);
       }
     }
-    float* p = part + (((int64_t)b * n_blk + blk) * 128 + tid) * 3;
+    float* p = part + (((int64_t)b * n_blk + blk) * 128 + tid) * 4;
     p[0] = (float)nv;
-    p[1] = mean;
-    p[2] = m2;
+    p[1] = c;
+    p[2] = sh;
+    p[3] = m2;
   }
 }
 
@@ -158,10 +160,10 @@ __global__ void __launch_bounds__(256) mel_normalize_kernel(float* __restrict__ 
   if (threadIdx.x == 0) {
     double n = 0, mean = 0, m2 = 0;
     for (int k = 0; k < n_blk; ++k) {
-      const float* p = part + (((int64_t)b * n_blk + k) * 128 + m) * 3;
+      const float* p = part + (((int64_t)b * n_blk + k) * 128 + m) * 4;
       double nb = p[0];
       if (nb <= 0) continue;
-      double mb = p[1], m2b = p[2];
+      double mb = (double)p[1] + (double)p[2] / nb, m2b = p[3];
       double nt = n + nb, d = mb - mean;
       mean += d * nb / nt;
       m2 += m2b + d * d * n * nb / nt;
@@ -196,7 +198,7 @@ cudaError_t launch_mel(const float* audio, int B, int64_t n_max, const MelArgs& 
 size_t mel_part_floats(int B, int64_t n_max) {
   const int T_cols = (int)(1 + n_max / 160);
   const int n_blk = (T_cols + MEL_FB - 1) / MEL_FB;
-  return (size_t)B * n_blk * 128 * 3;
+  return (size_t)B * n_blk * 128 * 4;
 }
 
 }  // namespace sf

@@ -63,10 +63,12 @@ __device__ __forceinline__ void masked_scores(const float* p, float* out) {
   for (int s = 0; s < 4; ++s) out[s] = (s == top && p[top] > 0.5f) ? lo[s] + (tot - l1m[s]) : -INFINITY;
 }
 
-// Exact per-speaker top-k over sc[n][4] in shared memory.  kept[t] = speaker
-// or -1; then slot sources src[0 .. 4k) (candidate index or -1 - s).
+// Exact per-speaker top-k over sc[n][4] in shared memory.  kept[t] = bit
+// mask of the speakers that keep frame t; then slot sources src[0 .. 4k):
+// kept frames in ascending index (a frame kept by two speakers appears
+// twice), then placeholders -1 - s in speaker order.
 __device__ void select_core(const float* sc, int n, int k, int* kept, int* src, int* cnt) {
-  for (int t = threadIdx.x; t < n; t += blockDim.x) kept[t] = -1;
+  for (int t = threadIdx.x; t < n; t += blockDim.x) kept[t] = 0;
   if (threadIdx.x < 4) cnt[threadIdx.x] = 0;
   __syncthreads();
   for (int idx = threadIdx.x; idx < n * 4; idx += blockDim.x) {
@@ -78,17 +80,18 @@ __device__ void select_core(const float* sc, int n, int k, int* kept, int* src, 
       const float v2 = sc[t2 * 4 + s];
       rank += (v2 > v) || (v2 == v && t2 < t);
     }
-    if (rank < k) kept[t] = s;
+    if (rank < k) atomicOr(&kept[t], 1 << s);
   }
   __syncthreads();
   if (threadIdx.x == 0) {
     int p = 0;
     int per[4] = {0, 0, 0, 0};
     for (int t = 0; t < n; ++t)
-      if (kept[t] >= 0) {
-        src[p++] = t;
-        per[kept[t]]++;
-      }
+      for (int s = 0; s < 4; ++s)
+        if (kept[t] & (1 << s)) {
+          src[p++] = t;
+          per[s]++;
+        }
     for (int s = 0; s < 4; ++s)
       for (int j = per[s]; j < k; ++j) src[p++] = -1 - s;
     for (int s = 0; s < 4; ++s) cnt[s] = per[s];
