@@ -162,6 +162,25 @@ SF_API const char* sf_status_str(sf_status s);
 SF_API sf_status sf_mel(sf_engine* e, const float* d_audio, const int64_t* h_len, int B, int64_t n_max,
                  float* d_mel, int64_t* h_mel_len, void* cuda_stream);
 
+/* Allocation-free front-end.  The pages have no counterpart to this call: it
+ * exists for callers that cannot allocate device memory when they compute
+ * features (a pre-budgeted memory pool they do not own, a plugin inside
+ * another framework's CUDA context, a real-time thread that must not block
+ * in cudaMalloc/cudaFree).  Same arguments, layout and result as sf_mel, but
+ * no engine is needed and nothing is allocated: the call's scratch (clip
+ * lengths and per-tile statistics) is a fixed 8 MiB static device array in
+ * libsf.so that every GPU loading the library keeps until exit.
+ * Limits: B <= 64 clips and B * ceil((1 + n_max/160) / 32) <= 4096 frame
+ * tiles (e.g. 10 clips of 120 s); larger requests return SF_ESHAPE.
+ * The first call on a device takes the array's device address and uploads
+ * the FFT/window/filterbank tables with a blocking copy: make it before any
+ * CUDA stream capture.  All calls share the array and it keeps the last
+ * call's contents, so calls whose GPU work overlaps (on different streams or
+ * threads) race and corrupt each other; order them on one stream.  No error
+ * message is kept (there is no engine): the status code is the report. */
+SF_API sf_status sf_mel_noalloc(const float* d_audio, const int64_t* h_len, int B, int64_t n_max, float* d_mel,
+                                int64_t* h_mel_len, void* cuda_stream);
+
 /* ------------------------------------------------- exported-method split */
 
 /* pre_encode ("Exported Methods / pre_encode": chunk (1, T, 128) -> embs

@@ -49,7 +49,7 @@ EXPORTED = ["sf_default_config", "sf_create", "sf_create_from_file", "sf_destroy
             "sf_last_error", "sf_status_str", "sf_mel", "sf_pre_encode", "sf_encode", "sf_forward_offline",
             "sf_forward_offline_host", "sf_stream_create", "sf_stream_destroy", "sf_stream_reset",
             "sf_stream_window", "sf_stream_step", "sf_stream_get_state", "sf_stream_set_state",
-            "sf_stream_update", "sf_select_topk", "sf_profile_enable", "sf_profile_read"]
+            "sf_stream_update", "sf_select_topk", "sf_profile_enable", "sf_profile_read", "sf_mel_noalloc"]
 
 
 class SFError(RuntimeError):
@@ -85,6 +85,7 @@ def _load():
         "sf_select_topk": ([VP, VP, VP, I, I, I, VP, VP], I),
         "sf_profile_enable": ([VP, I], I),
         "sf_profile_read": ([VP, P(sf_kernel_stat), I, P(I), I], I),
+        "sf_mel_noalloc": ([VP, VP, I, I64, VP, VP, VP], I),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -154,6 +155,15 @@ def sf_mel(eng, audio, lengths, mel, stream=None):
     out_len = np.zeros_like(lengths)
     B, N = audio.shape
     _check(lib.sf_mel(eng, _ptr(audio), _ptr(lengths), B, N, _ptr(mel), _ptr(out_len), _stream(stream)), eng)
+    return out_len
+
+
+def sf_mel_noalloc(audio, lengths, mel, stream=None):
+    """Allocation-free front-end (no engine); same result as sf_mel."""
+    lengths = np.ascontiguousarray(lengths, np.int64)
+    out_len = np.zeros_like(lengths)
+    B, N = audio.shape
+    _check(lib.sf_mel_noalloc(_ptr(audio), _ptr(lengths), B, N, _ptr(mel), _ptr(out_len), _stream(stream)))
     return out_len
 
 
