@@ -282,6 +282,21 @@ SF_API sf_status sf_stream_update(sf_stream* s, const float* d_preds, const void
 SF_API sf_status sf_select_topk(sf_engine* e, const float* d_scores, const int* h_n, int n_sets, int stride, int k,
                          int* d_src, void* cuda_stream);
 
+/* ------------------------------------------------------------ diagnostics */
+
+/* Synchronise `cuda_stream` and read (then clear) the engine's device error
+ * word: SF_ETIMEOUT if a kernel's bounded wait gave up, SF_EDEVICE if a
+ * device-side index check skipped an access, SF_OK otherwise. */
+SF_API sf_status sf_check(sf_engine* e, void* cuda_stream);
+
+/* The engine's dense projection alone, for tests and kernel benchmarks:
+ *   d_C f32 [M x N] (out) = d_A bf16 [M x K] (row stride lda) .
+ *       d_W bf16 [N x K]^T + d_bias f32 [N] (may be NULL)
+ * path 1 = tcgen05/TMEM/TMA kernel (the engine's), 0 = mma.sync kernel.
+ * Requires N % 16 == 0, K % 64 == 0, lda % 8 == 0, 16-byte aligned A/W. */
+SF_API sf_status sf_gemm_bf16(sf_engine* e, const void* d_A, int lda, const void* d_W, int M, int N, int K,
+                              const float* d_bias, float* d_C, int path, void* cuda_stream);
+
 /* ---------------------------------------------------------------- profiling */
 
 /* Per kernel class: launches, device time between CUDA events recorded on

@@ -49,7 +49,8 @@ EXPORTED = ["sf_default_config", "sf_create", "sf_create_from_file", "sf_destroy
             "sf_last_error", "sf_status_str", "sf_mel", "sf_pre_encode", "sf_encode", "sf_forward_offline",
             "sf_forward_offline_host", "sf_stream_create", "sf_stream_destroy", "sf_stream_reset",
             "sf_stream_window", "sf_stream_step", "sf_stream_get_state", "sf_stream_set_state",
-            "sf_stream_update", "sf_select_topk", "sf_profile_enable", "sf_profile_read", "sf_mel_noalloc"]
+            "sf_stream_update", "sf_select_topk", "sf_profile_enable", "sf_profile_read", "sf_mel_noalloc",
+            "sf_check", "sf_gemm_bf16"]
 
 
 class SFError(RuntimeError):
@@ -86,6 +87,8 @@ def _load():
         "sf_profile_enable": ([VP, I], I),
         "sf_profile_read": ([VP, P(sf_kernel_stat), I, P(I), I], I),
         "sf_mel_noalloc": ([VP, VP, I, I64, VP, VP, VP], I),
+        "sf_check": ([VP, VP], I),
+        "sf_gemm_bf16": ([VP, VP, I, VP, I, I, I, VP, VP, I, VP], I),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -265,3 +268,14 @@ def sf_profile_read(eng, reset=True):
     n = ctypes.c_int()
     _check(lib.sf_profile_read(eng, arr, 32, ctypes.byref(n), int(bool(reset))), eng)
     return {arr[i].name.decode(): (arr[i].launches, arr[i].ms, arr[i].flops, arr[i].bytes) for i in range(n.value)}
+
+
+def sf_check(eng, stream=None):
+    _check(lib.sf_check(eng, _stream(stream)), eng)
+
+
+def sf_gemm_bf16(eng, A, W, C, bias=None, path=1, stream=None):
+    M, K = A.shape
+    N = W.shape[0]
+    _check(lib.sf_gemm_bf16(eng, _ptr(A), A.stride(0), _ptr(W), M, N, K, _ptr(bias), _ptr(C), path,
+                            _stream(stream)), eng)

@@ -311,8 +311,6 @@ cudaError_t launch_relpos_attention<float>(const float* qkv, const float* ptab, 
   if (M <= 0) return cudaSuccess;
   const int s_cap = R;   // no sequence is longer than the position table
   const size_t smem = (size_t)4 * (s_cap + 128) * 4;
-  cudaError_t e = cudaFuncSetAttribute(attn_f32_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
   attn_f32_kernel<64, true><<<dim3((M + 3) / 4, 8), 128, smem, st>>>(qkv, 512, ptab, R, u, v, ctx, seq, M, s_cap);
   return cudaGetLastError();
 }
@@ -331,8 +329,6 @@ cudaError_t launch_mha<float>(const float* qkv, float* ctx, const SeqTable* seq,
   if (M <= 0) return cudaSuccess;
   const int s_cap = g_att_s_cap;
   const size_t smem = (size_t)4 * (s_cap + 128) * 4;
-  cudaError_t e = cudaFuncSetAttribute(attn_f32_kernel<24, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
   attn_f32_kernel<24, false><<<dim3((M + 3) / 4, 8), 128, smem, st>>>(qkv, 192, nullptr, 0, nullptr, nullptr, ctx, seq,
                                                                       M, s_cap);
   return cudaGetLastError();
@@ -347,6 +343,14 @@ cudaError_t launch_mha<bf16>(const bf16* qkv, bf16* ctx, const SeqTable* seq, in
 }
 
 void attention_set_max_seq(int s) { g_att_s_cap = s; }
+
+// fp32 path: one score row of up to R floats per warp (4 warps per CTA).
+cudaError_t attention_init_f32_attributes(int R) {
+  const int smem = 4 * (R + 128) * 4;
+  cudaError_t e = cudaFuncSetAttribute(attn_f32_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(attn_f32_kernel<24, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+}
 
 cudaError_t attention_init_attributes() {
   cudaError_t e = cudaFuncSetAttribute(attn_bf16_kernel<64, 64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,

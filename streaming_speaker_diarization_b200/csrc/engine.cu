@@ -31,10 +31,16 @@
 
 using namespace sf;
 
+// Source line of the first CUDA call that failed in the current API call
+// (reported by sf_last_error).
+static int g_fail_line = 0;
 #define CK(x)                                   \
   do {                                          \
     cudaError_t _e = (x);                       \
-    if (_e != cudaSuccess) return _e;           \
+    if (_e != cudaSuccess) {                    \
+      if (!g_fail_line) g_fail_line = __LINE__; \
+      return _e;                                \
+    }                                           \
   } while (0)
 
 namespace {
@@ -146,6 +152,7 @@ struct sf_engine {
   cudaEvent_t desc_ev = nullptr;
   bool desc_pending = false;
   int* d_err = nullptr;
+  int gemm_path = 1;      // bf16 GEMMs: 1 = tcgen05 (default), 0 = mma.sync
   Weights<float> wf;
   Weights<bf16> wb;
   // profiling: launch/work counters always; event pairs when prof is set
@@ -157,6 +164,22 @@ struct sf_engine {
   std::vector<cudaEvent_t> pool;
   size_t pool_used = 0;
   double att_s2 = 0;      // sum of squared sequence lengths of the current call
+  double ms_acc[K_COUNT] = {};   // event time already read back (graph replays)
+  // CUDA graphs: one per launch shape, replayed; invalidated when the workspace moves
+  bool use_graphs = true;
+  bool capturing = false;
+  cudaStream_t cap_stream = nullptr;     // graphs are captured here, launched on the caller's stream
+  std::vector<cudaEvent_t> cap_events;   // events created for the graph being captured
+  uint64_t ws_gen = 0;
+  struct GraphEntry {
+    cudaGraphExec_t exec = nullptr;
+    uint64_t gen = 0;
+    int64_t launches[K_COUNT] = {};
+    double flops[K_COUNT] = {}, bytes[K_COUNT] = {};
+    std::vector<ProfRec> recs;
+    std::vector<cudaEvent_t> events;
+  };
+  std::unordered_map<std::string, GraphEntry> graphs;
   // workspace (grow-only)
   Buf mel, part, audio, sub1, sub2a, sub2b, sub3a, sub3b, emb, x, h, big, ctx, x2, h2, probs, out;
 };
@@ -178,8 +201,10 @@ sf_status fail(sf_engine* e, sf_status s, const std::string& msg) {
   return s;
 }
 sf_status cuda_fail(sf_engine* e, cudaError_t c, const char* where) {
-  return fail(e, c == cudaErrorMemoryAllocation ? SF_ENOMEM : SF_ECUDA,
-              std::string(where) + ": " + cudaGetErrorString(c));
+  std::string msg = std::string(where) + ": " + cudaGetErrorString(c);
+  if (g_fail_line) msg += " (engine.cu:" + std::to_string(g_fail_line) + ")";
+  g_fail_line = 0;
+  return fail(e, c == cudaErrorMemoryAllocation ? SF_ENOMEM : SF_ECUDA, msg);
 }
 
 cudaEvent_t pool_event(sf_engine* e) {
@@ -189,6 +214,13 @@ cudaEvent_t pool_event(sf_engine* e) {
     e->pool.push_back(ev);
   }
   return e->pool[e->pool_used++];
+}
+
+cudaEvent_t cap_event(sf_engine* e) {
+  cudaEvent_t ev;
+  if (cudaEventCreate(&ev) != cudaSuccess) return nullptr;
+  e->cap_events.push_back(ev);
+  return ev;
 }
 
 // Accounts one launch site: counters always, an event pair when profiling.
@@ -201,10 +233,11 @@ struct Scope {
     e->kflops[cls] += flops;
     e->kbytes[cls] += bytes;
     if (e->prof) {
-      cudaEvent_t a = pool_event(e);
-      b = pool_event(e);
+      cudaEvent_t a = e->capturing ? cap_event(e) : pool_event(e);
+      b = e->capturing ? cap_event(e) : pool_event(e);
       if (a && b) {
-        cudaEventRecord(a, st);
+        // inside a capture, only an "external" record becomes an event node of the graph
+        cudaEventRecordWithFlags(a, st, e->capturing ? cudaEventRecordExternal : cudaEventRecordDefault);
         e->recs.push_back({cls, a, b});
       } else {
         b = nullptr;
@@ -212,7 +245,7 @@ struct Scope {
     }
   }
   ~Scope() {
-    if (b) cudaEventRecord(b, st);
+    if (b) cudaEventRecordWithFlags(b, st, e->capturing ? cudaEventRecordExternal : cudaEventRecordDefault);
   }
 };
 #define RUN(cls, nk, flops, bytes, call)                 \
@@ -221,8 +254,11 @@ struct Scope {
     CK(call);                                            \
   } while (0)
 
+uint64_t* g_ws_gen = nullptr;   // generation counter of the engine whose buffers ensure() grows
+
 cudaError_t ensure(Buf& b, size_t bytes) {
   if (bytes <= b.bytes) return cudaSuccess;
+  if (g_ws_gen) ++*g_ws_gen;
   if (b.p) CK(cudaFree(b.p));
   b.p = nullptr;
   b.bytes = 0;
@@ -521,12 +557,27 @@ cudaError_t gemm<bf16>(const bf16* A, int lda, const bf16* W, int M, int N, int 
 }
 
 template <typename T>
+cudaError_t gemm_dispatch(sf_engine* e, const T* A, int lda, const T* W, int M, int N, int K, const Epi& ep,
+                          cudaStream_t st);
+template <>
+cudaError_t gemm_dispatch<float>(sf_engine*, const float* A, int lda, const float* W, int M, int N, int K,
+                                 const Epi& ep, cudaStream_t st) {
+  return gemm_f32(A, lda, W, M, N, K, ep, st);
+}
+template <>
+cudaError_t gemm_dispatch<bf16>(sf_engine* e, const bf16* A, int lda, const bf16* W, int M, int N, int K,
+                                const Epi& ep, cudaStream_t st) {
+  if (e->gemm_path == 1 && N % 16 == 0) return gemm_bf16_tc(A, lda, W, M, N, K, ep, e->d_err, st);
+  return gemm_bf16_mma(A, lda, W, M, N, K, ep, st);
+}
+
+template <typename T>
 cudaError_t gemm_acc(sf_engine* e, const T* A, int lda, const T* W, int M, int N, int K, const Epi& ep,
                      cudaStream_t st) {
   const double a = sizeof(T);
   const double out_b = (ep.kind == EPI_RESID) ? 8.0 : (ep.kind == EPI_F32 ? 4.0 : (ep.kind == EPI_F32_AND_T ? 4.0 + a : (ep.kind == EPI_BIAS_GLU ? a / 2 : a)));
   RUN(K_GEMM, 1, 2.0 * M * N * K, ((double)M * K + (double)N * K) * a + (double)M * N * out_b,
-      gemm<T>(A, lda, W, M, N, K, ep, st));
+      gemm_dispatch<T>(e, A, lda, W, M, N, K, ep, st));
   return cudaSuccess;
 }
 
@@ -543,6 +594,8 @@ Epi epi(int kind, const float* bias, void* out, int ldo, float alpha = 1.f) {
 // ------------------------------------------------------------ descriptors
 DescBlock* desc_begin(sf_engine* e) {
   if (e->desc_pending) {
+    // the previous call's copy of the block must have left the pinned buffer;
+    // an error here is the stream's and resurfaces at its next launch check
     cudaEventSynchronize(e->desc_ev);
     e->desc_pending = false;
   }
@@ -550,10 +603,102 @@ DescBlock* desc_begin(sf_engine* e) {
 }
 cudaError_t desc_upload(sf_engine* e, cudaStream_t st) {
   CK(cudaMemcpyAsync(e->d_desc, e->h_desc, sizeof(DescBlock), cudaMemcpyHostToDevice, st));
-  CK(cudaEventRecord(e->desc_ev, st));
-  e->desc_pending = true;
+  if (!e->capturing) {   // a graph replay records the event after its launch (run_graph)
+    CK(cudaEventRecord(e->desc_ev, st));
+    e->desc_pending = true;
+  }
   return cudaSuccess;
 }
+void destroy_graphs(sf_engine* e) {
+  for (auto& kv : e->graphs) {
+    if (kv.second.exec) cudaGraphExecDestroy(kv.second.exec);
+    for (cudaEvent_t ev : kv.second.events) cudaEventDestroy(ev);
+  }
+  e->graphs.clear();
+}
+
+// Runs `enqueue` (which must only enqueue work on `st`: no allocation, no
+// synchronisation) through a CUDA graph cached under `key`: captured on
+// first use (or after the workspace moved), replayed afterwards.  Launch
+// counters of a replay are those recorded at capture; with profiling on,
+// the graph carries its own event pairs, read back after each replay.
+template <typename F>
+cudaError_t run_graph(sf_engine* e, std::string key, cudaStream_t st, F&& enqueue) {
+  if (!e->use_graphs) return enqueue(st);
+  key += e->prof ? "|p" : "|n";
+  auto it = e->graphs.find(key);
+  if (it != e->graphs.end() && it->second.gen != e->ws_gen) {
+    cudaGraphExecDestroy(it->second.exec);
+    for (cudaEvent_t ev : it->second.events) cudaEventDestroy(ev);
+    e->graphs.erase(it);
+    it = e->graphs.end();
+  }
+  if (it == e->graphs.end()) {
+    if (e->graphs.size() >= 256) destroy_graphs(e);
+    sf_engine::GraphEntry g;
+    int64_t l0[K_COUNT];
+    double f0[K_COUNT], b0[K_COUNT];
+    memcpy(l0, e->launches, sizeof(l0));
+    memcpy(f0, e->kflops, sizeof(f0));
+    memcpy(b0, e->kbytes, sizeof(b0));
+    std::vector<ProfRec> saved;
+    saved.swap(e->recs);
+    e->cap_events.clear();
+    e->capturing = true;
+    cudaError_t err = cudaStreamBeginCapture(e->cap_stream, cudaStreamCaptureModeThreadLocal);
+    if (err != cudaSuccess && !g_fail_line) g_fail_line = __LINE__;
+    if (err == cudaSuccess) {
+      cudaError_t qe = enqueue(e->cap_stream);
+      cudaGraph_t graph = nullptr;
+      err = cudaStreamEndCapture(e->cap_stream, &graph);
+      if (err != cudaSuccess && !g_fail_line) g_fail_line = __LINE__;
+      if (qe != cudaSuccess) err = qe;
+      if (err == cudaSuccess) {
+        err = cudaGraphInstantiate(&g.exec, graph, 0);
+        if (err != cudaSuccess && !g_fail_line) g_fail_line = __LINE__;
+      }
+      if (graph) cudaGraphDestroy(graph);
+    }
+    e->capturing = false;
+    g.recs.swap(e->recs);
+    e->recs.swap(saved);
+    g.events.swap(e->cap_events);
+    for (int k = 0; k < K_COUNT; ++k) {
+      g.launches[k] = e->launches[k] - l0[k];
+      g.flops[k] = e->kflops[k] - f0[k];
+      g.bytes[k] = e->kbytes[k] - b0[k];
+    }
+    memcpy(e->launches, l0, sizeof(l0));
+    memcpy(e->kflops, f0, sizeof(f0));
+    memcpy(e->kbytes, b0, sizeof(b0));
+    if (err != cudaSuccess) {
+      for (cudaEvent_t ev : g.events) cudaEventDestroy(ev);
+      cudaGetLastError();
+      return err;
+    }
+    g.gen = e->ws_gen;
+    it = e->graphs.emplace(key, std::move(g)).first;
+  }
+  sf_engine::GraphEntry& g = it->second;
+  CK(cudaGraphLaunch(g.exec, st));
+  CK(cudaEventRecord(e->desc_ev, st));
+  e->desc_pending = true;
+  for (int k = 0; k < K_COUNT; ++k) {
+    e->launches[k] += g.launches[k];
+    e->kflops[k] += g.flops[k];
+    e->kbytes[k] += g.bytes[k];
+  }
+  if (e->prof && !g.recs.empty()) {
+    CK(cudaStreamSynchronize(st));
+    for (const ProfRec& r : g.recs) {
+      float t = 0.f;
+      CK(cudaEventElapsedTime(&t, r.a, r.b));
+      e->ms_acc[r.cls] += t;
+    }
+  }
+  return cudaSuccess;
+}
+
 // Fill the sequence table from lengths; returns total rows and tile count.
 double sum_sq(const std::vector<int>& lens) {
   double s2 = 0;
@@ -578,17 +723,23 @@ void fill_seq(DescBlock* d, const std::vector<int>& lens, int& M, int& tiles) {
 // -------------------------------------------------------------- pipeline
 // ConvSubsampling of n_win windows (PreArgs in the descriptor) -> act
 // embeddings; output row (i, t) goes to out + (i * out_stride + t) * D.
+// Workspace of run_pre_encode (call before any capture).
+cudaError_t prep_pre_encode(sf_engine* e, int n_win, int64_t W_max, size_t a) {
+  const int T1 = (int)half_len(W_max), T2 = (int)half_len(T1), T3 = (int)half_len(T2);
+  CK(ensure(e->sub1, (size_t)n_win * T1 * 64 * 256 * a));
+  CK(ensure(e->sub2a, (size_t)n_win * T2 * 32 * 256 * a));
+  CK(ensure(e->sub2b, (size_t)n_win * T2 * 32 * 256 * a));
+  CK(ensure(e->sub3a, (size_t)n_win * T3 * 16 * 256 * a));
+  CK(ensure(e->sub3b, (size_t)n_win * T3 * 16 * 256 * a));
+  return cudaSuccess;
+}
+
 template <typename T>
 cudaError_t run_pre_encode(sf_engine* e, const float* feats, int64_t t_buf, int n_win, int64_t W_max, T* out,
                            int64_t out_stride, cudaStream_t st) {
   Weights<T>& W = weights<T>(e);
   const int D = e->cfg.d_model;
   const int T1 = (int)half_len(W_max), T2 = (int)half_len(T1), T3 = (int)half_len(T2);
-  CK(ensure(e->sub1, (size_t)n_win * T1 * 64 * 256 * sizeof(T)));
-  CK(ensure(e->sub2a, (size_t)n_win * T2 * 32 * 256 * sizeof(T)));
-  CK(ensure(e->sub2b, (size_t)n_win * T2 * 32 * 256 * sizeof(T)));
-  CK(ensure(e->sub3a, (size_t)n_win * T3 * 16 * 256 * sizeof(T)));
-  CK(ensure(e->sub3b, (size_t)n_win * T3 * 16 * 256 * sizeof(T)));
   PreArgs pa{e->d_desc->buf, e->d_desc->start, e->d_desc->frames};
   T* s1 = static_cast<T*>(e->sub1.p);
   T* s2a = static_cast<T*>(e->sub2a.p);
@@ -714,25 +865,35 @@ cudaError_t offline_impl(sf_engine* e, const float* d_audio, const std::vector<i
   CK(ensure(e->part, mel_part_floats(B, n_max) * 4));
   CK(ensure(e->emb, (size_t)B * T3 * e->cfg.d_model * sizeof(T)));
   CK(ensure_encode_ws(e, M));
-  CK(desc_upload(e, st));
-  MelArgs ma{e->d_desc->len};
-  RUN(K_MEL, 2, 0, (double)B * n_max * 4 + (double)B * 128 * T_cols * 4,
-      launch_mel(d_audio, B, n_max, ma, e->d_mel_tab, static_cast<float*>(e->mel.p), static_cast<float*>(e->part.p), st));
-  CK(run_pre_encode<T>(e, static_cast<float*>(e->mel.p), T_cols, B, L_max, static_cast<T*>(e->emb.p), T3, st));
-  StateBufs none{};
-  none.D = e->cfg.d_model;
-  RUN(K_ASSEMBLE, 1, 0, (double)M * e->cfg.d_model * (4 + sizeof(T)),
-      launch_assemble<T>(static_cast<float*>(e->x.p), &e->d_desc->seq, &e->d_desc->step, none,
-                         static_cast<T*>(e->emb.p), T3, M, st));
-  CK(run_encode<T>(e, M, tiles, static_cast<float*>(e->probs.p), st));
-  RUN(K_EXTRACT, 1, 0, (double)M * 16 + (double)B * Tp_max * 16,
-      launch_extract_rows(static_cast<float*>(e->probs.p), &e->d_desc->seq, nullptr, nullptr, nullptr, B, d_probs,
-                          Tp_max, st));
-  return cudaSuccess;
+  CK(prep_pre_encode(e, B, L_max, sizeof(T)));
+  std::string key = "off|" + std::to_string(B) + "|" + std::to_string(n_max) + "|" +
+                    std::to_string(reinterpret_cast<uintptr_t>(d_audio)) + "|" +
+                    std::to_string(reinterpret_cast<uintptr_t>(d_probs));
+  for (int b = 0; b < B; ++b) key += "|" + std::to_string(len[b]);
+  return run_graph(e, key, st, [&](cudaStream_t st) -> cudaError_t {
+    CK(desc_upload(e, st));
+    MelArgs ma{e->d_desc->len};
+    RUN(K_MEL, 2, 0, (double)B * n_max * 4 + (double)B * 128 * T_cols * 4,
+        launch_mel(d_audio, B, n_max, ma, e->d_mel_tab, static_cast<float*>(e->mel.p), static_cast<float*>(e->part.p), st));
+    CK(run_pre_encode<T>(e, static_cast<float*>(e->mel.p), T_cols, B, L_max, static_cast<T*>(e->emb.p), T3, st));
+    StateBufs none{};
+    none.D = e->cfg.d_model;
+    RUN(K_ASSEMBLE, 1, 0, (double)M * e->cfg.d_model * (4 + sizeof(T)),
+        launch_assemble<T>(static_cast<float*>(e->x.p), &e->d_desc->seq, &e->d_desc->step, none,
+                           static_cast<T*>(e->emb.p), T3, M, st));
+    CK(run_encode<T>(e, M, tiles, static_cast<float*>(e->probs.p), st));
+    RUN(K_EXTRACT, 1, 0, (double)M * 16 + (double)B * Tp_max * 16,
+        launch_extract_rows(static_cast<float*>(e->probs.p), &e->d_desc->seq, nullptr, nullptr, nullptr, B, d_probs,
+                            Tp_max, st));
+    return cudaSuccess;
+  });
 }
 
 sf_status check_engine(sf_engine* e) {
   if (!e) return SF_EINVAL;
+  g_ws_gen = &e->ws_gen;
+  g_fail_line = 0;
+  cudaGetLastError();   // start each call without a stale, non-sticky error
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev != e->device) cudaSetDevice(e->device);
   return SF_OK;
@@ -823,6 +984,10 @@ sf_status sf_create(const void* blob, uint64_t nbytes, const sf_config* cfg, sf_
   cudaError_t ce;
   if ((ce = gemm_init_attributes()) != cudaSuccess) return cuda_fail(e.get(), ce, "init"), SF_ECUDA;
   if ((ce = attention_init_attributes()) != cudaSuccess) return SF_ECUDA;
+  if ((ce = gemm_tc_init_attributes()) != cudaSuccess) return SF_ECUDA;
+  if ((ce = frontend_init_attributes()) != cudaSuccess) return SF_ECUDA;
+  if ((ce = attention_init_f32_attributes(e->R)) != cudaSuccess) return SF_ECUDA;
+  g_ws_gen = &e->ws_gen;
   std::unordered_map<std::string, TensorRef> m;
   std::string err;
   if (!parse_blob(blob, nbytes, m, err)) return SF_EFORMAT;
@@ -844,6 +1009,10 @@ sf_status sf_create(const void* blob, uint64_t nbytes, const sf_config* cfg, sf_
     return SF_ENOMEM;
   }
   memset(e->h_desc, 0, sizeof(DescBlock));
+  if (cudaStreamCreateWithFlags(&e->cap_stream, cudaStreamNonBlocking) != cudaSuccess) {
+    sf_destroy(e.release());
+    return SF_ECUDA;
+  }
   *out = e.release();
   return SF_OK;
 }
@@ -865,6 +1034,7 @@ sf_status sf_create_from_file(const char* path, const sf_config* cfg, sf_engine*
 sf_status sf_destroy(sf_engine* e) {
   if (!e) return SF_EINVAL;
   cudaDeviceSynchronize();
+  destroy_graphs(e);
   for (Buf* b : {&e->mel, &e->part, &e->audio, &e->sub1, &e->sub2a, &e->sub2b, &e->sub3a, &e->sub3b, &e->emb, &e->x,
                  &e->h, &e->big, &e->ctx, &e->x2, &e->h2, &e->probs, &e->out})
     if (b->p) cudaFree(b->p);
@@ -875,6 +1045,7 @@ sf_status sf_destroy(sf_engine* e) {
   if (e->h_desc) cudaFreeHost(e->h_desc);
   if (e->desc_ev) cudaEventDestroy(e->desc_ev);
   for (cudaEvent_t ev : e->pool) cudaEventDestroy(ev);
+  if (e->cap_stream) cudaStreamDestroy(e->cap_stream);
   if (e->d_err) cudaFree(e->d_err);
   delete e;
   return SF_OK;
@@ -936,13 +1107,21 @@ sf_status sf_forward_offline_host(sf_engine* e, const float* h_audio, const int6
   const size_t out_bytes = (size_t)B * Tp * 4 * 4;
   cudaError_t ce = ensure(e->audio, (size_t)B * n_max * 4);
   if (ce == cudaSuccess) ce = ensure(e->out, out_bytes);
+  if (ce != cudaSuccess && !g_fail_line) g_fail_line = __LINE__;
   if (ce == cudaSuccess) ce = cudaMemcpyAsync(e->audio.p, h_audio, (size_t)B * n_max * 4, cudaMemcpyHostToDevice, st);
+  if (ce != cudaSuccess && !g_fail_line) g_fail_line = __LINE__;
   if (ce == cudaSuccess)
     ce = e->cfg.precision == SF_BF16
              ? offline_impl<bf16>(e, static_cast<float*>(e->audio.p), len, B, n_max, static_cast<float*>(e->out.p), st)
              : offline_impl<float>(e, static_cast<float*>(e->audio.p), len, B, n_max, static_cast<float*>(e->out.p), st);
-  if (ce == cudaSuccess) ce = cudaMemcpyAsync(h_probs, e->out.p, out_bytes, cudaMemcpyDeviceToHost, st);
-  if (ce == cudaSuccess) ce = cudaStreamSynchronize(st);
+  if (ce == cudaSuccess) {
+    ce = cudaMemcpyAsync(h_probs, e->out.p, out_bytes, cudaMemcpyDeviceToHost, st);
+    if (ce != cudaSuccess && !g_fail_line) g_fail_line = __LINE__;
+  }
+  if (ce == cudaSuccess) {
+    ce = cudaStreamSynchronize(st);
+    if (ce != cudaSuccess && !g_fail_line) g_fail_line = __LINE__;
+  }
   if (ce != cudaSuccess) return cuda_fail(e, ce, "sf_forward_offline_host");
   if (h_out_len)
     for (int b = 0; b < B; ++b) h_out_len[b] = enc_frames(len[b] / 160);
@@ -967,7 +1146,8 @@ sf_status sf_pre_encode(sf_engine* e, const float* d_feats, int n_buf, int64_t t
     W_max = std::max(W_max, h_frames[i]);
   }
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
-  cudaError_t ce = desc_upload(e, st);
+  cudaError_t ce = prep_pre_encode(e, n, W_max, act_size(e));
+  if (ce == cudaSuccess) ce = desc_upload(e, st);
   if (ce == cudaSuccess)
     ce = e->cfg.precision == SF_BF16
              ? run_pre_encode<bf16>(e, d_feats, t_buf, n, W_max, static_cast<bf16*>(d_embs), emb_stride, st)
@@ -1002,6 +1182,35 @@ sf_status sf_encode(sf_engine* e, const void* d_embs, const int* h_seq_len, int 
   return SF_OK;
 }
 
+sf_status sf_check(sf_engine* e, void* cuda_stream) {
+  if (check_engine(e) != SF_OK) return SF_EINVAL;
+  cudaError_t ce = cudaStreamSynchronize(static_cast<cudaStream_t>(cuda_stream));
+  if (ce != cudaSuccess) return cuda_fail(e, ce, "sf_check");
+  int w = 0;
+  ce = cudaMemcpy(&w, e->d_err, sizeof(int), cudaMemcpyDeviceToHost);
+  if (ce == cudaSuccess && w) ce = cudaMemset(e->d_err, 0, sizeof(int));
+  if (ce != cudaSuccess) return cuda_fail(e, ce, "sf_check");
+  if (w & ERR_TIMEOUT) return fail(e, SF_ETIMEOUT, "a bounded device wait gave up");
+  if (w) return fail(e, SF_EDEVICE, "a device-side check failed (error word " + std::to_string(w) + ")");
+  return SF_OK;
+}
+
+sf_status sf_gemm_bf16(sf_engine* e, const void* d_A, int lda, const void* d_W, int M, int N, int K,
+                       const float* d_bias, float* d_C, int path, void* cuda_stream) {
+  if (check_engine(e) != SF_OK) return SF_EINVAL;
+  if (!d_A || !d_W || !d_C) return fail(e, SF_EINVAL, "null pointer argument");
+  if (M < 1 || N < 16 || K < 64 || N % 16 || K % 64 || lda < K || lda % 8 || (path != 0 && path != 1))
+    return fail(e, SF_ESHAPE, "sf_gemm_bf16: M >= 1, N % 16 == 0, K % 64 == 0, lda >= K, lda % 8 == 0, path 0/1");
+  Epi ep = epi(EPI_F32, d_bias, d_C, N);
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  const bf16* A = static_cast<const bf16*>(d_A);
+  const bf16* W = static_cast<const bf16*>(d_W);
+  cudaError_t ce = path == 1 ? gemm_bf16_tc(A, lda, W, M, N, K, ep, e->d_err, st)
+                             : gemm_bf16_mma(A, lda, W, M, N, K, ep, st);
+  if (ce != cudaSuccess) return cuda_fail(e, ce, "sf_gemm_bf16");
+  return SF_OK;
+}
+
 sf_status sf_profile_enable(sf_engine* e, int enable) {
   if (!e) return SF_EINVAL;
   e->prof = enable != 0;
@@ -1011,6 +1220,7 @@ sf_status sf_profile_enable(sf_engine* e, int enable) {
 sf_status sf_profile_read(sf_engine* e, sf_kernel_stat* out, int max, int* n_out, int reset) {
   if (!e || !n_out || (max > 0 && !out)) return SF_EINVAL;
   double ms[K_COUNT] = {};
+  for (int k = 0; k < K_COUNT; ++k) ms[k] = e->ms_acc[k];
   for (const ProfRec& r : e->recs) {
     float t = 0.f;
     if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess)
@@ -1033,7 +1243,7 @@ sf_status sf_profile_read(sf_engine* e, sf_kernel_stat* out, int max, int* n_out
   }
   *n_out = n;
   if (reset) {
-    for (int k = 0; k < K_COUNT; ++k) e->launches[k] = 0, e->kflops[k] = e->kbytes[k] = 0;
+    for (int k = 0; k < K_COUNT; ++k) e->launches[k] = 0, e->kflops[k] = e->kbytes[k] = e->ms_acc[k] = 0;
     e->recs.clear();
     e->pool_used = 0;
   }
@@ -1140,20 +1350,27 @@ cudaError_t stream_step_impl(sf_stream* s, const float* d_feats, int64_t t_buf, 
   const int T3 = (int)enc_frames(W_max);
   CK(ensure(e->emb, (size_t)n * T3 * e->cfg.d_model * sizeof(T)));
   CK(ensure_encode_ws(e, M));
-  CK(desc_upload(e, st));
-  if (n < s->n) CK(cudaMemsetAsync(d_chunk_probs, 0, (size_t)s->n * s->p.chunk_len * 4 * 4, st));
-  CK(run_pre_encode<T>(e, d_feats, t_buf, n, W_max, static_cast<T*>(e->emb.p), T3, st));
-  RUN(K_ASSEMBLE, 1, 0, (double)M * e->cfg.d_model * (4 + sizeof(T)),
-      launch_assemble<T>(static_cast<float*>(e->x.p), &e->d_desc->seq, &e->d_desc->step, s->sb,
-                         static_cast<T*>(e->emb.p), T3, M, st));
-  CK(run_encode<T>(e, M, tiles, static_cast<float*>(e->probs.p), st));
-  RUN(K_EXTRACT, 1, 0, (double)n * s->p.chunk_len * 32,
-      launch_extract_rows(static_cast<float*>(e->probs.p), &e->d_desc->seq, e->d_desc->first, e->d_desc->count,
-                          e->d_desc->dst, n, d_chunk_probs, s->p.chunk_len, st));
-  RUN(K_UPDATE, 1, 0, 0,
-      launch_state_update<T>(static_cast<float*>(e->probs.p), &e->d_desc->seq, &e->d_desc->step, s->sb,
-                             static_cast<T*>(e->emb.p), T3, n, nullptr, nullptr, nullptr, 0, st));
-  return cudaSuccess;
+  CK(prep_pre_encode(e, n, W_max, sizeof(T)));
+  std::string key = "st|" + std::to_string(reinterpret_cast<uintptr_t>(s)) + "|" + std::to_string(n) + "|" +
+                    std::to_string(M) + "|" + std::to_string(tiles) + "|" + std::to_string(W_max) + "|" +
+                    std::to_string(t_buf) + "|" + std::to_string(reinterpret_cast<uintptr_t>(d_feats)) + "|" +
+                    std::to_string(reinterpret_cast<uintptr_t>(d_chunk_probs));
+  return run_graph(e, key, st, [&](cudaStream_t st) -> cudaError_t {
+    CK(desc_upload(e, st));
+    if (n < s->n) CK(cudaMemsetAsync(d_chunk_probs, 0, (size_t)s->n * s->p.chunk_len * 4 * 4, st));
+    CK(run_pre_encode<T>(e, d_feats, t_buf, n, W_max, static_cast<T*>(e->emb.p), T3, st));
+    RUN(K_ASSEMBLE, 1, 0, (double)M * e->cfg.d_model * (4 + sizeof(T)),
+        launch_assemble<T>(static_cast<float*>(e->x.p), &e->d_desc->seq, &e->d_desc->step, s->sb,
+                           static_cast<T*>(e->emb.p), T3, M, st));
+    CK(run_encode<T>(e, M, tiles, static_cast<float*>(e->probs.p), st));
+    RUN(K_EXTRACT, 1, 0, (double)n * s->p.chunk_len * 32,
+        launch_extract_rows(static_cast<float*>(e->probs.p), &e->d_desc->seq, e->d_desc->first, e->d_desc->count,
+                            e->d_desc->dst, n, d_chunk_probs, s->p.chunk_len, st));
+    RUN(K_UPDATE, 1, 0, 0,
+        launch_state_update<T>(static_cast<float*>(e->probs.p), &e->d_desc->seq, &e->d_desc->step, s->sb,
+                               static_cast<T*>(e->emb.p), T3, n, nullptr, nullptr, nullptr, 0, st));
+    return cudaSuccess;
+  });
 }
 
 }  // namespace

@@ -179,17 +179,24 @@ __global__ void __launch_bounds__(256) mel_normalize_kernel(float* __restrict__ 
   for (int t = threadIdx.x; t < T_cols; t += blockDim.x) row[t] = (t < L) ? (row[t] - mu) * inv : 0.f;
 }
 
+constexpr size_t MEL_SMEM =
+    (size_t)MEL_SPAN * 4 + 128 * 8 + 258 * 8 + 512 * 4 + 8 * 256 * 8 + 128 * (MEL_FB + 1) * 4;
+
+cudaError_t frontend_init_attributes() {
+  return cudaFuncSetAttribute(mel_frames_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)MEL_SMEM);
+}
+
 cudaError_t launch_mel(const float* audio, int B, int64_t n_max, const MelArgs& args, const MelTables* tab,
                        float* mel, float* part, cudaStream_t st) {
   const int T_cols = (int)(1 + n_max / 160);
   const int n_blk = (T_cols + MEL_FB - 1) / MEL_FB;
-  const size_t smem = (size_t)MEL_SPAN * 4 + 128 * 8 + 258 * 8 + 512 * 4 + 8 * 256 * 8 + 128 * (MEL_FB + 1) * 4;
-  static bool attr_set = false;
+  const size_t smem = MEL_SMEM;
+  static bool attr_set = false;   // first use outside an engine (sf_mel_noalloc)
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(mel_frames_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = frontend_init_attributes();
     if (e != cudaSuccess) return e;
-    attr_set = true;
   }
+  attr_set = true;
   mel_frames_kernel<<<dim3(n_blk, B), 256, smem, st>>>(audio, n_max, args, tab, mel, part, T_cols, n_blk);
   mel_normalize_kernel<<<dim3(128, B), 256, 0, st>>>(mel, part, args, T_cols, n_blk);
   return cudaGetLastError();

@@ -24,6 +24,7 @@ struct MelArgs {
 cudaError_t launch_mel(const float* audio, int B, int64_t n_max, const MelArgs& args, const MelTables* tab,
                        float* mel, float* part, cudaStream_t st);
 size_t mel_part_floats(int B, int64_t n_max);
+cudaError_t frontend_init_attributes();
 void build_mel_tables(MelTables* t);   // host
 
 }  // namespace sf

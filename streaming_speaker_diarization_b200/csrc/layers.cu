@@ -6,31 +6,52 @@
 
 namespace sf {
 
-// One warp per row; lane j holds elements j, j + 32, ... (coalesced).
-template <typename T, int D>
+// One warp per row; lane j holds VEC-wide vectors j, j + 32, ... (coalesced).
+template <typename T, int D, int VEC>
 __global__ void __launch_bounds__(256) layernorm_kernel(float* __restrict__ x, const float* __restrict__ g,
                                                         const float* __restrict__ b, int M, bool write_x,
                                                         T* __restrict__ h) {
-  constexpr int V = D / 32;
+  constexpr int NV = D / (32 * VEC);
   const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= M) return;
   float* xr = x + (int64_t)row * D;
-  float v[V];
+  float v[NV][VEC];
   float s = 0.f;
 #pragma unroll
-  for (int j = 0; j < V; ++j) { v[j] = xr[lane + 32 * j]; s += v[j]; }
+  for (int j = 0; j < NV; ++j) {
+    const int c = (lane + 32 * j) * VEC;
+    if (VEC == 4) {
+      const float4 t = *reinterpret_cast<const float4*>(xr + c);
+      v[j][0] = t.x; v[j][1] = t.y; v[j][2 % VEC] = t.z; v[j][3 % VEC] = t.w;
+    } else {
+      const float2 t = *reinterpret_cast<const float2*>(xr + c);
+      v[j][0] = t.x; v[j][1 % VEC] = t.y;
+    }
+#pragma unroll
+    for (int k = 0; k < VEC; ++k) s += v[j][k];
+  }
   const float mean = warp_sum(s) * (1.0f / D);
   float q = 0.f;
 #pragma unroll
-  for (int j = 0; j < V; ++j) { const float d = v[j] - mean; q = fmaf(d, d, q); }
+  for (int j = 0; j < NV; ++j)
+#pragma unroll
+    for (int k = 0; k < VEC; ++k) { const float d = v[j][k] - mean; q = fmaf(d, d, q); }
   const float inv = 1.0f / sqrtf(warp_sum(q) * (1.0f / D) + 1e-5f);
 #pragma unroll
-  for (int j = 0; j < V; ++j) {
-    const int c = lane + 32 * j;
-    const float y = (v[j] - mean) * inv * g[c] + b[c];
-    if (write_x) xr[c] = y;
-    if (h) h[(int64_t)row * D + c] = from_f<T>(y);
+  for (int j = 0; j < NV; ++j) {
+    const int c = (lane + 32 * j) * VEC;
+    float y[VEC];
+#pragma unroll
+    for (int k = 0; k < VEC; ++k) y[k] = (v[j][k] - mean) * inv * g[c + k] + b[c + k];
+    if (write_x) {
+      if (VEC == 4) *reinterpret_cast<float4*>(xr + c) = make_float4(y[0], y[1 % VEC], y[2 % VEC], y[3 % VEC]);
+      else *reinterpret_cast<float2*>(xr + c) = make_float2(y[0], y[1 % VEC]);
+    }
+    if (h) {
+#pragma unroll
+      for (int k = 0; k < VEC; ++k) h[(int64_t)row * D + c + k] = from_f<T>(y[k]);
+    }
   }
 }
 
@@ -39,8 +60,8 @@ cudaError_t launch_layernorm(float* x, const float* g, const float* b, int M, in
                              cudaStream_t st) {
   if (M <= 0) return cudaSuccess;
   const int grid = (M + 7) / 8;
-  if (D == 512) layernorm_kernel<T, 512><<<grid, 256, 0, st>>>(x, g, b, M, write_x, h);
-  else if (D == 192) layernorm_kernel<T, 192><<<grid, 256, 0, st>>>(x, g, b, M, write_x, h);
+  if (D == 512) layernorm_kernel<T, 512, 4><<<grid, 256, 0, st>>>(x, g, b, M, write_x, h);
+  else if (D == 192) layernorm_kernel<T, 192, 2><<<grid, 256, 0, st>>>(x, g, b, M, write_x, h);
   else return cudaErrorInvalidValue;
   return cudaGetLastError();
 }
@@ -61,31 +82,52 @@ template <> struct Vec2<bf16> {
   static __device__ __forceinline__ float hi(__nv_bfloat162 v) { return __high2float(v); }
 };
 
-// Each thread: two channels over DW_ROWS rows; taps outside the row's
-// sequence read as zero.
-constexpr int DW_ROWS = 32;
+// Each thread: two channels x DW_ROWS consecutive rows; the DW_ROWS + K - 1
+// input rows they need are loaded once into registers.  Taps outside the
+// output row's sequence read as zero.
+constexpr int DW_ROWS = 8;
+constexpr int DW_KMAX = 9;
 template <typename T>
-__global__ void __launch_bounds__(256) dwconv1d_kernel(const T* __restrict__ in, T* __restrict__ out,
+__global__ void __launch_bounds__(128) dwconv1d_kernel(const T* __restrict__ in, T* __restrict__ out,
                                                        const float* __restrict__ w, const float* __restrict__ bias,
                                                        int M, int D, int K, const SeqTable* __restrict__ seq) {
-  const int c = 2 * (blockIdx.y * 256 + threadIdx.x);
+  const int c = 2 * (blockIdx.y * 128 + threadIdx.x);
   if (c >= D) return;
   const int r0 = blockIdx.x * DW_ROWS;
   const int pad = (K - 1) / 2;
-  float w0[16], w1[16];
-  for (int j = 0; j < K; ++j) { w0[j] = w[c * K + j]; w1[j] = w[(c + 1) * K + j]; }
+  float w0[DW_KMAX], w1[DW_KMAX];
+#pragma unroll
+  for (int j = 0; j < DW_KMAX; ++j) {
+    w0[j] = j < K ? w[c * K + j] : 0.f;
+    w1[j] = j < K ? w[(c + 1) * K + j] : 0.f;
+  }
   const float b0 = bias[c], b1 = bias[c + 1];
+  float x0[DW_ROWS + DW_KMAX - 1], x1[DW_ROWS + DW_KMAX - 1];
+#pragma unroll
+  for (int i = 0; i < DW_ROWS + DW_KMAX - 1; ++i) {
+    const int ri = r0 - pad + i;
+    x0[i] = x1[i] = 0.f;
+    if (ri >= 0 && ri < M && i < DW_ROWS + K - 1) {
+      const auto v = Vec2<T>::load(in + (int64_t)ri * D + c);
+      x0[i] = Vec2<T>::lo(v);
+      x1[i] = Vec2<T>::hi(v);
+    }
+  }
   int s = seq_of_row(seq, r0 < M ? r0 : M - 1);
-  for (int r = r0; r < min(r0 + DW_ROWS, M); ++r) {
+#pragma unroll
+  for (int k = 0; k < DW_ROWS; ++k) {
+    const int r = r0 + k;
+    if (r >= M) break;
     while (r >= seq->off[s + 1]) ++s;
     const int sb = seq->off[s], se = seq->off[s + 1];
     float a0 = b0, a1 = b1;
-    for (int j = 0; j < K; ++j) {
+#pragma unroll
+    for (int j = 0; j < DW_KMAX; ++j) {
       const int ri = r + j - pad;
-      if (ri < sb || ri >= se) continue;
-      const auto v = Vec2<T>::load(in + (int64_t)ri * D + c);
-      a0 = fmaf(w0[j], Vec2<T>::lo(v), a0);
-      a1 = fmaf(w1[j], Vec2<T>::hi(v), a1);
+      if (j < K && ri >= sb && ri < se) {
+        a0 = fmaf(w0[j], x0[k + j], a0);
+        a1 = fmaf(w1[j], x1[k + j], a1);
+      }
     }
     a0 = a0 / (1.f + expf(-a0));
     a1 = a1 / (1.f + expf(-a1));
@@ -97,9 +139,9 @@ template <typename T>
 cudaError_t launch_dwconv1d(const T* in, T* out, const float* w, const float* b, int M, int D, int K,
                             const SeqTable* seq, cudaStream_t st) {
   if (M <= 0) return cudaSuccess;
-  if (K > 16 || (D % 2)) return cudaErrorInvalidValue;
-  dim3 grid((M + DW_ROWS - 1) / DW_ROWS, (D / 2 + 255) / 256);
-  dwconv1d_kernel<T><<<grid, 256, 0, st>>>(in, out, w, b, M, D, K, seq);
+  if (K > DW_KMAX || (D % 2)) return cudaErrorInvalidValue;
+  dim3 grid((M + DW_ROWS - 1) / DW_ROWS, (D / 2 + 127) / 128);
+  dwconv1d_kernel<T><<<grid, 128, 0, st>>>(in, out, w, b, M, D, K, seq);
   return cudaGetLastError();
 }
 

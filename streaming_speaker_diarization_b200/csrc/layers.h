@@ -34,6 +34,11 @@ cudaError_t gemm_f32(const float* A, int lda, const float* W, int M, int N, int 
 cudaError_t gemm_bf16_mma(const bf16* A, int lda, const bf16* W, int M, int N, int K, const Epi& e,
                           cudaStream_t st);
 cudaError_t gemm_init_attributes();
+// tcgen05 / TMEM / TMA path (sm_100a); err = device error word (may be null).
+cudaError_t gemm_bf16_tc(const bf16* A, int lda, const bf16* W, int M, int N, int K, const Epi& e, int* err,
+                         cudaStream_t st);
+cudaError_t gemm_tc_init_attributes();
+int gemm_tc_pick_bn(int M, int N);
 
 // --------------------------------------------------------- subsampling
 struct PreArgs {        // device arrays, one entry per window
@@ -72,6 +77,7 @@ cudaError_t launch_to_f32(const T* in, float* out, int64_t n, cudaStream_t st);
 cudaError_t launch_extract_rows(const float* packed, const SeqTable* seq, const int* d_first, const int* d_count,
                                 const int* d_dst, int n_seq, float* out, int t_max, cudaStream_t st);
 void attention_set_max_seq(int s);
+cudaError_t attention_init_f32_attributes(int R);
 
 // ------------------------------------------------------------- attention
 // Relative-position MHSA (d_model 512, 8 heads of 64) over packed sequences.

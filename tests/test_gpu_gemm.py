@@ -1,0 +1,56 @@
+"""GPU: the tcgen05/TMEM/TMA GEMM and the mma.sync GEMM against a float64
+reference of the same bf16 operands (relative error bound of fp32
+accumulation over K terms: 1e-5 x sqrt(K) is generous; we use 2e-4 abs on
+O(1) outputs), on the engine's shapes, ragged M and every tile width."""
+import numpy as np
+import pytest
+
+pytestmark = pytest.mark.gpu
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():
+    pytest.skip("no CUDA device", allow_module_level=True)
+from streaming_speaker_diarization_b200 import binding as b  # noqa: E402
+from _helpers import make_engine, tiny_weights  # noqa: E402
+
+
+@pytest.fixture(scope="module")
+def eng():
+    e = make_engine(tiny_weights(), 1, 2, 2)
+    yield e
+    b.sf_destroy(e)
+
+
+SHAPES = [(1125, 2048, 512), (1125, 512, 2048), (1125, 1536, 512), (1125, 192, 192), (1125, 576, 192),
+          (1, 64, 64), (333, 768, 192), (128, 128, 128), (129, 256, 4096), (24896, 1024, 512), (70, 16, 64)]
+
+
+@pytest.mark.parametrize("M,N,K", SHAPES)
+@pytest.mark.parametrize("path", [1, 0])
+def test_gemm_vs_float64(eng, M, N, K, path):
+    g = torch.Generator().manual_seed(M * 7 + N * 3 + K)
+    A = (torch.randn(M, K, generator=g) / np.sqrt(K)).to(torch.bfloat16)
+    W = torch.randn(N, K, generator=g).to(torch.bfloat16)
+    bias = torch.randn(N, generator=g)
+    ref = A.double().numpy() @ W.double().numpy().T + bias.double().numpy()
+    C = torch.full((M, N), float("nan"), device="cuda")
+    b.sf_gemm_bf16(eng, A.cuda(), W.cuda(), C, bias=bias.cuda(), path=path)
+    b.sf_check(eng)
+    err = np.max(np.abs(C.cpu().numpy() - ref))
+    assert err <= 2e-4 * max(1.0, np.sqrt(K / 512)), err
+
+
+def test_gemm_tc_strided_a(eng):
+    """A with a row stride larger than K (a column slice of a wider matrix)."""
+    M, N, K = 300, 128, 256
+    g = torch.Generator().manual_seed(3)
+    big = torch.randn(M, 3 * K, generator=g).to(torch.bfloat16)
+    W = torch.randn(N, K, generator=g).to(torch.bfloat16)
+    A = big.cuda()
+    C = torch.zeros((M, N), device="cuda")
+    sub = A[:, K:2 * K]
+    rc = b.lib.sf_gemm_bf16(eng, sub.data_ptr(), A.stride(0), W.cuda().data_ptr(), M, N, K, None, C.data_ptr(), 1,
+                            torch.cuda.current_stream().cuda_stream)
+    assert rc == 0
+    b.sf_check(eng)
+    ref = big[:, K:2 * K].double().numpy() @ W.double().numpy().T
+    assert np.max(np.abs(C.cpu().numpy() - ref)) < 2e-3
