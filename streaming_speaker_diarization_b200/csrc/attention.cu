@@ -118,12 +118,38 @@ __device__ __forceinline__ void load_rows(bf16* dst, const bf16* src, int64_t ld
   }
 }
 
+__device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void* src, bool pred) {
+  const int sz = pred ? 16 : 0;
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(sz) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit_() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N> __device__ __forceinline__ void cp_async_wait_() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+
+// Asynchronous version of load_rows (no bias add): rows outside [lo, hi) and
+// dims >= HD arrive as zeros.
+template <int HD, int HDP, int LDS>
+__device__ __forceinline__ void load_rows_async(bf16* dst, const bf16* src, int64_t ld, int row0, int nrows, int lo,
+                                                int hi) {
+  constexpr int CH = HDP / 8;
+  for (int e = threadIdx.x; e < nrows * CH; e += blockDim.x) {
+    const int rr = e / CH, ch = e % CH;
+    const int row = row0 + rr;
+    const bool ok = row >= lo && row < hi && ch * 8 < HD;
+    const bf16* g = ok ? src + (int64_t)row * ld + ch * 8 : src;
+    cp_async16_zfill(s_u32(dst + rr * LDS + ch * 8), g, ok);
+  }
+}
+
 template <int HD, int HDP, bool REL>
 struct AttCfg {
   static constexpr int LDS = HDP + 8;
   static constexpr int TILE = 64 * LDS;                       // bf16 elements
   static constexpr int NQ = REL ? 2 : 1;
-  static constexpr int SMEM = (NQ * TILE + 2 * TILE + (REL ? 2 * TILE : 0)) * 2 + (REL ? 4 * 16 * 80 * 4 : 0);
+  // Q (+Qv) once; K, V and the 128-row relative slice double-buffered
+  static constexpr int BUF = 2 * TILE + (REL ? 2 * TILE : 0);
+  static constexpr int SMEM = (NQ * TILE + 2 * BUF) * 2 + (REL ? 4 * 16 * 80 * 4 : 0);
 };
 
 template <int HD, int HDP, bool REL>
@@ -136,10 +162,8 @@ __global__ void __launch_bounds__(128) attn_bf16_kernel(const bf16* __restrict__
   extern __shared__ float4 att_smem4[];
   bf16* sQu = reinterpret_cast<bf16*>(att_smem4);
   bf16* sQv = sQu + (REL ? C::TILE : 0);
-  bf16* sK = sQu + C::NQ * C::TILE;
-  bf16* sV = sK + C::TILE;
-  bf16* sP = sV + C::TILE;                                   // 128 rows (REL)
-  float* sBD = reinterpret_cast<float*>(sP + (REL ? 2 * C::TILE : 0));
+  bf16* sBuf = sQu + C::NQ * C::TILE;                         // 2 x [K | V | P(128 rows, REL)]
+  float* sBD = reinterpret_cast<float*>(sBuf + 2 * C::BUF);
 
   const int g_tile = blockIdx.x, h = blockIdx.y;
   const int s = seq_of_tile(seq, g_tile);
@@ -171,14 +195,23 @@ __global__ void __launch_bounds__(128) attn_bf16_kernel(const bf16* __restrict__
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
   const float sl2 = 1.4426950408889634f / sqrtf((float)HD);
 
-  for (int j0 = 0; j0 < S; j0 += 64) {
+  auto prefetch = [&](int j0, int buf) {
+    bf16* k_ = sBuf + buf * C::BUF;
+    load_rows_async<HD, HDP, LDS>(k_, Kg, ld, j0, 64, 0, S);
+    load_rows_async<HD, HDP, LDS>(k_ + C::TILE, Vg, ld, j0, 64, 0, S);
+    if (REL) load_rows_async<HD, HDP, LDS>(k_ + 2 * C::TILE, ptab + h * HD, D, i0 - j0 - 63 + R - 1, 128, 0, 2 * R - 1);
+    cp_async_commit_();
+  };
+  prefetch(0, 0);
+  for (int j0 = 0, it = 0; j0 < S; j0 += 64, ++it) {
+    // tile it+1 streams in while tile it is used
+    if (j0 + 64 < S) prefetch(j0 + 64, (it + 1) & 1);
+    else cp_async_commit_();
+    cp_async_wait_<1>();
     __syncthreads();
-    load_rows<HD, HDP, LDS>(sK, Kg, ld, j0, 64, 0, S, nullptr);
-    load_rows<HD, HDP, LDS>(sV, Vg, ld, j0, 64, 0, S, nullptr);
-    const int rbase = i0 - j0 - 63;   // relative distance of P slice row 0
-    if (REL) load_rows<HD, HDP, LDS>(sP, ptab + h * HD, D, rbase + R - 1, 128, 0, 2 * R - 1, nullptr);
-    __syncthreads();
-
+    const bf16* sK = sBuf + (it & 1) * C::BUF;
+    const bf16* sV = sK + C::TILE;
+    const bf16* sP = sK + 2 * C::TILE;
     float sc[8][4];
 #pragma unroll
     for (int n = 0; n < 8; ++n) sc[n][0] = sc[n][1] = sc[n][2] = sc[n][3] = 0.f;
@@ -281,7 +314,9 @@ __global__ void __launch_bounds__(128) attn_bf16_kernel(const bf16* __restrict__
         mma16816(o[2 * np + 1], a, b[2], b[3]);
       }
     }
+    __syncthreads();   // everyone is done with this buffer before it is refilled
   }
+  cp_async_wait_<0>();
   l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
   l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
   l1 += __shfl_xor_sync(0xffffffffu, l1, 1);

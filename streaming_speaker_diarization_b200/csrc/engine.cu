@@ -125,6 +125,8 @@ struct Arena {
 }  // namespace
 
 namespace {
+constexpr size_t SPLIT_WS_BYTES = (size_t)40 << 20;
+constexpr int SPLIT_CNT = 1 << 16;
 enum KClass : int {
   K_MEL = 0, K_CONV1, K_DW2D, K_GEMM, K_ATT_REL, K_ATT_MHA, K_LN, K_DW1D, K_HEAD, K_ASSEMBLE, K_EXTRACT,
   K_UPDATE, K_TOF32, K_SELECT, K_COUNT
@@ -153,6 +155,9 @@ struct sf_engine {
   bool desc_pending = false;
   int* d_err = nullptr;
   int gemm_path = 1;      // bf16 GEMMs: 1 = tcgen05 (default), 0 = mma.sync
+  float* d_split_ws = nullptr;   // split-K partial tiles of the tcgen05 GEMM
+  int* d_split_cnt = nullptr;    // their per-tile arrival counters (kept at zero between launches)
+  TcScratch tc_scratch() const { return TcScratch{d_err, d_split_ws, SPLIT_WS_BYTES, d_split_cnt, SPLIT_CNT}; }
   Weights<float> wf;
   Weights<bf16> wb;
   // profiling: launch/work counters always; event pairs when prof is set
@@ -567,7 +572,7 @@ cudaError_t gemm_dispatch<float>(sf_engine*, const float* A, int lda, const floa
 template <>
 cudaError_t gemm_dispatch<bf16>(sf_engine* e, const bf16* A, int lda, const bf16* W, int M, int N, int K,
                                 const Epi& ep, cudaStream_t st) {
-  if (e->gemm_path == 1 && N % 16 == 0) return gemm_bf16_tc(A, lda, W, M, N, K, ep, e->d_err, st);
+  if (e->gemm_path == 1 && N % 16 == 0) return gemm_bf16_tc(A, lda, W, M, N, K, ep, e->tc_scratch(), st);
   return gemm_bf16_mma(A, lda, W, M, N, K, ep, st);
 }
 
@@ -1004,7 +1009,10 @@ sf_status sf_create(const void* blob, uint64_t nbytes, const sf_config* cfg, sf_
       cudaMallocHost(&e->h_desc, sizeof(DescBlock)) != cudaSuccess ||
       cudaMalloc(&e->d_desc, sizeof(DescBlock)) != cudaSuccess ||
       cudaEventCreateWithFlags(&e->desc_ev, cudaEventDisableTiming) != cudaSuccess ||
-      cudaMalloc(&e->d_err, sizeof(int)) != cudaSuccess || cudaMemset(e->d_err, 0, sizeof(int)) != cudaSuccess) {
+      cudaMalloc(&e->d_err, sizeof(int)) != cudaSuccess || cudaMemset(e->d_err, 0, sizeof(int)) != cudaSuccess ||
+      cudaMalloc(&e->d_split_ws, SPLIT_WS_BYTES) != cudaSuccess ||
+      cudaMalloc(&e->d_split_cnt, SPLIT_CNT * sizeof(int)) != cudaSuccess ||
+      cudaMemset(e->d_split_cnt, 0, SPLIT_CNT * sizeof(int)) != cudaSuccess) {
     sf_destroy(e.release());
     return SF_ENOMEM;
   }
@@ -1047,6 +1055,8 @@ sf_status sf_destroy(sf_engine* e) {
   for (cudaEvent_t ev : e->pool) cudaEventDestroy(ev);
   if (e->cap_stream) cudaStreamDestroy(e->cap_stream);
   if (e->d_err) cudaFree(e->d_err);
+  if (e->d_split_ws) cudaFree(e->d_split_ws);
+  if (e->d_split_cnt) cudaFree(e->d_split_cnt);
   delete e;
   return SF_OK;
 }
@@ -1205,7 +1215,7 @@ sf_status sf_gemm_bf16(sf_engine* e, const void* d_A, int lda, const void* d_W, 
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
   const bf16* A = static_cast<const bf16*>(d_A);
   const bf16* W = static_cast<const bf16*>(d_W);
-  cudaError_t ce = path == 1 ? gemm_bf16_tc(A, lda, W, M, N, K, ep, e->d_err, st)
+  cudaError_t ce = path == 1 ? gemm_bf16_tc(A, lda, W, M, N, K, ep, e->tc_scratch(), st)
                              : gemm_bf16_mma(A, lda, W, M, N, K, ep, st);
   if (ce != cudaSuccess) return cuda_fail(e, ce, "sf_gemm_bf16");
   return SF_OK;

@@ -52,4 +52,50 @@ __device__ __forceinline__ void epi_store2(const Epi& e, int r, int c, float v0,
   }
 }
 
+// Four consecutive columns c .. c + 3 of row r (c % 4 == 0, c + 3 < N),
+// bias already added; kind fixed at compile time.
+template <int EK, typename T>
+__device__ __forceinline__ void epi_store4(const Epi& e, int r, int c, float4 v) {
+  const int64_t orow = e.rpg ? (int64_t)(r / e.rpg) * e.gstride + (r % e.rpg) : (int64_t)r;
+  if (EK == EPI_BIAS_RELU) {
+    v.x = fmaxf(v.x, 0.f); v.y = fmaxf(v.y, 0.f); v.z = fmaxf(v.z, 0.f); v.w = fmaxf(v.w, 0.f);
+  }
+  if (EK == EPI_BIAS_SWISH) {
+    v.x = v.x / (1.f + expf(-v.x)); v.y = v.y / (1.f + expf(-v.y));
+    v.z = v.z / (1.f + expf(-v.z)); v.w = v.w / (1.f + expf(-v.w));
+  }
+  if (EK == EPI_BIAS || EK == EPI_BIAS_RELU || EK == EPI_BIAS_SWISH) {
+    T* o = reinterpret_cast<T*>(e.out) + orow * e.ldo + c;
+    if (sizeof(T) == 2) {
+      __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
+      uint2 pk;
+      pk.x = *reinterpret_cast<uint32_t*>(&a);
+      pk.y = *reinterpret_cast<uint32_t*>(&b);
+      *reinterpret_cast<uint2*>(o) = pk;
+    } else {
+      *reinterpret_cast<float4*>(o) = v;
+    }
+  } else if (EK == EPI_BIAS_GLU) {
+    T* o = reinterpret_cast<T*>(e.out) + orow * e.ldo + (c >> 1);
+    const float g0 = v.x / (1.f + expf(-v.y)), g1 = v.z / (1.f + expf(-v.w));
+    if (sizeof(T) == 2) {
+      __nv_bfloat162 a = __floats2bfloat162_rn(g0, g1);
+      *reinterpret_cast<__nv_bfloat162*>(o) = a;
+    } else {
+      *reinterpret_cast<float2*>(o) = make_float2(g0, g1);
+    }
+  } else if (EK == EPI_RESID) {
+    float4* o = reinterpret_cast<float4*>(reinterpret_cast<float*>(e.out) + orow * e.ldo + c);
+    float4 x = *o;
+    x.x += e.alpha * v.x; x.y += e.alpha * v.y; x.z += e.alpha * v.z; x.w += e.alpha * v.w;
+    *o = x;
+  } else {   // EPI_F32, EPI_F32_AND_T
+    *reinterpret_cast<float4*>(reinterpret_cast<float*>(e.out) + orow * e.ldo + c) = v;
+    if (EK == EPI_F32_AND_T) {
+      T* o2 = reinterpret_cast<T*>(e.out2) + orow * e.ldo2 + c;
+      o2[0] = from_f<T>(v.x); o2[1] = from_f<T>(v.y); o2[2] = from_f<T>(v.z); o2[3] = from_f<T>(v.w);
+    }
+  }
+}
+
 }  // namespace sf

@@ -157,20 +157,39 @@ __global__ void __launch_bounds__(256) mel_normalize_kernel(float* __restrict__ 
   const int m = blockIdx.x, b = blockIdx.y;
   const int L = (int)(args.len[b] / 160);
   __shared__ float s_mu, s_inv;
-  if (threadIdx.x == 0) {
-    double n = 0, mean = 0, m2 = 0;
-    for (int k = 0; k < n_blk; ++k) {
-      const float* p = part + (((int64_t)b * n_blk + k) * 128 + m) * 4;
-      double nb = p[0];
-      if (nb <= 0) continue;
-      double mb = (double)p[1] + (double)p[2] / nb, m2b = p[3];
-      double nt = n + nb, d = mb - mean;
-      mean += d * nb / nt;
-      m2 += m2b + d * d * n * nb / nt;
-      n = nt;
+  __shared__ double sn[256], smean[256], sm2[256];
+  // Chan's pairwise merge of the per-tile (count, mean, M2): each thread
+  // merges a strided subset, then a fixed shared-memory tree (deterministic).
+  double n = 0, mean = 0, m2 = 0;
+  for (int k = threadIdx.x; k < n_blk; k += blockDim.x) {
+    const float* p = part + (((int64_t)b * n_blk + k) * 128 + m) * 4;
+    const double nb = p[0];
+    if (nb <= 0) continue;
+    const double mb = (double)p[1] + (double)p[2] / nb, m2b = p[3];
+    const double nt = n + nb, d = mb - mean;
+    mean += d * nb / nt;
+    m2 += m2b + d * d * n * nb / nt;
+    n = nt;
+  }
+  sn[threadIdx.x] = n;
+  smean[threadIdx.x] = mean;
+  sm2[threadIdx.x] = m2;
+  __syncthreads();
+  for (int w = blockDim.x / 2; w > 0; w >>= 1) {
+    if (threadIdx.x < w) {
+      const double na = sn[threadIdx.x], nb = sn[threadIdx.x + w];
+      if (nb > 0) {
+        const double nt = na + nb, d = smean[threadIdx.x + w] - smean[threadIdx.x];
+        smean[threadIdx.x] += d * nb / nt;
+        sm2[threadIdx.x] += sm2[threadIdx.x + w] + d * d * na * nb / nt;
+        sn[threadIdx.x] = nt;
+      }
     }
-    double sd = (L > 1) ? sqrt(m2 / (double)(L - 1)) : 0.0;
-    s_mu = (float)mean;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    const double sd = (L > 1) ? sqrt(sm2[0] / (double)(L - 1)) : 0.0;
+    s_mu = (float)smean[0];
     s_inv = (float)(1.0 / (sd + 1e-5));
   }
   __syncthreads();

@@ -114,12 +114,99 @@ struct TcCfg {
   static constexpr int A_BYTES = TC_BM * TC_BK * 2;
   static constexpr int B_BYTES = BN * TC_BK * 2;
   static constexpr int SMEM = 1024 + STAGES * (A_BYTES + B_BYTES) + 256;
+  static_assert(STAGES * (A_BYTES + B_BYTES) >= 4 * 32 * 68 * 4, "epilogue staging reuses the pipeline buffers");
 };
+
+// Epilogue of one warp's 32 rows: per 64-column chunk, the accumulator block
+// goes TMEM -> registers -> shared tile (row stride 68 floats: conflict-free
+// 16-byte writes by row and reads by column), then each lane writes 4
+// consecutive columns of 2 rows per step (bias preloaded for its columns).
+// With split-K the raw partial tile goes to `part` instead.
+template <int EK, int BN>
+__device__ __forceinline__ void epilogue_tile(const Epi& e, uint32_t tmem, float* stage, float* part, int M, int N,
+                                              int m0, int n0, int q, int lane, int S) {
+  const int l4 = lane & 15, rh = lane >> 4;
+#pragma unroll 1
+  for (int c0 = 0; c0 < BN; c0 += 64) {
+    uint32_t v[16];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(c0 + 16 * h), v);
+#pragma unroll
+      for (int j = 0; j < 16; j += 4)
+        *reinterpret_cast<float4*>(stage + lane * 68 + 16 * h + j) =
+            make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]), __uint_as_float(v[j + 2]),
+                        __uint_as_float(v[j + 3]));
+    }
+    __syncwarp();
+    const int c = n0 + c0 + 4 * l4;
+    if (S == 1) {
+      float4 bv = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (e.bias && c < N) bv = *reinterpret_cast<const float4*>(e.bias + c);
+#pragma unroll 4
+      for (int i = 0; i < 16; ++i) {
+        const int rr = 2 * i + rh;
+        const int row = m0 + 32 * q + rr;
+        float4 t = *reinterpret_cast<const float4*>(stage + rr * 68 + 4 * l4);
+        t.x += bv.x; t.y += bv.y; t.z += bv.z; t.w += bv.w;
+        if (row < M && c < N) epi_store4<EK, bf16>(e, row, c, t);
+      }
+    } else {
+#pragma unroll 4
+      for (int i = 0; i < 16; ++i) {
+        const int rr = 2 * i + rh;
+        *reinterpret_cast<float4*>(part + (int64_t)(32 * q + rr) * BN + c0 + 4 * l4) =
+            *reinterpret_cast<const float4*>(stage + rr * 68 + 4 * l4);
+      }
+    }
+    __syncwarp();
+  }
+}
+
+// Split-K finish: sum the S partial tiles (fixed order z = 0 .. S-1, so the
+// result does not depend on which CTA arrives last) and apply the epilogue.
+template <int EK, int BN>
+__device__ __forceinline__ void reduce_tile(const Epi& e, const float* base, int M, int N, int m0, int n0, int q,
+                                            int lane, int S) {
+  const int l4 = lane & 15, rh = lane >> 4;
+#pragma unroll 1
+  for (int c0 = 0; c0 < BN; c0 += 64) {
+    const int c = n0 + c0 + 4 * l4;
+    float4 bv = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (e.bias && c < N) bv = *reinterpret_cast<const float4*>(e.bias + c);
+#pragma unroll 1
+    for (int i0 = 0; i0 < 16; i0 += 4) {
+      float4 acc[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int zz = 0; zz < S; ++zz) {
+        float4 t[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int rr = 2 * (i0 + k) + rh;
+          t[k] = __ldcg(reinterpret_cast<const float4*>(base + ((int64_t)zz * TC_BM + 32 * q + rr) * BN + c0 + 4 * l4));
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          acc[k].x += t[k].x; acc[k].y += t[k].y; acc[k].z += t[k].z; acc[k].w += t[k].w;
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int row = m0 + 32 * q + 2 * (i0 + k) + rh;
+        float4 t = acc[k];
+        t.x += bv.x; t.y += bv.y; t.z += bv.z; t.w += bv.w;
+        if (row < M && c < N) epi_store4<EK, bf16>(e, row, c, t);
+      }
+    }
+  }
+}
 
 template <int BN, int STAGES>
 __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__ CUtensorMap ta,
                                                          const __grid_constant__ CUtensorMap tb, int M, int N, int K,
-                                                         Epi e, int* err) {
+                                                         Epi e, int* err, float* __restrict__ split_ws,
+                                                         int* __restrict__ split_cnt) {
   using C = TcCfg<BN, STAGES>;
   extern __shared__ uint8_t tc_smem[];
   uint8_t* sm = tc_smem + ((1024 - (su32(tc_smem) & 1023)) & 1023);
@@ -133,7 +220,11 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m0 = blockIdx.y * TC_BM, n0 = blockIdx.x * BN;
-  const int KB = (K + TC_BK - 1) / TC_BK;
+  // split-K: this CTA covers k-blocks [kb0, kb1) of the tile's K range
+  const int KB_all = (K + TC_BK - 1) / TC_BK;
+  const int S = gridDim.z, z = blockIdx.z;
+  const int kb0 = (int)((int64_t)KB_all * z / S), kb1 = (int)((int64_t)KB_all * (z + 1) / S);
+  const int KB = kb1 - kb0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -166,8 +257,8 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
           break;
         }
         mbar_expect_tx(&full[s], C::A_BYTES + C::B_BYTES);
-        tma_load_2d(sA + s * C::A_BYTES, &ta, &full[s], kb * TC_BK, m0);
-        tma_load_2d(sB + s * C::B_BYTES, &tb, &full[s], kb * TC_BK, n0);
+        tma_load_2d(sA + s * C::A_BYTES, &ta, &full[s], (kb0 + kb) * TC_BK, m0);
+        tma_load_2d(sB + s * C::B_BYTES, &tb, &full[s], (kb0 + kb) * TC_BK, n0);
         ++issued;
       }
       if (*abort_flag) {   // let this CTA's own loads land before the shared memory is released
@@ -204,26 +295,44 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
     // instruction).  The pipeline buffers are free once the accumulator is
     // complete, so the tiles reuse them.
     const int q = warp & 3;            // TMEM lane quarter this warp may access
-    float* stage = reinterpret_cast<float*>(sm) + q * (32 * 65);
+    float* stage = reinterpret_cast<float*>(sm) + q * (32 * 68);
+    volatile int* last_flag = abort_flag + 1;
     if (mbar_wait(accf, 0, abort_flag) && !*abort_flag) {
       tc_fence_after();
-#pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 64) {
-        uint32_t v[16];
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(c0 + 16 * h), v);
-#pragma unroll
-          for (int j = 0; j < 16; ++j) stage[lane * 65 + 16 * h + j] = __uint_as_float(v[j]);
+      const int tile = blockIdx.y * gridDim.x + blockIdx.x;
+      float* part = split_ws + ((int64_t)tile * S + z) * TC_BM * BN;
+      switch (e.kind) {
+        case EPI_BIAS: epilogue_tile<EPI_BIAS, BN>(e, tmem, stage, part, M, N, m0, n0, q, lane, S); break;
+        case EPI_BIAS_RELU: epilogue_tile<EPI_BIAS_RELU, BN>(e, tmem, stage, part, M, N, m0, n0, q, lane, S); break;
+        case EPI_BIAS_SWISH: epilogue_tile<EPI_BIAS_SWISH, BN>(e, tmem, stage, part, M, N, m0, n0, q, lane, S); break;
+        case EPI_BIAS_GLU: epilogue_tile<EPI_BIAS_GLU, BN>(e, tmem, stage, part, M, N, m0, n0, q, lane, S); break;
+        case EPI_RESID: epilogue_tile<EPI_RESID, BN>(e, tmem, stage, part, M, N, m0, n0, q, lane, S); break;
+        case EPI_F32: epilogue_tile<EPI_F32, BN>(e, tmem, stage, part, M, N, m0, n0, q, lane, S); break;
+        default: epilogue_tile<EPI_F32_AND_T, BN>(e, tmem, stage, part, M, N, m0, n0, q, lane, S); break;
+      }
+      if (S > 1) {
+        // the last CTA of the tile to arrive sums the partials in split order
+        __threadfence();
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (threadIdx.x == 64) {
+          const int prev = atomicAdd(&split_cnt[tile], 1);
+          *last_flag = (prev == S - 1) ? 1 : 0;
+          if (prev == S - 1) split_cnt[tile] = 0;   // ready for the next launch
         }
-        __syncwarp();
-        const int c = n0 + c0 + 2 * lane;
-#pragma unroll 4
-        for (int rr = 0; rr < 32; ++rr) {
-          const int row = m0 + 32 * q + rr;
-          if (row < M && c < N) epi_store2<bf16>(e, row, c, stage[rr * 65 + 2 * lane], stage[rr * 65 + 2 * lane + 1]);
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (*last_flag) {
+          __threadfence();
+          const float* base = split_ws + (int64_t)tile * S * TC_BM * BN;
+          switch (e.kind) {
+            case EPI_BIAS: reduce_tile<EPI_BIAS, BN>(e, base, M, N, m0, n0, q, lane, S); break;
+            case EPI_BIAS_RELU: reduce_tile<EPI_BIAS_RELU, BN>(e, base, M, N, m0, n0, q, lane, S); break;
+            case EPI_BIAS_SWISH: reduce_tile<EPI_BIAS_SWISH, BN>(e, base, M, N, m0, n0, q, lane, S); break;
+            case EPI_BIAS_GLU: reduce_tile<EPI_BIAS_GLU, BN>(e, base, M, N, m0, n0, q, lane, S); break;
+            case EPI_RESID: reduce_tile<EPI_RESID, BN>(e, base, M, N, m0, n0, q, lane, S); break;
+            case EPI_F32: reduce_tile<EPI_F32, BN>(e, base, M, N, m0, n0, q, lane, S); break;
+            default: reduce_tile<EPI_F32_AND_T, BN>(e, base, M, N, m0, n0, q, lane, S); break;
+          }
         }
-        __syncwarp();
       }
     } else {
       *abort_flag = 1;
@@ -266,48 +375,64 @@ cudaError_t make_map(CUtensorMap* m, const void* base, int rows, int cols, int l
 }
 
 template <int BN, int STAGES>
-cudaError_t launch_tc(const bf16* A, int lda, const bf16* W, int M, int N, int K, const Epi& e, int* err,
-                      cudaStream_t st) {
+cudaError_t launch_tc(const bf16* A, int lda, const bf16* W, int M, int N, int K, int splits, const Epi& e,
+                      const TcScratch& sc, cudaStream_t st) {
   CUtensorMap ta, tb;
   cudaError_t r = make_map(&ta, A, M, K, lda, TC_BM);
   if (r != cudaSuccess) return r;
   r = make_map(&tb, W, N, K, K, BN);
   if (r != cudaSuccess) return r;
-  dim3 grid((N + BN - 1) / BN, (M + TC_BM - 1) / TC_BM);
-  gemm_tc_kernel<BN, STAGES><<<grid, 192, TcCfg<BN, STAGES>::SMEM, st>>>(ta, tb, M, N, K, e, err);
+  dim3 grid((N + BN - 1) / BN, (M + TC_BM - 1) / TC_BM, splits);
+  gemm_tc_kernel<BN, STAGES><<<grid, 192, TcCfg<BN, STAGES>::SMEM, st>>>(ta, tb, M, N, K, e, sc.err, sc.ws, sc.cnt);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-// Tile width: the widest of 256 / 128 / 64 that does not cost extra waves of
-// 148 SMs (cost ~ waves x (BN + 32), 32 standing for the per-tile A traffic).
-int gemm_tc_pick_bn(int M, int N) {
+// Tile width BN and split count S from a cost model of this kernel on 148
+// SMs, calibrated with per-phase timestamps on B200: per CTA ~1.4 us of
+// set-up and first-load latency, ~0.28 us per 64-wide k-block (bounded by
+// loads in flight, nearly independent of BN), and an epilogue of ~1.4 / 2.1 /
+// 3.8 us for BN = 64 / 128 / 256; a split-K partial round trip costs about
+// (BN / 64) x (1.5 + 0.9 S) us.  Splits need scratch and at most 2 waves.
+void gemm_tc_plan(int M, int N, int K, const TcScratch& sc, int* bn_out, int* s_out) {
   const int tm = (M + TC_BM - 1) / TC_BM;
-  int best = 64;
-  double best_cost = 1e30;
+  const int KB = (K + TC_BK - 1) / TC_BK;
+  double best = 1e30;
+  int bb = 64, bs = 1;
   for (int bn : {256, 128, 64}) {
     const int tiles = tm * ((N + bn - 1) / bn);
-    const int waves = (tiles + 147) / 148;
-    const double cost = (double)waves * (bn + 32);
-    if (cost < best_cost) {
-      best_cost = cost;
-      best = bn;
+    for (int sp : {1, 2, 3, 4}) {
+      if (sp > 1 && (!sc.ws || !sc.cnt || sp > KB || (int64_t)tiles * sp > 2 * 148 ||
+                     (size_t)tiles * sp * TC_BM * bn * 4 > sc.ws_bytes || tiles > sc.cnt_len))
+        continue;
+      const int waves = (tiles * sp + 147) / 148;
+      const int kb_per = (KB + sp - 1) / sp;
+      const double epi = sp == 1 ? (bn == 64 ? 1.4 : bn == 128 ? 2.1 : 3.8) : (bn / 64.0) * (1.5 + 0.9 * sp);
+      const double t = waves * (1.4 + 0.28 * kb_per + epi);
+      if (t < best * 0.97) {
+        best = t;
+        bb = bn;
+        bs = sp;
+      }
     }
   }
-  return best;
+  *bn_out = bb;
+  *s_out = bs;
 }
 
-cudaError_t gemm_bf16_tc(const bf16* A, int lda, const bf16* W, int M, int N, int K, const Epi& e, int* err,
-                         cudaStream_t st) {
+cudaError_t gemm_bf16_tc(const bf16* A, int lda, const bf16* W, int M, int N, int K, const Epi& e,
+                         const TcScratch& sc, cudaStream_t st) {
   if (M <= 0) return cudaSuccess;
   if (N % 16 || K % 8) return cudaErrorInvalidValue;
   cudaError_t r = get_encoder();
   if (r != cudaSuccess) return r;
-  switch (gemm_tc_pick_bn(M, N)) {
-    case 256: return launch_tc<256, 4>(A, lda, W, M, N, K, e, err, st);
-    case 128: return launch_tc<128, 6>(A, lda, W, M, N, K, e, err, st);
-    default: return launch_tc<64, 8>(A, lda, W, M, N, K, e, err, st);
+  int bn, sp;
+  gemm_tc_plan(M, N, K, sc, &bn, &sp);
+  switch (bn) {
+    case 256: return launch_tc<256, 4>(A, lda, W, M, N, K, sp, e, sc, st);
+    case 128: return launch_tc<128, 6>(A, lda, W, M, N, K, sp, e, sc, st);
+    default: return launch_tc<64, 8>(A, lda, W, M, N, K, sp, e, sc, st);
   }
 }
 

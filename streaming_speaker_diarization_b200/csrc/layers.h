@@ -34,11 +34,21 @@ cudaError_t gemm_f32(const float* A, int lda, const float* W, int M, int N, int 
 cudaError_t gemm_bf16_mma(const bf16* A, int lda, const bf16* W, int M, int N, int K, const Epi& e,
                           cudaStream_t st);
 cudaError_t gemm_init_attributes();
-// tcgen05 / TMEM / TMA path (sm_100a); err = device error word (may be null).
-cudaError_t gemm_bf16_tc(const bf16* A, int lda, const bf16* W, int M, int N, int K, const Epi& e, int* err,
-                         cudaStream_t st);
+// Scratch of the tcgen05 GEMM: error word, split-K partial tiles and the
+// per-tile arrival counters (zero between launches; the last CTA of a tile
+// resets its counter).  ws/cnt may be null: no split-K then.
+struct TcScratch {
+  int* err;
+  float* ws;
+  size_t ws_bytes;
+  int* cnt;
+  int cnt_len;
+};
+// tcgen05 / TMEM / TMA path (sm_100a).
+cudaError_t gemm_bf16_tc(const bf16* A, int lda, const bf16* W, int M, int N, int K, const Epi& e,
+                         const TcScratch& sc, cudaStream_t st);
 cudaError_t gemm_tc_init_attributes();
-int gemm_tc_pick_bn(int M, int N);
+void gemm_tc_plan(int M, int N, int K, const TcScratch& sc, int* bn, int* splits);
 
 // --------------------------------------------------------- subsampling
 struct PreArgs {        // device arrays, one entry per window

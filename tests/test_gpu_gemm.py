@@ -20,8 +20,11 @@ def eng():
     b.sf_destroy(e)
 
 
+# engine shapes at the 90 s workload (M = 1125), streaming batches, ragged M,
+# every tile width and split-K counts 1..8 (e.g. (300, 64, 4096): 3 tiles -> 8 splits)
 SHAPES = [(1125, 2048, 512), (1125, 512, 2048), (1125, 1536, 512), (1125, 192, 192), (1125, 576, 192),
-          (1, 64, 64), (333, 768, 192), (128, 128, 128), (129, 256, 4096), (24896, 1024, 512), (70, 16, 64)]
+          (1125, 192, 768), (1125, 512, 4096), (1, 64, 64), (333, 768, 192), (128, 128, 128), (129, 256, 4096),
+          (24896, 1024, 512), (70, 16, 64), (300, 64, 4096), (2000, 256, 1024)]
 
 
 @pytest.mark.parametrize("M,N,K", SHAPES)
@@ -54,3 +57,20 @@ def test_gemm_tc_strided_a(eng):
     b.sf_check(eng)
     ref = big[:, K:2 * K].double().numpy() @ W.double().numpy().T
     assert np.max(np.abs(C.cpu().numpy() - ref)) < 2e-3
+
+
+def test_gemm_tc_split_k_is_deterministic(eng):
+    """Split-K partials are summed in split order by whichever CTA arrives
+    last: repeated launches must agree bit for bit."""
+    M, N, K = 1125, 512, 2048
+    g = torch.Generator().manual_seed(11)
+    A = (torch.randn(M, K, generator=g) / 40).to(torch.bfloat16).cuda()
+    W = torch.randn(N, K, generator=g).to(torch.bfloat16).cuda()
+    outs = []
+    for _ in range(4):
+        C = torch.zeros((M, N), device="cuda")
+        b.sf_gemm_bf16(eng, A, W, C, path=1)
+        outs.append(C.cpu())
+    b.sf_check(eng)
+    for o in outs[1:]:
+        assert torch.equal(o, outs[0])
