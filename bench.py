@@ -104,6 +104,73 @@ def cpu_baseline(audio, seconds=30.0):
                       f"({dt:.1f} s)"}
 
 
+STREAM_WORKLOADS = [
+    # (name, preset chunk/right/fifo/update/cache, workload index, streams, seconds)
+    ("Low preset (6/7/188/144/188, 1.04 s latency), 64 streams x 60 s, 2-4 speakers", (6, 7, 188, 144, 188), 2, 64, 60.0),
+    ("Very high preset (340/40/40/300/188, 30.4 s latency), 16 streams x 600 s, 4 speakers, 20% overlap, arrivals",
+     (340, 40, 40, 300, 188), 3, 16, 600.0),
+]
+
+
+def streaming_bench(b, torch, eng_blob, rank, world, local):
+    """Streaming throughput: front-end over each stream's clip, then every
+    step of every stream (pre_encode on the new window, encoder on
+    [cache | FIFO | chunk], state update) until all streams finish.  A first
+    pass captures each step shape's CUDA graph; the streams are reset and the
+    second pass is timed with CUDA events."""
+    from streaming_speaker_diarization_b200 import dist as sd
+    from synth import clip_for_config
+    out = []
+    for name, preset, idx, n_total, dur in STREAM_WORKLOADS:
+        lo, hi = sd.shard(n_total, rank, world)
+        n = hi - lo
+        audio_np, lens, _ = clip_for_config(idx)
+        audio_np, lens = np.ascontiguousarray(audio_np[lo:hi]), lens[lo:hi]
+        eng = b.sf_create(eng_blob, b.default_config(max_batch=max(n, 1)))
+        audio = torch.from_numpy(audio_np).cuda()
+        T = 1 + audio_np.shape[1] // 160
+        mel = torch.empty((n, 128, T), device="cuda")
+        cp = torch.zeros((n, preset[0], 4), device="cuda")
+        st = b.sf_stream_create(eng, preset, n)
+        zero = np.zeros(n, np.int64)
+
+        def one_pass(times=None):
+            ml = b.sf_mel(eng, audio, lens, mel)
+            left = 1 + (ml - 1) // 8          # encoder frames each stream still has to emit
+            while (left > 0).any():
+                if times is not None:
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record()
+                n_out = b.sf_stream_step(eng, st, mel, zero, ml, cp)
+                if times is not None:
+                    e1.record()
+                    times.append((e0, e1))
+                left -= n_out
+            return ml
+
+        one_pass()
+        b.sf_stream_reset(st)
+        torch.cuda.synchronize()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        steps = []
+        t0.record()
+        one_pass(steps)
+        t1.record()
+        torch.cuda.synchronize()
+        ms = t0.elapsed_time(t1)
+        step_ms = [a.elapsed_time(c) for a, c in steps]
+        audio_s = float(lens.sum()) / 16000.0
+        value = sd.throughput(audio_s, ms)
+        out.append({"workload": name, "value": value, "unit": UNIT, "streams": n_total, "steps": len(step_ms),
+                    "ms_total": sd.max_over_ranks(ms), "step_ms_p50": float(np.median(step_ms)),
+                    "step_ms_p95": float(np.percentile(step_ms, 95))})
+        b.sf_stream_destroy(st)
+        b.sf_destroy(eng)
+        del audio, mel
+        torch.cuda.empty_cache()
+    return out
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return 0
@@ -140,6 +207,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--pdl", type=int, default=0, help="programmatic dependent launch between kernels (0/1)")
+    ap.add_argument("--no-streaming", action="store_true", help="skip the streaming workloads")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
@@ -159,6 +228,7 @@ def main():
     audio_np, lens, _ = clip_for_config(1)
     w = make_weights(FULL, seed=0)
     eng = b.sf_create(weights_blob(w), b.default_config(max_batch=1))
+    b.sf_set_option(eng, b.SF_OPT_PDL, args.pdl)
     st = torch.cuda.current_stream()
     audio = torch.from_numpy(audio_np).cuda()
     probs = torch.zeros((1, 1125, 4), device="cuda")
@@ -188,22 +258,28 @@ def main():
     step_ms = [a.elapsed_time(c) for a, c in ev]
     stats = b.sf_profile_read(eng, reset=True)
     launches = int(sum(v[0] for v in stats.values()))
+    from streaming_speaker_diarization_b200 import dist as sd
     total_ms = float(sum(step_ms))
-    t = torch.tensor([total_ms], device="cuda", dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    max_ms = float(t.item())
+    max_ms = sd.max_over_ranks(total_ms, "cuda")
     audio_s = 90.0 * args.steps * world
-    value = audio_s / (max_ms / 1000.0)
+    value = sd.throughput(90.0 * args.steps, total_ms, "cuda")
 
-    # per-kernel attribution: the same K steps again with CUDA events around every launch
-    b.sf_profile_enable(eng, True)
+    # per-kernel attribution: the same K steps again with CUDA events around
+    # every launch (shares), then with events around the GEMM launches only
+    # (the roofline's kernel time, without event nodes between the others)
+    b.sf_profile_enable(eng, 1)
     for i in range(args.steps):
         flush.zero_()
         b.sf_forward_offline(eng, audio, lens, probs)
     torch.cuda.synchronize()
     prof = b.sf_profile_read(eng, reset=True)
-    b.sf_profile_enable(eng, False)
+    b.sf_profile_enable(eng, 2 * (1 << 3))      # class 3 = gemm
+    for i in range(args.steps):
+        flush.zero_()
+        b.sf_forward_offline(eng, audio, lens, probs)
+    torch.cuda.synchronize()
+    prof_gemm = b.sf_profile_read(eng, reset=True)
+    b.sf_profile_enable(eng, 0)
 
     # end to end through the host-memory entry point (H2D + compute + D2H every step)
     h_audio = torch.from_numpy(audio_np).pin_memory()
@@ -218,13 +294,10 @@ def main():
         e2e_ev[i][1].record(st)
     barrier()
     e2e_ms = float(sum(a.elapsed_time(c) for a, c in e2e_ev))
-    te = torch.tensor([e2e_ms], device="cuda", dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_value = audio_s / (float(te.item()) / 1000.0)
+    e2e_value = sd.throughput(90.0 * args.steps, e2e_ms, "cuda")
 
     pk, pk_kind = peaks()
-    g = prof.get("gemm", (0, 0.0, 0.0, 0.0))
+    g = prof_gemm.get("gemm", (0, 0.0, 0.0, 0.0))
     timed_s = max_ms / 1000.0
     peak_tf = pk["bf16_tflops_sustained"] if timed_s > 1.0 else pk["bf16_tflops"]
     achieved = (g[2] / (g[1] / 1000.0)) / 1e12 if g[1] > 0 else None
@@ -246,11 +319,13 @@ def main():
                     "d2h_bytes_per_step": int(h_probs.numel() * 4)},
             "step_ms_p50": float(np.median(step_ms)), "step_ms_p95": float(np.percentile(step_ms, 95)),
             "kernels": kernels}
+    b.sf_destroy(eng)
+    if not args.no_streaming:
+        line["streaming"] = streaming_bench(b, torch, weights_blob(w), rank, world, local)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(audio_np)
     if rank == 0:
         print(json.dumps(line), flush=True)
-    b.sf_destroy(eng)
     if world > 1:
         dist.destroy_process_group()
     return 0

@@ -282,6 +282,16 @@ SF_API sf_status sf_stream_update(sf_stream* s, const float* d_preds, const void
 SF_API sf_status sf_select_topk(sf_engine* e, const float* d_scores, const int* h_n, int n_sets, int stride, int k,
                          int* d_src, void* cuda_stream);
 
+/* ---------------------------------------------------------------- options */
+
+enum {
+  SF_OPT_GRAPHS = 1,     /* 1 (default): capture each call shape once as a CUDA graph and
+                            replay it; 0: launch kernel by kernel */
+  SF_OPT_PDL = 2,        /* 1: programmatic dependent launch between kernels; 0 (default) */
+  SF_OPT_GEMM_PATH = 3   /* bf16 projections: 1 (default) tcgen05/TMEM/TMA kernel, 0 mma.sync */
+};
+SF_API sf_status sf_set_option(sf_engine* e, int option, int value);
+
 /* ------------------------------------------------------------ diagnostics */
 
 /* Synchronise `cuda_stream` and read (then clear) the engine's device error
@@ -312,8 +322,12 @@ typedef struct {
 } sf_kernel_stat;
 
 /* Launch counting is always on.  enable = 1 also brackets every launch with
- * a pair of CUDA events (adds a few microseconds of event records per
- * launch; use for attribution, not for end-to-end timing). */
+ * a pair of CUDA events (each pair adds a few microseconds; use for
+ * attribution, not for end-to-end timing); enable = 2 * mask brackets only
+ * the kernel classes whose bit is set in `mask` (bit k = the k-th class in
+ * the order mel, conv1, dwconv3x3s2, gemm, attention_relpos, attention_mha,
+ * layernorm, dwconv1d, head_out, assemble, extract, state_update, to_f32,
+ * select_topk); enable = 0 stops recording. */
 SF_API sf_status sf_profile_enable(sf_engine* e, int enable);
 /* Synchronise on the recorded events and report one entry per kernel class
  * with at least one launch since the last reset (at most `max` entries,

@@ -17,6 +17,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libsf.so")
 
 SF_FP32, SF_BF16 = 0, 1
+SF_OPT_GRAPHS, SF_OPT_PDL, SF_OPT_GEMM_PATH = 1, 2, 3
 STATUS = {0: "SF_OK", 1: "SF_EINVAL", 2: "SF_ESHAPE", 3: "SF_ENOMEM", 4: "SF_ECUDA", 5: "SF_ESTATE",
           6: "SF_ETIMEOUT", 7: "SF_EDEVICE", 8: "SF_EFORMAT"}
 
@@ -50,7 +51,7 @@ EXPORTED = ["sf_default_config", "sf_create", "sf_create_from_file", "sf_destroy
             "sf_forward_offline_host", "sf_stream_create", "sf_stream_destroy", "sf_stream_reset",
             "sf_stream_window", "sf_stream_step", "sf_stream_get_state", "sf_stream_set_state",
             "sf_stream_update", "sf_select_topk", "sf_profile_enable", "sf_profile_read", "sf_mel_noalloc",
-            "sf_check", "sf_gemm_bf16"]
+            "sf_check", "sf_gemm_bf16", "sf_set_option"]
 
 
 class SFError(RuntimeError):
@@ -88,6 +89,7 @@ def _load():
         "sf_profile_read": ([VP, P(sf_kernel_stat), I, P(I), I], I),
         "sf_mel_noalloc": ([VP, VP, I, I64, VP, VP, VP], I),
         "sf_check": ([VP, VP], I),
+        "sf_set_option": ([VP, I, I], I),
         "sf_gemm_bf16": ([VP, VP, I, VP, I, I, I, VP, VP, I, VP], I),
     }
     for name, (args, res) in sig.items():
@@ -258,8 +260,9 @@ def sf_select_topk(eng, scores, n, k, src, stream=None):
     _check(lib.sf_select_topk(eng, _ptr(scores), _ptr(n), n_sets, stride, k, _ptr(src), _stream(stream)), eng)
 
 
-def sf_profile_enable(eng, enable=True):
-    _check(lib.sf_profile_enable(eng, int(bool(enable))), eng)
+def sf_profile_enable(eng, enable=1):
+    """0 = off, 1 = every kernel class, 2 * mask = the classes in mask."""
+    _check(lib.sf_profile_enable(eng, int(enable)), eng)
 
 
 def sf_profile_read(eng, reset=True):
@@ -279,3 +282,7 @@ def sf_gemm_bf16(eng, A, W, C, bias=None, path=1, stream=None):
     N = W.shape[0]
     _check(lib.sf_gemm_bf16(eng, _ptr(A), A.stride(0), _ptr(W), M, N, K, _ptr(bias), _ptr(C), path,
                             _stream(stream)), eng)
+
+
+def sf_set_option(eng, option, value):
+    _check(lib.sf_set_option(eng, option, value), eng)

@@ -24,6 +24,7 @@ __global__ void __launch_bounds__(128) attn_f32_kernel(const float* __restrict__
                                                        const float* __restrict__ u, const float* __restrict__ vb,
                                                        float* __restrict__ ctx, const SeqTable* __restrict__ seq,
                                                        int M, int s_cap) {
+  SF_PDL_ENTRY();
   extern __shared__ float att_smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r = blockIdx.x * 4 + warp;
@@ -157,6 +158,7 @@ __global__ void __launch_bounds__(128) attn_bf16_kernel(const bf16* __restrict__
                                                         const bf16* __restrict__ ptab, int R,
                                                         const float* __restrict__ u, const float* __restrict__ vb,
                                                         bf16* __restrict__ ctx, const SeqTable* __restrict__ seq) {
+  SF_PDL_ENTRY();
   using C = AttCfg<HD, HDP, REL>;
   constexpr int LDS = C::LDS;
   extern __shared__ float4 att_smem4[];
@@ -346,7 +348,7 @@ cudaError_t launch_relpos_attention<float>(const float* qkv, const float* ptab, 
   if (M <= 0) return cudaSuccess;
   const int s_cap = R;   // no sequence is longer than the position table
   const size_t smem = (size_t)4 * (s_cap + 128) * 4;
-  attn_f32_kernel<64, true><<<dim3((M + 3) / 4, 8), 128, smem, st>>>(qkv, 512, ptab, R, u, v, ctx, seq, M, s_cap);
+  CK_LAUNCH(launch_k(attn_f32_kernel<64, true>, dim3(dim3((M + 3) / 4, 8)), dim3(128), smem, st, qkv, 512, ptab, R, u, v, ctx, seq, M, s_cap));
   return cudaGetLastError();
 }
 
@@ -354,8 +356,8 @@ template <>
 cudaError_t launch_relpos_attention<bf16>(const bf16* qkv, const bf16* ptab, int R, const float* u, const float* v,
                                           bf16* ctx, const SeqTable* seq, int n_tiles, int M, cudaStream_t st) {
   if (M <= 0) return cudaSuccess;
-  attn_bf16_kernel<64, 64, true><<<dim3(n_tiles, 8), 128, AttCfg<64, 64, true>::SMEM, st>>>(qkv, 512, ptab, R, u, v,
-                                                                                             ctx, seq);
+  CK_LAUNCH(launch_k(attn_bf16_kernel<64, 64, true>, dim3(dim3(n_tiles, 8)), dim3(128), AttCfg<64, 64, true>::SMEM, st, qkv, 512, ptab, R, u, v,
+                                                                                             ctx, seq));
   return cudaGetLastError();
 }
 
@@ -364,16 +366,16 @@ cudaError_t launch_mha<float>(const float* qkv, float* ctx, const SeqTable* seq,
   if (M <= 0) return cudaSuccess;
   const int s_cap = g_att_s_cap;
   const size_t smem = (size_t)4 * (s_cap + 128) * 4;
-  attn_f32_kernel<24, false><<<dim3((M + 3) / 4, 8), 128, smem, st>>>(qkv, 192, nullptr, 0, nullptr, nullptr, ctx, seq,
-                                                                      M, s_cap);
+  CK_LAUNCH(launch_k(attn_f32_kernel<24, false>, dim3(dim3((M + 3) / 4, 8)), dim3(128), smem, st, qkv, 192, nullptr, 0, nullptr, nullptr, ctx, seq,
+                                                                      M, s_cap));
   return cudaGetLastError();
 }
 
 template <>
 cudaError_t launch_mha<bf16>(const bf16* qkv, bf16* ctx, const SeqTable* seq, int n_tiles, int M, cudaStream_t st) {
   if (M <= 0) return cudaSuccess;
-  attn_bf16_kernel<24, 32, false><<<dim3(n_tiles, 8), 128, AttCfg<24, 32, false>::SMEM, st>>>(
-      qkv, 192, nullptr, 0, nullptr, nullptr, ctx, seq);
+  CK_LAUNCH(launch_k(attn_bf16_kernel<24, 32, false>, dim3(dim3(n_tiles, 8)), dim3(128), AttCfg<24, 32, false>::SMEM, st, 
+      qkv, 192, nullptr, 0, nullptr, nullptr, ctx, seq));
   return cudaGetLastError();
 }
 

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 namespace sf {
 
 typedef __nv_bfloat16 bf16;
@@ -72,6 +74,43 @@ __device__ __forceinline__ int seq_of_tile(const SeqTable* __restrict__ st, int 
 
 __device__ __forceinline__ void set_err(int* err, int bit) {
   if (err) atomicOr(err, bit);
+}
+
+// Programmatic dependent launch: every kernel waits for its predecessor's
+// memory before its first global access, then lets its successor launch (the
+// successor's prologue overlaps this kernel; at most two grids are in flight).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+#define SF_PDL_ENTRY() \
+  do {                 \
+    sf::pdl_wait();    \
+    sf::pdl_trigger(); \
+  } while (0)
+
+#define CK_LAUNCH(x)                  \
+  do {                                \
+    cudaError_t _le = (x);            \
+    if (_le != cudaSuccess) return _le; \
+  } while (0)
+
+// Launch mode of the calling engine (set at each API entry): 0 = plain
+// stream order, 1 = programmatic dependent launch.
+extern int g_launch_pdl;
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                            Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = g_launch_pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 }  // namespace sf

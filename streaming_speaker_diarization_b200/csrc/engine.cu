@@ -31,6 +31,10 @@
 
 using namespace sf;
 
+namespace sf {
+int g_launch_pdl = 0;
+}
+
 // Source line of the first CUDA call that failed in the current API call
 // (reported by sf_last_error).
 static int g_fail_line = 0;
@@ -162,6 +166,7 @@ struct sf_engine {
   Weights<bf16> wb;
   // profiling: launch/work counters always; event pairs when prof is set
   bool prof = false;
+  uint32_t prof_mask = 0;       // kernel classes bracketed with events
   int64_t launches[K_COUNT] = {};
   double kflops[K_COUNT] = {};
   double kbytes[K_COUNT] = {};
@@ -172,6 +177,7 @@ struct sf_engine {
   double ms_acc[K_COUNT] = {};   // event time already read back (graph replays)
   // CUDA graphs: one per launch shape, replayed; invalidated when the workspace moves
   bool use_graphs = true;
+  int use_pdl = 0;
   bool capturing = false;
   cudaStream_t cap_stream = nullptr;     // graphs are captured here, launched on the caller's stream
   std::vector<cudaEvent_t> cap_events;   // events created for the graph being captured
@@ -237,7 +243,7 @@ struct Scope {
     e->launches[cls] += n_kernels;
     e->kflops[cls] += flops;
     e->kbytes[cls] += bytes;
-    if (e->prof) {
+    if (e->prof && ((e->prof_mask >> cls) & 1u)) {
       cudaEvent_t a = e->capturing ? cap_event(e) : pool_event(e);
       b = e->capturing ? cap_event(e) : pool_event(e);
       if (a && b) {
@@ -630,7 +636,8 @@ void destroy_graphs(sf_engine* e) {
 template <typename F>
 cudaError_t run_graph(sf_engine* e, std::string key, cudaStream_t st, F&& enqueue) {
   if (!e->use_graphs) return enqueue(st);
-  key += e->prof ? "|p" : "|n";
+  key += e->prof ? "|p" + std::to_string(e->prof_mask) : "|n";
+  key += e->use_pdl ? "|pdl" : "";
   auto it = e->graphs.find(key);
   if (it != e->graphs.end() && it->second.gen != e->ws_gen) {
     cudaGraphExecDestroy(it->second.exec);
@@ -898,6 +905,7 @@ sf_status check_engine(sf_engine* e) {
   if (!e) return SF_EINVAL;
   g_ws_gen = &e->ws_gen;
   g_fail_line = 0;
+  sf::g_launch_pdl = e->use_pdl;
   cudaGetLastError();   // start each call without a stale, non-sticky error
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev != e->device) cudaSetDevice(e->device);
@@ -1221,9 +1229,25 @@ sf_status sf_gemm_bf16(sf_engine* e, const void* d_A, int lda, const void* d_W, 
   return SF_OK;
 }
 
+sf_status sf_set_option(sf_engine* e, int option, int value) {
+  if (check_engine(e) != SF_OK) return SF_EINVAL;
+  switch (option) {
+    case SF_OPT_GRAPHS: e->use_graphs = value != 0; break;
+    case SF_OPT_PDL: e->use_pdl = value != 0; break;
+    case SF_OPT_GEMM_PATH:
+      if (value != 0 && value != 1) return fail(e, SF_EINVAL, "gemm path must be 0 or 1");
+      e->gemm_path = value;
+      break;
+    default: return fail(e, SF_EINVAL, "unknown option");
+  }
+  sf::g_launch_pdl = e->use_pdl;
+  return SF_OK;
+}
+
 sf_status sf_profile_enable(sf_engine* e, int enable) {
   if (!e) return SF_EINVAL;
   e->prof = enable != 0;
+  e->prof_mask = enable == 1 ? 0xffffffffu : (uint32_t)enable >> 1;
   return SF_OK;
 }
 

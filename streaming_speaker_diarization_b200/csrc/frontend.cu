@@ -28,6 +28,7 @@ __global__ void __launch_bounds__(256) mel_frames_kernel(const float* __restrict
                                                           const MelArgs args, const MelTables* __restrict__ tab,
                                                           float* __restrict__ mel, float* __restrict__ part,
                                                           int T_cols, int n_blk) {
+  SF_PDL_ENTRY();
   extern __shared__ float4 mel_smem[];
   float* y = reinterpret_cast<float*>(mel_smem);               // [MEL_SPAN]
   float2* tw256 = reinterpret_cast<float2*>(y + MEL_SPAN);      // [128]
@@ -154,6 +155,7 @@ __global__ void __launch_bounds__(256) mel_frames_kernel(const float* __restrict
 
 __global__ void __launch_bounds__(256) mel_normalize_kernel(float* __restrict__ mel, const float* __restrict__ part,
                                                             const MelArgs args, int T_cols, int n_blk) {
+  SF_PDL_ENTRY();
   const int m = blockIdx.x, b = blockIdx.y;
   const int L = (int)(args.len[b] / 160);
   __shared__ float s_mu, s_inv;
@@ -216,8 +218,8 @@ cudaError_t launch_mel(const float* audio, int B, int64_t n_max, const MelArgs& 
     if (e != cudaSuccess) return e;
   }
   attr_set = true;
-  mel_frames_kernel<<<dim3(n_blk, B), 256, smem, st>>>(audio, n_max, args, tab, mel, part, T_cols, n_blk);
-  mel_normalize_kernel<<<dim3(128, B), 256, 0, st>>>(mel, part, args, T_cols, n_blk);
+  CK_LAUNCH(launch_k(mel_frames_kernel, dim3(dim3(n_blk, B)), dim3(256), smem, st, audio, n_max, args, tab, mel, part, T_cols, n_blk));
+  CK_LAUNCH(launch_k(mel_normalize_kernel, dim3(dim3(128, B)), dim3(256), 0, st, mel, part, args, T_cols, n_blk));
   return cudaGetLastError();
 }
 

@@ -17,6 +17,7 @@ namespace sf {
 // ------------------------------------------------------------- fp32 SIMT
 __global__ void __launch_bounds__(256) gemm_simt_kernel(const float* __restrict__ A, int lda,
                                                         const float* __restrict__ W, int M, int N, int K, Epi e) {
+  SF_PDL_ENTRY();
   constexpr int BM = 64, BN = 64, BK = 16;
   __shared__ float As[BK][BM + 4];
   __shared__ float Bs[BK][BN + 4];
@@ -85,6 +86,7 @@ constexpr int MM_SMEM = MM_STAGES * (MM_BM + MM_BN) * MM_LD * 2;
 
 __global__ void __launch_bounds__(256) gemm_mma_kernel(const bf16* __restrict__ A, int lda,
                                                        const bf16* __restrict__ W, int M, int N, int K, Epi e) {
+  SF_PDL_ENTRY();
   extern __shared__ float4 mm_smem[];
   bf16* sA = reinterpret_cast<bf16*>(mm_smem);
   bf16* sB = sA + MM_STAGES * MM_BM * MM_LD;
@@ -173,14 +175,14 @@ __global__ void __launch_bounds__(256) gemm_mma_kernel(const bf16* __restrict__ 
 cudaError_t gemm_f32(const float* A, int lda, const float* W, int M, int N, int K, const Epi& e, cudaStream_t st) {
   if (M <= 0) return cudaSuccess;
   dim3 grid((N + 63) / 64, (M + 63) / 64);
-  gemm_simt_kernel<<<grid, 256, 0, st>>>(A, lda, W, M, N, K, e);
+  CK_LAUNCH(launch_k(gemm_simt_kernel, dim3(grid), dim3(256), 0, st, A, lda, W, M, N, K, e));
   return cudaGetLastError();
 }
 
 cudaError_t gemm_bf16_mma(const bf16* A, int lda, const bf16* W, int M, int N, int K, const Epi& e, cudaStream_t st) {
   if (M <= 0) return cudaSuccess;
   dim3 grid((N + MM_BN - 1) / MM_BN, (M + MM_BM - 1) / MM_BM);
-  gemm_mma_kernel<<<grid, 256, MM_SMEM, st>>>(A, lda, W, M, N, K, e);
+  CK_LAUNCH(launch_k(gemm_mma_kernel, dim3(grid), dim3(256), MM_SMEM, st, A, lda, W, M, N, K, e));
   return cudaGetLastError();
 }
 

@@ -227,6 +227,8 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
   const int KB = kb1 - kb0;
 
   if (threadIdx.x == 0) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&ta)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tb)) : "memory");
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
@@ -246,6 +248,8 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // set-up above overlaps the previous kernel; global memory only from here
+  SF_PDL_ENTRY();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -383,7 +387,7 @@ cudaError_t launch_tc(const bf16* A, int lda, const bf16* W, int M, int N, int K
   r = make_map(&tb, W, N, K, K, BN);
   if (r != cudaSuccess) return r;
   dim3 grid((N + BN - 1) / BN, (M + TC_BM - 1) / TC_BM, splits);
-  gemm_tc_kernel<BN, STAGES><<<grid, 192, TcCfg<BN, STAGES>::SMEM, st>>>(ta, tb, M, N, K, e, sc.err, sc.ws, sc.cnt);
+  CK_LAUNCH(launch_k(gemm_tc_kernel<BN, STAGES>, dim3(grid), dim3(192), TcCfg<BN, STAGES>::SMEM, st, ta, tb, M, N, K, e, sc.err, sc.ws, sc.cnt));
   return cudaGetLastError();
 }
 

@@ -11,6 +11,7 @@ template <typename T, int D, int VEC>
 __global__ void __launch_bounds__(256) layernorm_kernel(float* __restrict__ x, const float* __restrict__ g,
                                                         const float* __restrict__ b, int M, bool write_x,
                                                         T* __restrict__ h) {
+  SF_PDL_ENTRY();
   constexpr int NV = D / (32 * VEC);
   const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -60,8 +61,8 @@ cudaError_t launch_layernorm(float* x, const float* g, const float* b, int M, in
                              cudaStream_t st) {
   if (M <= 0) return cudaSuccess;
   const int grid = (M + 7) / 8;
-  if (D == 512) layernorm_kernel<T, 512, 4><<<grid, 256, 0, st>>>(x, g, b, M, write_x, h);
-  else if (D == 192) layernorm_kernel<T, 192, 2><<<grid, 256, 0, st>>>(x, g, b, M, write_x, h);
+  if (D == 512) CK_LAUNCH(launch_k(layernorm_kernel<T, 512, 4>, dim3(grid), dim3(256), 0, st, x, g, b, M, write_x, h));
+  else if (D == 192) CK_LAUNCH(launch_k(layernorm_kernel<T, 192, 2>, dim3(grid), dim3(256), 0, st, x, g, b, M, write_x, h));
   else return cudaErrorInvalidValue;
   return cudaGetLastError();
 }
@@ -91,6 +92,7 @@ template <typename T>
 __global__ void __launch_bounds__(128) dwconv1d_kernel(const T* __restrict__ in, T* __restrict__ out,
                                                        const float* __restrict__ w, const float* __restrict__ bias,
                                                        int M, int D, int K, const SeqTable* __restrict__ seq) {
+  SF_PDL_ENTRY();
   const int c = 2 * (blockIdx.y * 128 + threadIdx.x);
   if (c >= D) return;
   const int r0 = blockIdx.x * DW_ROWS;
@@ -141,7 +143,7 @@ cudaError_t launch_dwconv1d(const T* in, T* out, const float* w, const float* b,
   if (M <= 0) return cudaSuccess;
   if (K > DW_KMAX || (D % 2)) return cudaErrorInvalidValue;
   dim3 grid((M + DW_ROWS - 1) / DW_ROWS, (D / 2 + 127) / 128);
-  dwconv1d_kernel<T><<<grid, 128, 0, st>>>(in, out, w, b, M, D, K, seq);
+  CK_LAUNCH(launch_k(dwconv1d_kernel<T>, dim3(grid), dim3(128), 0, st, in, out, w, b, M, D, K, seq));
   return cudaGetLastError();
 }
 
@@ -150,6 +152,7 @@ template <typename T>
 __global__ void __launch_bounds__(256) head_out_kernel(const T* __restrict__ h, const float* __restrict__ w,
                                                        const float* __restrict__ b, float* __restrict__ probs,
                                                        int M, int E) {
+  SF_PDL_ENTRY();
   const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= M) return;
@@ -175,12 +178,13 @@ template <typename T>
 cudaError_t launch_head_out(const T* h, const float* w, const float* b, float* probs, int M, int E,
                             cudaStream_t st) {
   if (M <= 0) return cudaSuccess;
-  head_out_kernel<T><<<(M + 7) / 8, 256, 0, st>>>(h, w, b, probs, M, E);
+  CK_LAUNCH(launch_k(head_out_kernel<T>, dim3((M + 7) / 8), dim3(256), 0, st, h, w, b, probs, M, E));
   return cudaGetLastError();
 }
 
 template <typename T>
 __global__ void to_f32_kernel(const T* __restrict__ in, float* __restrict__ out, int64_t n) {
+  SF_PDL_ENTRY();
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
     out[i] = to_f<T>(in[i]);
 }
@@ -190,13 +194,14 @@ cudaError_t launch_to_f32(const T* in, float* out, int64_t n, cudaStream_t st) {
   if (n <= 0) return cudaSuccess;
   const int64_t want = (n + 255) / 256;
   const int64_t blocks = want < 148 * 16 ? want : 148 * 16;
-  to_f32_kernel<T><<<(int)blocks, 256, 0, st>>>(in, out, n);
+  CK_LAUNCH(launch_k(to_f32_kernel<T>, dim3((int)blocks), dim3(256), 0, st, in, out, n));
   return cudaGetLastError();
 }
 
 __global__ void extract_rows_kernel(const float* __restrict__ packed, const SeqTable* __restrict__ seq,
                                     const int* __restrict__ first, const int* __restrict__ count,
                                     const int* __restrict__ dst, float* __restrict__ out, int t_max) {
+  SF_PDL_ENTRY();
   const int s = blockIdx.y;
   const int t = blockIdx.x * blockDim.x + threadIdx.x;
   if (t >= t_max) return;
@@ -211,8 +216,8 @@ __global__ void extract_rows_kernel(const float* __restrict__ packed, const SeqT
 cudaError_t launch_extract_rows(const float* packed, const SeqTable* seq, const int* d_first, const int* d_count,
                                 const int* d_dst, int n_seq, float* out, int t_max, cudaStream_t st) {
   if (n_seq <= 0 || t_max <= 0) return cudaSuccess;
-  extract_rows_kernel<<<dim3((t_max + 127) / 128, n_seq), 128, 0, st>>>(packed, seq, d_first, d_count, d_dst, out,
-                                                                         t_max);
+  CK_LAUNCH(launch_k(extract_rows_kernel, dim3(dim3((t_max + 127) / 128, n_seq)), dim3(128), 0, st, packed, seq, d_first, d_count, d_dst, out,
+                                                                         t_max));
   return cudaGetLastError();
 }
 

@@ -21,6 +21,7 @@ template <typename T>
 __global__ void __launch_bounds__(128) assemble_kernel(float* __restrict__ x, const SeqTable* __restrict__ seq,
                                                        const StepDesc* __restrict__ sd, StateBufs sb,
                                                        const T* __restrict__ emb, int emb_stride) {
+  SF_PDL_ENTRY();
   const int r = blockIdx.x;
   const int D = sb.D;
   const int i = seq_of_row(seq, r);
@@ -41,7 +42,7 @@ template <typename T>
 cudaError_t launch_assemble(float* x, const SeqTable* seq, const StepDesc* sd, const StateBufs& sb, const T* emb,
                             int emb_stride, int M, cudaStream_t st) {
   if (M <= 0) return cudaSuccess;
-  assemble_kernel<T><<<M, 128, 0, st>>>(x, seq, sd, sb, emb, emb_stride);
+  CK_LAUNCH(launch_k(assemble_kernel<T>, dim3(M), dim3(128), 0, st, x, seq, sd, sb, emb, emb_stride));
   return cudaGetLastError();
 }
 
@@ -106,6 +107,7 @@ __global__ void __launch_bounds__(256) state_update_kernel(const float* __restri
                                                            const T* __restrict__ emb, int emb_stride,
                                                            float* scores_out, int* src_out,
                                                            const float* scores_in, int score_stride) {
+  SF_PDL_ENTRY();
   __shared__ float sc[CAND_MAX * 4];
   __shared__ int kept[CAND_MAX];
   __shared__ int src[CAND_MAX];
@@ -218,13 +220,14 @@ cudaError_t launch_state_update(const float* probs, const SeqTable* seq, const S
                                 const T* emb, int emb_stride, int n_seq, float* scores_out, int* src_out,
                                 const float* scores_in, int score_stride, cudaStream_t st) {
   if (n_seq <= 0) return cudaSuccess;
-  state_update_kernel<T><<<n_seq, 256, 0, st>>>(probs, seq, sd, sb, emb, emb_stride, scores_out, src_out, scores_in,
-                                                score_stride);
+  CK_LAUNCH(launch_k(state_update_kernel<T>, dim3(n_seq), dim3(256), 0, st, probs, seq, sd, sb, emb, emb_stride, scores_out, src_out, scores_in,
+                                                score_stride));
   return cudaGetLastError();
 }
 
 __global__ void __launch_bounds__(256) select_topk_kernel(const float* __restrict__ scores, const int* __restrict__ n,
                                                           int stride, int k, int* __restrict__ src_out) {
+  SF_PDL_ENTRY();
   __shared__ float sc[CAND_MAX * 4];
   __shared__ int kept[CAND_MAX];
   __shared__ int src[CAND_MAX];
@@ -240,7 +243,7 @@ __global__ void __launch_bounds__(256) select_topk_kernel(const float* __restric
 cudaError_t launch_select_topk(const float* scores, const int* n, int n_sets, int stride, int k, int* src,
                                cudaStream_t st) {
   if (n_sets <= 0) return cudaSuccess;
-  select_topk_kernel<<<n_sets, 256, 0, st>>>(scores, n, stride, k, src);
+  CK_LAUNCH(launch_k(select_topk_kernel, dim3(n_sets), dim3(256), 0, st, scores, n, stride, k, src));
   return cudaGetLastError();
 }
 

@@ -17,6 +17,7 @@ template <typename T>
 __global__ void __launch_bounds__(256) conv1_kernel(const float* __restrict__ feats, int64_t t_buf, PreArgs args,
                                                      const float* __restrict__ w, const float* __restrict__ bias,
                                                      T* __restrict__ out, int T1max) {
+  SF_PDL_ENTRY();
   constexpr int R = 4;                 // output rows per CTA
   __shared__ float patch[2 * R + 1][130];
   const int i = blockIdx.y;
@@ -61,6 +62,7 @@ __global__ void __launch_bounds__(256) dwconv3x3s2_kernel(const T* __restrict__ 
                                                           T* __restrict__ out, int Tout_max, int Fout, PreArgs args,
                                                           int stage, const float* __restrict__ w,
                                                           const float* __restrict__ bias) {
+  SF_PDL_ENTRY();
   const int t = blockIdx.x, i = blockIdx.y, c = threadIdx.x;
   int64_t l = args.frames[i];
   for (int s = 0; s < stage; ++s) l = 1 + (l - 1) / 2;     // valid rows of the input stage
@@ -90,14 +92,14 @@ __global__ void __launch_bounds__(256) dwconv3x3s2_kernel(const T* __restrict__ 
 template <typename T>
 cudaError_t launch_conv1(const float* feats, int64_t t_buf, const PreArgs& a, int n_win, const float* w,
                          const float* b, T* out, int T1max, cudaStream_t st) {
-  conv1_kernel<T><<<dim3((T1max + 3) / 4, n_win), 256, 0, st>>>(feats, t_buf, a, w, b, out, T1max);
+  CK_LAUNCH(launch_k(conv1_kernel<T>, dim3(dim3((T1max + 3) / 4, n_win)), dim3(256), 0, st, feats, t_buf, a, w, b, out, T1max));
   return cudaGetLastError();
 }
 
 template <typename T>
 cudaError_t launch_dwconv3x3s2(const T* in, int Tin_max, int Fin, T* out, int Tout_max, int Fout, const PreArgs& a,
                                int n_win, int stage, const float* w, const float* b, cudaStream_t st) {
-  dwconv3x3s2_kernel<T><<<dim3(Tout_max, n_win), 256, 0, st>>>(in, Tin_max, Fin, out, Tout_max, Fout, a, stage, w, b);
+  CK_LAUNCH(launch_k(dwconv3x3s2_kernel<T>, dim3(dim3(Tout_max, n_win)), dim3(256), 0, st, in, Tin_max, Fin, out, Tout_max, Fout, a, stage, w, b));
   return cudaGetLastError();
 }
 
