@@ -126,7 +126,7 @@ def streaming_bench(b, torch, eng_blob, rank, world, local):
         n = hi - lo
         audio_np, lens, _ = clip_for_config(idx)
         audio_np, lens = np.ascontiguousarray(audio_np[lo:hi]), lens[lo:hi]
-        eng = b.sf_create(eng_blob, b.default_config(max_batch=max(n, 1)))
+        eng = b.sf_create(eng_blob, b.default_config(max_batch=max(n, 1), max_samples=int(audio_np.shape[1])))
         audio = torch.from_numpy(audio_np).cuda()
         T = 1 + audio_np.shape[1] // 160
         mel = torch.empty((n, 128, T), device="cuda")
