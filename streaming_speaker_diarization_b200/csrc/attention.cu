@@ -6,7 +6,9 @@
 // Transformer: plain MHSA, head dim 24.
 //
 // bf16 path (flash-style, mma.sync m16n8k16): one CTA = 64 query rows of one
-// sequence x one head, 4 warps of 16 rows.  Per 64-key tile the warp computes
+// sequence x one head, 8 warps: two groups of 4 warps (16 query rows each)
+// take alternate 64-key tiles and merge their partial softmax state at the
+// end.  Per 64-key tile the warp computes
 // AC = (Q+u) K^T (16 x 64) and, for the relative term, BD = (Q+v) P^T over
 // the 80 relative distances its 16 rows x 64 keys can take; BD goes through
 // a per-warp shared tile and is read back along the i - j diagonal.  Online
@@ -132,9 +134,9 @@ template <int N> __device__ __forceinline__ void cp_async_wait_() {
 // dims >= HD arrive as zeros.
 template <int HD, int HDP, int LDS>
 __device__ __forceinline__ void load_rows_async(bf16* dst, const bf16* src, int64_t ld, int row0, int nrows, int lo,
-                                                int hi) {
+                                                int hi, int tid, int nthr) {
   constexpr int CH = HDP / 8;
-  for (int e = threadIdx.x; e < nrows * CH; e += blockDim.x) {
+  for (int e = tid; e < nrows * CH; e += nthr) {
     const int rr = e / CH, ch = e % CH;
     const int row = row0 + rr;
     const bool ok = row >= lo && row < hi && ch * 8 < HD;
@@ -148,13 +150,16 @@ struct AttCfg {
   static constexpr int LDS = HDP + 8;
   static constexpr int TILE = 64 * LDS;                       // bf16 elements
   static constexpr int NQ = REL ? 2 : 1;
-  // Q (+Qv) once; K, V and the 128-row relative slice double-buffered
+  // Q (+Qv) once; per warp group, K, V and the 128-row relative slice
+  // double-buffered; per warp a 16 x 80 fp32 tile of relative scores
   static constexpr int BUF = 2 * TILE + (REL ? 2 * TILE : 0);
-  static constexpr int SMEM = (NQ * TILE + 2 * BUF) * 2 + (REL ? 4 * 16 * 80 * 4 : 0);
+  static constexpr int SMEM = (NQ * TILE + 2 * 2 * BUF) * 2 + (REL ? 8 * 16 * 80 * 4 : 0);
+  static constexpr int MERGE_FLOATS = 128 * (4 + 4 * (HDP / 8));   // group 1's (m, l, O) handed to group 0
+  static_assert(MERGE_FLOATS * 4 <= 2 * BUF * 2, "merge area fits in one group's buffers");
 };
 
 template <int HD, int HDP, bool REL>
-__global__ void __launch_bounds__(128) attn_bf16_kernel(const bf16* __restrict__ qkv, int D,
+__global__ void __launch_bounds__(256) attn_bf16_kernel(const bf16* __restrict__ qkv, int D,
                                                         const bf16* __restrict__ ptab, int R,
                                                         const float* __restrict__ u, const float* __restrict__ vb,
                                                         bf16* __restrict__ ctx, const SeqTable* __restrict__ seq) {
@@ -164,14 +169,17 @@ __global__ void __launch_bounds__(128) attn_bf16_kernel(const bf16* __restrict__
   extern __shared__ float4 att_smem4[];
   bf16* sQu = reinterpret_cast<bf16*>(att_smem4);
   bf16* sQv = sQu + (REL ? C::TILE : 0);
-  bf16* sBuf = sQu + C::NQ * C::TILE;                         // 2 x [K | V | P(128 rows, REL)]
-  float* sBD = reinterpret_cast<float*>(sBuf + 2 * C::BUF);
+  bf16* sBuf0 = sQu + C::NQ * C::TILE;                        // per group: 2 x [K | V | P(128 rows, REL)]
+  float* sBD = reinterpret_cast<float*>(sBuf0 + 2 * 2 * C::BUF);
 
   const int g_tile = blockIdx.x, h = blockIdx.y;
   const int s = seq_of_tile(seq, g_tile);
   const int sb = seq->off[s], S = seq->off[s + 1] - sb;
   const int i0 = (g_tile - seq->tile_off[s]) * 64;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int grp = warp >> 2, wq = warp & 3;     // key-tile group, 16-row query slice
+  const int gtid = threadIdx.x & 127;
+  bf16* sBuf = sBuf0 + grp * 2 * C::BUF;
   const int g = lane >> 2, q = lane & 3;
   const int64_t ld = 3 * D;
   const bf16* Qg = qkv + (int64_t)sb * ld + h * HD;
@@ -185,7 +193,7 @@ __global__ void __launch_bounds__(128) attn_bf16_kernel(const bf16* __restrict__
   uint32_t aqu[KS][4], aqv[REL ? KS : 1][4];
 #pragma unroll
   for (int ks = 0; ks < KS; ++ks) {
-    const int row = warp * 16 + (lane & 15), col = ks * 16 + (lane >> 4) * 8;
+    const int row = wq * 16 + (lane & 15), col = ks * 16 + (lane >> 4) * 8;
     ldsm4(s_u32(sQu + row * LDS + col), aqu[ks]);
     if (REL) ldsm4(s_u32(sQv + row * LDS + col), aqv[ks]);
   }
@@ -197,21 +205,28 @@ __global__ void __launch_bounds__(128) attn_bf16_kernel(const bf16* __restrict__
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
   const float sl2 = 1.4426950408889634f / sqrtf((float)HD);
 
+  // group `grp` takes key tiles grp, grp + 2, ...; each group double-buffers its own tiles
   auto prefetch = [&](int j0, int buf) {
     bf16* k_ = sBuf + buf * C::BUF;
-    load_rows_async<HD, HDP, LDS>(k_, Kg, ld, j0, 64, 0, S);
-    load_rows_async<HD, HDP, LDS>(k_ + C::TILE, Vg, ld, j0, 64, 0, S);
-    if (REL) load_rows_async<HD, HDP, LDS>(k_ + 2 * C::TILE, ptab + h * HD, D, i0 - j0 - 63 + R - 1, 128, 0, 2 * R - 1);
+    load_rows_async<HD, HDP, LDS>(k_, Kg, ld, j0, 64, 0, S, gtid, 128);
+    load_rows_async<HD, HDP, LDS>(k_ + C::TILE, Vg, ld, j0, 64, 0, S, gtid, 128);
+    if (REL)
+      load_rows_async<HD, HDP, LDS>(k_ + 2 * C::TILE, ptab + h * HD, D, i0 - j0 - 63 + R - 1, 128, 0, 2 * R - 1,
+                                    gtid, 128);
     cp_async_commit_();
   };
-  prefetch(0, 0);
-  for (int j0 = 0, it = 0; j0 < S; j0 += 64, ++it) {
-    // tile it+1 streams in while tile it is used
-    if (j0 + 64 < S) prefetch(j0 + 64, (it + 1) & 1);
+  auto group_sync = [&]() { asm volatile("bar.sync %0, 128;" ::"r"(1 + grp) : "memory"); };
+  if (grp * 64 < S) prefetch(grp * 64, 0);
+  else cp_async_commit_();
+  for (int k = 0;; ++k) {
+    const int j0 = (grp + 2 * k) * 64;
+    if (j0 >= S) break;
+    // tile k+1 of this group streams in while tile k is used
+    if (j0 + 128 < S) prefetch(j0 + 128, (k + 1) & 1);
     else cp_async_commit_();
     cp_async_wait_<1>();
-    __syncthreads();
-    const bf16* sK = sBuf + (it & 1) * C::BUF;
+    group_sync();
+    const bf16* sK = sBuf + (k & 1) * C::BUF;
     const bf16* sV = sK + C::TILE;
     const bf16* sP = sK + 2 * C::TILE;
     float sc[8][4];
@@ -237,7 +252,7 @@ __global__ void __launch_bounds__(128) attn_bf16_kernel(const bf16* __restrict__
 #pragma unroll
         for (int np = 0; np < 5; ++np) {
           uint32_t b[4];
-          const int nrow = warp * 16 + np * 16 + (lane & 7) + ((lane >> 4) << 3);
+          const int nrow = wq * 16 + np * 16 + (lane & 7) + ((lane >> 4) << 3);
           const int col = ks * 16 + ((lane >> 3) & 1) * 8;
           ldsm4(s_u32(sP + nrow * LDS + col), b);
           mma16816(bd[2 * np], aqv[ks], b[0], b[1]);
@@ -316,15 +331,42 @@ __global__ void __launch_bounds__(128) attn_bf16_kernel(const bf16* __restrict__
         mma16816(o[2 * np + 1], a, b[2], b[3]);
       }
     }
-    __syncthreads();   // everyone is done with this buffer before it is refilled
+    group_sync();   // the whole group is done with this buffer before it is refilled
   }
   cp_async_wait_<0>();
   l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
   l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
   l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
   l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+  // group 1 hands its running max, sum and unnormalised output to group 0
+  // (same query rows, same lane layout) through its own, now idle, buffers
+  float* mg = reinterpret_cast<float*>(sBuf0 + 2 * C::BUF) + gtid * (4 + 4 * NO);
+  __syncthreads();
+  if (grp == 1) {
+    mg[0] = m0; mg[1] = m1; mg[2] = l0; mg[3] = l1;
+#pragma unroll
+    for (int n = 0; n < NO; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) mg[4 + 4 * n + e] = o[n][e];
+  }
+  __syncthreads();
+  if (grp == 1) return;
+  {
+    const float mb0 = mg[0], mb1 = mg[1], lb0 = mg[2], lb1 = mg[3];
+    const float n0 = fmaxf(m0, mb0), n1 = fmaxf(m1, mb1);   // m0/m1 are finite: group 0 saw key 0
+    const float ca0 = exp2f(m0 - n0), cb0 = exp2f(mb0 - n0), ca1 = exp2f(m1 - n1), cb1 = exp2f(mb1 - n1);
+    l0 = l0 * ca0 + lb0 * cb0;
+    l1 = l1 * ca1 + lb1 * cb1;
+#pragma unroll
+    for (int n = 0; n < NO; ++n) {
+      o[n][0] = o[n][0] * ca0 + mg[4 + 4 * n + 0] * cb0;
+      o[n][1] = o[n][1] * ca0 + mg[4 + 4 * n + 1] * cb0;
+      o[n][2] = o[n][2] * ca1 + mg[4 + 4 * n + 2] * cb1;
+      o[n][3] = o[n][3] * ca1 + mg[4 + 4 * n + 3] * cb1;
+    }
+  }
   const float inv0 = 1.f / l0, inv1 = 1.f / l1;
-  const int r0 = i0 + warp * 16 + g, r1 = r0 + 8;
+  const int r0 = i0 + wq * 16 + g, r1 = r0 + 8;
 #pragma unroll
   for (int n = 0; n < NO; ++n) {
     const int d = n * 8 + 2 * q;
@@ -356,7 +398,7 @@ template <>
 cudaError_t launch_relpos_attention<bf16>(const bf16* qkv, const bf16* ptab, int R, const float* u, const float* v,
                                           bf16* ctx, const SeqTable* seq, int n_tiles, int M, cudaStream_t st) {
   if (M <= 0) return cudaSuccess;
-  CK_LAUNCH(launch_k(attn_bf16_kernel<64, 64, true>, dim3(dim3(n_tiles, 8)), dim3(128), AttCfg<64, 64, true>::SMEM, st, qkv, 512, ptab, R, u, v,
+  CK_LAUNCH(launch_k(attn_bf16_kernel<64, 64, true>, dim3(dim3(n_tiles, 8)), dim3(256), AttCfg<64, 64, true>::SMEM, st, qkv, 512, ptab, R, u, v,
                                                                                              ctx, seq));
   return cudaGetLastError();
 }
@@ -374,7 +416,7 @@ cudaError_t launch_mha<float>(const float* qkv, float* ctx, const SeqTable* seq,
 template <>
 cudaError_t launch_mha<bf16>(const bf16* qkv, bf16* ctx, const SeqTable* seq, int n_tiles, int M, cudaStream_t st) {
   if (M <= 0) return cudaSuccess;
-  CK_LAUNCH(launch_k(attn_bf16_kernel<24, 32, false>, dim3(dim3(n_tiles, 8)), dim3(128), AttCfg<24, 32, false>::SMEM, st, 
+  CK_LAUNCH(launch_k(attn_bf16_kernel<24, 32, false>, dim3(dim3(n_tiles, 8)), dim3(256), AttCfg<24, 32, false>::SMEM, st, 
       qkv, 192, nullptr, 0, nullptr, nullptr, ctx, seq));
   return cudaGetLastError();
 }
