@@ -124,10 +124,10 @@ struct TcCfg {
 // With split-K the raw partial tile goes to `part` instead.
 template <int EK, int BN>
 __device__ __forceinline__ void epilogue_tile(const Epi& e, uint32_t tmem, float* stage, float* part, int M, int N,
-                                              int m0, int n0, int q, int lane, int S) {
+                                              int m0, int n0, int q, int lane, int S, int cbeg = 0, int cend = BN) {
   const int l4 = lane & 15, rh = lane >> 4;
 #pragma unroll 1
-  for (int c0 = 0; c0 < BN; c0 += 64) {
+  for (int c0 = cbeg; c0 < cend; c0 += 64) {
     uint32_t v[16];
 #pragma unroll
     for (int h = 0; h < 4; ++h) {
@@ -351,6 +351,166 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
   if (threadIdx.x == 0 && *abort_flag) set_err(err, ERR_TIMEOUT);
 }
 
+__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su32(b)) : "memory");
+}
+
+// Persistent variant for GEMMs with more tiles than SMs: each CTA walks the
+// tiles blockIdx.x, blockIdx.x + gridDim.x, ... (n fastest, so co-running CTAs
+// share A rows in L2).  Two TMEM accumulators of BN columns alternate between
+// tiles, so the epilogue of tile i overlaps the mainloop of tile i + 1; the
+// producer's ring of stages runs on across tiles.  Warps: 0 TMA producer,
+// 1 MMA issuer, 2-9 epilogue (two warps per TMEM lane quarter, each draining
+// half of the columns).  acc_full[a] is committed by the MMA thread;
+// acc_empty[a] collects one arrival per epilogue warp.
+template <int BN, int STAGES>
+struct TcpCfg {
+  static constexpr int A_BYTES = TC_BM * TC_BK * 2;
+  static constexpr int B_BYTES = BN * TC_BK * 2;
+  static constexpr int STAGE_FLOATS = 8 * 32 * 68;
+  static constexpr int SMEM = 1024 + STAGES * (A_BYTES + B_BYTES) + STAGE_FLOATS * 4 + 256;
+  static_assert(SMEM <= 232448, "shared memory per CTA");
+};
+
+template <int BN, int STAGES>
+__global__ void __launch_bounds__(320, 1) gemm_tcp_kernel(const __grid_constant__ CUtensorMap ta,
+                                                          const __grid_constant__ CUtensorMap tb, int M, int N, int K,
+                                                          Epi e, int* err) {
+  using C = TcpCfg<BN, STAGES>;
+  extern __shared__ uint8_t tc_smem[];
+  uint8_t* sm = tc_smem + ((1024 - (su32(tc_smem) & 1023)) & 1023);
+  uint8_t* sA = sm;
+  uint8_t* sB = sm + STAGES * C::A_BYTES;
+  float* stg = reinterpret_cast<float*>(sB + STAGES * C::B_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(stg + C::STAGE_FLOATS);
+  uint64_t* empty = full + STAGES;
+  uint64_t* accf = empty + STAGES;     // [2]
+  uint64_t* acce = accf + 2;           // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tiles_n = (N + BN - 1) / BN;
+  const int tiles = ((M + TC_BM - 1) / TC_BM) * tiles_n;
+  const int KB = (K + TC_BK - 1) / TC_BK;
+
+  if (threadIdx.x == 0) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&ta)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tb)) : "memory");
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&accf[a], 1);
+      mbar_init(&acce[a], 8);
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(tmem_slot)),
+                 "r"((uint32_t)(2 * BN))
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  SF_PDL_ENTRY();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int it = 0;
+      for (int tile = blockIdx.x; tile < tiles && !*abort_flag; tile += gridDim.x) {
+        const int m0 = (tile / tiles_n) * TC_BM, n0 = (tile % tiles_n) * BN;
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % STAGES, r = it / STAGES;
+          if (!mbar_wait(&empty[s], (r & 1) ^ 1, abort_flag)) {
+            *abort_flag = 1;
+            break;
+          }
+          mbar_expect_tx(&full[s], C::A_BYTES + C::B_BYTES);
+          tma_load_2d(sA + s * C::A_BYTES, &ta, &full[s], kb * TC_BK, m0);
+          tma_load_2d(sB + s * C::B_BYTES, &tb, &full[s], kb * TC_BK, n0);
+        }
+      }
+      if (*abort_flag) {   // let this CTA's own loads land before the shared memory is released
+        for (int k = it - STAGES > 0 ? it - STAGES : 0; k < it; ++k) {
+          const long long t0 = clock64();
+          while (!mbar_try_wait(&full[k % STAGES], (k / STAGES) & 1) && clock64() - t0 < WAIT_CYCLES) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(BN);
+      int it = 0, i = 0;
+      for (int tile = blockIdx.x; tile < tiles && !*abort_flag; tile += gridDim.x, ++i) {
+        const int a = i & 1, u = i >> 1;
+        if (!mbar_wait(&acce[a], (u & 1) ^ 1, abort_flag)) {
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t acc = tmem + (uint32_t)(a * BN);
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % STAGES, r = it / STAGES;
+          if (!mbar_wait(&full[s], r & 1, abort_flag)) {
+            *abort_flag = 1;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t ad = sw128_desc(su32(sA + s * C::A_BYTES));
+          const uint64_t bd = sw128_desc(su32(sB + s * C::B_BYTES));
+#pragma unroll
+          for (int k = 0; k < TC_BK / 16; ++k)
+            umma_bf16(acc, ad + (uint64_t)(2 * k), bd + (uint64_t)(2 * k), idesc, (kb | k) != 0);
+          umma_commit(&empty[s]);
+        }
+        umma_commit(&accf[a]);
+      }
+    }
+  } else {
+    const int q = warp & 3, hc = (warp - 2) >> 2;   // TMEM lane quarter, column half
+    float* stage = stg + (warp - 2) * (32 * 68);
+    int i = 0;
+    for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++i) {
+      const int a = i & 1, u = i >> 1;
+      if (!mbar_wait(&accf[a], u & 1, abort_flag) || *abort_flag) {
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const int m0 = (tile / tiles_n) * TC_BM, n0 = (tile % tiles_n) * BN;
+      const uint32_t acc = tmem + (uint32_t)(a * BN);
+      switch (e.kind) {
+        case EPI_BIAS: epilogue_tile<EPI_BIAS, BN>(e, acc, stage, nullptr, M, N, m0, n0, q, lane, 1, hc * BN / 2, (hc + 1) * BN / 2); break;
+        case EPI_BIAS_RELU: epilogue_tile<EPI_BIAS_RELU, BN>(e, acc, stage, nullptr, M, N, m0, n0, q, lane, 1, hc * BN / 2, (hc + 1) * BN / 2); break;
+        case EPI_BIAS_SWISH: epilogue_tile<EPI_BIAS_SWISH, BN>(e, acc, stage, nullptr, M, N, m0, n0, q, lane, 1, hc * BN / 2, (hc + 1) * BN / 2); break;
+        case EPI_BIAS_GLU: epilogue_tile<EPI_BIAS_GLU, BN>(e, acc, stage, nullptr, M, N, m0, n0, q, lane, 1, hc * BN / 2, (hc + 1) * BN / 2); break;
+        case EPI_RESID: epilogue_tile<EPI_RESID, BN>(e, acc, stage, nullptr, M, N, m0, n0, q, lane, 1, hc * BN / 2, (hc + 1) * BN / 2); break;
+        case EPI_F32: epilogue_tile<EPI_F32, BN>(e, acc, stage, nullptr, M, N, m0, n0, q, lane, 1, hc * BN / 2, (hc + 1) * BN / 2); break;
+        default: epilogue_tile<EPI_F32_AND_T, BN>(e, acc, stage, nullptr, M, N, m0, n0, q, lane, 1, hc * BN / 2, (hc + 1) * BN / 2); break;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acce[a]);   // this warp is done reading accumulator a
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"((uint32_t)(2 * BN))
+                 : "memory");
+  }
+  if (threadIdx.x == 0 && *abort_flag) set_err(err, ERR_TIMEOUT);
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 cudaError_t get_encoder() {
@@ -388,6 +548,23 @@ cudaError_t launch_tc(const bf16* A, int lda, const bf16* W, int M, int N, int K
   if (r != cudaSuccess) return r;
   dim3 grid((N + BN - 1) / BN, (M + TC_BM - 1) / TC_BM, splits);
   CK_LAUNCH(launch_k(gemm_tc_kernel<BN, STAGES>, dim3(grid), dim3(192), TcCfg<BN, STAGES>::SMEM, st, ta, tb, M, N, K, e, sc.err, sc.ws, sc.cnt));
+  return cudaGetLastError();
+}
+
+int g_num_sms = 148;
+
+template <int BN, int STAGES>
+cudaError_t launch_tcp(const bf16* A, int lda, const bf16* W, int M, int N, int K, const Epi& e, const TcScratch& sc,
+                       cudaStream_t st) {
+  CUtensorMap ta, tb;
+  cudaError_t r = make_map(&ta, A, M, K, lda, TC_BM);
+  if (r != cudaSuccess) return r;
+  r = make_map(&tb, W, N, K, K, BN);
+  if (r != cudaSuccess) return r;
+  const int tiles = ((M + TC_BM - 1) / TC_BM) * ((N + BN - 1) / BN);
+  const int grid = tiles < g_num_sms ? tiles : g_num_sms;
+  CK_LAUNCH(launch_k(gemm_tcp_kernel<BN, STAGES>, dim3(grid), dim3(320), TcpCfg<BN, STAGES>::SMEM, st, ta, tb, M, N, K,
+                     e, sc.err));
   return cudaGetLastError();
 }
 
@@ -433,6 +610,12 @@ cudaError_t gemm_bf16_tc(const bf16* A, int lda, const bf16* W, int M, int N, in
   if (r != cudaSuccess) return r;
   int bn, sp;
   gemm_tc_plan(M, N, K, sc, &bn, &sp);
+  // more tiles than SMs: the persistent kernel overlaps each tile's epilogue
+  // with the next tile's mainloop
+  if (sp == 1 && N >= 128 && ((M + TC_BM - 1) / TC_BM) * ((N + bn - 1) / bn) > g_num_sms) {
+    if (N >= 256) return launch_tcp<256, 3>(A, lda, W, M, N, K, e, sc, st);
+    return launch_tcp<128, 4>(A, lda, W, M, N, K, e, sc, st);
+  }
   switch (bn) {
     case 256: return launch_tc<256, 4>(A, lda, W, M, N, K, sp, e, sc, st);
     case 128: return launch_tc<128, 6>(A, lda, W, M, N, K, sp, e, sc, st);
@@ -442,6 +625,14 @@ cudaError_t gemm_bf16_tc(const bf16* A, int lda, const bf16* W, int M, int N, in
 
 cudaError_t gemm_tc_init_attributes() {
   cudaError_t r = get_encoder();
+  if (r != cudaSuccess) return r;
+  int dev = 0, n_sm = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) ==
+                                                 cudaSuccess && n_sm > 0)
+    g_num_sms = n_sm;
+  r = cudaFuncSetAttribute(gemm_tcp_kernel<256, 3>, cudaFuncAttributeMaxDynamicSharedMemorySize, TcpCfg<256, 3>::SMEM);
+  if (r == cudaSuccess)
+    r = cudaFuncSetAttribute(gemm_tcp_kernel<128, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, TcpCfg<128, 4>::SMEM);
   if (r != cudaSuccess) return r;
   r = cudaFuncSetAttribute(gemm_tc_kernel<256, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        TcCfg<256, 4>::SMEM);

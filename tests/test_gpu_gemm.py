@@ -24,7 +24,9 @@ def eng():
 # every tile width and split-K counts 1..8 (e.g. (300, 64, 4096): 3 tiles -> 8 splits)
 SHAPES = [(1125, 2048, 512), (1125, 512, 2048), (1125, 1536, 512), (1125, 192, 192), (1125, 576, 192),
           (1125, 192, 768), (1125, 512, 4096), (1, 64, 64), (333, 768, 192), (128, 128, 128), (129, 256, 4096),
-          (24896, 1024, 512), (70, 16, 64), (300, 64, 4096), (2000, 256, 1024)]
+          (24896, 1024, 512), (70, 16, 64), (300, 64, 4096), (2000, 256, 1024),
+          # more tiles than SMs: persistent kernel, BN 256 / 128, ragged M and N tails
+          (20000, 192, 256), (19001, 256, 512), (50000, 576, 192), (72000, 256, 256)]
 
 
 @pytest.mark.parametrize("M,N,K", SHAPES)
