@@ -76,16 +76,13 @@ __device__ __forceinline__ void set_err(int* err, int bit) {
   if (err) atomicOr(err, bit);
 }
 
-// Programmatic dependent launch: every kernel waits for its predecessor's
-// memory before its first global access, then lets its successor launch (the
-// successor's prologue overlaps this kernel; at most two grids are in flight).
+// Programmatic dependent launch (when enabled): every kernel waits for its
+// predecessor's memory before its first global access.  The GEMMs let their
+// successor launch once their last MMA is issued, so the successor's launch
+// and set-up overlap the epilogue; other kernels release it when they exit.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-#define SF_PDL_ENTRY() \
-  do {                 \
-    sf::pdl_wait();    \
-    sf::pdl_trigger(); \
-  } while (0)
+#define SF_PDL_ENTRY() sf::pdl_wait()
 
 #define CK_LAUNCH(x)                  \
   do {                                \

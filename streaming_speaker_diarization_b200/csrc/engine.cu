@@ -787,28 +787,33 @@ cudaError_t run_encode(sf_engine* e, int M, int n_tiles, float* probs, cudaStrea
   T* ctx = static_cast<T*>(e->ctx.p);
   for (int l = 0; l < c.n_conformer; ++l) {
     const ConfW<T>& w = W.conf[l];
-    RUN(K_LN, 1, 0, (double)M * D * (4 + sizeof(T) + (false ? 4 : 0)),
-        launch_layernorm<T>(x, w.ff1_g, w.ff1_b, M, D, false, h, st));
+    if (l == 0)   // later layers get this LN fused into the previous layer's final LN
+      RUN(K_LN, 1, 0, (double)M * D * (4 + sizeof(T)), launch_layernorm<T>(x, w.ff1_g, w.ff1_b, M, D, false, h, st));
     CK(gemm_acc<T>(e, h, D, w.ff1_w1, M, DFF, D, epi(EPI_BIAS_SWISH, w.ff1_b1, big, DFF), st));
     CK(gemm_acc<T>(e, big, DFF, w.ff1_w2, M, D, DFF, epi(EPI_RESID, w.ff1_b2, x, D, 0.5f), st));
-    RUN(K_LN, 1, 0, (double)M * D * (4 + sizeof(T) + (false ? 4 : 0)),
+    RUN(K_LN, 1, 0, (double)M * D * (4 + sizeof(T)),
         launch_layernorm<T>(x, w.att_g, w.att_b, M, D, false, h, st));
     CK(gemm_acc<T>(e, h, D, w.wqkv, M, 3 * D, D, epi(EPI_BIAS, w.bqkv, big, 3 * D), st));
     RUN(K_ATT_REL, 1, 6.0 * e->att_s2 * D, (double)M * 4 * D * sizeof(T),
         launch_relpos_attention<T>(big, w.ptab, e->R, w.pu, w.pv, ctx, seq, n_tiles, M, st));
     CK(gemm_acc<T>(e, ctx, D, w.wo, M, D, D, epi(EPI_RESID, w.bo, x, D, 1.f), st));
-    RUN(K_LN, 1, 0, (double)M * D * (4 + sizeof(T) + (false ? 4 : 0)),
+    RUN(K_LN, 1, 0, (double)M * D * (4 + sizeof(T)),
         launch_layernorm<T>(x, w.conv_g, w.conv_b, M, D, false, h, st));
     CK(gemm_acc<T>(e, h, D, w.pw1, M, 2 * D, D, epi(EPI_BIAS_GLU, w.pw1_b, ctx, D), st));
     RUN(K_DW1D, 1, 2.0 * M * D * c.conv_kernel, (double)M * D * 2 * sizeof(T),
         launch_dwconv1d<T>(ctx, h, w.dw_w, w.dw_b, M, D, c.conv_kernel, seq, st));
     CK(gemm_acc<T>(e, h, D, w.pw2, M, D, D, epi(EPI_RESID, w.pw2_b, x, D, 1.f), st));
-    RUN(K_LN, 1, 0, (double)M * D * (4 + sizeof(T) + (false ? 4 : 0)),
+    RUN(K_LN, 1, 0, (double)M * D * (4 + sizeof(T)),
         launch_layernorm<T>(x, w.ff2_g, w.ff2_b, M, D, false, h, st));
     CK(gemm_acc<T>(e, h, D, w.ff2_w1, M, DFF, D, epi(EPI_BIAS_SWISH, w.ff2_b1, big, DFF), st));
     CK(gemm_acc<T>(e, big, DFF, w.ff2_w2, M, D, DFF, epi(EPI_RESID, w.ff2_b2, x, D, 0.5f), st));
-    RUN(K_LN, 1, 0, (double)M * D * (4 + sizeof(T) + (true ? 4 : 0)),
-        launch_layernorm<T>(x, w.out_g, w.out_b, M, D, true, h, st));
+    if (l + 1 < c.n_conformer) {   // layer-final LN, then the next layer's FFN1 LN, in one pass
+      const ConfW<T>& wn = W.conf[l + 1];
+      RUN(K_LN, 1, 0, (double)M * D * (4 + 4 + sizeof(T)),
+          launch_layernorm<T>(x, w.out_g, w.out_b, M, D, true, h, st, wn.ff1_g, wn.ff1_b));
+    } else {
+      RUN(K_LN, 1, 0, (double)M * D * (4 + 4 + sizeof(T)), launch_layernorm<T>(x, w.out_g, w.out_b, M, D, true, h, st));
+    }
   }
   float* x2 = static_cast<float*>(e->x2.p);
   T* h2 = static_cast<T*>(e->h2.p);

@@ -291,6 +291,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
         umma_commit(&empty[s]);
       }
       umma_commit(accf);   // arrives once every MMA issued above has completed
+      pdl_trigger();
     }
   } else {
     // Epilogue: per 64-column chunk, each warp copies its 32 x 64 accumulator
@@ -473,6 +474,7 @@ __global__ void __launch_bounds__(320, 1) gemm_tcp_kernel(const __grid_constant_
         }
         umma_commit(&accf[a]);
       }
+      pdl_trigger();
     }
   } else {
     const int q = warp & 3, hc = (warp - 2) >> 2;   // TMEM lane quarter, column half

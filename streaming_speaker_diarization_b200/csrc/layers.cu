@@ -7,10 +7,14 @@
 namespace sf {
 
 // One warp per row; lane j holds VEC-wide vectors j, j + 32, ... (coalesced).
+// With g2/b2 set, a second LayerNorm follows on the first one's output (the
+// conformer's layer-final LN and the next layer's first LN): x gets LN1(x),
+// h gets LN2(LN1(x)).
 template <typename T, int D, int VEC>
 __global__ void __launch_bounds__(256) layernorm_kernel(float* __restrict__ x, const float* __restrict__ g,
                                                         const float* __restrict__ b, int M, bool write_x,
-                                                        T* __restrict__ h) {
+                                                        T* __restrict__ h, const float* __restrict__ g2,
+                                                        const float* __restrict__ b2) {
   SF_PDL_ENTRY();
   constexpr int NV = D / (32 * VEC);
   const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
@@ -39,6 +43,36 @@ __global__ void __launch_bounds__(256) layernorm_kernel(float* __restrict__ x, c
 #pragma unroll
     for (int k = 0; k < VEC; ++k) { const float d = v[j][k] - mean; q = fmaf(d, d, q); }
   const float inv = 1.0f / sqrtf(warp_sum(q) * (1.0f / D) + 1e-5f);
+  if (g2) {   // x <- LN1(x) kept in registers, then the statistics of LN2 over it
+    float s2 = 0.f;
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+      const int c = (lane + 32 * j) * VEC;
+#pragma unroll
+      for (int k = 0; k < VEC; ++k) {
+        v[j][k] = (v[j][k] - mean) * inv * g[c + k] + b[c + k];
+        s2 += v[j][k];
+      }
+      if (VEC == 4)
+        *reinterpret_cast<float4*>(xr + c) = make_float4(v[j][0], v[j][1 % VEC], v[j][2 % VEC], v[j][3 % VEC]);
+      else
+        *reinterpret_cast<float2*>(xr + c) = make_float2(v[j][0], v[j][1 % VEC]);
+    }
+    const float mean2 = warp_sum(s2) * (1.0f / D);
+    float q2 = 0.f;
+#pragma unroll
+    for (int j = 0; j < NV; ++j)
+#pragma unroll
+      for (int k = 0; k < VEC; ++k) { const float dd = v[j][k] - mean2; q2 = fmaf(dd, dd, q2); }
+    const float inv2 = 1.0f / sqrtf(warp_sum(q2) * (1.0f / D) + 1e-5f);
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+      const int c = (lane + 32 * j) * VEC;
+#pragma unroll
+      for (int k = 0; k < VEC; ++k) h[(int64_t)row * D + c + k] = from_f<T>((v[j][k] - mean2) * inv2 * g2[c + k] + b2[c + k]);
+    }
+    return;
+  }
 #pragma unroll
   for (int j = 0; j < NV; ++j) {
     const int c = (lane + 32 * j) * VEC;
@@ -58,11 +92,14 @@ __global__ void __launch_bounds__(256) layernorm_kernel(float* __restrict__ x, c
 
 template <typename T>
 cudaError_t launch_layernorm(float* x, const float* g, const float* b, int M, int D, bool write_x, T* h,
-                             cudaStream_t st) {
+                             cudaStream_t st, const float* g2, const float* b2) {
   if (M <= 0) return cudaSuccess;
+  if (g2 && (!h || !b2)) return cudaErrorInvalidValue;
   const int grid = (M + 7) / 8;
-  if (D == 512) CK_LAUNCH(launch_k(layernorm_kernel<T, 512, 4>, dim3(grid), dim3(256), 0, st, x, g, b, M, write_x, h));
-  else if (D == 192) CK_LAUNCH(launch_k(layernorm_kernel<T, 192, 2>, dim3(grid), dim3(256), 0, st, x, g, b, M, write_x, h));
+  if (D == 512)
+    CK_LAUNCH(launch_k(layernorm_kernel<T, 512, 4>, dim3(grid), dim3(256), 0, st, x, g, b, M, write_x, h, g2, b2));
+  else if (D == 192)
+    CK_LAUNCH(launch_k(layernorm_kernel<T, 192, 2>, dim3(grid), dim3(256), 0, st, x, g, b, M, write_x, h, g2, b2));
   else return cudaErrorInvalidValue;
   return cudaGetLastError();
 }
@@ -221,8 +258,10 @@ cudaError_t launch_extract_rows(const float* packed, const SeqTable* seq, const 
   return cudaGetLastError();
 }
 
-template cudaError_t launch_layernorm<float>(float*, const float*, const float*, int, int, bool, float*, cudaStream_t);
-template cudaError_t launch_layernorm<bf16>(float*, const float*, const float*, int, int, bool, bf16*, cudaStream_t);
+template cudaError_t launch_layernorm<float>(float*, const float*, const float*, int, int, bool, float*, cudaStream_t,
+                                             const float*, const float*);
+template cudaError_t launch_layernorm<bf16>(float*, const float*, const float*, int, int, bool, bf16*, cudaStream_t,
+                                            const float*, const float*);
 template cudaError_t launch_dwconv1d<float>(const float*, float*, const float*, const float*, int, int, int, const SeqTable*, cudaStream_t);
 template cudaError_t launch_dwconv1d<bf16>(const bf16*, bf16*, const float*, const float*, int, int, int, const SeqTable*, cudaStream_t);
 template cudaError_t launch_head_out<float>(const float*, const float*, const float*, float*, int, int, cudaStream_t);

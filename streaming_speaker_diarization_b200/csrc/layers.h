@@ -66,9 +66,10 @@ cudaError_t launch_dwconv3x3s2(const T* in, int Tin_max, int Fin, T* out, int To
 
 // ------------------------------------------------------- norms / elementwise
 // x (f32, M x D) -> optional in-place LN(x) (f32) and/or h = act(LN(x)).
+// With g2/b2: x <- LN1(x) and h = act(LN2(LN1(x))) in one pass.
 template <typename T>
 cudaError_t launch_layernorm(float* x, const float* g, const float* b, int M, int D, bool write_x, T* h,
-                             cudaStream_t st);
+                             cudaStream_t st, const float* g2 = nullptr, const float* b2 = nullptr);
 // Conformer depthwise conv (k=9, zero padding at sequence edges) with the
 // folded BatchNorm and swish: in/out act (M x D).
 template <typename T>
