@@ -6,6 +6,36 @@
 
 namespace sf {
 
+// VEC consecutive floats at p (VEC = 2 or 4, aligned).
+template <int VEC>
+__device__ __forceinline__ void ld_vec(const float* p, float* v) {
+  if (VEC == 4) {
+    const float4 t = *reinterpret_cast<const float4*>(p);
+    v[0] = t.x; v[1 % VEC] = t.y; v[2 % VEC] = t.z; v[3 % VEC] = t.w;
+  } else {
+    const float2 t = *reinterpret_cast<const float2*>(p);
+    v[0] = t.x; v[1 % VEC] = t.y;
+  }
+}
+template <int VEC>
+__device__ __forceinline__ void st_vec(float* p, const float* v) {
+  if (VEC == 4) *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1 % VEC], v[2 % VEC], v[3 % VEC]);
+  else *reinterpret_cast<float2*>(p) = make_float2(v[0], v[1 % VEC]);
+}
+template <int VEC>
+__device__ __forceinline__ void st_vec(bf16* p, const float* v) {
+  const __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1 % VEC]);
+  if (VEC == 4) {
+    const __nv_bfloat162 c = __floats2bfloat162_rn(v[2 % VEC], v[3 % VEC]);
+    uint2 pk;
+    pk.x = *reinterpret_cast<const uint32_t*>(&a);
+    pk.y = *reinterpret_cast<const uint32_t*>(&c);
+    *reinterpret_cast<uint2*>(p) = pk;
+  } else {
+    *reinterpret_cast<__nv_bfloat162*>(p) = a;
+  }
+}
+
 // One warp per row; lane j holds VEC-wide vectors j, j + 32, ... (coalesced).
 // With g2/b2 set, a second LayerNorm follows on the first one's output (the
 // conformer's layer-final LN and the next layer's first LN): x gets LN1(x),
@@ -21,18 +51,12 @@ __global__ void __launch_bounds__(256) layernorm_kernel(float* __restrict__ x, c
   const int lane = threadIdx.x & 31;
   if (row >= M) return;
   float* xr = x + (int64_t)row * D;
+  T* hr = h ? h + (int64_t)row * D : nullptr;
   float v[NV][VEC];
   float s = 0.f;
 #pragma unroll
   for (int j = 0; j < NV; ++j) {
-    const int c = (lane + 32 * j) * VEC;
-    if (VEC == 4) {
-      const float4 t = *reinterpret_cast<const float4*>(xr + c);
-      v[j][0] = t.x; v[j][1] = t.y; v[j][2 % VEC] = t.z; v[j][3 % VEC] = t.w;
-    } else {
-      const float2 t = *reinterpret_cast<const float2*>(xr + c);
-      v[j][0] = t.x; v[j][1 % VEC] = t.y;
-    }
+    ld_vec<VEC>(xr + (lane + 32 * j) * VEC, v[j]);
 #pragma unroll
     for (int k = 0; k < VEC; ++k) s += v[j][k];
   }
@@ -43,50 +67,39 @@ __global__ void __launch_bounds__(256) layernorm_kernel(float* __restrict__ x, c
 #pragma unroll
     for (int k = 0; k < VEC; ++k) { const float d = v[j][k] - mean; q = fmaf(d, d, q); }
   const float inv = 1.0f / sqrtf(warp_sum(q) * (1.0f / D) + 1e-5f);
-  if (g2) {   // x <- LN1(x) kept in registers, then the statistics of LN2 over it
-    float s2 = 0.f;
-#pragma unroll
-    for (int j = 0; j < NV; ++j) {
-      const int c = (lane + 32 * j) * VEC;
-#pragma unroll
-      for (int k = 0; k < VEC; ++k) {
-        v[j][k] = (v[j][k] - mean) * inv * g[c + k] + b[c + k];
-        s2 += v[j][k];
-      }
-      if (VEC == 4)
-        *reinterpret_cast<float4*>(xr + c) = make_float4(v[j][0], v[j][1 % VEC], v[j][2 % VEC], v[j][3 % VEC]);
-      else
-        *reinterpret_cast<float2*>(xr + c) = make_float2(v[j][0], v[j][1 % VEC]);
-    }
-    const float mean2 = warp_sum(s2) * (1.0f / D);
-    float q2 = 0.f;
-#pragma unroll
-    for (int j = 0; j < NV; ++j)
-#pragma unroll
-      for (int k = 0; k < VEC; ++k) { const float dd = v[j][k] - mean2; q2 = fmaf(dd, dd, q2); }
-    const float inv2 = 1.0f / sqrtf(warp_sum(q2) * (1.0f / D) + 1e-5f);
-#pragma unroll
-    for (int j = 0; j < NV; ++j) {
-      const int c = (lane + 32 * j) * VEC;
-#pragma unroll
-      for (int k = 0; k < VEC; ++k) h[(int64_t)row * D + c + k] = from_f<T>((v[j][k] - mean2) * inv2 * g2[c + k] + b2[c + k]);
-    }
-    return;
-  }
+  float s2 = 0.f;
 #pragma unroll
   for (int j = 0; j < NV; ++j) {
     const int c = (lane + 32 * j) * VEC;
-    float y[VEC];
+    float gg[VEC], bb[VEC];
+    ld_vec<VEC>(g + c, gg);
+    ld_vec<VEC>(b + c, bb);
 #pragma unroll
-    for (int k = 0; k < VEC; ++k) y[k] = (v[j][k] - mean) * inv * g[c + k] + b[c + k];
-    if (write_x) {
-      if (VEC == 4) *reinterpret_cast<float4*>(xr + c) = make_float4(y[0], y[1 % VEC], y[2 % VEC], y[3 % VEC]);
-      else *reinterpret_cast<float2*>(xr + c) = make_float2(y[0], y[1 % VEC]);
+    for (int k = 0; k < VEC; ++k) {
+      v[j][k] = (v[j][k] - mean) * inv * gg[k] + bb[k];
+      s2 += v[j][k];
     }
-    if (h) {
+    if (write_x || g2) st_vec<VEC>(xr + c, v[j]);
+    if (!g2 && hr) st_vec<VEC>(hr + c, v[j]);
+  }
+  if (!g2) return;
+  // x <- LN1(x) (stored above), then LN2 over it into h
+  const float mean2 = warp_sum(s2) * (1.0f / D);
+  float q2 = 0.f;
 #pragma unroll
-      for (int k = 0; k < VEC; ++k) h[(int64_t)row * D + c + k] = from_f<T>(y[k]);
-    }
+  for (int j = 0; j < NV; ++j)
+#pragma unroll
+    for (int k = 0; k < VEC; ++k) { const float dd = v[j][k] - mean2; q2 = fmaf(dd, dd, q2); }
+  const float inv2 = 1.0f / sqrtf(warp_sum(q2) * (1.0f / D) + 1e-5f);
+#pragma unroll
+  for (int j = 0; j < NV; ++j) {
+    const int c = (lane + 32 * j) * VEC;
+    float gg[VEC], bb[VEC], y[VEC];
+    ld_vec<VEC>(g2 + c, gg);
+    ld_vec<VEC>(b2 + c, bb);
+#pragma unroll
+    for (int k = 0; k < VEC; ++k) y[k] = (v[j][k] - mean2) * inv2 * gg[k] + bb[k];
+    st_vec<VEC>(hr + c, y);
   }
 }
 
