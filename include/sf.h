@@ -300,12 +300,16 @@ SF_API sf_status sf_set_option(sf_engine* e, int option, int value);
 SF_API sf_status sf_check(sf_engine* e, void* cuda_stream);
 
 /* The engine's dense projection alone, for tests and kernel benchmarks:
- *   d_C f32 [M x N] (out) = d_A bf16 [M x K] (row stride lda) .
+ *   d_C [M x N] (out) = d_A bf16 [M x K] (row stride lda) .
  *       d_W bf16 [N x K]^T + d_bias f32 [N] (may be NULL)
- * path 1 = tcgen05/TMEM/TMA kernel (the engine's), 0 = mma.sync kernel.
+ * path 1 = tcgen05/TMEM/TMA kernel (the engine's), 0 = mma.sync kernel,
+ * both writing f32 C.  The engine's fused epilogues on the tcgen05 kernel:
+ * path 2 = bf16 C; 3 = residual update, f32 C [M x N] += result; 4 = bf16
+ * C = swish(result); 5 = gated linear unit, bf16 C [M x N/2] with
+ * C[:, j] = r[:, 2j] * sigmoid(r[:, 2j + 1]) (value/gate columns interleaved).
  * Requires N % 16 == 0, K % 64 == 0, lda % 8 == 0, 16-byte aligned A/W. */
 SF_API sf_status sf_gemm_bf16(sf_engine* e, const void* d_A, int lda, const void* d_W, int M, int N, int K,
-                              const float* d_bias, float* d_C, int path, void* cuda_stream);
+                              const float* d_bias, void* d_C, int path, void* cuda_stream);
 
 /* ---------------------------------------------------------------- profiling */
 

@@ -1219,16 +1219,17 @@ sf_status sf_check(sf_engine* e, void* cuda_stream) {
 }
 
 sf_status sf_gemm_bf16(sf_engine* e, const void* d_A, int lda, const void* d_W, int M, int N, int K,
-                       const float* d_bias, float* d_C, int path, void* cuda_stream) {
+                       const float* d_bias, void* d_C, int path, void* cuda_stream) {
   if (check_engine(e) != SF_OK) return SF_EINVAL;
   if (!d_A || !d_W || !d_C) return fail(e, SF_EINVAL, "null pointer argument");
-  if (M < 1 || N < 16 || K < 64 || N % 16 || K % 64 || lda < K || lda % 8 || (path != 0 && path != 1))
-    return fail(e, SF_ESHAPE, "sf_gemm_bf16: M >= 1, N % 16 == 0, K % 64 == 0, lda >= K, lda % 8 == 0, path 0/1");
-  Epi ep = epi(EPI_F32, d_bias, d_C, N);
+  if (M < 1 || N < 16 || K < 64 || N % 16 || K % 64 || lda < K || lda % 8 || path < 0 || path > 5)
+    return fail(e, SF_ESHAPE, "sf_gemm_bf16: M >= 1, N % 16 == 0, K % 64 == 0, lda >= K, lda % 8 == 0, path 0..5");
+  static const int kinds[6] = {EPI_F32, EPI_F32, EPI_BIAS, EPI_RESID, EPI_BIAS_SWISH, EPI_BIAS_GLU};
+  Epi ep = epi(kinds[path], d_bias, d_C, path == 5 ? N / 2 : N);
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
   const bf16* A = static_cast<const bf16*>(d_A);
   const bf16* W = static_cast<const bf16*>(d_W);
-  cudaError_t ce = path == 1 ? gemm_bf16_tc(A, lda, W, M, N, K, ep, e->tc_scratch(), st)
+  cudaError_t ce = path >= 1 ? gemm_bf16_tc(A, lda, W, M, N, K, ep, e->tc_scratch(), st)
                              : gemm_bf16_mma(A, lda, W, M, N, K, ep, st);
   if (ce != cudaSuccess) return cuda_fail(e, ce, "sf_gemm_bf16");
   return SF_OK;

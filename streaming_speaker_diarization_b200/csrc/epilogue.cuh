@@ -52,6 +52,23 @@ __device__ __forceinline__ void epi_store2(const Epi& e, int r, int c, float v0,
   }
 }
 
+// Logistic sigmoid for an output of type T.  A bf16 output keeps 8
+// significant bits, so the hardware exp2 approximation and an approximate
+// reciprocal (relative error ~1e-7 each) are far inside its rounding; an
+// f32 output takes expf and an IEEE division.  Large negative x gives
+// exp(-x) = inf and a sigmoid of exactly 0.
+template <typename T>
+__device__ __forceinline__ float sigm(float x) {
+  if (sizeof(T) == 2) return __fdividef(1.f, 1.f + __expf(-x));
+  return 1.f / (1.f + expf(-x));
+}
+
+// Pointer to element (r, c) of an f32 output with the row remap applied.
+__device__ __forceinline__ float* epi_f32_ptr(const Epi& e, int r, int c) {
+  const int64_t orow = e.rpg ? (int64_t)(r / e.rpg) * e.gstride + (r % e.rpg) : (int64_t)r;
+  return reinterpret_cast<float*>(e.out) + orow * e.ldo + c;
+}
+
 // Four consecutive columns c .. c + 3 of row r (c % 4 == 0, c + 3 < N),
 // bias already added; kind fixed at compile time.
 template <int EK, typename T>
@@ -61,8 +78,7 @@ __device__ __forceinline__ void epi_store4(const Epi& e, int r, int c, float4 v)
     v.x = fmaxf(v.x, 0.f); v.y = fmaxf(v.y, 0.f); v.z = fmaxf(v.z, 0.f); v.w = fmaxf(v.w, 0.f);
   }
   if (EK == EPI_BIAS_SWISH) {
-    v.x = v.x / (1.f + expf(-v.x)); v.y = v.y / (1.f + expf(-v.y));
-    v.z = v.z / (1.f + expf(-v.z)); v.w = v.w / (1.f + expf(-v.w));
+    v.x *= sigm<T>(v.x); v.y *= sigm<T>(v.y); v.z *= sigm<T>(v.z); v.w *= sigm<T>(v.w);
   }
   if (EK == EPI_BIAS || EK == EPI_BIAS_RELU || EK == EPI_BIAS_SWISH) {
     T* o = reinterpret_cast<T*>(e.out) + orow * e.ldo + c;
@@ -77,7 +93,7 @@ __device__ __forceinline__ void epi_store4(const Epi& e, int r, int c, float4 v)
     }
   } else if (EK == EPI_BIAS_GLU) {
     T* o = reinterpret_cast<T*>(e.out) + orow * e.ldo + (c >> 1);
-    const float g0 = v.x / (1.f + expf(-v.y)), g1 = v.z / (1.f + expf(-v.w));
+    const float g0 = v.x * sigm<T>(v.y), g1 = v.z * sigm<T>(v.w);
     if (sizeof(T) == 2) {
       __nv_bfloat162 a = __floats2bfloat162_rn(g0, g1);
       *reinterpret_cast<__nv_bfloat162*>(o) = a;

@@ -140,7 +140,34 @@ __device__ __forceinline__ void epilogue_tile(const Epi& e, uint32_t tmem, float
     }
     __syncwarp();
     const int c = n0 + c0 + 4 * l4;
-    if (S == 1) {
+    if (S == 1 && EK == EPI_RESID) {
+      // residual update: 8 loads of x issued before the first store so
+      // their latencies overlap (a load after a store to the same array
+      // would otherwise wait for it)
+      float4 bv = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (e.bias && c < N) bv = *reinterpret_cast<const float4*>(e.bias + c);
+#pragma unroll 1
+      for (int i0 = 0; i0 < 16; i0 += 8) {
+        float4 xv[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int row = m0 + 32 * q + 2 * (i0 + i) + rh;
+          if (row < M && c < N) xv[i] = *reinterpret_cast<const float4*>(epi_f32_ptr(e, row, c));
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int rr = 2 * (i0 + i) + rh;
+          const int row = m0 + 32 * q + rr;
+          const float4 t = *reinterpret_cast<const float4*>(stage + rr * 68 + 4 * l4);
+          if (row < M && c < N) {
+            float4 x = xv[i];
+            x.x += e.alpha * (t.x + bv.x); x.y += e.alpha * (t.y + bv.y);
+            x.z += e.alpha * (t.z + bv.z); x.w += e.alpha * (t.w + bv.w);
+            *reinterpret_cast<float4*>(epi_f32_ptr(e, row, c)) = x;
+          }
+        }
+      }
+    } else if (S == 1) {
       float4 bv = make_float4(0.f, 0.f, 0.f, 0.f);
       if (e.bias && c < N) bv = *reinterpret_cast<const float4*>(e.bias + c);
 #pragma unroll 4

@@ -76,3 +76,45 @@ def test_gemm_tc_split_k_is_deterministic(eng):
     b.sf_check(eng)
     for o in outs[1:]:
         assert torch.equal(o, outs[0])
+
+
+@pytest.mark.parametrize("M,N,K", [(1125, 2048, 512), (20000, 192, 256), (19001, 256, 512), (333, 768, 192)])
+def test_gemm_tc_bf16_output(eng, M, N, K):
+    """Path 2: the engine's bf16 projection epilogue; each output is the
+    float64 result rounded to bf16 (within one bf16 ulp of it)."""
+    g = torch.Generator().manual_seed(M + N + K)
+    A = (torch.randn(M, K, generator=g) / np.sqrt(K)).to(torch.bfloat16)
+    W = torch.randn(N, K, generator=g).to(torch.bfloat16)
+    bias = torch.randn(N, generator=g)
+    ref = A.double().numpy() @ W.double().numpy().T + bias.double().numpy()
+    C = torch.full((M, N), float("nan"), device="cuda", dtype=torch.bfloat16)
+    b.sf_gemm_bf16(eng, A.cuda(), W.cuda(), C, bias=bias.cuda(), path=2)
+    b.sf_check(eng)
+    got = C.float().cpu().numpy()
+    assert np.all(np.abs(got - ref) <= np.abs(ref) * 2.0 ** -8 + 2e-4)
+
+
+@pytest.mark.parametrize("M,N,K", [(1125, 1024, 512), (20000, 192, 256), (19001, 512, 512)])
+@pytest.mark.parametrize("path", [3, 4, 5])
+def test_gemm_tc_fused_epilogues(eng, M, N, K, path):
+    """Paths 3-5: residual update (f32), swish (bf16) and gated linear unit
+    (bf16, interleaved value/gate columns) against float64."""
+    g = torch.Generator().manual_seed(M + 3 * N + K + path)
+    A = (torch.randn(M, K, generator=g) / np.sqrt(K)).to(torch.bfloat16)
+    W = torch.randn(N, K, generator=g).to(torch.bfloat16)
+    bias = torch.randn(N, generator=g)
+    r = A.double().numpy() @ W.double().numpy().T + bias.double().numpy()
+    if path == 3:
+        x0 = torch.randn(M, N, generator=g)
+        C = x0.cuda()
+        ref, tol_rel, tol_abs = x0.double().numpy() + r, 0.0, 4e-4
+    elif path == 4:
+        C = torch.full((M, N), float("nan"), device="cuda", dtype=torch.bfloat16)
+        ref, tol_rel, tol_abs = r / (1 + np.exp(-r)), 2.0 ** -8, 2e-4
+    else:
+        C = torch.full((M, N // 2), float("nan"), device="cuda", dtype=torch.bfloat16)
+        ref, tol_rel, tol_abs = r[:, 0::2] / (1 + np.exp(-r[:, 1::2])), 2.0 ** -8, 2e-4
+    b.sf_gemm_bf16(eng, A.cuda(), W.cuda(), C, bias=bias.cuda(), path=path)
+    b.sf_check(eng)
+    got = C.float().cpu().numpy()
+    assert np.all(np.abs(got - ref) <= np.abs(ref) * tol_rel + tol_abs)
