@@ -288,7 +288,13 @@ enum {
   SF_OPT_GRAPHS = 1,     /* 1 (default): capture each call shape once as a CUDA graph and
                             replay it; 0: launch kernel by kernel */
   SF_OPT_PDL = 2,        /* 1: programmatic dependent launch between kernels; 0 (default) */
-  SF_OPT_GEMM_PATH = 3   /* bf16 projections: 1 (default) tcgen05/TMEM/TMA kernel, 0 mma.sync */
+  SF_OPT_GEMM_PATH = 3,  /* bf16 projections on the tcgen05/TMEM/TMA kernels: 1 (default) with
+                            multi-wave projections of K >= 1024 and width >= 256 on CTA
+                            pairs (tcgen05 cta_group::2, 256-row tiles), 2 every multi-wave
+                            projection on CTA pairs, 3 single CTAs only; 0 the mma.sync
+                            kernel */
+  SF_OPT_GEMM_PAIR_BN = 4 /* tile width of the CTA-pair kernel: 0 (default) chosen per shape,
+                             or 128, 192, 256 */
 };
 SF_API sf_status sf_set_option(sf_engine* e, int option, int value);
 

@@ -158,7 +158,9 @@ struct sf_engine {
   cudaEvent_t desc_ev = nullptr;
   bool desc_pending = false;
   int* d_err = nullptr;
-  int gemm_path = 1;      // bf16 GEMMs: 1 = tcgen05 (default), 0 = mma.sync
+  int gemm_path = 1;      // bf16 GEMMs: tcgen05 with CTA pairs 1 = where faster (default), 2 = always,
+                          // 3 = never; 0 = mma.sync
+  int pair_bn = 0;        // CTA-pair tile width (0 = planned)
   float* d_split_ws = nullptr;   // split-K partial tiles of the tcgen05 GEMM
   int* d_split_cnt = nullptr;    // their per-tile arrival counters (kept at zero between launches)
   TcScratch tc_scratch() const { return TcScratch{d_err, d_split_ws, SPLIT_WS_BYTES, d_split_cnt, SPLIT_CNT}; }
@@ -578,7 +580,7 @@ cudaError_t gemm_dispatch<float>(sf_engine*, const float* A, int lda, const floa
 template <>
 cudaError_t gemm_dispatch<bf16>(sf_engine* e, const bf16* A, int lda, const bf16* W, int M, int N, int K,
                                 const Epi& ep, cudaStream_t st) {
-  if (e->gemm_path == 1 && N % 16 == 0) return gemm_bf16_tc(A, lda, W, M, N, K, ep, e->tc_scratch(), st);
+  if (e->gemm_path >= 1 && N % 16 == 0) return gemm_bf16_tc(A, lda, W, M, N, K, ep, e->tc_scratch(), st);
   return gemm_bf16_mma(A, lda, W, M, N, K, ep, st);
 }
 
@@ -638,6 +640,7 @@ cudaError_t run_graph(sf_engine* e, std::string key, cudaStream_t st, F&& enqueu
   if (!e->use_graphs) return enqueue(st);
   key += e->prof ? "|p" + std::to_string(e->prof_mask) : "|n";
   key += e->use_pdl ? "|pdl" : "";
+  key += "|g" + std::to_string(e->gemm_path) + "." + std::to_string(e->pair_bn);
   auto it = e->graphs.find(key);
   if (it != e->graphs.end() && it->second.gen != e->ws_gen) {
     cudaGraphExecDestroy(it->second.exec);
@@ -911,6 +914,8 @@ sf_status check_engine(sf_engine* e) {
   g_ws_gen = &e->ws_gen;
   g_fail_line = 0;
   sf::g_launch_pdl = e->use_pdl;
+  sf::g_gemm_pairs = e->gemm_path == 2 ? 2 : e->gemm_path == 3 ? 0 : 1;
+  sf::g_gemm_pair_bn = e->pair_bn;
   cudaGetLastError();   // start each call without a stale, non-sticky error
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev != e->device) cudaSetDevice(e->device);
@@ -1241,12 +1246,19 @@ sf_status sf_set_option(sf_engine* e, int option, int value) {
     case SF_OPT_GRAPHS: e->use_graphs = value != 0; break;
     case SF_OPT_PDL: e->use_pdl = value != 0; break;
     case SF_OPT_GEMM_PATH:
-      if (value != 0 && value != 1) return fail(e, SF_EINVAL, "gemm path must be 0 or 1");
+      if (value < 0 || value > 3) return fail(e, SF_EINVAL, "gemm path must be 0, 1, 2 or 3");
       e->gemm_path = value;
+      break;
+    case SF_OPT_GEMM_PAIR_BN:
+      if (value != 0 && value != 128 && value != 192 && value != 256)
+        return fail(e, SF_EINVAL, "pair tile width must be 0, 128, 192 or 256");
+      e->pair_bn = value;
       break;
     default: return fail(e, SF_EINVAL, "unknown option");
   }
   sf::g_launch_pdl = e->use_pdl;
+  sf::g_gemm_pairs = e->gemm_path == 2 ? 2 : e->gemm_path == 3 ? 0 : 1;
+  sf::g_gemm_pair_bn = e->pair_bn;
   return SF_OK;
 }
 

@@ -117,48 +117,54 @@ struct TcCfg {
   static_assert(STAGES * (A_BYTES + B_BYTES) >= 4 * 32 * 68 * 4, "epilogue staging reuses the pipeline buffers");
 };
 
-// Epilogue of one warp's 32 rows: per 64-column chunk, the accumulator block
-// goes TMEM -> registers -> shared tile (row stride 68 floats: conflict-free
-// 16-byte writes by row and reads by column), then each lane writes 4
-// consecutive columns of 2 rows per step (bias preloaded for its columns).
-// With split-K the raw partial tile goes to `part` instead.
-template <int EK, int BN>
+// Epilogue of one warp's 32 rows: per CW-column chunk (CW = 64 or 32), the
+// accumulator block goes TMEM -> registers -> shared tile (row stride CW + 4
+// floats: conflict-free 16-byte writes by row and reads by column), then
+// each lane writes 4 consecutive columns of one row per step, CW / 4 lanes
+// per row (bias preloaded for its columns).  With split-K the raw partial
+// tile goes to `part` instead.
+template <int EK, int BN, int CW = 64>
 __device__ __forceinline__ void epilogue_tile(const Epi& e, uint32_t tmem, float* stage, float* part, int M, int N,
                                               int m0, int n0, int q, int lane, int S, int cbeg = 0, int cend = BN) {
-  const int l4 = lane & 15, rh = lane >> 4;
+  constexpr int LD = CW + 4;          // staged row stride (floats)
+  constexpr int LPR = CW / 4;         // lanes per row
+  constexpr int RPI = 32 / LPR;       // rows per store instruction
+  constexpr int NI = 32 / RPI;        // store steps per chunk
+  const int l4 = lane % LPR, rh = lane / LPR;
 #pragma unroll 1
-  for (int c0 = cbeg; c0 < cend; c0 += 64) {
+  for (int c0 = cbeg; c0 < cend; c0 += CW) {
     uint32_t v[16];
 #pragma unroll
-    for (int h = 0; h < 4; ++h) {
+    for (int h = 0; h < CW / 16; ++h) {
       tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(c0 + 16 * h), v);
 #pragma unroll
       for (int j = 0; j < 16; j += 4)
-        *reinterpret_cast<float4*>(stage + lane * 68 + 16 * h + j) =
+        *reinterpret_cast<float4*>(stage + lane * LD + 16 * h + j) =
             make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]), __uint_as_float(v[j + 2]),
                         __uint_as_float(v[j + 3]));
     }
     __syncwarp();
     const int c = n0 + c0 + 4 * l4;
     if (S == 1 && EK == EPI_RESID) {
-      // residual update: 8 loads of x issued before the first store so
+      // residual update: NI / 2 loads of x issued before the first store so
       // their latencies overlap (a load after a store to the same array
       // would otherwise wait for it)
       float4 bv = make_float4(0.f, 0.f, 0.f, 0.f);
       if (e.bias && c < N) bv = *reinterpret_cast<const float4*>(e.bias + c);
+      constexpr int NB = NI / 2;
 #pragma unroll 1
-      for (int i0 = 0; i0 < 16; i0 += 8) {
-        float4 xv[8];
+      for (int i0 = 0; i0 < NI; i0 += NB) {
+        float4 xv[NB];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int row = m0 + 32 * q + 2 * (i0 + i) + rh;
+        for (int i = 0; i < NB; ++i) {
+          const int row = m0 + 32 * q + RPI * (i0 + i) + rh;
           if (row < M && c < N) xv[i] = *reinterpret_cast<const float4*>(epi_f32_ptr(e, row, c));
         }
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int rr = 2 * (i0 + i) + rh;
+        for (int i = 0; i < NB; ++i) {
+          const int rr = RPI * (i0 + i) + rh;
           const int row = m0 + 32 * q + rr;
-          const float4 t = *reinterpret_cast<const float4*>(stage + rr * 68 + 4 * l4);
+          const float4 t = *reinterpret_cast<const float4*>(stage + rr * LD + 4 * l4);
           if (row < M && c < N) {
             float4 x = xv[i];
             x.x += e.alpha * (t.x + bv.x); x.y += e.alpha * (t.y + bv.y);
@@ -171,19 +177,19 @@ __device__ __forceinline__ void epilogue_tile(const Epi& e, uint32_t tmem, float
       float4 bv = make_float4(0.f, 0.f, 0.f, 0.f);
       if (e.bias && c < N) bv = *reinterpret_cast<const float4*>(e.bias + c);
 #pragma unroll 4
-      for (int i = 0; i < 16; ++i) {
-        const int rr = 2 * i + rh;
+      for (int i = 0; i < NI; ++i) {
+        const int rr = RPI * i + rh;
         const int row = m0 + 32 * q + rr;
-        float4 t = *reinterpret_cast<const float4*>(stage + rr * 68 + 4 * l4);
+        float4 t = *reinterpret_cast<const float4*>(stage + rr * LD + 4 * l4);
         t.x += bv.x; t.y += bv.y; t.z += bv.z; t.w += bv.w;
         if (row < M && c < N) epi_store4<EK, bf16>(e, row, c, t);
       }
     } else {
 #pragma unroll 4
-      for (int i = 0; i < 16; ++i) {
-        const int rr = 2 * i + rh;
+      for (int i = 0; i < NI; ++i) {
+        const int rr = RPI * i + rh;
         *reinterpret_cast<float4*>(part + (int64_t)(32 * q + rr) * BN + c0 + 4 * l4) =
-            *reinterpret_cast<const float4*>(stage + rr * 68 + 4 * l4);
+            *reinterpret_cast<const float4*>(stage + rr * LD + 4 * l4);
       }
     }
     __syncwarp();
@@ -516,14 +522,15 @@ __global__ void __launch_bounds__(320, 1) gemm_tcp_kernel(const __grid_constant_
       tc_fence_after();
       const int m0 = (tile / tiles_n) * TC_BM, n0 = (tile % tiles_n) * BN;
       const uint32_t acc = tmem + (uint32_t)(a * BN);
+      const int cb = hc * BN / 2, ce = cb + BN / 2;
       switch (e.kind) {
-        case EPI_BIAS: epilogue_tile<EPI_BIAS, BN>(e, acc, stage, nullptr, M, N, m0, n0, q, lane, 1, hc * BN / 2, (hc + 1) * BN / 2); break;
-        case EPI_BIAS_RELU: epilogue_tile<EPI_BIAS_RELU, BN>(e, acc, stage, nullptr, M, N, m0, n0, q, lane, 1, hc * BN / 2, (hc + 1) * BN / 2); break;
-        case EPI_BIAS_SWISH: epilogue_tile<EPI_BIAS_SWISH, BN>(e, acc, stage, nullptr, M, N, m0, n0, q, lane, 1, hc * BN / 2, (hc + 1) * BN / 2); break;
-        case EPI_BIAS_GLU: epilogue_tile<EPI_BIAS_GLU, BN>(e, acc, stage, nullptr, M, N, m0, n0, q, lane, 1, hc * BN / 2, (hc + 1) * BN / 2); break;
-        case EPI_RESID: epilogue_tile<EPI_RESID, BN>(e, acc, stage, nullptr, M, N, m0, n0, q, lane, 1, hc * BN / 2, (hc + 1) * BN / 2); break;
-        case EPI_F32: epilogue_tile<EPI_F32, BN>(e, acc, stage, nullptr, M, N, m0, n0, q, lane, 1, hc * BN / 2, (hc + 1) * BN / 2); break;
-        default: epilogue_tile<EPI_F32_AND_T, BN>(e, acc, stage, nullptr, M, N, m0, n0, q, lane, 1, hc * BN / 2, (hc + 1) * BN / 2); break;
+        case EPI_BIAS: epilogue_tile<EPI_BIAS, BN>(e, acc, stage, nullptr, M, N, m0, n0, q, lane, 1, cb, ce); break;
+        case EPI_BIAS_RELU: epilogue_tile<EPI_BIAS_RELU, BN>(e, acc, stage, nullptr, M, N, m0, n0, q, lane, 1, cb, ce); break;
+        case EPI_BIAS_SWISH: epilogue_tile<EPI_BIAS_SWISH, BN>(e, acc, stage, nullptr, M, N, m0, n0, q, lane, 1, cb, ce); break;
+        case EPI_BIAS_GLU: epilogue_tile<EPI_BIAS_GLU, BN>(e, acc, stage, nullptr, M, N, m0, n0, q, lane, 1, cb, ce); break;
+        case EPI_RESID: epilogue_tile<EPI_RESID, BN>(e, acc, stage, nullptr, M, N, m0, n0, q, lane, 1, cb, ce); break;
+        case EPI_F32: epilogue_tile<EPI_F32, BN>(e, acc, stage, nullptr, M, N, m0, n0, q, lane, 1, cb, ce); break;
+        default: epilogue_tile<EPI_F32_AND_T, BN>(e, acc, stage, nullptr, M, N, m0, n0, q, lane, 1, cb, ce); break;
       }
       tc_fence_before();
       __syncwarp();
@@ -535,6 +542,247 @@ __global__ void __launch_bounds__(320, 1) gemm_tcp_kernel(const __grid_constant_
   if (warp == 1) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"((uint32_t)(2 * BN))
+                 : "memory");
+  }
+  if (threadIdx.x == 0 && *abort_flag) set_err(err, ERR_TIMEOUT);
+}
+
+// ---------------------------------------------------------------------------
+// CTA-pair variant (tcgen05 cta_group::2): a cluster of two CTAs on two SMs
+// computes one 256 x BN tile.  Each CTA loads its own 128 rows of A and its
+// own BN/2 rows of W per k-block; the even CTA (rank 0) issues M = 256
+// MMAs that read both CTAs' shared tiles, and each CTA's TMEM receives its
+// 128 rows x BN accumulator.  Per output element each SM moves 2/3 of the
+// operand bytes of the single-CTA 128 x 256 tile, so the same shared memory
+// holds half again as many k-blocks in flight.
+//   rank 0 warp 0 / rank 1 warp 0: TMA producers; both signal rank 0's
+//     full[s] (rank 0 arms it with both CTAs' bytes);
+//   rank 0 warp 1: MMA issuer; tcgen05.commit multicast frees empty[s] and
+//     publishes acc_full[a] in both CTAs;
+//   warps 2-9 of both CTAs: epilogue of their own 128 rows; each warp
+//     arrives on rank 0's acc_empty[a] (16 arrivals per phase).
+// Waits are bounded like the single-CTA kernels.  If either CTA gave up, both
+// hold their shared memory ~200 us after the closing cluster barrier so that
+// copies and MMAs still in flight land before it is released.  The loads
+// carry no multicast.
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Address of the same shared variable in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// TMA load into this CTA's shared memory whose completion is signalled on an
+// mbarrier that may live in the peer CTA (cluster address).
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
+      "[%2];" ::"r"(su32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void umma_bf16_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                               uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive once on the mbarrier at this offset in both CTAs of the pair when
+// every MMA issued so far has completed.
+__device__ __forceinline__ void umma_commit_pair(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          su32(bar)),
+      "h"((uint16_t)3)
+      : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+}
+__device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+constexpr int PAIR_BM = 256;
+
+template <int BN, int STAGES>
+struct Tc2Cfg {
+  static constexpr int CW = 32;        // epilogue chunk width (columns)
+  static constexpr int A_BYTES = TC_BM * TC_BK * 2;
+  static constexpr int B_BYTES = (BN / 2) * TC_BK * 2;
+  static constexpr int STAGE_FLOATS = 8 * 32 * (CW + 4);
+  static constexpr int SMEM = 1024 + STAGES * (A_BYTES + B_BYTES) + STAGE_FLOATS * 4 + 256;
+  // TMEM columns: two accumulators, rounded up to a power of two
+  static constexpr uint32_t TMEM_COLS = 2 * BN <= 256 ? 256u : 512u;
+  static_assert(SMEM <= 232448, "shared memory per CTA");
+  static_assert(BN % 64 == 0 && BN <= 256 && (BN / 2) % 32 == 0, "pair tile width");
+  static_assert(B_BYTES % 1024 == 0, "stage buffers stay 1024-byte aligned for the 128-byte swizzle");
+};
+
+// M = 256 instruction descriptor (bf16 x bf16 -> f32, K-major operands).
+__host__ __device__ constexpr uint32_t idesc_bf16_m256(int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(PAIR_BM >> 4) << 24);
+}
+
+template <int BN, int STAGES>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
+    gemm_tc2_kernel(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtensorMap tb, int M, int N,
+                    int K, Epi e, int* err) {
+  using C = Tc2Cfg<BN, STAGES>;
+  extern __shared__ uint8_t tc_smem[];
+  uint8_t* sm = tc_smem + ((1024 - (su32(tc_smem) & 1023)) & 1023);
+  uint8_t* sA = sm;
+  uint8_t* sB = sm + STAGES * C::A_BYTES;
+  float* stg = reinterpret_cast<float*>(sB + STAGES * C::B_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(stg + C::STAGE_FLOATS);
+  uint64_t* empty = full + STAGES;
+  uint64_t* accf = empty + STAGES;     // [2]
+  uint64_t* acce = accf + 2;           // [2], used in rank 0
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* peer_abort = abort_flag + 1;   // written by the other CTA at teardown
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int tiles_n = (N + BN - 1) / BN;
+  const int tiles = ((M + PAIR_BM - 1) / PAIR_BM) * tiles_n;
+  const int KB = (K + TC_BK - 1) / TC_BK;
+
+  if (threadIdx.x == 0) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&ta)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tb)) : "memory");
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&accf[a], 1);
+      mbar_init(&acce[a], 16);
+    }
+    *abort_flag = 0;
+    *peer_abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(tmem_slot)),
+                 "r"(C::TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncwarp();
+  cluster_sync_all();   // both CTAs' barriers initialised and TMEM allocated
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  SF_PDL_ENTRY();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int it = 0;
+      for (int tile = pair; tile < tiles && !*abort_flag; tile += npairs) {
+        const int m0 = (tile / tiles_n) * PAIR_BM + TC_BM * (int)rank;
+        const int n0 = (tile % tiles_n) * BN + (BN / 2) * (int)rank;
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % STAGES, r = it / STAGES;
+          if (!mbar_wait(&empty[s], (r & 1) ^ 1, abort_flag)) {
+            *abort_flag = 1;
+            break;
+          }
+          if (rank == 0) mbar_expect_tx(&full[s], 2 * (C::A_BYTES + C::B_BYTES));
+          const uint32_t fb = mapa_shared(su32(&full[s]), 0);
+          tma_load_2d_pair(sA + s * C::A_BYTES, &ta, fb, kb * TC_BK, m0);
+          tma_load_2d_pair(sB + s * C::B_BYTES, &tb, fb, kb * TC_BK, n0);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t idesc = idesc_bf16_m256(BN);
+      int it = 0, i = 0;
+      for (int tile = pair; tile < tiles && !*abort_flag; tile += npairs, ++i) {
+        const int a = i & 1, u = i >> 1;
+        if (!mbar_wait(&acce[a], (u & 1) ^ 1, abort_flag)) {
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t acc = tmem + (uint32_t)(a * BN);
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % STAGES, r = it / STAGES;
+          if (!mbar_wait(&full[s], r & 1, abort_flag)) {
+            *abort_flag = 1;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t ad = sw128_desc(su32(sA + s * C::A_BYTES));
+          const uint64_t bd = sw128_desc(su32(sB + s * C::B_BYTES));
+#pragma unroll
+          for (int k = 0; k < TC_BK / 16; ++k)
+            umma_bf16_pair(acc, ad + (uint64_t)(2 * k), bd + (uint64_t)(2 * k), idesc, (kb | k) != 0);
+          umma_commit_pair(&empty[s]);
+        }
+        umma_commit_pair(&accf[a]);
+      }
+      pdl_trigger();
+    }
+  } else {
+    const int q = warp & 3, hc = (warp - 2) >> 2;   // TMEM lane quarter, column half
+    float* stage = stg + (warp - 2) * (32 * (C::CW + 4));
+    int i = 0;
+    for (int tile = pair; tile < tiles; tile += npairs, ++i) {
+      const int a = i & 1, u = i >> 1;
+      if (!mbar_wait(&accf[a], u & 1, abort_flag) || *abort_flag) {
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const int m0 = (tile / tiles_n) * PAIR_BM + TC_BM * (int)rank, n0 = (tile % tiles_n) * BN;
+      const uint32_t acc = tmem + (uint32_t)(a * BN);
+      const int cb = hc * BN / 2, ce = cb + BN / 2;
+      switch (e.kind) {
+        case EPI_BIAS: epilogue_tile<EPI_BIAS, BN, C::CW>(e, acc, stage, nullptr, M, N, m0, n0, q, lane, 1, cb, ce); break;
+        case EPI_BIAS_RELU: epilogue_tile<EPI_BIAS_RELU, BN, C::CW>(e, acc, stage, nullptr, M, N, m0, n0, q, lane, 1, cb, ce); break;
+        case EPI_BIAS_SWISH: epilogue_tile<EPI_BIAS_SWISH, BN, C::CW>(e, acc, stage, nullptr, M, N, m0, n0, q, lane, 1, cb, ce); break;
+        case EPI_BIAS_GLU: epilogue_tile<EPI_BIAS_GLU, BN, C::CW>(e, acc, stage, nullptr, M, N, m0, n0, q, lane, 1, cb, ce); break;
+        case EPI_RESID: epilogue_tile<EPI_RESID, BN, C::CW>(e, acc, stage, nullptr, M, N, m0, n0, q, lane, 1, cb, ce); break;
+        case EPI_F32: epilogue_tile<EPI_F32, BN, C::CW>(e, acc, stage, nullptr, M, N, m0, n0, q, lane, 1, cb, ce); break;
+        default: epilogue_tile<EPI_F32_AND_T, BN, C::CW>(e, acc, stage, nullptr, M, N, m0, n0, q, lane, 1, cb, ce); break;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(su32(&acce[a]), 0));   // accumulator a drained here
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort_flag) st_cluster_u32(mapa_shared(su32((const void*)peer_abort), rank ^ 1u), 1u);
+  __syncwarp();
+  cluster_sync_all();   // no CTA leaves while its peer may still signal its barriers
+  if (*abort_flag || *peer_abort) {
+    // a wait gave up: copies or MMAs may still be in flight into either CTA
+    uint64_t t0, t1;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+    do {
+      __nanosleep(10000);
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t1));
+    } while (t1 - t0 < 200000ull);
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::TMEM_COLS)
                  : "memory");
   }
   if (threadIdx.x == 0 && *abort_flag) set_err(err, ERR_TIMEOUT);
@@ -597,7 +845,49 @@ cudaError_t launch_tcp(const bf16* A, int lda, const bf16* W, int M, int N, int 
   return cudaGetLastError();
 }
 
+int g_max_pairs = 0;   // co-resident CTA pairs of gemm_tc2_kernel (0: not queried)
+
+template <int BN, int STAGES>
+cudaError_t launch_tc2(const bf16* A, int lda, const bf16* W, int M, int N, int K, const Epi& e, const TcScratch& sc,
+                       cudaStream_t st) {
+  CUtensorMap ta, tb;
+  cudaError_t r = make_map(&ta, A, M, K, lda, TC_BM);
+  if (r != cudaSuccess) return r;
+  r = make_map(&tb, W, N, K, K, BN / 2);
+  if (r != cudaSuccess) return r;
+  const int tiles = ((M + PAIR_BM - 1) / PAIR_BM) * ((N + BN - 1) / BN);
+  const int cap = g_max_pairs > 0 ? g_max_pairs : g_num_sms / 2;
+  const int pairs = tiles < cap ? tiles : cap;
+  CK_LAUNCH(launch_k(gemm_tc2_kernel<BN, STAGES>, dim3(2 * pairs), dim3(320), Tc2Cfg<BN, STAGES>::SMEM, st, ta, tb, M,
+                     N, K, e, sc.err));
+  return cudaGetLastError();
+}
+
 }  // namespace
+
+int g_gemm_pairs = 1;
+int g_gemm_pair_bn = 0;
+
+// Pair tile width for a multi-wave GEMM on the CTA-pair kernel: the fewest
+// estimated microseconds over BN = 256 / 192 / 128, counting whole rounds of
+// tiles over the co-resident pairs (the last round is as long as a full one)
+// and per tile a fixed ~1 us plus a per-k-block time that shrinks with BN.
+int gemm_pair_plan(int M, int N, int K) {
+  const int pairs = g_max_pairs > 0 ? g_max_pairs : g_num_sms / 2;
+  const int tm = (M + PAIR_BM - 1) / PAIR_BM, KB = (K + TC_BK - 1) / TC_BK;
+  double best = 1e30;
+  int bb = 256;
+  for (int bn : {256, 192, 128}) {
+    const int tiles = tm * ((N + bn - 1) / bn);
+    const int rounds = (tiles + pairs - 1) / pairs;
+    const double t = rounds * (1.0 + KB * (bn == 256 ? 0.40 : bn == 192 ? 0.33 : 0.27));
+    if (t < best * 0.98) {
+      best = t;
+      bb = bn;
+    }
+  }
+  return bb;
+}
 
 // Tile width BN and split count S from a cost model of this kernel on 148
 // SMs, calibrated with per-phase timestamps on B200: per CTA ~1.4 us of
@@ -642,6 +932,16 @@ cudaError_t gemm_bf16_tc(const bf16* A, int lda, const bf16* W, int M, int N, in
   // more tiles than SMs: the persistent kernel overlaps each tile's epilogue
   // with the next tile's mainloop
   if (sp == 1 && N >= 128 && ((M + TC_BM - 1) / TC_BM) * ((N + bn - 1) / bn) > g_num_sms) {
+    // CTA pairs: every such GEMM in mode 2; in mode 1 those with K >= 1024
+    // and N >= 256, where the pair kernel's deeper operand ring wins (the
+    // single-CTA kernel leads on shorter K, whose time goes to the epilogue)
+    if (g_gemm_pairs == 2 || (g_gemm_pairs == 1 && K >= 1024 && N >= 256)) {
+      switch (g_gemm_pair_bn ? g_gemm_pair_bn : gemm_pair_plan(M, N, K)) {
+        case 256: return launch_tc2<256, 5>(A, lda, W, M, N, K, e, sc, st);
+        case 192: return launch_tc2<192, 6>(A, lda, W, M, N, K, e, sc, st);
+        default: return launch_tc2<128, 7>(A, lda, W, M, N, K, e, sc, st);
+      }
+    }
     if (N >= 256) return launch_tcp<256, 3>(A, lda, W, M, N, K, e, sc, st);
     return launch_tcp<128, 4>(A, lda, W, M, N, K, e, sc, st);
   }
@@ -659,6 +959,21 @@ cudaError_t gemm_tc_init_attributes() {
   if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) ==
                                                  cudaSuccess && n_sm > 0)
     g_num_sms = n_sm;
+  r = cudaFuncSetAttribute(gemm_tc2_kernel<256, 5>, cudaFuncAttributeMaxDynamicSharedMemorySize, Tc2Cfg<256, 5>::SMEM);
+  if (r == cudaSuccess)
+    r = cudaFuncSetAttribute(gemm_tc2_kernel<192, 6>, cudaFuncAttributeMaxDynamicSharedMemorySize, Tc2Cfg<192, 6>::SMEM);
+  if (r == cudaSuccess)
+    r = cudaFuncSetAttribute(gemm_tc2_kernel<128, 7>, cudaFuncAttributeMaxDynamicSharedMemorySize, Tc2Cfg<128, 7>::SMEM);
+  if (r != cudaSuccess) return r;
+  {   // every configuration holds one CTA per SM: the same number of co-resident pairs
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (g_num_sms / 2));
+    cfg.blockDim = dim3(320);
+    cfg.dynamicSmemBytes = Tc2Cfg<256, 5>::SMEM;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, gemm_tc2_kernel<256, 5>, &cfg) == cudaSuccess && n > 0) g_max_pairs = n;
+    cudaGetLastError();
+  }
   r = cudaFuncSetAttribute(gemm_tcp_kernel<256, 3>, cudaFuncAttributeMaxDynamicSharedMemorySize, TcpCfg<256, 3>::SMEM);
   if (r == cudaSuccess)
     r = cudaFuncSetAttribute(gemm_tcp_kernel<128, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, TcpCfg<128, 4>::SMEM);

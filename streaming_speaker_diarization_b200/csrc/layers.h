@@ -48,6 +48,12 @@ struct TcScratch {
 cudaError_t gemm_bf16_tc(const bf16* A, int lda, const bf16* W, int M, int N, int K, const Epi& e,
                          const TcScratch& sc, cudaStream_t st);
 cudaError_t gemm_tc_init_attributes();
+// Multi-wave bf16 GEMMs on the CTA-pair (cta_group::2) kernel: 0 never, 1
+// where it is faster (K >= 1024, N >= 256), 2 always; set from the calling
+// engine's options at each API entry.
+extern int g_gemm_pairs;
+// Pair tile width forced for those GEMMs (128, 192 or 256); 0 = planned.
+extern int g_gemm_pair_bn;
 void gemm_tc_plan(int M, int N, int K, const TcScratch& sc, int* bn, int* splits);
 
 // --------------------------------------------------------- subsampling

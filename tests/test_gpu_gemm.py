@@ -26,7 +26,9 @@ SHAPES = [(1125, 2048, 512), (1125, 512, 2048), (1125, 1536, 512), (1125, 192, 1
           (1125, 192, 768), (1125, 512, 4096), (1, 64, 64), (333, 768, 192), (128, 128, 128), (129, 256, 4096),
           (24896, 1024, 512), (70, 16, 64), (300, 64, 4096), (2000, 256, 1024),
           # more tiles than SMs: persistent kernel, BN 256 / 128, ragged M and N tails
-          (20000, 192, 256), (19001, 256, 512), (50000, 576, 192), (72000, 256, 256)]
+          (20000, 192, 256), (19001, 256, 512), (50000, 576, 192), (72000, 256, 256),
+          # K >= 1024, N >= 256, multi-wave: CTA pairs on the default path
+          (20608, 512, 2048)]
 
 
 @pytest.mark.parametrize("M,N,K", SHAPES)
@@ -99,12 +101,56 @@ def test_gemm_tc_bf16_output(eng, M, N, K):
 def test_gemm_tc_fused_epilogues(eng, M, N, K, path):
     """Paths 3-5: residual update (f32), swish (bf16) and gated linear unit
     (bf16, interleaved value/gate columns) against float64."""
+    _check_fused(eng, M, N, K, path)
+
+
+@pytest.fixture(scope="module", params=[0, 128, 192, 256])
+def eng_pairs(request):
+    """Engine on the CTA-pair GEMM path: planned tile width (0) or forced."""
+    e = make_engine(tiny_weights(), 1, 2, 2)
+    b.sf_set_option(e, b.SF_OPT_GEMM_PATH, 2)
+    b.sf_set_option(e, b.SF_OPT_GEMM_PAIR_BN, request.param)
+    yield e
+    b.sf_destroy(e)
+
+
+# multi-wave shapes with N >= 256 (the CTA-pair kernel): ragged last pair tile
+# whose second CTA is entirely past M (19001 = 74 x 256 + 57), N not a
+# multiple of 256 (the second CTA's weight rows of the last tile all past N),
+# long K, many tiles per pair
+PAIR_SHAPES = [(19001, 256, 512), (20000, 320, 256), (24896, 1024, 512), (20608, 512, 2048), (72000, 256, 256),
+               (20608, 2048, 512), (20608, 192, 768), (20608, 576, 192), (33000, 192, 192)]
+
+
+@pytest.mark.parametrize("M,N,K", PAIR_SHAPES)
+def test_gemm_tc_pairs_vs_float64(eng_pairs, M, N, K):
+    g = torch.Generator().manual_seed(M * 5 + N * 3 + K)
+    A = (torch.randn(M, K, generator=g) / np.sqrt(K)).to(torch.bfloat16)
+    W = torch.randn(N, K, generator=g).to(torch.bfloat16)
+    bias = torch.randn(N, generator=g)
+    ref = A.double().numpy() @ W.double().numpy().T + bias.double().numpy()
+    C = torch.full((M, N), float("nan"), device="cuda")
+    b.sf_gemm_bf16(eng_pairs, A.cuda(), W.cuda(), C, bias=bias.cuda(), path=1)
+    b.sf_check(eng_pairs)
+    err = np.max(np.abs(C.cpu().numpy() - ref))
+    assert err <= 2e-4 * max(1.0, np.sqrt(K / 512)), err
+
+
+@pytest.mark.parametrize("path", [2, 3, 4, 5])
+def test_gemm_tc_pairs_fused_epilogues(eng_pairs, path):
+    _check_fused(eng_pairs, 20608, 1024, 512, path)
+
+
+def _check_fused(eng, M, N, K, path):
     g = torch.Generator().manual_seed(M + 3 * N + K + path)
     A = (torch.randn(M, K, generator=g) / np.sqrt(K)).to(torch.bfloat16)
     W = torch.randn(N, K, generator=g).to(torch.bfloat16)
     bias = torch.randn(N, generator=g)
     r = A.double().numpy() @ W.double().numpy().T + bias.double().numpy()
-    if path == 3:
+    if path == 2:
+        C = torch.full((M, N), float("nan"), device="cuda", dtype=torch.bfloat16)
+        ref, tol_rel, tol_abs = r, 2.0 ** -8, 2e-4
+    elif path == 3:
         x0 = torch.randn(M, N, generator=g)
         C = x0.cuda()
         ref, tol_rel, tol_abs = x0.double().numpy() + r, 0.0, 4e-4
