@@ -293,8 +293,10 @@ enum {
                             pairs (tcgen05 cta_group::2, 256-row tiles), 2 every multi-wave
                             projection on CTA pairs, 3 single CTAs only; 0 the mma.sync
                             kernel */
-  SF_OPT_GEMM_PAIR_BN = 4 /* tile width of the CTA-pair kernel: 0 (default) chosen per shape,
-                             or 128, 192, 256 */
+  SF_OPT_GEMM_PAIR_BN = 4, /* tile width of the CTA-pair kernel: 0 (default) chosen per shape,
+                              or 128, 192, 256 */
+  SF_OPT_ATTN_PATH = 5    /* bf16 relative-position attention: 1 (default) tcgen05/TMEM/TMA
+                             kernel, 0 mma.sync kernel */
 };
 SF_API sf_status sf_set_option(sf_engine* e, int option, int value);
 
@@ -316,6 +318,23 @@ SF_API sf_status sf_check(sf_engine* e, void* cuda_stream);
  * Requires N % 16 == 0, K % 64 == 0, lda % 8 == 0, 16-byte aligned A/W. */
 SF_API sf_status sf_gemm_bf16(sf_engine* e, const void* d_A, int lda, const void* d_W, int M, int N, int K,
                               const float* d_bias, void* d_C, int path, void* cuda_stream);
+
+/* The engine's relative-position self-attention alone (bf16 engines), for
+ * tests and kernel benchmarks ("Streaming Sortformer Diarizer" model card,
+ * FastConformer encoder: relative-position MHSA, d_model 512, 8 heads of 64):
+ *   d_qkv  bf16 [M x 1536]  rows of the n packed sequences (h_seq_len[i]
+ *                           rows each, M = their sum), columns q | k | v,
+ *                           head h at columns 64h .. 64h + 63 of each part
+ *   d_ptab bf16 [(2R-1) x 512]  projected relative-position rows; row
+ *                           i - j + R - 1 holds distance i - j
+ *   d_u, d_v f32 [512]      per-head position biases (pos_bias_u / _v)
+ *   d_ctx  bf16 [M x 512] (out)  softmax_j(((q_i+u).k_j + (q_i+v).p_(i-j))/8) v_j
+ * Sequence lengths must lie in [1, R]; path 1 = tcgen05 kernel, 0 = mma.sync.
+ * Pointers 16-byte aligned.  Uses the engine's descriptor block (ordered on
+ * `cuda_stream` with the engine's other calls). */
+SF_API sf_status sf_attention_relpos(sf_engine* e, const void* d_qkv, const void* d_ptab, int R, const float* d_u,
+                                     const float* d_v, const int* h_seq_len, int n, void* d_ctx, int path,
+                                     void* cuda_stream);
 
 /* ---------------------------------------------------------------- profiling */
 

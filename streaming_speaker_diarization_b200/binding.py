@@ -17,7 +17,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libsf.so")
 
 SF_FP32, SF_BF16 = 0, 1
-SF_OPT_GRAPHS, SF_OPT_PDL, SF_OPT_GEMM_PATH, SF_OPT_GEMM_PAIR_BN = 1, 2, 3, 4
+SF_OPT_GRAPHS, SF_OPT_PDL, SF_OPT_GEMM_PATH, SF_OPT_GEMM_PAIR_BN, SF_OPT_ATTN_PATH = 1, 2, 3, 4, 5
 STATUS = {0: "SF_OK", 1: "SF_EINVAL", 2: "SF_ESHAPE", 3: "SF_ENOMEM", 4: "SF_ECUDA", 5: "SF_ESTATE",
           6: "SF_ETIMEOUT", 7: "SF_EDEVICE", 8: "SF_EFORMAT"}
 
@@ -51,7 +51,7 @@ EXPORTED = ["sf_default_config", "sf_create", "sf_create_from_file", "sf_destroy
             "sf_forward_offline_host", "sf_stream_create", "sf_stream_destroy", "sf_stream_reset",
             "sf_stream_window", "sf_stream_step", "sf_stream_get_state", "sf_stream_set_state",
             "sf_stream_update", "sf_select_topk", "sf_profile_enable", "sf_profile_read", "sf_mel_noalloc",
-            "sf_check", "sf_gemm_bf16", "sf_set_option"]
+            "sf_check", "sf_gemm_bf16", "sf_set_option", "sf_attention_relpos"]
 
 
 class SFError(RuntimeError):
@@ -91,6 +91,7 @@ def _load():
         "sf_check": ([VP, VP], I),
         "sf_set_option": ([VP, I, I], I),
         "sf_gemm_bf16": ([VP, VP, I, VP, I, I, I, VP, VP, I, VP], I),
+        "sf_attention_relpos": ([VP, VP, VP, I, VP, VP, VP, I, VP, I, VP], I),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -282,6 +283,12 @@ def sf_gemm_bf16(eng, A, W, C, bias=None, path=1, stream=None):
     N = W.shape[0]
     _check(lib.sf_gemm_bf16(eng, _ptr(A), A.stride(0), _ptr(W), M, N, K, _ptr(bias), _ptr(C), path,
                             _stream(stream)), eng)
+
+
+def sf_attention_relpos(eng, qkv, ptab, R, u, v, seq_len, ctx, path=1, stream=None):
+    seq_len = np.ascontiguousarray(seq_len, np.int32)
+    _check(lib.sf_attention_relpos(eng, _ptr(qkv), _ptr(ptab), R, _ptr(u), _ptr(v), _ptr(seq_len), len(seq_len),
+                                   _ptr(ctx), path, _stream(stream)), eng)
 
 
 def sf_set_option(eng, option, value):

@@ -1,0 +1,384 @@
+// Relative-position MHSA on the Blackwell tensor cores (tcgen05 MMA with TMEM
+// accumulators, TMA loads), bf16 operands, fp32 scores and softmax, head dim
+// 64.  Same arithmetic as the FastConformer attention of the "Streaming
+// Sortformer Diarizer" model (relative-position MHSA):
+//   score(i, j) = ((q_i + u) . k_j + (q_i + v) . p_(i-j)) / sqrt(64),
+//   out_i = sum_j softmax_j(score(i, .)) v_j   over the keys of i's sequence.
+//
+// One CTA = 128 query rows [i0, i0 + 128) of one sequence x one head.  Per
+// 64-key tile [j0, j0 + 64):
+//   AC = (Q+u) K^T    M 128, N  64, K 64   TMEM columns [0, 64)
+//   BD = (Q+v) Pw^T   M 128, N 192, K 64   TMEM columns [64, 256)
+//        Pw = position-table rows for distances i0 - j0 - 63 .. i0 - j0 + 128,
+//        i.e. every i - j of the tile (row r, key c: BD column r - c + 63)
+//   O_t = P V         M 128, N  64, K 64   TMEM columns 256 + 64 (t % 2)
+// Warps: 0 loads K, V and Pw with TMA into a two-stage ring; 1 issues the
+// MMAs (one thread); 2-5 run the softmax, thread = query row = TMEM lane.  A
+// warp's 32 rows need a 96-column band of BD; it is staged in shared memory
+// (row stride 100 floats: conflict-free by rows and along the diagonal) and
+// read back at column r - c + 63.  The softmax is online in the exp2 domain
+// (scale folded in); P goes to shared memory as bf16 (the A operand of P.V);
+// O accumulates in registers, rescaled before each tile's P.V is added.
+// Every wait is bounded: a wait that runs out raises ERR_TIMEOUT, the CTA
+// drains its own copies and frees its TMEM.
+#include "common.cuh"
+#include "layers.h"
+#include "tcgen05.cuh"
+
+namespace sf {
+namespace {
+
+constexpr int AQ = 128;      // query rows per CTA
+constexpr int AK = 64;       // keys per tile
+constexpr int AHD = 64;      // head dim
+constexpr int APW = 192;     // position-table rows per tile (distances r - c)
+constexpr int ANB = 2;       // K / V / Pw ring stages
+constexpr int BD_LD = 100;   // staged BD row stride (floats)
+
+struct AttTc {
+  static constexpr int Q_BYTES = AQ * AHD * 2;      // 16 KB, K-major, 128-byte swizzle
+  static constexpr int K_BYTES = AK * AHD * 2;      //  8 KB
+  static constexpr int V_BYTES = AK * AHD * 2;      //  8 KB (MN-major B operand)
+  static constexpr int PW_BYTES = APW * AHD * 2;    // 24 KB
+  static constexpr int STAGE = K_BYTES + V_BYTES + PW_BYTES;
+  static constexpr int P_BYTES = AQ * AK * 2;       // 16 KB
+  static constexpr int OFF_QU = 0;
+  static constexpr int OFF_QV = Q_BYTES;
+  static constexpr int OFF_RING = 2 * Q_BYTES;
+  static constexpr int OFF_P = OFF_RING + ANB * STAGE;
+  static constexpr int OFF_BD = OFF_P + 2 * P_BYTES;
+  static constexpr int BD_BYTES = 4 * 32 * BD_LD * 4;
+  static constexpr int OFF_BAR = OFF_BD + BD_BYTES;
+  static constexpr int SMEM = 1024 + OFF_BAR + 256;
+  static_assert(STAGE % 1024 == 0 && OFF_P % 1024 == 0 && OFF_RING % 1024 == 0, "swizzled tiles 1024-aligned");
+  static_assert(SMEM <= 232448, "shared memory per CTA");
+};
+
+// Shared-memory descriptor of an MN-major operand with 128-byte swizzle:
+// rows of 64 bf16 along N (one swizzle atom wide), consecutive K rows 128
+// bytes apart, 8-row groups 1024 bytes apart (stride byte offset).
+__device__ __forceinline__ uint64_t sw128_desc_mn(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFF) >> 4);
+  d |= (uint64_t)(8192 >> 4) << 16;          // leading byte offset: next atom along N (not reached, N = 64)
+  d |= (uint64_t)(1024 >> 4) << 32;          // stride byte offset: next 8 rows along K
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
+// Byte offset of element (row, col) (col in bf16 units, < 64) of a K-major
+// tile with 128-byte rows and the 128-byte swizzle (16-byte chunk index
+// XOR row % 8), as TMA writes it and tcgen05 reads it.
+__device__ __forceinline__ uint32_t sw128_off(int row, int chunk) {
+  return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(192, 1) attn_relpos_tc_kernel(const __grid_constant__ CUtensorMap t_qkv,
+                                                                const __grid_constant__ CUtensorMap t_pos,
+                                                                const bf16* __restrict__ qkv, int D, int R,
+                                                                const float* __restrict__ u,
+                                                                const float* __restrict__ vb, bf16* __restrict__ ctx,
+                                                                const SeqTable* __restrict__ seq, int* err) {
+  using L = AttTc;
+  extern __shared__ uint8_t at_smem[];
+  uint8_t* sm = at_smem + ((1024 - (su32(at_smem) & 1023)) & 1023);
+  uint8_t* sQu = sm + L::OFF_QU;
+  uint8_t* sQv = sm + L::OFF_QV;
+  uint8_t* sRing = sm + L::OFF_RING;
+  uint8_t* sP = sm + L::OFF_P;
+  float* sBD = reinterpret_cast<float*>(sm + L::OFF_BD);
+  uint64_t* kv_full = reinterpret_cast<uint64_t*>(sm + L::OFF_BAR);   // [ANB]
+  uint64_t* kv_empty = kv_full + ANB;                                  // [ANB]
+  uint64_t* s_full = kv_empty + ANB;
+  uint64_t* s_free = s_full + 1;
+  uint64_t* p_full = s_free + 1;                                       // [2]
+  uint64_t* pv_full = p_full + 2;                                      // [2]
+  uint64_t* q_ready = pv_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_ready + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.y;
+  const int s = seq_of_tile2(seq, blockIdx.x);
+  const int sb = seq->off[s], S = seq->off[s + 1] - sb;
+  const int i0 = (blockIdx.x - seq->tile2_off[s]) * AQ;
+  const int T = (S + AK - 1) / AK;   // key tiles
+
+  if (threadIdx.x == 0) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&t_qkv)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&t_pos)) : "memory");
+    for (int b = 0; b < ANB; ++b) {
+      mbar_init(&kv_full[b], 1);
+      mbar_init(&kv_empty[b], 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(s_free, 4);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&p_full[b], 4);
+      mbar_init(&pv_full[b], 1);
+    }
+    mbar_init(q_ready, 4);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(tmem_slot)),
+                 "r"(512u)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  SF_PDL_ENTRY();
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- loads
+    if (lane == 0) {
+      int t = 0;
+      for (; t < T && !*abort_flag; ++t) {
+        const int b = t % ANB, r = t / ANB, j0 = t * AK;
+        if (!mbar_wait(&kv_empty[b], (r & 1) ^ 1, abort_flag)) {
+          *abort_flag = 1;
+          break;
+        }
+        uint8_t* st = sRing + b * L::STAGE;
+        mbar_expect_tx(&kv_full[b], L::STAGE);
+        tma_load_2d(st, &t_qkv, &kv_full[b], D + h * AHD, sb + j0);                       // K rows j0 ..
+        tma_load_2d(st + L::K_BYTES, &t_qkv, &kv_full[b], 2 * D + h * AHD, sb + j0);      // V rows j0 ..
+        tma_load_2d(st + L::K_BYTES + L::V_BYTES, &t_pos, &kv_full[b], h * AHD,
+                    i0 - j0 - (AK - 1) + R - 1);                                            // distances
+      }
+      if (*abort_flag) {   // let this CTA's own loads land before its shared memory is released
+        for (int k = t - ANB > 0 ? t - ANB : 0; k < t; ++k) {
+          const long long c0 = clock64();
+          while (!mbar_try_wait(&kv_full[k % ANB], (k / ANB) & 1) && clock64() - c0 < WAIT_CYCLES) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------------------- MMAs
+    if (lane == 0) {
+      constexpr uint32_t id_s = idesc_bf16_mn(AQ, AK, false);
+      constexpr uint32_t id_bd = idesc_bf16_mn(AQ, APW, false);
+      constexpr uint32_t id_pv = idesc_bf16_mn(AQ, AHD, true);
+      const uint32_t tm_s = tmem, tm_bd = tmem + AK;
+      const uint64_t dqu = sw128_desc(su32(sQu)), dqv = sw128_desc(su32(sQv));
+      bool ok = mbar_wait(q_ready, 0, abort_flag);
+      auto issue_pv = [&](int t) -> bool {
+        const int pb = t & 1, b = t % ANB;
+        if (!mbar_wait(&p_full[pb], (t >> 1) & 1, abort_flag)) return false;
+        tc_fence_after();
+        const uint64_t dp = sw128_desc(su32(sP + pb * L::P_BYTES));
+        const uint64_t dv = sw128_desc_mn(su32(sRing + b * L::STAGE + L::K_BYTES));
+#pragma unroll
+        for (int k = 0; k < AK / 16; ++k)   // K (keys) 16 at a time: +32 bytes in P, +16 rows (2048 bytes) in V
+          umma_bf16(tmem + 256 + 64 * pb, dp + (uint64_t)(2 * k), dv + (uint64_t)(128 * k), id_pv, k != 0);
+        umma_commit(&pv_full[pb]);
+        umma_commit(&kv_empty[b]);   // K, V and Pw of tile t are no longer read
+        return true;
+      };
+      for (int t = 0; ok && t < T; ++t) {
+        const int b = t % ANB;
+        if (!mbar_wait(&kv_full[b], (t / ANB) & 1, abort_flag)) { ok = false; break; }
+        if (t > 0 && !mbar_wait(s_free, (t - 1) & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        uint8_t* st = sRing + b * L::STAGE;
+        const uint64_t dk = sw128_desc(su32(st)), dpw = sw128_desc(su32(st + L::K_BYTES + L::V_BYTES));
+#pragma unroll
+        for (int k = 0; k < AHD / 16; ++k) umma_bf16(tm_s, dqu + (uint64_t)(2 * k), dk + (uint64_t)(2 * k), id_s, k != 0);
+#pragma unroll
+        for (int k = 0; k < AHD / 16; ++k)
+          umma_bf16(tm_bd, dqv + (uint64_t)(2 * k), dpw + (uint64_t)(2 * k), id_bd, k != 0);
+        umma_commit(s_full);
+        if (t > 0 && !issue_pv(t - 1)) { ok = false; break; }
+      }
+      if (ok && T > 0) ok = issue_pv(T - 1);
+      if (!ok) *abort_flag = 1;
+    }
+  } else {
+    // -------------------------------------------------------------- softmax
+    const int q = warp & 3;                        // TMEM lane quarter of this warp
+    const int r = 32 * q + lane;                   // query row in the tile = TMEM lane
+    const int i = i0 + r;
+    const bool row_ok = i < S;
+    const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+    // (Q + u) and (Q + v) rows, rounded to bf16, into the swizzled A tiles
+    {
+      const bf16* qrow = qkv + (int64_t)(sb + (row_ok ? i : 0)) * (3 * D) + h * AHD;
+      const float* uh = u + h * AHD;
+      const float* vh = vb + h * AHD;
+#pragma unroll
+      for (int c = 0; c < AHD / 8; ++c) {
+        uint4 raw = make_uint4(0, 0, 0, 0);
+        if (row_ok) raw = *reinterpret_cast<const uint4*>(qrow + 8 * c);
+        const bf16* qv8 = reinterpret_cast<const bf16*>(&raw);
+        uint32_t wu[4], wv[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int d = 8 * c + 2 * k;
+          const float a0 = __bfloat162float(qv8[2 * k]), a1 = __bfloat162float(qv8[2 * k + 1]);
+          __nv_bfloat162 hu = __floats2bfloat162_rn(row_ok ? a0 + uh[d] : 0.f, row_ok ? a1 + uh[d + 1] : 0.f);
+          __nv_bfloat162 hv = __floats2bfloat162_rn(row_ok ? a0 + vh[d] : 0.f, row_ok ? a1 + vh[d + 1] : 0.f);
+          wu[k] = *reinterpret_cast<uint32_t*>(&hu);
+          wv[k] = *reinterpret_cast<uint32_t*>(&hv);
+        }
+        *reinterpret_cast<uint4*>(sQu + sw128_off(r, c)) = make_uint4(wu[0], wu[1], wu[2], wu[3]);
+        *reinterpret_cast<uint4*>(sQv + sw128_off(r, c)) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // visible to the tensor cores
+      __syncwarp();
+      if (lane == 0) mbar_arrive(q_ready);
+    }
+
+    float* stg = sBD + (warp - 2) * 32 * BD_LD;
+    const float sl2 = 1.4426950408889634f * 0.125f;   // log2(e) / sqrt(64)
+    float m_run = -INFINITY, l_run = 0.f;
+    float o[AHD];
+#pragma unroll
+    for (int d = 0; d < AHD; ++d) o[d] = 0.f;
+    bool ok = true;
+    for (int t = 0; t < T; ++t) {
+      const int j0 = t * AK;
+      if (!mbar_wait(s_full, t & 1, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      float sc[AK];
+      {
+        uint32_t v[16];
+#pragma unroll
+        for (int hq = 0; hq < AK / 16; ++hq) {
+          tmem_ld16(tmem + lane_base + 16 * hq, v);
+#pragma unroll
+          for (int k = 0; k < 16; ++k) sc[16 * hq + k] = __uint_as_float(v[k]);
+        }
+        // this warp's BD band: columns 32q .. 32q + 95 of BD, one row per lane
+#pragma unroll
+        for (int hq = 0; hq < 6; ++hq) {
+          tmem_ld16(tmem + lane_base + (uint32_t)(AK + 32 * q + 16 * hq), v);
+#pragma unroll
+          for (int k = 0; k < 16; k += 4)
+            *reinterpret_cast<float4*>(stg + lane * BD_LD + 16 * hq + k) =
+                make_float4(__uint_as_float(v[k]), __uint_as_float(v[k + 1]), __uint_as_float(v[k + 2]),
+                            __uint_as_float(v[k + 3]));
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_free);   // AC / BD of tile t read out of TMEM
+      // key c of row r: BD column r - c + 63 = staged column lane + 63 - c
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < AK; ++c) {
+        float x = (sc[c] + stg[lane * (BD_LD + 1) + (AK - 1) - c]) * sl2;
+        if (j0 + c >= S) x = -INFINITY;
+        sc[c] = x;
+        mx = fmaxf(mx, x);
+      }
+      const float m_new = fmaxf(m_run, mx);   // finite: key j0 < S
+      const float alpha = exp2f(m_run - m_new);
+      float ps = 0.f;
+#pragma unroll
+      for (int c = 0; c < AK; ++c) {
+        sc[c] = exp2f(sc[c] - m_new);
+        ps += sc[c];
+      }
+      l_run = l_run * alpha + ps;
+      m_run = m_new;
+      // P row as bf16 into the swizzled A tile of P.V (buffer t % 2; its
+      // previous tile's P.V completed before iteration t - 1 read its result)
+      uint8_t* pt = sP + (t & 1) * L::P_BYTES;
+#pragma unroll
+      for (int ch = 0; ch < AK / 8; ++ch) {
+        uint32_t w4[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          __nv_bfloat162 hp = __floats2bfloat162_rn(sc[8 * ch + 2 * k], sc[8 * ch + 2 * k + 1]);
+          w4[k] = *reinterpret_cast<uint32_t*>(&hp);
+        }
+        *reinterpret_cast<uint4*>(pt + sw128_off(r, ch)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[t & 1]);
+      // O (relative to m_(t-1)) += P_(t-1) V_(t-1), then rescale to m_t
+      if (t > 0) {
+        const int pb = (t - 1) & 1;
+        if (!mbar_wait(&pv_full[pb], ((t - 1) >> 1) & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t v[16];
+#pragma unroll
+        for (int hq = 0; hq < AHD / 16; ++hq) {
+          tmem_ld16(tmem + lane_base + (uint32_t)(256 + 64 * pb + 16 * hq), v);
+#pragma unroll
+          for (int k = 0; k < 16; ++k) o[16 * hq + k] = (o[16 * hq + k] + __uint_as_float(v[k])) * alpha;
+        }
+      }
+    }
+    if (ok && T > 0) {
+      const int pb = (T - 1) & 1;
+      if (mbar_wait(&pv_full[pb], ((T - 1) >> 1) & 1, abort_flag)) {
+        tc_fence_after();
+        uint32_t v[16];
+#pragma unroll
+        for (int hq = 0; hq < AHD / 16; ++hq) {
+          tmem_ld16(tmem + lane_base + (uint32_t)(256 + 64 * pb + 16 * hq), v);
+#pragma unroll
+          for (int k = 0; k < 16; ++k) o[16 * hq + k] += __uint_as_float(v[k]);
+        }
+      } else {
+        ok = false;
+      }
+    }
+    if (!ok) {
+      *abort_flag = 1;
+    } else if (row_ok) {
+      const float inv = 1.f / l_run;
+      uint4* dst = reinterpret_cast<uint4*>(ctx + (int64_t)(sb + i) * D + h * AHD);
+#pragma unroll
+      for (int c = 0; c < AHD / 8; ++c) {
+        uint32_t w4[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          __nv_bfloat162 ho = __floats2bfloat162_rn(o[8 * c + 2 * k] * inv, o[8 * c + 2 * k + 1] * inv);
+          w4[k] = *reinterpret_cast<uint32_t*>(&ho);
+        }
+        dst[c] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512u) : "memory");
+  }
+  if (threadIdx.x == 0 && *abort_flag) set_err(err, ERR_TIMEOUT);
+}
+
+cudaError_t launch_relpos_attention_tc(const bf16* qkv, const bf16* ptab, int R, const float* u, const float* v,
+                                       bf16* ctx, const SeqTable* seq, int n_tiles2, int M, int* err,
+                                       cudaStream_t st) {
+  if (M <= 0 || n_tiles2 <= 0) return cudaSuccess;
+  constexpr int D = 512;
+  CUtensorMap t_qkv, t_pos;
+  cudaError_t r = make_bf16_map_sw128(&t_qkv, qkv, M, 3 * D, 3 * D, AK);
+  if (r != cudaSuccess) return r;
+  r = make_bf16_map_sw128(&t_pos, ptab, 2 * R - 1, D, D, APW);
+  if (r != cudaSuccess) return r;
+  CK_LAUNCH(launch_k(attn_relpos_tc_kernel, dim3(n_tiles2, 8), dim3(192), AttTc::SMEM, st, t_qkv, t_pos, qkv, D, R, u,
+                     v, ctx, seq, err));
+  return cudaGetLastError();
+}
+
+cudaError_t attention_tc_init_attributes() {
+  return cudaFuncSetAttribute(attn_relpos_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, AttTc::SMEM);
+}
+
+}  // namespace sf

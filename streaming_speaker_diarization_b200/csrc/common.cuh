@@ -23,13 +23,15 @@ constexpr int MAX_SEQ = 512;   // sequences / streams per call
 constexpr int ATT_TILE = 64;   // query rows per attention CTA
 
 // Packed-sequence table in device memory: sequence s occupies rows
-// [off[s], off[s+1]) of the token matrix; its attention query tiles are
-// global tiles [tile_off[s], tile_off[s+1]).
+// [off[s], off[s+1]) of the token matrix; its 64-row attention query tiles
+// are global tiles [tile_off[s], tile_off[s+1]), its 128-row tiles
+// [tile2_off[s], tile2_off[s+1]).
 struct SeqTable {
   int n_seq;
   int total;
   int off[MAX_SEQ + 1];
   int tile_off[MAX_SEQ + 1];
+  int tile2_off[MAX_SEQ + 1];
 };
 
 template <typename T> __device__ __forceinline__ float to_f(T x);
@@ -60,6 +62,14 @@ __device__ __forceinline__ int seq_of_row(const SeqTable* __restrict__ st, int r
   while (lo < hi) {
     int mid = (lo + hi + 1) >> 1;
     if (st->off[mid] <= r) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+__device__ __forceinline__ int seq_of_tile2(const SeqTable* __restrict__ st, int g) {
+  int lo = 0, hi = st->n_seq - 1;
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if (st->tile2_off[mid] <= g) lo = mid; else hi = mid - 1;
   }
   return lo;
 }

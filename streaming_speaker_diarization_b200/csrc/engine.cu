@@ -161,6 +161,7 @@ struct sf_engine {
   int gemm_path = 1;      // bf16 GEMMs: tcgen05 with CTA pairs 1 = where faster (default), 2 = always,
                           // 3 = never; 0 = mma.sync
   int pair_bn = 0;        // CTA-pair tile width (0 = planned)
+  int attn_path = 1;      // bf16 relative-position attention: 1 = tcgen05, 0 = mma.sync
   float* d_split_ws = nullptr;   // split-K partial tiles of the tcgen05 GEMM
   int* d_split_cnt = nullptr;    // their per-tile arrival counters (kept at zero between launches)
   TcScratch tc_scratch() const { return TcScratch{d_err, d_split_ws, SPLIT_WS_BYTES, d_split_cnt, SPLIT_CNT}; }
@@ -176,6 +177,7 @@ struct sf_engine {
   std::vector<cudaEvent_t> pool;
   size_t pool_used = 0;
   double att_s2 = 0;      // sum of squared sequence lengths of the current call
+  int att_tiles2 = 0;     // 128-row attention query tiles of the current call
   double ms_acc[K_COUNT] = {};   // event time already read back (graph replays)
   // CUDA graphs: one per launch shape, replayed; invalidated when the workspace moves
   bool use_graphs = true;
@@ -584,6 +586,21 @@ cudaError_t gemm_dispatch<bf16>(sf_engine* e, const bf16* A, int lda, const bf16
   return gemm_bf16_mma(A, lda, W, M, N, K, ep, st);
 }
 
+// Relative-position attention: the bf16 engine runs it on tcgen05 unless the
+// mma.sync kernel is selected (SF_OPT_ATTN_PATH = 0).
+template <typename T>
+cudaError_t relpos_attention(sf_engine* e, const T* qkv, const T* ptab, const float* pu, const float* pv, T* ctx,
+                             const SeqTable* seq, int n_tiles, int M, cudaStream_t st) {
+  return launch_relpos_attention<T>(qkv, ptab, e->R, pu, pv, ctx, seq, n_tiles, M, st);
+}
+template <>
+cudaError_t relpos_attention<bf16>(sf_engine* e, const bf16* qkv, const bf16* ptab, const float* pu, const float* pv,
+                                   bf16* ctx, const SeqTable* seq, int n_tiles, int M, cudaStream_t st) {
+  if (e->attn_path == 1)
+    return launch_relpos_attention_tc(qkv, ptab, e->R, pu, pv, ctx, seq, e->att_tiles2, M, e->d_err, st);
+  return launch_relpos_attention<bf16>(qkv, ptab, e->R, pu, pv, ctx, seq, n_tiles, M, st);
+}
+
 template <typename T>
 cudaError_t gemm_acc(sf_engine* e, const T* A, int lda, const T* W, int M, int N, int K, const Epi& ep,
                      cudaStream_t st) {
@@ -640,7 +657,7 @@ cudaError_t run_graph(sf_engine* e, std::string key, cudaStream_t st, F&& enqueu
   if (!e->use_graphs) return enqueue(st);
   key += e->prof ? "|p" + std::to_string(e->prof_mask) : "|n";
   key += e->use_pdl ? "|pdl" : "";
-  key += "|g" + std::to_string(e->gemm_path) + "." + std::to_string(e->pair_bn);
+  key += "|g" + std::to_string(e->gemm_path) + "." + std::to_string(e->pair_bn) + "|a" + std::to_string(e->attn_path);
   auto it = e->graphs.find(key);
   if (it != e->graphs.end() && it->second.gen != e->ws_gen) {
     cudaGraphExecDestroy(it->second.exec);
@@ -724,14 +741,18 @@ void fill_seq(DescBlock* d, const std::vector<int>& lens, int& M, int& tiles) {
   d->seq.n_seq = (int)lens.size();
   M = 0;
   tiles = 0;
+  int tiles2 = 0;
   for (size_t i = 0; i < lens.size(); ++i) {
     d->seq.off[i] = M;
     d->seq.tile_off[i] = tiles;
+    d->seq.tile2_off[i] = tiles2;
     M += lens[i];
     tiles += (lens[i] + ATT_TILE - 1) / ATT_TILE;
+    tiles2 += (lens[i] + 2 * ATT_TILE - 1) / (2 * ATT_TILE);
   }
   d->seq.off[lens.size()] = M;
   d->seq.tile_off[lens.size()] = tiles;
+  d->seq.tile2_off[lens.size()] = tiles2;
   d->seq.total = M;
 }
 
@@ -798,7 +819,7 @@ cudaError_t run_encode(sf_engine* e, int M, int n_tiles, float* probs, cudaStrea
         launch_layernorm<T>(x, w.att_g, w.att_b, M, D, false, h, st));
     CK(gemm_acc<T>(e, h, D, w.wqkv, M, 3 * D, D, epi(EPI_BIAS, w.bqkv, big, 3 * D), st));
     RUN(K_ATT_REL, 1, 6.0 * e->att_s2 * D, (double)M * 4 * D * sizeof(T),
-        launch_relpos_attention<T>(big, w.ptab, e->R, w.pu, w.pv, ctx, seq, n_tiles, M, st));
+        relpos_attention<T>(e, big, w.ptab, w.pu, w.pv, ctx, seq, n_tiles, M, st));
     CK(gemm_acc<T>(e, ctx, D, w.wo, M, D, D, epi(EPI_RESID, w.bo, x, D, 1.f), st));
     RUN(K_LN, 1, 0, (double)M * D * (4 + sizeof(T)),
         launch_layernorm<T>(x, w.conv_g, w.conv_b, M, D, false, h, st));
@@ -879,6 +900,7 @@ cudaError_t offline_impl(sf_engine* e, const float* d_audio, const std::vector<i
   int M, tiles;
   fill_seq(d, tp, M, tiles);
   e->att_s2 = sum_sq(tp);
+  e->att_tiles2 = d->seq.tile2_off[d->seq.n_seq];
   const int T3 = (int)enc_frames(L_max);
   const int Tp_max = (int)enc_frames(n_max / 160);
   CK(ensure(e->mel, (size_t)B * 128 * T_cols * 4));
@@ -1007,6 +1029,7 @@ sf_status sf_create(const void* blob, uint64_t nbytes, const sf_config* cfg, sf_
   cudaError_t ce;
   if ((ce = gemm_init_attributes()) != cudaSuccess) return cuda_fail(e.get(), ce, "init"), SF_ECUDA;
   if ((ce = attention_init_attributes()) != cudaSuccess) return SF_ECUDA;
+  if ((ce = attention_tc_init_attributes()) != cudaSuccess) return SF_ECUDA;
   if ((ce = gemm_tc_init_attributes()) != cudaSuccess) return SF_ECUDA;
   if ((ce = frontend_init_attributes()) != cudaSuccess) return SF_ECUDA;
   if ((ce = attention_init_f32_attributes(e->R)) != cudaSuccess) return SF_ECUDA;
@@ -1195,6 +1218,7 @@ sf_status sf_encode(sf_engine* e, const void* d_embs, const int* h_seq_len, int 
   int M, tiles;
   fill_seq(d, lens, M, tiles);
   e->att_s2 = sum_sq(lens);
+  e->att_tiles2 = d->seq.tile2_off[d->seq.n_seq];
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
   cudaError_t ce = ensure_encode_ws(e, M);
   if (ce == cudaSuccess) ce = desc_upload(e, st);
@@ -1240,6 +1264,34 @@ sf_status sf_gemm_bf16(sf_engine* e, const void* d_A, int lda, const void* d_W, 
   return SF_OK;
 }
 
+sf_status sf_attention_relpos(sf_engine* e, const void* d_qkv, const void* d_ptab, int R, const float* d_u,
+                              const float* d_v, const int* h_seq_len, int n, void* d_ctx, int path,
+                              void* cuda_stream) {
+  if (check_engine(e) != SF_OK) return SF_EINVAL;
+  if (!d_qkv || !d_ptab || !d_u || !d_v || !h_seq_len || !d_ctx) return fail(e, SF_EINVAL, "null pointer argument");
+  if (e->cfg.precision != SF_BF16) return fail(e, SF_ESTATE, "sf_attention_relpos needs a bf16 engine");
+  if (n < 1 || n > MAX_SEQ || (path != 0 && path != 1) || R < 1) return fail(e, SF_ESHAPE, "sequence count, path or R");
+  if ((reinterpret_cast<uintptr_t>(d_qkv) | reinterpret_cast<uintptr_t>(d_ptab) | reinterpret_cast<uintptr_t>(d_ctx)) & 15)
+    return fail(e, SF_EINVAL, "qkv, ptab and ctx must be 16-byte aligned");
+  std::vector<int> lens(h_seq_len, h_seq_len + n);
+  for (int v : lens)
+    if (v < 1 || v > R) return fail(e, SF_ESHAPE, "sequence length must be in [1, R]");
+  DescBlock* d = desc_begin(e);
+  int M, tiles;
+  fill_seq(d, lens, M, tiles);
+  const int tiles2 = d->seq.tile2_off[n];
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  cudaError_t ce = desc_upload(e, st);
+  const bf16* qkv = static_cast<const bf16*>(d_qkv);
+  const bf16* ptab = static_cast<const bf16*>(d_ptab);
+  bf16* ctx = static_cast<bf16*>(d_ctx);
+  if (ce == cudaSuccess)
+    ce = path == 1 ? launch_relpos_attention_tc(qkv, ptab, R, d_u, d_v, ctx, &e->d_desc->seq, tiles2, M, e->d_err, st)
+                   : launch_relpos_attention<bf16>(qkv, ptab, R, d_u, d_v, ctx, &e->d_desc->seq, tiles, M, st);
+  if (ce != cudaSuccess) return cuda_fail(e, ce, "sf_attention_relpos");
+  return SF_OK;
+}
+
 sf_status sf_set_option(sf_engine* e, int option, int value) {
   if (check_engine(e) != SF_OK) return SF_EINVAL;
   switch (option) {
@@ -1248,6 +1300,10 @@ sf_status sf_set_option(sf_engine* e, int option, int value) {
     case SF_OPT_GEMM_PATH:
       if (value < 0 || value > 3) return fail(e, SF_EINVAL, "gemm path must be 0, 1, 2 or 3");
       e->gemm_path = value;
+      break;
+    case SF_OPT_ATTN_PATH:
+      if (value != 0 && value != 1) return fail(e, SF_EINVAL, "attention path must be 0 or 1");
+      e->attn_path = value;
       break;
     case SF_OPT_GEMM_PAIR_BN:
       if (value != 0 && value != 128 && value != 192 && value != 256)
@@ -1360,6 +1416,7 @@ void fill_step(sf_stream* s, DescBlock* d, const StepPlan& pl, int& M, int& tile
   }
   fill_seq(d, lens, M, tiles);
   s->e->att_s2 = sum_sq(lens);
+  s->e->att_tiles2 = d->seq.tile2_off[d->seq.n_seq];
 }
 
 // Host bookkeeping after a state update (sizes are data-independent).
@@ -1404,7 +1461,8 @@ cudaError_t stream_step_impl(sf_stream* s, const float* d_feats, int64_t t_buf, 
   CK(ensure_encode_ws(e, M));
   CK(prep_pre_encode(e, n, W_max, sizeof(T)));
   std::string key = "st|" + std::to_string(reinterpret_cast<uintptr_t>(s)) + "|" + std::to_string(n) + "|" +
-                    std::to_string(M) + "|" + std::to_string(tiles) + "|" + std::to_string(W_max) + "|" +
+                    std::to_string(M) + "|" + std::to_string(tiles) + "|" + std::to_string(e->att_tiles2) + "|" +
+                    std::to_string(W_max) + "|" +
                     std::to_string(t_buf) + "|" + std::to_string(reinterpret_cast<uintptr_t>(d_feats)) + "|" +
                     std::to_string(reinterpret_cast<uintptr_t>(d_chunk_probs));
   return run_graph(e, key, st, [&](cudaStream_t st) -> cudaError_t {

@@ -1,5 +1,6 @@
 // Launchers of the engine's kernels (host-callable, stream-ordered).
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -48,6 +49,9 @@ struct TcScratch {
 cudaError_t gemm_bf16_tc(const bf16* A, int lda, const bf16* W, int M, int N, int K, const Epi& e,
                          const TcScratch& sc, cudaStream_t st);
 cudaError_t gemm_tc_init_attributes();
+// 2-D bf16 tensor map (row-major [rows x cols], row stride ld elements), box
+// box_rows x 64 columns, 128-byte swizzle, zero fill outside the matrix.
+cudaError_t make_bf16_map_sw128(CUtensorMap* m, const void* base, int rows, int cols, int ld, int box_rows);
 // Multi-wave bf16 GEMMs on the CTA-pair (cta_group::2) kernel: 0 never, 1
 // where it is faster (K >= 1024, N >= 256), 2 always; set from the calling
 // engine's options at each API entry.
@@ -107,5 +111,12 @@ cudaError_t launch_relpos_attention(const T* qkv, const T* ptab, int R, const fl
 template <typename T>
 cudaError_t launch_mha(const T* qkv, T* ctx, const SeqTable* seq, int n_tiles, int M, cudaStream_t st);
 cudaError_t attention_init_attributes();
+// bf16 relative-position MHSA on tcgen05 (one CTA per 128 query rows x head;
+// n_tiles2 = 128-row tiles of the sequence table); err gets ERR_TIMEOUT if
+// a bounded wait gives up.
+cudaError_t launch_relpos_attention_tc(const bf16* qkv, const bf16* ptab, int R, const float* u, const float* v,
+                                       bf16* ctx, const SeqTable* seq, int n_tiles2, int M, int* err,
+                                       cudaStream_t st);
+cudaError_t attention_tc_init_attributes();
 
 }  // namespace sf
