@@ -10,10 +10,13 @@
 //   AC = (Q+u) K^T    M 128, N  64, K 64   TMEM columns [0, 64)
 //   BD = (Q+v) Pw^T   M 128, N 192, K 64   TMEM columns [64, 256)
 //        Pw = position-table rows for distances i0 - j0 - 63 .. i0 - j0 + 128,
-//        i.e. every i - j of the tile (row r, key c: BD column r - c + 63)
+//        i.e. every i - j of the tile (row r, key c: BD column r - c + 63),
+//        as three 64-row blocks; consecutive key tiles share two of them, so
+//        each tile loads one new block (three N = 64 MMAs, one per block)
 //   O_t = P V         M 128, N  64, K 64   TMEM columns 256 + 64 (t % 2)
-// Warps: 0 loads K, V and Pw with TMA into a two-stage ring; 1 issues the
-// MMAs (one thread); 2-5 run the softmax, thread = query row = TMEM lane.  A
+// Warps: 0 loads K and V (three-stage ring) and the position blocks (five-
+// slot ring) with TMA; 1 issues the MMAs (one thread); 2-5 run the softmax,
+// thread = query row = TMEM lane.  A
 // warp's 32 rows need a 96-column band of BD; it is staged in shared memory
 // (row stride 100 floats: conflict-free by rows and along the diagonal) and
 // read back at column r - c + 63.  The softmax is online in the exp2 domain
@@ -32,25 +35,27 @@ constexpr int AQ = 128;      // query rows per CTA
 constexpr int AK = 64;       // keys per tile
 constexpr int AHD = 64;      // head dim
 constexpr int APW = 192;     // position-table rows per tile (distances r - c)
-constexpr int ANB = 2;       // K / V / Pw ring stages
+constexpr int ANB = 3;       // K / V ring stages
+constexpr int NPW = ANB + 2; // 64-row position blocks held (tile t reads blocks t - 2 .. t)
 constexpr int BD_LD = 100;   // staged BD row stride (floats)
 
 struct AttTc {
   static constexpr int Q_BYTES = AQ * AHD * 2;      // 16 KB, K-major, 128-byte swizzle
   static constexpr int K_BYTES = AK * AHD * 2;      //  8 KB
   static constexpr int V_BYTES = AK * AHD * 2;      //  8 KB (MN-major B operand)
-  static constexpr int PW_BYTES = APW * AHD * 2;    // 24 KB
-  static constexpr int STAGE = K_BYTES + V_BYTES + PW_BYTES;
+  static constexpr int PB_BYTES = 64 * AHD * 2;     //  8 KB position block
+  static constexpr int STAGE = K_BYTES + V_BYTES;
   static constexpr int P_BYTES = AQ * AK * 2;       // 16 KB
   static constexpr int OFF_QU = 0;
   static constexpr int OFF_QV = Q_BYTES;
   static constexpr int OFF_RING = 2 * Q_BYTES;
-  static constexpr int OFF_P = OFF_RING + ANB * STAGE;
+  static constexpr int OFF_PW = OFF_RING + ANB * STAGE;
+  static constexpr int OFF_P = OFF_PW + NPW * PB_BYTES;
   static constexpr int OFF_BD = OFF_P + 2 * P_BYTES;
   static constexpr int BD_BYTES = 4 * 32 * BD_LD * 4;
   static constexpr int OFF_BAR = OFF_BD + BD_BYTES;
   static constexpr int SMEM = 1024 + OFF_BAR + 256;
-  static_assert(STAGE % 1024 == 0 && OFF_P % 1024 == 0 && OFF_RING % 1024 == 0, "swizzled tiles 1024-aligned");
+  static_assert(STAGE % 1024 == 0 && OFF_P % 1024 == 0 && OFF_PW % 1024 == 0, "swizzled tiles 1024-aligned");
   static_assert(SMEM <= 232448, "shared memory per CTA");
 };
 
@@ -90,9 +95,11 @@ __global__ void __launch_bounds__(192, 1) attn_relpos_tc_kernel(const __grid_con
   uint8_t* sRing = sm + L::OFF_RING;
   uint8_t* sP = sm + L::OFF_P;
   float* sBD = reinterpret_cast<float*>(sm + L::OFF_BD);
-  uint64_t* kv_full = reinterpret_cast<uint64_t*>(sm + L::OFF_BAR);   // [ANB]
+  uint8_t* sPw = sm + L::OFF_PW;
+  uint64_t* kv_full = reinterpret_cast<uint64_t*>(sm + L::OFF_BAR);   // [ANB] K, V (+ new position blocks)
   uint64_t* kv_empty = kv_full + ANB;                                  // [ANB]
-  uint64_t* s_full = kv_empty + ANB;
+  uint64_t* pw_empty = kv_empty + ANB;                                 // [NPW]
+  uint64_t* s_full = pw_empty + NPW;
   uint64_t* s_free = s_full + 1;
   uint64_t* p_full = s_free + 1;                                       // [2]
   uint64_t* pv_full = p_full + 2;                                      // [2]
@@ -114,6 +121,7 @@ __global__ void __launch_bounds__(192, 1) attn_relpos_tc_kernel(const __grid_con
       mbar_init(&kv_full[b], 1);
       mbar_init(&kv_empty[b], 1);
     }
+    for (int b = 0; b < NPW; ++b) mbar_init(&pw_empty[b], 1);
     mbar_init(s_full, 1);
     mbar_init(s_free, 4);
     for (int b = 0; b < 2; ++b) {
@@ -147,12 +155,23 @@ __global__ void __launch_bounds__(192, 1) attn_relpos_tc_kernel(const __grid_con
           *abort_flag = 1;
           break;
         }
+        // position block k = distances i0 - 64k - 63 .. i0 - 64k, slot (k + 2) % NPW;
+        // tile 0 brings blocks -2, -1, 0, tile t > 0 block t
+        const int k_lo = t == 0 ? -2 : t;
+        bool got = true;
+        for (int k = k_lo; k <= t && got; ++k)
+          got = mbar_wait(&pw_empty[(k + 2) % NPW], (((k + 2) / NPW) & 1) ^ 1, abort_flag);
+        if (!got) {
+          *abort_flag = 1;
+          break;
+        }
         uint8_t* st = sRing + b * L::STAGE;
-        mbar_expect_tx(&kv_full[b], L::STAGE);
+        mbar_expect_tx(&kv_full[b], L::STAGE + (t - k_lo + 1) * L::PB_BYTES);
         tma_load_2d(st, &t_qkv, &kv_full[b], D + h * AHD, sb + j0);                       // K rows j0 ..
         tma_load_2d(st + L::K_BYTES, &t_qkv, &kv_full[b], 2 * D + h * AHD, sb + j0);      // V rows j0 ..
-        tma_load_2d(st + L::K_BYTES + L::V_BYTES, &t_pos, &kv_full[b], h * AHD,
-                    i0 - j0 - (AK - 1) + R - 1);                                            // distances
+        for (int k = k_lo; k <= t; ++k)
+          tma_load_2d(sPw + ((k + 2) % NPW) * L::PB_BYTES, &t_pos, &kv_full[b], h * AHD,
+                      i0 - 64 * k - (AK - 1) + R - 1);
       }
       if (*abort_flag) {   // let this CTA's own loads land before its shared memory is released
         for (int k = t - ANB > 0 ? t - ANB : 0; k < t; ++k) {
@@ -166,7 +185,7 @@ __global__ void __launch_bounds__(192, 1) attn_relpos_tc_kernel(const __grid_con
     // ----------------------------------------------------------------- MMAs
     if (lane == 0) {
       constexpr uint32_t id_s = idesc_bf16_mn(AQ, AK, false);
-      constexpr uint32_t id_bd = idesc_bf16_mn(AQ, APW, false);
+      constexpr uint32_t id_bd = idesc_bf16_mn(AQ, 64, false);
       constexpr uint32_t id_pv = idesc_bf16_mn(AQ, AHD, true);
       const uint32_t tm_s = tmem, tm_bd = tmem + AK;
       const uint64_t dqu = sw128_desc(su32(sQu)), dqv = sw128_desc(su32(sQv));
@@ -190,13 +209,19 @@ __global__ void __launch_bounds__(192, 1) attn_relpos_tc_kernel(const __grid_con
         if (t > 0 && !mbar_wait(s_free, (t - 1) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
         uint8_t* st = sRing + b * L::STAGE;
-        const uint64_t dk = sw128_desc(su32(st)), dpw = sw128_desc(su32(st + L::K_BYTES + L::V_BYTES));
+        const uint64_t dk = sw128_desc(su32(st));
 #pragma unroll
         for (int k = 0; k < AHD / 16; ++k) umma_bf16(tm_s, dqu + (uint64_t)(2 * k), dk + (uint64_t)(2 * k), id_s, k != 0);
+        // BD columns 64 m .. 64 m + 63 <- position block t - m
 #pragma unroll
-        for (int k = 0; k < AHD / 16; ++k)
-          umma_bf16(tm_bd, dqv + (uint64_t)(2 * k), dpw + (uint64_t)(2 * k), id_bd, k != 0);
+        for (int m = 0; m < 3; ++m) {
+          const uint64_t dpw = sw128_desc(su32(sPw + ((t - m + 2 + NPW) % NPW) * L::PB_BYTES));
+#pragma unroll
+          for (int k = 0; k < AHD / 16; ++k)
+            umma_bf16(tm_bd + 64 * m, dqv + (uint64_t)(2 * k), dpw + (uint64_t)(2 * k), id_bd, k != 0);
+        }
         umma_commit(s_full);
+        umma_commit(&pw_empty[t % NPW]);   // block t - 2 is read for the last time by tile t
         if (t > 0 && !issue_pv(t - 1)) { ok = false; break; }
       }
       if (ok && T > 0) ok = issue_pv(T - 1);
@@ -209,6 +234,10 @@ __global__ void __launch_bounds__(192, 1) attn_relpos_tc_kernel(const __grid_con
     const int i = i0 + r;
     const bool row_ok = i < S;
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+    // bounded wait with a warp-uniform outcome (the tcgen05.ld that follow are warp-collective)
+    auto warp_wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+    };
     // (Q + u) and (Q + v) rows, rounded to bf16, into the swizzled A tiles
     {
       const bf16* qrow = qkv + (int64_t)(sb + (row_ok ? i : 0)) * (3 * D) + h * AHD;
@@ -246,27 +275,28 @@ __global__ void __launch_bounds__(192, 1) attn_relpos_tc_kernel(const __grid_con
     bool ok = true;
     for (int t = 0; t < T; ++t) {
       const int j0 = t * AK;
-      if (!mbar_wait(s_full, t & 1, abort_flag)) { ok = false; break; }
+      if (!warp_wait(s_full, t & 1)) { ok = false; break; }
       tc_fence_after();
       float sc[AK];
       {
-        uint32_t v[16];
-#pragma unroll
-        for (int hq = 0; hq < AK / 16; ++hq) {
-          tmem_ld16(tmem + lane_base + 16 * hq, v);
-#pragma unroll
-          for (int k = 0; k < 16; ++k) sc[16 * hq + k] = __uint_as_float(v[k]);
-        }
         // this warp's BD band: columns 32q .. 32q + 95 of BD, one row per lane
+        // (wide TMEM loads: one wait per load instruction)
+        uint32_t v[64];
+        tmem_ld64(tmem + lane_base + (uint32_t)(AK + 32 * q), v);
 #pragma unroll
-        for (int hq = 0; hq < 6; ++hq) {
-          tmem_ld16(tmem + lane_base + (uint32_t)(AK + 32 * q + 16 * hq), v);
+        for (int k = 0; k < 64; k += 4)
+          *reinterpret_cast<float4*>(stg + lane * BD_LD + k) =
+              make_float4(__uint_as_float(v[k]), __uint_as_float(v[k + 1]), __uint_as_float(v[k + 2]),
+                          __uint_as_float(v[k + 3]));
+        tmem_ld32(tmem + lane_base + (uint32_t)(AK + 32 * q + 64), v);
 #pragma unroll
-          for (int k = 0; k < 16; k += 4)
-            *reinterpret_cast<float4*>(stg + lane * BD_LD + 16 * hq + k) =
-                make_float4(__uint_as_float(v[k]), __uint_as_float(v[k + 1]), __uint_as_float(v[k + 2]),
-                            __uint_as_float(v[k + 3]));
-        }
+        for (int k = 0; k < 32; k += 4)
+          *reinterpret_cast<float4*>(stg + lane * BD_LD + 64 + k) =
+              make_float4(__uint_as_float(v[k]), __uint_as_float(v[k + 1]), __uint_as_float(v[k + 2]),
+                          __uint_as_float(v[k + 3]));
+        tmem_ld64(tmem + lane_base, v);
+#pragma unroll
+        for (int k = 0; k < AK; ++k) sc[k] = __uint_as_float(v[k]);
       }
       tc_fence_before();
       __syncwarp();
@@ -310,28 +340,22 @@ __global__ void __launch_bounds__(192, 1) attn_relpos_tc_kernel(const __grid_con
       // O (relative to m_(t-1)) += P_(t-1) V_(t-1), then rescale to m_t
       if (t > 0) {
         const int pb = (t - 1) & 1;
-        if (!mbar_wait(&pv_full[pb], ((t - 1) >> 1) & 1, abort_flag)) { ok = false; break; }
+        if (!warp_wait(&pv_full[pb], ((t - 1) >> 1) & 1)) { ok = false; break; }
         tc_fence_after();
-        uint32_t v[16];
+        uint32_t v[AHD];
+        tmem_ld64(tmem + lane_base + (uint32_t)(256 + 64 * pb), v);
 #pragma unroll
-        for (int hq = 0; hq < AHD / 16; ++hq) {
-          tmem_ld16(tmem + lane_base + (uint32_t)(256 + 64 * pb + 16 * hq), v);
-#pragma unroll
-          for (int k = 0; k < 16; ++k) o[16 * hq + k] = (o[16 * hq + k] + __uint_as_float(v[k])) * alpha;
-        }
+        for (int k = 0; k < AHD; ++k) o[k] = (o[k] + __uint_as_float(v[k])) * alpha;
       }
     }
     if (ok && T > 0) {
       const int pb = (T - 1) & 1;
-      if (mbar_wait(&pv_full[pb], ((T - 1) >> 1) & 1, abort_flag)) {
+      if (warp_wait(&pv_full[pb], ((T - 1) >> 1) & 1)) {
         tc_fence_after();
-        uint32_t v[16];
+        uint32_t v[AHD];
+        tmem_ld64(tmem + lane_base + (uint32_t)(256 + 64 * pb), v);
 #pragma unroll
-        for (int hq = 0; hq < AHD / 16; ++hq) {
-          tmem_ld16(tmem + lane_base + (uint32_t)(256 + 64 * pb + 16 * hq), v);
-#pragma unroll
-          for (int k = 0; k < 16; ++k) o[16 * hq + k] += __uint_as_float(v[k]);
-        }
+        for (int k = 0; k < AHD; ++k) o[k] += __uint_as_float(v[k]);
       } else {
         ok = false;
       }
@@ -370,7 +394,7 @@ cudaError_t launch_relpos_attention_tc(const bf16* qkv, const bf16* ptab, int R,
   CUtensorMap t_qkv, t_pos;
   cudaError_t r = make_bf16_map_sw128(&t_qkv, qkv, M, 3 * D, 3 * D, AK);
   if (r != cudaSuccess) return r;
-  r = make_bf16_map_sw128(&t_pos, ptab, 2 * R - 1, D, D, APW);
+  r = make_bf16_map_sw128(&t_pos, ptab, 2 * R - 1, D, D, 64);
   if (r != cudaSuccess) return r;
   CK_LAUNCH(launch_k(attn_relpos_tc_kernel, dim3(n_tiles2, 8), dim3(192), AttTc::SMEM, st, t_qkv, t_pos, qkv, D, R, u,
                      v, ctx, seq, err));

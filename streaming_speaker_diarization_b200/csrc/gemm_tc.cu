@@ -56,13 +56,13 @@ __device__ __forceinline__ void epilogue_tile(const Epi& e, uint32_t tmem, float
   const int l4 = lane % LPR, rh = lane / LPR;
 #pragma unroll 1
   for (int c0 = cbeg; c0 < cend; c0 += CW) {
-    uint32_t v[16];
+    {
+      uint32_t v[CW];   // one wide TMEM load (one wait) per chunk
+      if (CW == 64) tmem_ld64(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)c0, v);
+      else tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)c0, v);
 #pragma unroll
-    for (int h = 0; h < CW / 16; ++h) {
-      tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(c0 + 16 * h), v);
-#pragma unroll
-      for (int j = 0; j < 16; j += 4)
-        *reinterpret_cast<float4*>(stage + lane * LD + 16 * h + j) =
+      for (int j = 0; j < CW; j += 4)
+        *reinterpret_cast<float4*>(stage + lane * LD + j) =
             make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]), __uint_as_float(v[j + 2]),
                         __uint_as_float(v[j + 3]));
     }
