@@ -72,6 +72,14 @@ __device__ __forceinline__ uint64_t sw128_desc_mn(uint32_t saddr) {
   return d;
 }
 
+// 2^x with the hardware approximation (ex2.approx.ftz.f32: relative error
+// ~2^-22, far inside the bf16 rounding of P; 2^-inf = 0).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // Byte offset of element (row, col) (col in bf16 units, < 64) of a K-major
 // tile with 128-byte rows and the 128-byte swizzle (16-byte chunk index
 // XOR row % 8), as TMA writes it and tcgen05 reads it.
@@ -303,19 +311,28 @@ __global__ void __launch_bounds__(192, 1) attn_relpos_tc_kernel(const __grid_con
       if (lane == 0) mbar_arrive(s_free);   // AC / BD of tile t read out of TMEM
       // key c of row r: BD column r - c + 63 = staged column lane + 63 - c
       float mx = -INFINITY;
+      if (j0 + AK <= S) {
 #pragma unroll
-      for (int c = 0; c < AK; ++c) {
-        float x = (sc[c] + stg[lane * (BD_LD + 1) + (AK - 1) - c]) * sl2;
-        if (j0 + c >= S) x = -INFINITY;
-        sc[c] = x;
-        mx = fmaxf(mx, x);
+        for (int c = 0; c < AK; ++c) {
+          const float x = (sc[c] + stg[lane * (BD_LD + 1) + (AK - 1) - c]) * sl2;
+          sc[c] = x;
+          mx = fmaxf(mx, x);
+        }
+      } else {   // last tile: keys past the sequence end get no weight
+#pragma unroll
+        for (int c = 0; c < AK; ++c) {
+          float x = (sc[c] + stg[lane * (BD_LD + 1) + (AK - 1) - c]) * sl2;
+          if (j0 + c >= S) x = -INFINITY;
+          sc[c] = x;
+          mx = fmaxf(mx, x);
+        }
       }
       const float m_new = fmaxf(m_run, mx);   // finite: key j0 < S
-      const float alpha = exp2f(m_run - m_new);
+      const float alpha = ex2_approx(m_run - m_new);
       float ps = 0.f;
 #pragma unroll
       for (int c = 0; c < AK; ++c) {
-        sc[c] = exp2f(sc[c] - m_new);
+        sc[c] = ex2_approx(sc[c] - m_new);
         ps += sc[c];
       }
       l_run = l_run * alpha + ps;

@@ -119,6 +119,19 @@ __device__ __forceinline__ void epilogue_tile(const Epi& e, uint32_t tmem, float
   }
 }
 
+// A residual epilogue reads the f32 block it updates: ask L2 for this warp's
+// share (rows r0 .. r0 + nrows, columns c0 .. c0 + ncols) while the
+// accumulator is still being computed, so the epilogue's loads hit L2.
+__device__ __forceinline__ void prefetch_resid(const Epi& e, int M, int N, int r0, int nrows, int c0, int ncols,
+                                               int lane) {
+  if (e.kind != EPI_RESID) return;
+  const int lpr = (ncols + 31) / 32;   // 128-byte lines per row
+  for (int k = lane; k < nrows * lpr; k += 32) {
+    const int r = r0 + k / lpr, c = c0 + (k % lpr) * 32;
+    if (r < M && c < N) asm volatile("prefetch.global.L2 [%0];" ::"l"(epi_f32_ptr(e, r, c)));
+  }
+}
+
 // Split-K finish: sum the S partial tiles (fixed order z = 0 .. S-1, so the
 // result does not depend on which CTA arrives last) and apply the epilogue.
 template <int EK, int BN>
@@ -258,6 +271,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
     const int q = warp & 3;            // TMEM lane quarter this warp may access
     float* stage = reinterpret_cast<float*>(sm) + q * (32 * 68);
     volatile int* last_flag = abort_flag + 1;
+    prefetch_resid(e, M, N, m0 + 32 * q, 32, n0, BN, lane);
     if (mbar_wait(accf, 0, abort_flag) && !*abort_flag) {
       tc_fence_after();
       const int tile = blockIdx.y * gridDim.x + blockIdx.x;
@@ -435,12 +449,13 @@ __global__ void __launch_bounds__(320, 1) gemm_tcp_kernel(const __grid_constant_
     int i = 0;
     for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++i) {
       const int a = i & 1, u = i >> 1;
+      const int m0 = (tile / tiles_n) * TC_BM, n0 = (tile % tiles_n) * BN;
+      prefetch_resid(e, M, N, m0 + 32 * q, 32, n0 + hc * BN / 2, BN / 2, lane);
       if (!mbar_wait(&accf[a], u & 1, abort_flag) || *abort_flag) {
         *abort_flag = 1;
         break;
       }
       tc_fence_after();
-      const int m0 = (tile / tiles_n) * TC_BM, n0 = (tile % tiles_n) * BN;
       const uint32_t acc = tmem + (uint32_t)(a * BN);
       const int cb = hc * BN / 2, ce = cb + BN / 2;
       switch (e.kind) {
@@ -664,12 +679,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
     int i = 0;
     for (int tile = pair; tile < tiles; tile += npairs, ++i) {
       const int a = i & 1, u = i >> 1;
+      const int m0 = (tile / tiles_n) * PAIR_BM + TC_BM * (int)rank, n0 = (tile % tiles_n) * BN;
+      prefetch_resid(e, M, N, m0 + 32 * q, 32, n0 + hc * BN / 2, BN / 2, lane);
       if (!mbar_wait(&accf[a], u & 1, abort_flag) || *abort_flag) {
         *abort_flag = 1;
         break;
       }
       tc_fence_after();
-      const int m0 = (tile / tiles_n) * PAIR_BM + TC_BM * (int)rank, n0 = (tile % tiles_n) * BN;
       const uint32_t acc = tmem + (uint32_t)(a * BN);
       const int cb = hc * BN / 2, ce = cb + BN / 2;
       switch (e.kind) {

@@ -1,0 +1,95 @@
+"""Kernel micro-benchmarks through the C ABI's single-op entry points.
+
+    python -m streaming_speaker_diarization_b200.kbench gemm M N K [--epi E] [--path P] [--reps R]
+    python -m streaming_speaker_diarization_b200.kbench attn N_SEQ LEN [--path P] [--reps R]
+
+`gemm` runs sf_gemm_bf16 (E: 1 f32 out, 2 bf16 out, 3 residual update, 4
+swish, 5 gated linear unit; P: SF_OPT_GEMM_PATH, 1 = tcgen05 with CTA pairs
+where faster, 2 = CTA pairs always, 3 = single CTAs, 0 = mma.sync); `attn`
+runs sf_attention_relpos on N_SEQ packed sequences of LEN rows (P: 1 tcgen05,
+0 mma.sync).  Operands are seeded random values on the device; three warm-up
+launches, then REPS launches queued behind a GPU sleep (so host launch
+overhead is hidden) and timed with CUDA events on the current stream.  Also
+the driver for single-kernel ncu captures (small REPS)."""
+from __future__ import annotations
+
+import argparse
+
+import numpy as np
+
+
+def _engine(b, max_batch):
+    from synth import TINY, make_weights, weights_blob
+    cfg = b.default_config(n_conformer=TINY.n_conformer, n_transformer=TINY.n_transformer, precision=1,
+                           max_batch=max_batch)
+    return b.sf_create(weights_blob(make_weights(TINY, seed=0)), cfg)
+
+
+def _time(torch, fn, reps):
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda._sleep(2_000_000)
+    s.record()
+    for _ in range(reps):
+        fn()
+    e.record()
+    torch.cuda.synchronize()
+    return s.elapsed_time(e) / reps
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    sub = ap.add_subparsers(dest="op", required=True)
+    g = sub.add_parser("gemm")
+    g.add_argument("M", type=int)
+    g.add_argument("N", type=int)
+    g.add_argument("K", type=int)
+    g.add_argument("--epi", type=int, default=2)
+    g.add_argument("--path", type=int, default=1)
+    g.add_argument("--reps", type=int, default=20)
+    a = sub.add_parser("attn")
+    a.add_argument("n_seq", type=int)
+    a.add_argument("length", type=int)
+    a.add_argument("--path", type=int, default=1)
+    a.add_argument("--reps", type=int, default=20)
+    args = ap.parse_args(argv)
+
+    import torch
+    from streaming_speaker_diarization_b200 import binding as b
+    gen = torch.Generator(device="cuda").manual_seed(0)
+    if args.op == "gemm":
+        eng = _engine(b, 8)
+        M, N, K = args.M, args.N, args.K
+        if args.path == 0:
+            args.epi = 1   # the mma.sync kernel writes f32 only
+        b.sf_set_option(eng, b.SF_OPT_GEMM_PATH, args.path)
+        A = torch.randn(M, K, device="cuda", generator=gen).to(torch.bfloat16)
+        W = torch.randn(N, K, device="cuda", generator=gen).to(torch.bfloat16)
+        cols = N // 2 if args.epi == 5 else N
+        C = torch.zeros(M, cols, device="cuda", dtype=torch.float32 if args.epi in (1, 3) else torch.bfloat16)
+        path = args.epi if args.path else 0   # sf_gemm_bf16 path: the epilogue, or 0 = mma.sync
+        ms = _time(torch, lambda: b.sf_gemm_bf16(eng, A, W, C, path=path), args.reps)
+        print(f"gemm M={M} N={N} K={K} epi={args.epi} path={args.path}: {ms * 1e3:.1f} us/launch, "
+              f"{2 * M * N * K / ms / 1e9:.1f} TFLOP/s")
+    else:
+        n, L = args.n_seq, args.length
+        eng = _engine(b, max(n, 8))
+        R = max(L, 756)
+        qkv = torch.randn(n * L, 1536, device="cuda", generator=gen).to(torch.bfloat16)
+        ptab = torch.randn(2 * R - 1, 512, device="cuda", generator=gen).to(torch.bfloat16)
+        u = 0.5 * torch.randn(512, device="cuda", generator=gen)
+        v = 0.5 * torch.randn(512, device="cuda", generator=gen)
+        ctx = torch.empty(n * L, 512, device="cuda", dtype=torch.bfloat16)
+        lens = np.full(n, L, np.int32)
+        ms = _time(torch, lambda: b.sf_attention_relpos(eng, qkv, ptab, R, u, v, lens, ctx, path=args.path), args.reps)
+        flops = 3 * 2 * n * L * L * 512
+        print(f"attn n={n} L={L} path={args.path}: {ms * 1e3:.1f} us/launch, {flops / ms / 1e9:.1f} TFLOP/s "
+              f"(3 x 2 x L^2 x 512 per sequence)")
+    b.sf_check(eng)
+    b.sf_destroy(eng)
+
+
+if __name__ == "__main__":
+    main()
