@@ -134,10 +134,18 @@ template <> struct Vec2<bf16> {
 };
 
 // Each thread: two channels x DW_ROWS consecutive rows; the DW_ROWS + K - 1
-// input rows they need are loaded once into registers.  Taps outside the
-// output row's sequence read as zero.
-constexpr int DW_ROWS = 8;
+// input rows they need are loaded once into registers (32-row blocks keep
+// the halo re-read at K - 1 rows per 32 and the weight loads amortised).
+// Taps outside the output row's sequence read as zero.  Swish: exact expf and
+// division for f32 outputs; for bf16 outputs the hardware exp2 and an
+// approximate reciprocal (relative error ~1e-7, far inside bf16 rounding).
+constexpr int DW_ROWS = 32;
 constexpr int DW_KMAX = 9;
+template <typename T>
+__device__ __forceinline__ float dw_swish(float a) {
+  if (sizeof(T) == 2) return a * __fdividef(1.f, 1.f + __expf(-a));
+  return a / (1.f + expf(-a));
+}
 template <typename T>
 __global__ void __launch_bounds__(128) dwconv1d_kernel(const T* __restrict__ in, T* __restrict__ out,
                                                        const float* __restrict__ w, const float* __restrict__ bias,
@@ -149,9 +157,9 @@ __global__ void __launch_bounds__(128) dwconv1d_kernel(const T* __restrict__ in,
   const int pad = (K - 1) / 2;
   float w0[DW_KMAX], w1[DW_KMAX];
 #pragma unroll
-  for (int j = 0; j < DW_KMAX; ++j) {
-    w0[j] = j < K ? w[c * K + j] : 0.f;
-    w1[j] = j < K ? w[(c + 1) * K + j] : 0.f;
+  for (int j = 0; j < DW_KMAX; ++j) {   // channels c, c + 1: 2K consecutive floats at c * K
+    w0[j] = j < K ? w[(int64_t)c * K + j] : 0.f;
+    w1[j] = j < K ? w[(int64_t)c * K + K + j] : 0.f;
   }
   const float b0 = bias[c], b1 = bias[c + 1];
   float x0[DW_ROWS + DW_KMAX - 1], x1[DW_ROWS + DW_KMAX - 1];
@@ -166,24 +174,36 @@ __global__ void __launch_bounds__(128) dwconv1d_kernel(const T* __restrict__ in,
     }
   }
   int s = seq_of_row(seq, r0 < M ? r0 : M - 1);
+  int sb = seq->off[s], se = seq->off[s + 1];
 #pragma unroll
   for (int k = 0; k < DW_ROWS; ++k) {
     const int r = r0 + k;
     if (r >= M) break;
-    while (r >= seq->off[s + 1]) ++s;
-    const int sb = seq->off[s], se = seq->off[s + 1];
+    if (r >= se) {   // next sequence (rows are packed sequence after sequence)
+      while (r >= seq->off[s + 1]) ++s;
+      sb = seq->off[s];
+      se = seq->off[s + 1];
+    }
     float a0 = b0, a1 = b1;
+    if (r - pad >= sb && r + pad < se) {   // interior row: every tap inside the sequence
 #pragma unroll
-    for (int j = 0; j < DW_KMAX; ++j) {
-      const int ri = r + j - pad;
-      if (j < K && ri >= sb && ri < se) {
-        a0 = fmaf(w0[j], x0[k + j], a0);
-        a1 = fmaf(w1[j], x1[k + j], a1);
+      for (int j = 0; j < DW_KMAX; ++j) {
+        if (j < K) {
+          a0 = fmaf(w0[j], x0[k + j], a0);
+          a1 = fmaf(w1[j], x1[k + j], a1);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < DW_KMAX; ++j) {
+        const int ri = r + j - pad;
+        if (j < K && ri >= sb && ri < se) {
+          a0 = fmaf(w0[j], x0[k + j], a0);
+          a1 = fmaf(w1[j], x1[k + j], a1);
+        }
       }
     }
-    a0 = a0 / (1.f + expf(-a0));
-    a1 = a1 / (1.f + expf(-a1));
-    Vec2<T>::store(out + (int64_t)r * D + c, a0, a1);
+    Vec2<T>::store(out + (int64_t)r * D + c, dw_swish<T>(a0), dw_swish<T>(a1));
   }
 }
 
