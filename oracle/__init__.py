@@ -26,3 +26,4 @@ from .model import (encoder_frames, subsample, rel_pos_table, rel_pos_mhsa, conf
                     transformer_layer, head, encode, forward_offline, layer_norm, W)
 from .streaming import (Preset, PRESETS, StreamState, compress_scores, select_topk,  # noqa: F401
                         compress_cache, stream_step, stream_run, state_update)
+from .postprocess import SegParams, binarize, speaker_segments, segments  # noqa: F401
