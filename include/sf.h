@@ -282,6 +282,45 @@ SF_API sf_status sf_stream_update(sf_stream* s, const float* d_preds, const void
 SF_API sf_status sf_select_topk(sf_engine* e, const float* d_scores, const int* h_n, int n_sets, int stride, int k,
                          int* d_src, void* cuda_stream);
 
+/* ----------------------------------------------------------- segments */
+
+/* Post-processing of frame probabilities into speaker segments ("Streaming
+ * Sortformer Diarizer" model card, Output: diarize() turns the (B, T/8, 4)
+ * sigmoid probabilities into [start_seconds, end_seconds, speaker_index]
+ * segments by VAD-style thresholding and smoothing; NeMo API page,
+ * SortformerEncLabelModel.diarize).  Per clip and speaker, in this order:
+ *   1. hysteresis: a run starts at a frame with p > onset and ends before the
+ *      first later frame with p <= offset (onset = offset: active <=> p > it);
+ *   2. a run of encoder frames a..b covers [0.08 a, 0.08 (b + 1)) seconds;
+ *   3. padding: start - pad_onset (>= 0), end + pad_offset (<= 0.08 n_frames);
+ *   4. a segment joins the previous one when it starts at or before its end
+ *      or less than min_duration_off after it;
+ *   5. merged segments shorter than min_duration_on are dropped.
+ * Times are float64 with each product and sum rounded separately. */
+typedef struct sf_seg_params {
+  float onset, offset;                       /* onset >= offset, both in [0, 1] */
+  double pad_onset, pad_offset;              /* seconds, >= 0 */
+  double min_duration_on, min_duration_off;  /* seconds, >= 0 */
+} sf_seg_params;
+
+/* Defaults: onset = offset = 0.5, no padding, no duration limits. */
+SF_API sf_status sf_default_seg_params(sf_seg_params* out);
+
+/*   d_probs    f32 [n][stride_t][4]  per-clip probabilities (sf_forward_offline's
+ *                                    output layout, or chunk outputs gathered by
+ *                                    the caller)
+ *   h_n_frames i32 [n] host          frames of each clip, 0 <= n_frames <= stride_t
+ *   d_segs     f64 [n][4][max_seg][2] (out)  start, end seconds, in time order
+ *   d_counts   i32 [n][4] (out)      segments found per clip and speaker; may
+ *                                    exceed max_seg, only the first max_seg
+ *                                    are stored
+ * 1 <= n <= 512.  Device buffers are the caller's; the
+ * engine's descriptor block carries the frame counts (ordered on
+ * `cuda_stream` with the engine's other calls). */
+SF_API sf_status sf_segments(sf_engine* e, const float* d_probs, int stride_t, const int* h_n_frames, int n,
+                             const sf_seg_params* params, int max_seg, double* d_segs, int* d_counts,
+                             void* cuda_stream);
+
 /* ---------------------------------------------------------------- options */
 
 enum {

@@ -41,6 +41,12 @@ class sf_state_view(ctypes.Structure):
                 ("d_fifo_emb", ctypes.c_void_p), ("d_fifo_preds", ctypes.c_void_p), ("d_sil_mean", ctypes.c_void_p)]
 
 
+class sf_seg_params(ctypes.Structure):
+    _fields_ = [("onset", ctypes.c_float), ("offset", ctypes.c_float), ("pad_onset", ctypes.c_double),
+                ("pad_offset", ctypes.c_double), ("min_duration_on", ctypes.c_double),
+                ("min_duration_off", ctypes.c_double)]
+
+
 class sf_kernel_stat(ctypes.Structure):
     _fields_ = [("name", ctypes.c_char * 32), ("launches", ctypes.c_int64), ("ms", ctypes.c_double),
                 ("flops", ctypes.c_double), ("bytes", ctypes.c_double)]
@@ -51,7 +57,8 @@ EXPORTED = ["sf_default_config", "sf_create", "sf_create_from_file", "sf_destroy
             "sf_forward_offline_host", "sf_stream_create", "sf_stream_destroy", "sf_stream_reset",
             "sf_stream_window", "sf_stream_step", "sf_stream_get_state", "sf_stream_set_state",
             "sf_stream_update", "sf_select_topk", "sf_profile_enable", "sf_profile_read", "sf_mel_noalloc",
-            "sf_check", "sf_gemm_bf16", "sf_set_option", "sf_attention_relpos"]
+            "sf_check", "sf_gemm_bf16", "sf_set_option", "sf_attention_relpos", "sf_default_seg_params",
+            "sf_segments"]
 
 
 class SFError(RuntimeError):
@@ -92,6 +99,8 @@ def _load():
         "sf_set_option": ([VP, I, I], I),
         "sf_gemm_bf16": ([VP, VP, I, VP, I, I, I, VP, VP, I, VP], I),
         "sf_attention_relpos": ([VP, VP, VP, I, VP, VP, VP, I, VP, I, VP], I),
+        "sf_default_seg_params": ([P(sf_seg_params)], I),
+        "sf_segments": ([VP, VP, I, VP, I, P(sf_seg_params), I, VP, VP, VP], I),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -289,6 +298,27 @@ def sf_attention_relpos(eng, qkv, ptab, R, u, v, seq_len, ctx, path=1, stream=No
     seq_len = np.ascontiguousarray(seq_len, np.int32)
     _check(lib.sf_attention_relpos(eng, _ptr(qkv), _ptr(ptab), R, _ptr(u), _ptr(v), _ptr(seq_len), len(seq_len),
                                    _ptr(ctx), path, _stream(stream)), eng)
+
+
+def seg_params(**kw):
+    p = sf_seg_params()
+    _check(lib.sf_default_seg_params(ctypes.byref(p)))
+    for k, v in kw.items():
+        setattr(p, k, v)
+    return p
+
+
+def sf_segments(eng, probs, n_frames, params=None, max_seg=256, stream=None):
+    """probs: device f32 [n, T, 4]; returns (segs f64 [n, 4, max_seg, 2], counts i32 [n, 4]) on the device."""
+    import torch
+    n, T = probs.shape[0], probs.shape[1]
+    n_frames = np.ascontiguousarray(n_frames, np.int32)
+    segs = torch.zeros((n, 4, max_seg, 2), dtype=torch.float64, device=probs.device)
+    counts = torch.zeros((n, 4), dtype=torch.int32, device=probs.device)
+    p = params if params is not None else seg_params()
+    _check(lib.sf_segments(eng, _ptr(probs), T, _ptr(n_frames), n, ctypes.byref(p), max_seg, _ptr(segs),
+                           _ptr(counts), _stream(stream)), eng)
+    return segs, counts
 
 
 def sf_set_option(eng, option, value):

@@ -38,6 +38,7 @@ constexpr int APW = 192;     // position-table rows per tile (distances r - c)
 constexpr int ANB = 3;       // K / V ring stages
 constexpr int NPW = ANB + 2; // 64-row position blocks held (tile t reads blocks t - 2 .. t)
 constexpr int BD_LD = 100;   // staged BD row stride (floats)
+constexpr int PSTR = AHD + 4; // key-split partial row: O[64], m, l, 2 pad (16-byte aligned rows)
 
 struct AttTc {
   static constexpr int Q_BYTES = AQ * AHD * 2;      // 16 KB, K-major, 128-byte swizzle
@@ -94,7 +95,9 @@ __global__ void __launch_bounds__(192, 1) attn_relpos_tc_kernel(const __grid_con
                                                                 const bf16* __restrict__ qkv, int D, int R,
                                                                 const float* __restrict__ u,
                                                                 const float* __restrict__ vb, bf16* __restrict__ ctx,
-                                                                const SeqTable* __restrict__ seq, int* err) {
+                                                                const SeqTable* __restrict__ seq, int* err, int ks,
+                                                                float* __restrict__ part_ws,
+                                                                int* __restrict__ part_cnt) {
   using L = AttTc;
   extern __shared__ uint8_t at_smem[];
   uint8_t* sm = at_smem + ((1024 - (su32(at_smem) & 1023)) & 1023);
@@ -120,7 +123,11 @@ __global__ void __launch_bounds__(192, 1) attn_relpos_tc_kernel(const __grid_con
   const int s = seq_of_tile2(seq, blockIdx.x);
   const int sb = seq->off[s], S = seq->off[s + 1] - sb;
   const int i0 = (blockIdx.x - seq->tile2_off[s]) * AQ;
-  const int T = (S + AK - 1) / AK;   // key tiles
+  const int T = (S + AK - 1) / AK;   // key tiles of the sequence
+  // key split: this CTA takes key tiles [t0, t0 + Tl) (blockIdx.z of ks);
+  // ring stages and barrier phases count local tiles tt = t - t0
+  const int t0 = (int)((int64_t)T * blockIdx.z / ks);
+  const int Tl = (int)((int64_t)T * (blockIdx.z + 1) / ks) - t0;
 
   if (threadIdx.x == 0) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&t_qkv)) : "memory");
@@ -156,33 +163,34 @@ __global__ void __launch_bounds__(192, 1) attn_relpos_tc_kernel(const __grid_con
   if (warp == 0) {
     // ---------------------------------------------------------------- loads
     if (lane == 0) {
-      int t = 0;
-      for (; t < T && !*abort_flag; ++t) {
-        const int b = t % ANB, r = t / ANB, j0 = t * AK;
+      int tt = 0;
+      for (; tt < Tl && !*abort_flag; ++tt) {
+        const int t = t0 + tt, b = tt % ANB, r = tt / ANB, j0 = t * AK;
         if (!mbar_wait(&kv_empty[b], (r & 1) ^ 1, abort_flag)) {
           *abort_flag = 1;
           break;
         }
-        // position block k = distances i0 - 64k - 63 .. i0 - 64k, slot (k + 2) % NPW;
-        // tile 0 brings blocks -2, -1, 0, tile t > 0 block t
-        const int k_lo = t == 0 ? -2 : t;
+        // position block k = distances i0 - 64k - 63 .. i0 - 64k; local index
+        // lb = k - t0 + 2, slot lb % NPW; the first tile brings blocks
+        // t0 - 2 .. t0, later tiles block t
+        const int lb_lo = tt == 0 ? 0 : tt + 2, lb_hi = tt + 2;
         bool got = true;
-        for (int k = k_lo; k <= t && got; ++k)
-          got = mbar_wait(&pw_empty[(k + 2) % NPW], (((k + 2) / NPW) & 1) ^ 1, abort_flag);
+        for (int lb = lb_lo; lb <= lb_hi && got; ++lb)
+          got = mbar_wait(&pw_empty[lb % NPW], ((lb / NPW) & 1) ^ 1, abort_flag);
         if (!got) {
           *abort_flag = 1;
           break;
         }
         uint8_t* st = sRing + b * L::STAGE;
-        mbar_expect_tx(&kv_full[b], L::STAGE + (t - k_lo + 1) * L::PB_BYTES);
+        mbar_expect_tx(&kv_full[b], L::STAGE + (lb_hi - lb_lo + 1) * L::PB_BYTES);
         tma_load_2d(st, &t_qkv, &kv_full[b], D + h * AHD, sb + j0);                       // K rows j0 ..
         tma_load_2d(st + L::K_BYTES, &t_qkv, &kv_full[b], 2 * D + h * AHD, sb + j0);      // V rows j0 ..
-        for (int k = k_lo; k <= t; ++k)
-          tma_load_2d(sPw + ((k + 2) % NPW) * L::PB_BYTES, &t_pos, &kv_full[b], h * AHD,
-                      i0 - 64 * k - (AK - 1) + R - 1);
+        for (int lb = lb_lo; lb <= lb_hi; ++lb)
+          tma_load_2d(sPw + (lb % NPW) * L::PB_BYTES, &t_pos, &kv_full[b], h * AHD,
+                      i0 - 64 * (lb + t0 - 2) - (AK - 1) + R - 1);
       }
       if (*abort_flag) {   // let this CTA's own loads land before its shared memory is released
-        for (int k = t - ANB > 0 ? t - ANB : 0; k < t; ++k) {
+        for (int k = tt - ANB > 0 ? tt - ANB : 0; k < tt; ++k) {
           const long long c0 = clock64();
           while (!mbar_try_wait(&kv_full[k % ANB], (k / ANB) & 1) && clock64() - c0 < WAIT_CYCLES) {
           }
@@ -191,16 +199,16 @@ __global__ void __launch_bounds__(192, 1) attn_relpos_tc_kernel(const __grid_con
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMAs
-    if (lane == 0) {
+    if (lane == 0 && Tl > 0) {
       constexpr uint32_t id_s = idesc_bf16_mn(AQ, AK, false);
       constexpr uint32_t id_bd = idesc_bf16_mn(AQ, 64, false);
       constexpr uint32_t id_pv = idesc_bf16_mn(AQ, AHD, true);
       const uint32_t tm_s = tmem, tm_bd = tmem + AK;
       const uint64_t dqu = sw128_desc(su32(sQu)), dqv = sw128_desc(su32(sQv));
       bool ok = mbar_wait(q_ready, 0, abort_flag);
-      auto issue_pv = [&](int t) -> bool {
-        const int pb = t & 1, b = t % ANB;
-        if (!mbar_wait(&p_full[pb], (t >> 1) & 1, abort_flag)) return false;
+      auto issue_pv = [&](int tt) -> bool {
+        const int pb = tt & 1, b = tt % ANB;
+        if (!mbar_wait(&p_full[pb], (tt >> 1) & 1, abort_flag)) return false;
         tc_fence_after();
         const uint64_t dp = sw128_desc(su32(sP + pb * L::P_BYTES));
         const uint64_t dv = sw128_desc_mn(su32(sRing + b * L::STAGE + L::K_BYTES));
@@ -211,28 +219,28 @@ __global__ void __launch_bounds__(192, 1) attn_relpos_tc_kernel(const __grid_con
         umma_commit(&kv_empty[b]);   // K, V and Pw of tile t are no longer read
         return true;
       };
-      for (int t = 0; ok && t < T; ++t) {
-        const int b = t % ANB;
-        if (!mbar_wait(&kv_full[b], (t / ANB) & 1, abort_flag)) { ok = false; break; }
-        if (t > 0 && !mbar_wait(s_free, (t - 1) & 1, abort_flag)) { ok = false; break; }
+      for (int tt = 0; ok && tt < Tl; ++tt) {
+        const int b = tt % ANB;
+        if (!mbar_wait(&kv_full[b], (tt / ANB) & 1, abort_flag)) { ok = false; break; }
+        if (tt > 0 && !mbar_wait(s_free, (tt - 1) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
         uint8_t* st = sRing + b * L::STAGE;
         const uint64_t dk = sw128_desc(su32(st));
 #pragma unroll
         for (int k = 0; k < AHD / 16; ++k) umma_bf16(tm_s, dqu + (uint64_t)(2 * k), dk + (uint64_t)(2 * k), id_s, k != 0);
-        // BD columns 64 m .. 64 m + 63 <- position block t - m
+        // BD columns 64 m .. 64 m + 63 <- position block t - m (local index tt + 2 - m)
 #pragma unroll
         for (int m = 0; m < 3; ++m) {
-          const uint64_t dpw = sw128_desc(su32(sPw + ((t - m + 2 + NPW) % NPW) * L::PB_BYTES));
+          const uint64_t dpw = sw128_desc(su32(sPw + ((tt + 2 - m) % NPW) * L::PB_BYTES));
 #pragma unroll
           for (int k = 0; k < AHD / 16; ++k)
             umma_bf16(tm_bd + 64 * m, dqv + (uint64_t)(2 * k), dpw + (uint64_t)(2 * k), id_bd, k != 0);
         }
         umma_commit(s_full);
-        umma_commit(&pw_empty[t % NPW]);   // block t - 2 is read for the last time by tile t
-        if (t > 0 && !issue_pv(t - 1)) { ok = false; break; }
+        umma_commit(&pw_empty[tt % NPW]);   // block t - 2 (local tt) is read for the last time by tile t
+        if (tt > 0 && !issue_pv(tt - 1)) { ok = false; break; }
       }
-      if (ok && T > 0) ok = issue_pv(T - 1);
+      if (ok) ok = issue_pv(Tl - 1);
       if (!ok) *abort_flag = 1;
     }
   } else {
@@ -247,7 +255,7 @@ __global__ void __launch_bounds__(192, 1) attn_relpos_tc_kernel(const __grid_con
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
     };
     // (Q + u) and (Q + v) rows, rounded to bf16, into the swizzled A tiles
-    {
+    if (Tl > 0) {
       const bf16* qrow = qkv + (int64_t)(sb + (row_ok ? i : 0)) * (3 * D) + h * AHD;
       const float* uh = u + h * AHD;
       const float* vh = vb + h * AHD;
@@ -281,9 +289,9 @@ __global__ void __launch_bounds__(192, 1) attn_relpos_tc_kernel(const __grid_con
 #pragma unroll
     for (int d = 0; d < AHD; ++d) o[d] = 0.f;
     bool ok = true;
-    for (int t = 0; t < T; ++t) {
-      const int j0 = t * AK;
-      if (!warp_wait(s_full, t & 1)) { ok = false; break; }
+    for (int tt = 0; tt < Tl; ++tt) {
+      const int j0 = (t0 + tt) * AK;
+      if (!warp_wait(s_full, tt & 1)) { ok = false; break; }
       tc_fence_after();
       float sc[AK];
       {
@@ -339,7 +347,7 @@ __global__ void __launch_bounds__(192, 1) attn_relpos_tc_kernel(const __grid_con
       m_run = m_new;
       // P row as bf16 into the swizzled A tile of P.V (buffer t % 2; its
       // previous tile's P.V completed before iteration t - 1 read its result)
-      uint8_t* pt = sP + (t & 1) * L::P_BYTES;
+      uint8_t* pt = sP + (tt & 1) * L::P_BYTES;
 #pragma unroll
       for (int ch = 0; ch < AK / 8; ++ch) {
         uint32_t w4[4];
@@ -353,11 +361,11 @@ __global__ void __launch_bounds__(192, 1) attn_relpos_tc_kernel(const __grid_con
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[t & 1]);
+      if (lane == 0) mbar_arrive(&p_full[tt & 1]);
       // O (relative to m_(t-1)) += P_(t-1) V_(t-1), then rescale to m_t
-      if (t > 0) {
-        const int pb = (t - 1) & 1;
-        if (!warp_wait(&pv_full[pb], ((t - 1) >> 1) & 1)) { ok = false; break; }
+      if (tt > 0) {
+        const int pb = (tt - 1) & 1;
+        if (!warp_wait(&pv_full[pb], ((tt - 1) >> 1) & 1)) { ok = false; break; }
         tc_fence_after();
         uint32_t v[AHD];
         tmem_ld64(tmem + lane_base + (uint32_t)(256 + 64 * pb), v);
@@ -365,9 +373,9 @@ __global__ void __launch_bounds__(192, 1) attn_relpos_tc_kernel(const __grid_con
         for (int k = 0; k < AHD; ++k) o[k] = (o[k] + __uint_as_float(v[k])) * alpha;
       }
     }
-    if (ok && T > 0) {
-      const int pb = (T - 1) & 1;
-      if (warp_wait(&pv_full[pb], ((T - 1) >> 1) & 1)) {
+    if (ok && Tl > 0) {
+      const int pb = (Tl - 1) & 1;
+      if (warp_wait(&pv_full[pb], ((Tl - 1) >> 1) & 1)) {
         tc_fence_after();
         uint32_t v[AHD];
         tmem_ld64(tmem + lane_base + (uint32_t)(256 + 64 * pb), v);
@@ -377,20 +385,63 @@ __global__ void __launch_bounds__(192, 1) attn_relpos_tc_kernel(const __grid_con
         ok = false;
       }
     }
-    if (!ok) {
-      *abort_flag = 1;
-    } else if (row_ok) {
-      const float inv = 1.f / l_run;
+    if (!ok) *abort_flag = 1;
+    auto store_row = [&](const float* ov, float l) {
+      const float inv = 1.f / l;
       uint4* dst = reinterpret_cast<uint4*>(ctx + (int64_t)(sb + i) * D + h * AHD);
 #pragma unroll
       for (int c = 0; c < AHD / 8; ++c) {
         uint32_t w4[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          __nv_bfloat162 ho = __floats2bfloat162_rn(o[8 * c + 2 * k] * inv, o[8 * c + 2 * k + 1] * inv);
+          __nv_bfloat162 ho = __floats2bfloat162_rn(ov[8 * c + 2 * k] * inv, ov[8 * c + 2 * k + 1] * inv);
           w4[k] = *reinterpret_cast<uint32_t*>(&ho);
         }
         dst[c] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+      }
+    };
+    if (ks == 1) {
+      if (ok && row_ok) store_row(o, l_run);
+    } else {
+      // Key split: every CTA of a (query tile, head) leaves (O, m, l) of its
+      // key range in the workspace; the last one to arrive merges them in
+      // split order, so the result does not depend on the arrival order.
+      // (Also after a failed wait, so that the counter returns to zero.)
+      const int unit = blockIdx.x * 8 + h;
+      float* mine = part_ws + (((int64_t)unit * ks + blockIdx.z) * AQ + r) * PSTR;
+#pragma unroll
+      for (int d = 0; d < AHD; d += 4)
+        *reinterpret_cast<float4*>(mine + d) = make_float4(o[d], o[d + 1], o[d + 2], o[d + 3]);
+      mine[AHD] = m_run;
+      mine[AHD + 1] = l_run;
+      __threadfence();
+      volatile int* last_flag = abort_flag + 1;
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (warp == 2 && lane == 0) {
+        const int prev = atomicAdd(&part_cnt[unit], 1);
+        *last_flag = prev == ks - 1;
+        if (prev == ks - 1) part_cnt[unit] = 0;   // ready for the next launch
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (*last_flag) {
+        __threadfence();
+        const float* base = part_ws + ((int64_t)unit * ks * AQ + r) * PSTR;
+        float m = -INFINITY;
+        for (int zz = 0; zz < ks; ++zz) m = fmaxf(m, __ldcg(base + (int64_t)zz * AQ * PSTR + AHD));
+        float acc[AHD], l = 0.f;
+#pragma unroll
+        for (int d = 0; d < AHD; ++d) acc[d] = 0.f;
+        for (int zz = 0; zz < ks; ++zz) {
+          const float* pz = base + (int64_t)zz * AQ * PSTR;
+          const float wz = ex2_approx(__ldcg(pz + AHD) - m);   // empty key range: m_z = -inf, weight 0
+          l += wz * __ldcg(pz + AHD + 1);
+#pragma unroll
+          for (int d = 0; d < AHD; d += 4) {
+            const float4 v4 = __ldcg(reinterpret_cast<const float4*>(pz + d));
+            acc[d] += wz * v4.x; acc[d + 1] += wz * v4.y; acc[d + 2] += wz * v4.z; acc[d + 3] += wz * v4.w;
+          }
+        }
+        if (row_ok && !*abort_flag) store_row(acc, l);
       }
     }
   }
@@ -403,9 +454,13 @@ __global__ void __launch_bounds__(192, 1) attn_relpos_tc_kernel(const __grid_con
   if (threadIdx.x == 0 && *abort_flag) set_err(err, ERR_TIMEOUT);
 }
 
+namespace {
+int g_att_sms = 148;
+}
+
 cudaError_t launch_relpos_attention_tc(const bf16* qkv, const bf16* ptab, int R, const float* u, const float* v,
-                                       bf16* ctx, const SeqTable* seq, int n_tiles2, int M, int* err,
-                                       cudaStream_t st) {
+                                       bf16* ctx, const SeqTable* seq, int n_tiles2, int M, int max_len,
+                                       const TcScratch& sc, cudaStream_t st) {
   if (M <= 0 || n_tiles2 <= 0) return cudaSuccess;
   constexpr int D = 512;
   CUtensorMap t_qkv, t_pos;
@@ -413,12 +468,29 @@ cudaError_t launch_relpos_attention_tc(const bf16* qkv, const bf16* ptab, int R,
   if (r != cudaSuccess) return r;
   r = make_bf16_map_sw128(&t_pos, ptab, 2 * R - 1, D, D, 64);
   if (r != cudaSuccess) return r;
-  CK_LAUNCH(launch_k(attn_relpos_tc_kernel, dim3(n_tiles2, 8), dim3(192), AttTc::SMEM, st, t_qkv, t_pos, qkv, D, R, u,
-                     v, ctx, seq, err));
+  // fewer (query tile, head) units than SMs: split each unit's keys over up
+  // to 4 CTAs (no more splits than key tiles of the longest sequence),
+  // partials merged by the last CTA of the unit
+  const int units = n_tiles2 * 8;
+  int ks = 1;
+  if (sc.ws && sc.cnt && units < g_att_sms) {
+    ks = g_att_sms / units;
+    ks = ks < 4 ? ks : 4;
+    const int tmax = (max_len + AK - 1) / AK;
+    ks = ks < tmax ? ks : tmax;
+    if (ks < 1 || (size_t)units * ks * AQ * PSTR * 4 > sc.ws_bytes || units > sc.cnt_len / 2) ks = 1;
+  }
+  int* cnt = sc.cnt ? sc.cnt + sc.cnt_len / 2 : nullptr;   // upper half: the GEMM's split-K uses the lower
+  CK_LAUNCH(launch_k(attn_relpos_tc_kernel, dim3(n_tiles2, 8, ks), dim3(192), AttTc::SMEM, st, t_qkv, t_pos, qkv, D, R,
+                     u, v, ctx, seq, sc.err, ks, sc.ws, cnt));
   return cudaGetLastError();
 }
 
 cudaError_t attention_tc_init_attributes() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
+      n > 0)
+    g_att_sms = n;
   return cudaFuncSetAttribute(attn_relpos_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, AttTc::SMEM);
 }
 

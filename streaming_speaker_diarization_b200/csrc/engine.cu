@@ -178,6 +178,7 @@ struct sf_engine {
   size_t pool_used = 0;
   double att_s2 = 0;      // sum of squared sequence lengths of the current call
   int att_tiles2 = 0;     // 128-row attention query tiles of the current call
+  int att_max_len = 0;    // longest sequence of the current call
   double ms_acc[K_COUNT] = {};   // event time already read back (graph replays)
   // CUDA graphs: one per launch shape, replayed; invalidated when the workspace moves
   bool use_graphs = true;
@@ -597,7 +598,8 @@ template <>
 cudaError_t relpos_attention<bf16>(sf_engine* e, const bf16* qkv, const bf16* ptab, const float* pu, const float* pv,
                                    bf16* ctx, const SeqTable* seq, int n_tiles, int M, cudaStream_t st) {
   if (e->attn_path == 1)
-    return launch_relpos_attention_tc(qkv, ptab, e->R, pu, pv, ctx, seq, e->att_tiles2, M, e->d_err, st);
+    return launch_relpos_attention_tc(qkv, ptab, e->R, pu, pv, ctx, seq, e->att_tiles2, M, e->att_max_len,
+                                      e->tc_scratch(), st);
   return launch_relpos_attention<bf16>(qkv, ptab, e->R, pu, pv, ctx, seq, n_tiles, M, st);
 }
 
@@ -901,6 +903,9 @@ cudaError_t offline_impl(sf_engine* e, const float* d_audio, const std::vector<i
   fill_seq(d, tp, M, tiles);
   e->att_s2 = sum_sq(tp);
   e->att_tiles2 = d->seq.tile2_off[d->seq.n_seq];
+  e->att_max_len = 0;
+  for (int q_ = 0; q_ < d->seq.n_seq; ++q_)
+    e->att_max_len = std::max(e->att_max_len, d->seq.off[q_ + 1] - d->seq.off[q_]);
   const int T3 = (int)enc_frames(L_max);
   const int Tp_max = (int)enc_frames(n_max / 160);
   CK(ensure(e->mel, (size_t)B * 128 * T_cols * 4));
@@ -1219,6 +1224,9 @@ sf_status sf_encode(sf_engine* e, const void* d_embs, const int* h_seq_len, int 
   fill_seq(d, lens, M, tiles);
   e->att_s2 = sum_sq(lens);
   e->att_tiles2 = d->seq.tile2_off[d->seq.n_seq];
+  e->att_max_len = 0;
+  for (int q_ = 0; q_ < d->seq.n_seq; ++q_)
+    e->att_max_len = std::max(e->att_max_len, d->seq.off[q_ + 1] - d->seq.off[q_]);
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
   cudaError_t ce = ensure_encode_ws(e, M);
   if (ce == cudaSuccess) ce = desc_upload(e, st);
@@ -1286,9 +1294,38 @@ sf_status sf_attention_relpos(sf_engine* e, const void* d_qkv, const void* d_pta
   const bf16* ptab = static_cast<const bf16*>(d_ptab);
   bf16* ctx = static_cast<bf16*>(d_ctx);
   if (ce == cudaSuccess)
-    ce = path == 1 ? launch_relpos_attention_tc(qkv, ptab, R, d_u, d_v, ctx, &e->d_desc->seq, tiles2, M, e->d_err, st)
+    ce = path == 1 ? launch_relpos_attention_tc(qkv, ptab, R, d_u, d_v, ctx, &e->d_desc->seq, tiles2, M,
+                                                *std::max_element(lens.begin(), lens.end()), e->tc_scratch(), st)
                    : launch_relpos_attention<bf16>(qkv, ptab, R, d_u, d_v, ctx, &e->d_desc->seq, tiles, M, st);
   if (ce != cudaSuccess) return cuda_fail(e, ce, "sf_attention_relpos");
+  return SF_OK;
+}
+
+sf_status sf_default_seg_params(sf_seg_params* out) {
+  if (!out) return SF_EINVAL;
+  *out = sf_seg_params{0.5f, 0.5f, 0.0, 0.0, 0.0, 0.0};
+  return SF_OK;
+}
+
+sf_status sf_segments(sf_engine* e, const float* d_probs, int stride_t, const int* h_n_frames, int n,
+                      const sf_seg_params* prm, int max_seg, double* d_segs, int* d_counts, void* cuda_stream) {
+  if (check_engine(e) != SF_OK) return SF_EINVAL;
+  if (!d_probs || !h_n_frames || !prm || !d_segs || !d_counts) return fail(e, SF_EINVAL, "null pointer argument");
+  if (n < 1 || n > MAX_SEQ || stride_t < 1 || max_seg < 1) return fail(e, SF_ESHAPE, "n, stride_t or max_seg out of range");
+  if (!(prm->onset >= prm->offset) || !(prm->offset >= 0.f) || !(prm->onset <= 1.f) || !(prm->pad_onset >= 0.0) ||
+      !(prm->pad_offset >= 0.0) || !(prm->min_duration_on >= 0.0) || !(prm->min_duration_off >= 0.0))
+    return fail(e, SF_EINVAL, "segment parameters: 0 <= offset <= onset <= 1, non-negative times");
+  DescBlock* d = desc_begin(e);
+  for (int i = 0; i < n; ++i) {
+    if (h_n_frames[i] < 0 || h_n_frames[i] > stride_t) return fail(e, SF_ESHAPE, "n_frames out of [0, stride_t]");
+    d->count[i] = h_n_frames[i];
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  SegArgs a{prm->onset, prm->offset, prm->pad_onset, prm->pad_offset, prm->min_duration_on, prm->min_duration_off,
+            max_seg};
+  cudaError_t ce = desc_upload(e, st);
+  if (ce == cudaSuccess) ce = launch_segments(d_probs, stride_t, e->d_desc->count, n, a, d_segs, d_counts, st);
+  if (ce != cudaSuccess) return cuda_fail(e, ce, "sf_segments");
   return SF_OK;
 }
 
@@ -1417,6 +1454,9 @@ void fill_step(sf_stream* s, DescBlock* d, const StepPlan& pl, int& M, int& tile
   fill_seq(d, lens, M, tiles);
   s->e->att_s2 = sum_sq(lens);
   s->e->att_tiles2 = d->seq.tile2_off[d->seq.n_seq];
+  s->e->att_max_len = 0;
+  for (int q_ = 0; q_ < d->seq.n_seq; ++q_)
+    s->e->att_max_len = std::max(s->e->att_max_len, d->seq.off[q_ + 1] - d->seq.off[q_]);
 }
 
 // Host bookkeeping after a state update (sizes are data-independent).

@@ -100,6 +100,19 @@ cudaError_t launch_extract_rows(const float* packed, const SeqTable* seq, const 
 void attention_set_max_seq(int s);
 cudaError_t attention_init_f32_attributes(int R);
 
+// ------------------------------------------------------- post-processing
+struct SegArgs {
+  float onset, offset;      // activity thresholds (onset >= offset)
+  double pad_on, pad_off;   // seconds added before / after each run
+  double min_on, min_off;   // shortest kept segment, shortest kept gap (s)
+  int max_seg;              // segments stored per (clip, speaker)
+};
+// probs f32 [n][stride_t][4], d_n_frames i32 [n] -> segs f64
+// [n][4][max_seg][2] (start, end seconds), counts i32 [n][4] (found, may
+// exceed max_seg; only the first max_seg are stored).
+cudaError_t launch_segments(const float* probs, int stride_t, const int* d_n_frames, int n, const SegArgs& a,
+                            double* segs, int* counts, cudaStream_t st);
+
 // ------------------------------------------------------------- attention
 // Relative-position MHSA (d_model 512, 8 heads of 64) over packed sequences.
 //   qkv act [M x 3*512] (q | k | v), ptab act [(2R-1) x 512] projected
@@ -111,12 +124,13 @@ cudaError_t launch_relpos_attention(const T* qkv, const T* ptab, int R, const fl
 template <typename T>
 cudaError_t launch_mha(const T* qkv, T* ctx, const SeqTable* seq, int n_tiles, int M, cudaStream_t st);
 cudaError_t attention_init_attributes();
-// bf16 relative-position MHSA on tcgen05 (one CTA per 128 query rows x head;
-// n_tiles2 = 128-row tiles of the sequence table); err gets ERR_TIMEOUT if
-// a bounded wait gives up.
+// bf16 relative-position MHSA on tcgen05 (one CTA per 128 query rows x head
+// x key split; n_tiles2 = 128-row tiles of the sequence table, max_len the
+// longest sequence); sc.err gets ERR_TIMEOUT if a bounded wait gives up;
+// sc.ws / the upper half of sc.cnt hold the key-split partials and counters.
 cudaError_t launch_relpos_attention_tc(const bf16* qkv, const bf16* ptab, int R, const float* u, const float* v,
-                                       bf16* ctx, const SeqTable* seq, int n_tiles2, int M, int* err,
-                                       cudaStream_t st);
+                                       bf16* ctx, const SeqTable* seq, int n_tiles2, int M, int max_len,
+                                       const TcScratch& sc, cudaStream_t st);
 cudaError_t attention_tc_init_attributes();
 
 }  // namespace sf

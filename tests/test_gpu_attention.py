@@ -115,3 +115,18 @@ def test_relpos_attention_rejects_bad_input(eng):
         _run(eng, qkv, ptab, 16, u, v, [17], 1)      # longer than R
     with pytest.raises(b.SFError):
         _run(eng, qkv, ptab, 16, u, v, [10], 2)      # unknown path
+
+
+@pytest.mark.parametrize("L", [1125, 300, 100, 65])
+def test_relpos_attention_key_split(eng, L):
+    """One sequence: fewer (query tile, head) units than SMs, so each unit's
+    keys are split over up to 4 CTAs (1125: 2 splits of 9 key tiles; 300: 4
+    splits over 5 tiles; 100 and 65: 2 splits of one tile) and the partial
+    softmax states are merged by the last CTA."""
+    R = 1200
+    qkv, ptab, u, v = _inputs(11 + L, [L], R)
+    got = _run(eng, qkv, ptab, R, u, v, [L], 1)
+    ref = _reference(qkv, ptab, R, u, v, [L], [0])[0]
+    assert np.max(np.abs(got - ref)) <= 1.5e-2
+    again = _run(eng, qkv, ptab, R, u, v, [L], 1)
+    assert np.array_equal(got, again)            # merge order fixed: bitwise repeatable
