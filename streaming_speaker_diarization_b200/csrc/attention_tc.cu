@@ -34,7 +34,6 @@ namespace {
 constexpr int AQ = 128;      // query rows per CTA
 constexpr int AK = 64;       // keys per tile
 constexpr int AHD = 64;      // head dim
-constexpr int APW = 192;     // position-table rows per tile (distances r - c)
 constexpr int ANB = 3;       // K / V ring stages
 constexpr int NPW = ANB + 2; // 64-row position blocks held (tile t reads blocks t - 2 .. t)
 constexpr int BD_LD = 100;   // staged BD row stride (floats)
@@ -44,7 +43,7 @@ struct AttTc {
   static constexpr int Q_BYTES = AQ * AHD * 2;      // 16 KB, K-major, 128-byte swizzle
   static constexpr int K_BYTES = AK * AHD * 2;      //  8 KB
   static constexpr int V_BYTES = AK * AHD * 2;      //  8 KB (MN-major B operand)
-  static constexpr int PB_BYTES = 64 * AHD * 2;     //  8 KB position block
+  static constexpr int PB_BYTES = 64 * AHD * 2;     //  8 KB position block (one of the 192 distances of a tile)
   static constexpr int STAGE = K_BYTES + V_BYTES;
   static constexpr int P_BYTES = AQ * AK * 2;       // 16 KB
   static constexpr int OFF_QU = 0;
@@ -95,9 +94,7 @@ __global__ void __launch_bounds__(192, 1) attn_relpos_tc_kernel(const __grid_con
                                                                 const bf16* __restrict__ qkv, int D, int R,
                                                                 const float* __restrict__ u,
                                                                 const float* __restrict__ vb, bf16* __restrict__ ctx,
-                                                                const SeqTable* __restrict__ seq, int* err, int ks,
-                                                                float* __restrict__ part_ws,
-                                                                int* __restrict__ part_cnt) {
+                                                                const SeqTable* __restrict__ seq, int* err, int ks) {
   using L = AttTc;
   extern __shared__ uint8_t at_smem[];
   uint8_t* sm = at_smem + ((1024 - (su32(at_smem) & 1023)) & 1023);
@@ -403,47 +400,83 @@ __global__ void __launch_bounds__(192, 1) attn_relpos_tc_kernel(const __grid_con
     if (ks == 1) {
       if (ok && row_ok) store_row(o, l_run);
     } else {
-      // Key split: every CTA of a (query tile, head) leaves (O, m, l) of its
-      // key range in the workspace; the last one to arrive merges them in
-      // split order, so the result does not depend on the arrival order.
-      // (Also after a failed wait, so that the counter returns to zero.)
-      const int unit = blockIdx.x * 8 + h;
-      float* mine = part_ws + (((int64_t)unit * ks + blockIdx.z) * AQ + r) * PSTR;
+      // Key split: the ks CTAs of a (query tile, head) form a cluster; each
+      // leaves (O, m, l) of its key range in its own shared memory (the BD
+      // staging area, free now) and the cluster's rank 0 merges them in rank
+      // order over distributed shared memory after the cluster barrier.
+      // Row r's slot overlaps another warp's BD band: all four softmax warps
+      // finish their last tile before any slot is written.
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      float* mine = sBD + r * PSTR;
 #pragma unroll
       for (int d = 0; d < AHD; d += 4)
         *reinterpret_cast<float4*>(mine + d) = make_float4(o[d], o[d + 1], o[d + 2], o[d + 3]);
       mine[AHD] = m_run;
       mine[AHD + 1] = l_run;
-      __threadfence();
-      volatile int* last_flag = abort_flag + 1;
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      if (warp == 2 && lane == 0) {
-        const int prev = atomicAdd(&part_cnt[unit], 1);
-        *last_flag = prev == ks - 1;
-        if (prev == ks - 1) part_cnt[unit] = 0;   // ready for the next launch
+    }
+  }
+  if (ks > 1) {
+    // every thread of every CTA of the cluster meets here (also after a failed wait)
+    __syncthreads();
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+    uint32_t crank;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(crank));
+    if (crank == 0 && warp >= 2 && !*abort_flag) {
+      const int q = warp & 3, r = 32 * q + lane, i = i0 + r;
+      const uint32_t row_addr = su32(sBD + r * PSTR);
+      auto ld_peer = [&](uint32_t rank, int off) -> float {
+        uint32_t a;
+        asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(row_addr + 4u * off), "r"(rank));
+        float v;
+        asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(a) : "memory");
+        return v;
+      };
+      float mz[4], lz[4];
+#pragma unroll
+      for (int zz = 0; zz < 4; ++zz) {
+        mz[zz] = zz < ks ? ld_peer(zz, AHD) : -INFINITY;
+        lz[zz] = zz < ks ? ld_peer(zz, AHD + 1) : 0.f;
       }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      if (*last_flag) {
-        __threadfence();
-        const float* base = part_ws + ((int64_t)unit * ks * AQ + r) * PSTR;
-        float m = -INFINITY;
-        for (int zz = 0; zz < ks; ++zz) m = fmaxf(m, __ldcg(base + (int64_t)zz * AQ * PSTR + AHD));
-        float acc[AHD], l = 0.f;
+      const float m = fmaxf(fmaxf(mz[0], mz[1]), fmaxf(mz[2], mz[3]));
+      float acc[AHD], l = 0.f;
 #pragma unroll
-        for (int d = 0; d < AHD; ++d) acc[d] = 0.f;
-        for (int zz = 0; zz < ks; ++zz) {
-          const float* pz = base + (int64_t)zz * AQ * PSTR;
-          const float wz = ex2_approx(__ldcg(pz + AHD) - m);   // empty key range: m_z = -inf, weight 0
-          l += wz * __ldcg(pz + AHD + 1);
+      for (int d = 0; d < AHD; ++d) acc[d] = 0.f;
 #pragma unroll
-          for (int d = 0; d < AHD; d += 4) {
-            const float4 v4 = __ldcg(reinterpret_cast<const float4*>(pz + d));
-            acc[d] += wz * v4.x; acc[d + 1] += wz * v4.y; acc[d + 2] += wz * v4.z; acc[d + 3] += wz * v4.w;
-          }
+      for (int zz = 0; zz < 4; ++zz) {
+        if (zz >= ks) break;
+        const float wz = ex2_approx(mz[zz] - m);   // an empty key range has m = -inf: weight 0
+        l += wz * lz[zz];
+#pragma unroll
+        for (int d = 0; d < AHD; d += 4) {
+          uint32_t a;
+          asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(row_addr + 4u * d), "r"((uint32_t)zz));
+          float4 v4;
+          asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                       : "=f"(v4.x), "=f"(v4.y), "=f"(v4.z), "=f"(v4.w)
+                       : "r"(a)
+                       : "memory");
+          acc[d] += wz * v4.x; acc[d + 1] += wz * v4.y; acc[d + 2] += wz * v4.z; acc[d + 3] += wz * v4.w;
         }
-        if (row_ok && !*abort_flag) store_row(acc, l);
+      }
+      if (i < S) {
+        const float inv = 1.f / l;
+        uint4* dst = reinterpret_cast<uint4*>(ctx + (int64_t)(sb + i) * D + h * AHD);
+#pragma unroll
+        for (int c = 0; c < AHD / 8; ++c) {
+          uint32_t w4[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            __nv_bfloat162 ho = __floats2bfloat162_rn(acc[8 * c + 2 * k] * inv, acc[8 * c + 2 * k + 1] * inv);
+            w4[k] = *reinterpret_cast<uint32_t*>(&ho);
+          }
+          dst[c] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        }
       }
     }
+    // no CTA leaves while rank 0 may still read its shared memory
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
   }
   tc_fence_before();
   __syncthreads();
@@ -456,6 +489,7 @@ __global__ void __launch_bounds__(192, 1) attn_relpos_tc_kernel(const __grid_con
 
 namespace {
 int g_att_sms = 148;
+int g_att_clusters[3] = {1, 0, 0};   // co-resident clusters of 1, 2, 4 CTAs (0: that split is off)
 }
 
 cudaError_t launch_relpos_attention_tc(const bf16* qkv, const bf16* ptab, int R, const float* u, const float* v,
@@ -468,21 +502,36 @@ cudaError_t launch_relpos_attention_tc(const bf16* qkv, const bf16* ptab, int R,
   if (r != cudaSuccess) return r;
   r = make_bf16_map_sw128(&t_pos, ptab, 2 * R - 1, D, D, 64);
   if (r != cudaSuccess) return r;
-  // fewer (query tile, head) units than SMs: split each unit's keys over up
-  // to 4 CTAs (no more splits than key tiles of the longest sequence),
-  // partials merged by the last CTA of the unit
+  // fewer (query tile, head) units than SMs: split each unit's keys over a
+  // cluster of 2 or 4 CTAs (no more splits than key tiles of the longest
+  // sequence), merged in the cluster's shared memory
   const int units = n_tiles2 * 8;
   int ks = 1;
-  if (sc.ws && sc.cnt && units < g_att_sms) {
-    ks = g_att_sms / units;
-    ks = ks < 4 ? ks : 4;
-    const int tmax = (max_len + AK - 1) / AK;
-    ks = ks < tmax ? ks : tmax;
-    if (ks < 1 || (size_t)units * ks * AQ * PSTR * 4 > sc.ws_bytes || units > sc.cnt_len / 2) ks = 1;
+  if (units < g_att_sms) {
+    const int want = g_att_sms / units, tmax = (max_len + AK - 1) / AK;
+    if (want >= 4 && tmax >= 4 && g_att_clusters[2] > 0) ks = 4;
+    else if (want >= 2 && tmax >= 2 && g_att_clusters[1] > 0) ks = 2;
   }
-  int* cnt = sc.cnt ? sc.cnt + sc.cnt_len / 2 : nullptr;   // upper half: the GEMM's split-K uses the lower
-  CK_LAUNCH(launch_k(attn_relpos_tc_kernel, dim3(n_tiles2, 8, ks), dim3(192), AttTc::SMEM, st, t_qkv, t_pos, qkv, D, R,
-                     u, v, ctx, seq, sc.err, ks, sc.ws, cnt));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(n_tiles2, 8, ks);
+  cfg.blockDim = dim3(192);
+  cfg.dynamicSmemBytes = AttTc::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  attr[na].id = cudaLaunchAttributeClusterDimension;
+  attr[na].val.clusterDim.x = 1;
+  attr[na].val.clusterDim.y = 1;
+  attr[na].val.clusterDim.z = ks;
+  ++na;
+  if (g_launch_pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  CK_LAUNCH(cudaLaunchKernelEx(&cfg, attn_relpos_tc_kernel, t_qkv, t_pos, qkv, D, R, u, v, ctx, seq, sc.err, ks));
   return cudaGetLastError();
 }
 
@@ -491,7 +540,25 @@ cudaError_t attention_tc_init_attributes() {
   if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
       n > 0)
     g_att_sms = n;
-  return cudaFuncSetAttribute(attn_relpos_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, AttTc::SMEM);
+  cudaError_t r = cudaFuncSetAttribute(attn_relpos_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, AttTc::SMEM);
+  if (r != cudaSuccess) return r;
+  for (int j = 1; j < 3; ++j) {   // can clusters of 2 and 4 CTAs be scheduled at all?
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1, 1, 1 << j);
+    cfg.blockDim = dim3(192);
+    cfg.dynamicSmemBytes = AttTc::SMEM;
+    cudaLaunchAttribute a;
+    a.id = cudaLaunchAttributeClusterDimension;
+    a.val.clusterDim.x = 1;
+    a.val.clusterDim.y = 1;
+    a.val.clusterDim.z = 1 << j;
+    cfg.attrs = &a;
+    cfg.numAttrs = 1;
+    int n_cl = 0;
+    g_att_clusters[j] = cudaOccupancyMaxActiveClusters(&n_cl, attn_relpos_tc_kernel, &cfg) == cudaSuccess ? n_cl : 0;
+    cudaGetLastError();
+  }
+  return cudaSuccess;
 }
 
 }  // namespace sf
