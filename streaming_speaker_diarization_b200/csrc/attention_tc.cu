@@ -22,6 +22,10 @@
 // read back at column r - c + 63.  The softmax is online in the exp2 domain
 // (scale folded in); P goes to shared memory as bf16 (the A operand of P.V);
 // O accumulates in registers, rescaled before each tile's P.V is added.
+// With fewer (query tile, head) units than SMs (one long sequence), each
+// unit's key tiles are split over a cluster of 2 or 4 CTAs; each keeps its
+// softmax state (O, m, l) in shared memory and the cluster's rank 0 merges
+// them in rank order over distributed shared memory.
 // Every wait is bounded: a wait that runs out raises ERR_TIMEOUT, the CTA
 // drains its own copies and frees its TMEM.
 #include "common.cuh"

@@ -126,8 +126,9 @@ cudaError_t launch_mha(const T* qkv, T* ctx, const SeqTable* seq, int n_tiles, i
 cudaError_t attention_init_attributes();
 // bf16 relative-position MHSA on tcgen05 (one CTA per 128 query rows x head
 // x key split; n_tiles2 = 128-row tiles of the sequence table, max_len the
-// longest sequence); sc.err gets ERR_TIMEOUT if a bounded wait gives up;
-// sc.ws / the upper half of sc.cnt hold the key-split partials and counters.
+// longest sequence); with fewer (tile, head) units than SMs each unit's keys
+// are split over a cluster of 2 or 4 CTAs merged in shared memory; sc.err
+// gets ERR_TIMEOUT if a bounded wait gives up.
 cudaError_t launch_relpos_attention_tc(const bf16* qkv, const bf16* ptab, int R, const float* u, const float* v,
                                        bf16* ctx, const SeqTable* seq, int n_tiles2, int M, int max_len,
                                        const TcScratch& sc, cudaStream_t st);
