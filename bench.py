@@ -40,6 +40,27 @@ CONFIG = {"workload": "offline forward, 1 clip x 90 s (16 kHz, 4 speakers, 15% o
           "l2": "flushed between timed steps (256 MiB write)"}
 
 
+# DRAM bytes (read + write) per projection launch of the offline forward,
+# from an ncu launch list of this workload (profiles/offline_90s_launch_list.md:
+# 815.3 MB over the 213 GEMM launches of one forward); valid only for the GEMM
+# sources it was taken with, null once they change.
+GEMM_TRAFFIC = {"bytes_per_launch": 815.3e6 / 213,
+                "sources_sha256": "9bad6df933c0cd329728f20224afdde012e864c83a7fc71d246a0dfde6e9963d"}
+
+
+def gemm_traffic_per_launch():
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(os.path.dirname(os.path.abspath(__file__)), "streaming_speaker_diarization_b200", "csrc")
+    try:
+        for f in ("gemm_tc.cu", "tcgen05.cuh", "epilogue.cuh"):
+            with open(os.path.join(csrc, f), "rb") as fh:
+                h.update(fh.read())
+    except OSError:
+        return None
+    return GEMM_TRAFFIC["bytes_per_launch"] if h.hexdigest() == GEMM_TRAFFIC["sources_sha256"] else None
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -298,11 +319,13 @@ def main():
 
     pk, pk_kind = peaks()
     g = prof_gemm.get("gemm", (0, 0.0, 0.0, 0.0))
+    traffic = gemm_traffic_per_launch()
     timed_s = max_ms / 1000.0
     peak_tf = pk["bf16_tflops_sustained"] if timed_s > 1.0 else pk["bf16_tflops"]
     achieved = (g[2] / (g[1] / 1000.0)) / 1e12 if g[1] > 0 else None
     roof = {"bound": "tensor", "kernel": "gemm (all projection launches)", "achieved": achieved, "peak": peak_tf,
-            "unit": "TFLOP/s", "frac": (achieved / peak_tf) if achieved else None, "traffic": None,
+            "unit": "TFLOP/s", "frac": (achieved / peak_tf) if achieved else None, "traffic": traffic,
+            "traffic_unit": "bytes per launch (DRAM read + write, mean over the forward's projections)",
             "peak_kind": f"{pk_kind} bf16 {'sustained' if timed_s > 1.0 else 'burst'}",
             "launches_per_step": g[0] / args.steps if args.steps else None,
             "ms_per_step": g[1] / args.steps if args.steps else None}
