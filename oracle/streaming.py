@@ -236,3 +236,71 @@ def stream_run(feats, L, w, preset, dt=np.float64, taps=None, max_steps=None):
         outs.append(stream_step(st, feats, L, w, preset, dt, taps))
         steps += 1
     return np.concatenate(outs), st
+
+
+# ---------------------------------------------------------------- audio in
+# Source: the Transformers "Nemotron 3 Diarization" streaming notes (the
+# processor is called on successive audio slices, the last one flagged as the
+# end of the session) and the NeMo API (streaming over features).  Reading:
+# a step's mel window is computed from the stream's continuous signal as the
+# offline front-end computes it (preemphasis from the stream start, centred
+# frames, zeros past the samples received so far) and normalised per bin over
+# the window's own frames (the clip normalisation applied to the window).
+
+def window_log_mel(audio, n_avail, m0, m1, dt=np.float64):
+    """Log-mel (128, m1 - m0) of frames m0 .. m1-1 of the first n_avail
+    samples of a stream: frame t is the 400-point Hann-windowed, 512-point
+    zero-padded segment centred on sample 160 t of the preemphasised signal
+    (zeros outside [0, n_avail)), power spectrum by direct DFT, Slaney mel,
+    log(x + 2^-24)."""
+    from .frontend import hann_window_512, log_mel, preemphasis
+    y = preemphasis(np.asarray(audio[:n_avail], dt), n_avail, dt)
+    need = 160 * (m1 - 1) + 512                       # last padded sample used
+    ypad = np.zeros(max(need, n_avail + 512), dt)
+    ypad[256:256 + n_avail] = y
+    win = hann_window_512(dt)
+    frames = np.stack([ypad[160 * t: 160 * t + 512] for t in range(m0, m1)]) * win
+    k = np.arange(257)[:, None] * np.arange(512)[None, :]
+    X = frames @ np.exp(-2j * np.pi * k / 512).T
+    return log_mel(np.abs(X) ** 2, dt)
+
+
+def stream_step_audio(st, audio, n_avail, final, w, preset, dt=np.float64, taps=None):
+    """One audio-in step of one stream with n_avail samples received (final:
+    no more will come).  Returns the chunk probabilities, or None when the
+    window is not complete yet (its last frame's samples have not all
+    arrived) and the stream is not final."""
+    from .frontend import normalize_per_bin
+    L = n_avail // 160
+    c0 = st.c0
+    need = 8 * (c0 + preset.chunk_len + preset.right_context)
+    lc, m0, m1 = chunk_window(c0, L, preset)
+    if not final and n_avail < 160 * need + 96:
+        return None
+    if m1 <= 8 * c0:
+        return None
+    feats = np.zeros((128, m1), dt)
+    feats[:, m0:m1] = normalize_per_bin(window_log_mel(audio, n_avail, m0, m1, dt), m1 - m0, dt)
+    return stream_step(st, feats, m1, w, preset, dt, taps)
+
+
+def stream_run_audio(audio, n_total, w, preset, arrivals, dt=np.float64, taps=None):
+    """A stream fed by audio arriving in pieces: arrivals = increasing sample
+    counts received before each step (the last equal to n_total, marked
+    final).  Steps every arrival until the stream finishes; returns (probs
+    (T', 4), emitted frames per step)."""
+    st = StreamState(dt=dt)
+    T_enc = 1 + (n_total // 160 - 1) // 8
+    outs, per_step = [], []
+    k = 0
+    while st.c0 < T_enc:
+        n_avail = int(arrivals[min(k, len(arrivals) - 1)])
+        final = n_avail >= n_total
+        out = stream_step_audio(st, audio, n_avail, final, w, preset, dt, taps)
+        per_step.append(0 if out is None else len(out))
+        if out is not None:
+            outs.append(out)
+        if out is None and final:
+            break
+        k += 1
+    return (np.concatenate(outs) if outs else np.zeros((0, 4), dt)), per_step
