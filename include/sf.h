@@ -252,6 +252,30 @@ SF_API sf_status sf_stream_window(const sf_stream* s, int id, int64_t h_total, i
 SF_API sf_status sf_stream_step(sf_stream* s, const float* d_feats, int64_t t_buf, const int64_t* h_feat_start,
                          const int64_t* h_feat_end, float* d_chunk_probs, int* h_n_out, void* cuda_stream);
 
+/* Audio-in streaming step: the step computes each stream's mel window
+ * itself from raw audio instead of taking features.  Reading (the HF
+ * streaming notes slice the audio per chunk and run the processor on each
+ * slice, without saying how features are normalised; the NeMo API streams
+ * features normalised over the whole clip): the window's frames m0 .. m1-1
+ * are the centred frames of the stream's continuous signal (preemphasis and
+ * STFT exactly as sf_mel, zeros past the audio received so far), normalised
+ * per bin over the window's own frames (same formula as sf_mel over a clip).
+ *   d_audio        f32 [n_streams][n_buf]  row = stream; column 0 holds sample
+ *                  h_audio_start[id] of that stream, h_audio_end[id] samples
+ *                  (absolute) have arrived
+ *   h_final        i32 [n_streams]  1 once the stream's audio has ended
+ * A stream steps when its window is complete: its last frame (chunk plus
+ * right context) has all its samples, i.e. audio_end >= 160 x (8 x (c0 +
+ * chunk_len + right_context)) + 96 with c0 the next encoder frame; a final
+ * stream steps with what it has and finishes after its last frame.  Other
+ * streams emit 0 frames; a call where no stream is ready does nothing and
+ * returns SF_OK.  The buffer row must start no later than sample
+ * 160 x m0 - 257 of the window (m0 = 8 x (c0 - 1), 0 for the first step).
+ * Outputs as sf_stream_step. */
+SF_API sf_status sf_stream_step_audio(sf_stream* s, const float* d_audio, int64_t n_buf,
+                                      const int64_t* h_audio_start, const int64_t* h_audio_end, const int* h_final,
+                                      float* d_chunk_probs, int* h_n_out, void* cuda_stream);
+
 /* Copy one stream's state out to / in from caller buffers (forward_for_export
  * style state injection).  Synchronise on `cuda_stream`. */
 SF_API sf_status sf_stream_get_state(sf_stream* s, int id, sf_state_view* v, void* cuda_stream);

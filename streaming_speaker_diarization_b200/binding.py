@@ -58,7 +58,7 @@ EXPORTED = ["sf_default_config", "sf_create", "sf_create_from_file", "sf_destroy
             "sf_stream_window", "sf_stream_step", "sf_stream_get_state", "sf_stream_set_state",
             "sf_stream_update", "sf_select_topk", "sf_profile_enable", "sf_profile_read", "sf_mel_noalloc",
             "sf_check", "sf_gemm_bf16", "sf_set_option", "sf_attention_relpos", "sf_default_seg_params",
-            "sf_segments"]
+            "sf_segments", "sf_stream_step_audio"]
 
 
 class SFError(RuntimeError):
@@ -101,6 +101,7 @@ def _load():
         "sf_attention_relpos": ([VP, VP, VP, I, VP, VP, VP, I, VP, I, VP], I),
         "sf_default_seg_params": ([P(sf_seg_params)], I),
         "sf_segments": ([VP, VP, I, VP, I, P(sf_seg_params), I, VP, VP, VP], I),
+        "sf_stream_step_audio": ([VP, VP, I64, VP, VP, VP, VP, VP, VP], I),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -245,6 +246,17 @@ def sf_stream_step(eng, st, feats, feat_start, feat_end, chunk_probs, stream=Non
     n_out = np.zeros(len(feat_start), np.int32)
     _check(lib.sf_stream_step(st, _ptr(feats), feats.shape[-1], _ptr(feat_start), _ptr(feat_end), _ptr(chunk_probs),
                               _ptr(n_out), _stream(stream)), eng)
+    return n_out
+
+
+def sf_stream_step_audio(eng, st, audio, audio_start, audio_end, final, chunk_probs, stream=None):
+    """audio: device f32 [n_streams, n_buf]; returns frames emitted per stream."""
+    audio_start = np.ascontiguousarray(audio_start, np.int64)
+    audio_end = np.ascontiguousarray(audio_end, np.int64)
+    final = np.ascontiguousarray(final, np.int32)
+    n_out = np.zeros(len(audio_start), np.int32)
+    _check(lib.sf_stream_step_audio(st, _ptr(audio), audio.shape[1], _ptr(audio_start), _ptr(audio_end), _ptr(final),
+                                    _ptr(chunk_probs), _ptr(n_out), _stream(stream)), eng)
     return n_out
 
 

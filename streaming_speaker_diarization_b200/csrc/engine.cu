@@ -83,6 +83,9 @@ struct DescBlock {
   int count[MAX_SEQ];
   int dst[MAX_SEQ];
   int n_cand[MAX_SEQ];
+  int64_t win_f0[MAX_SEQ];   // audio-in steps: first mel frame of each window
+  int64_t win_a0[MAX_SEQ];   //   absolute sample of the stream's buffer column 0
+  int win_nf[MAX_SEQ];       //   mel frames of the window
   StepDesc step;
 };
 
@@ -1481,9 +1484,20 @@ void commit_sizes(sf_stream* s, const StepPlan& pl) {
   }
 }
 
+// Audio-in step inputs: stream buffers [n_streams][n_buf] (row = stream id,
+// column 0 = absolute sample start[id], end[id] samples arrived) and each
+// planned window's first mel frame m0[i].
+struct AudioIn {
+  const float* audio;
+  int64_t n_buf;
+  const int64_t* start;
+  const int64_t* end;
+  std::vector<int64_t> m0;
+};
+
 template <typename T>
 cudaError_t stream_step_impl(sf_stream* s, const float* d_feats, int64_t t_buf, const StepPlan& pl,
-                             float* d_chunk_probs, cudaStream_t st) {
+                             float* d_chunk_probs, cudaStream_t st, const AudioIn* ain = nullptr) {
   sf_engine* e = s->e;
   DescBlock* d = desc_begin(e);
   const int n = (int)pl.sid.size();
@@ -1493,6 +1507,18 @@ cudaError_t stream_step_impl(sf_stream* s, const float* d_feats, int64_t t_buf, 
     d->start[i] = pl.m0[i];
     d->frames[i] = pl.W[i];
     W_max = std::max(W_max, pl.W[i]);
+  }
+  if (ain) {   // audio-in step: the windows' features are computed from audio first
+    for (int i = 0; i < n; ++i) {
+      d->len[i] = ain->end[pl.sid[i]];
+      d->win_f0[i] = ain->m0[i];
+      d->win_a0[i] = ain->start[pl.sid[i]];
+      d->win_nf[i] = (int)pl.W[i];
+    }
+    CK(ensure(e->mel, (size_t)s->n * 128 * W_max * 4));   // rows by stream id, as the pre-encode reads them
+    CK(ensure(e->part, (size_t)n * ((W_max + 31) / 32) * 128 * 4 * 4));
+    d_feats = static_cast<const float*>(e->mel.p);
+    t_buf = W_max;
   }
   int M, tiles;
   fill_step(s, d, pl, M, tiles);
@@ -1505,9 +1531,20 @@ cudaError_t stream_step_impl(sf_stream* s, const float* d_feats, int64_t t_buf, 
                     std::to_string(W_max) + "|" +
                     std::to_string(t_buf) + "|" + std::to_string(reinterpret_cast<uintptr_t>(d_feats)) + "|" +
                     std::to_string(reinterpret_cast<uintptr_t>(d_chunk_probs));
+  if (ain) key += "|a" + std::to_string(reinterpret_cast<uintptr_t>(ain->audio)) + "|" + std::to_string(ain->n_buf);
   return run_graph(e, key, st, [&](cudaStream_t st) -> cudaError_t {
     CK(desc_upload(e, st));
     if (n < s->n) CK(cudaMemsetAsync(d_chunk_probs, 0, (size_t)s->n * s->p.chunk_len * 4 * 4, st));
+    if (ain) {
+      MelArgs ma{e->d_desc->len};
+      ma.f0 = e->d_desc->win_f0;
+      ma.a0 = e->d_desc->win_a0;
+      ma.nf = e->d_desc->win_nf;
+      ma.row = e->d_desc->buf;
+      RUN(K_MEL, 2, 0, (double)n * W_max * (160 * 4 + 128 * 4),
+          launch_mel_windows(ain->audio, n, ain->n_buf, ma, e->d_mel_tab, static_cast<float*>(e->mel.p),
+                             static_cast<float*>(e->part.p), (int)W_max, st));
+    }
     CK(run_pre_encode<T>(e, d_feats, t_buf, n, W_max, static_cast<T*>(e->emb.p), T3, st));
     RUN(K_ASSEMBLE, 1, 0, (double)M * e->cfg.d_model * (4 + sizeof(T)),
         launch_assemble<T>(static_cast<float*>(e->x.p), &e->d_desc->seq, &e->d_desc->step, s->sb,
@@ -1705,6 +1742,63 @@ sf_status sf_stream_update(sf_stream* s, const float* d_preds, const void* d_new
                                           static_cast<float*>(e->emb.p), (int)new_stride, n, d_scores, d_src,
                                           d_scores_in, score_stride, st);
   if (ce != cudaSuccess) return cuda_fail(e, ce, "sf_stream_update");
+  commit_sizes(s, pl);
+  return SF_OK;
+}
+
+sf_status sf_stream_step_audio(sf_stream* s, const float* d_audio, int64_t n_buf, const int64_t* h_audio_start,
+                               const int64_t* h_audio_end, const int* h_final, float* d_chunk_probs, int* h_n_out,
+                               void* cuda_stream) {
+  if (!s) return SF_EINVAL;
+  sf_engine* e = s->e;
+  if (check_engine(e) != SF_OK) return SF_EINVAL;
+  if (!d_audio || !h_audio_start || !h_audio_end || !h_final || !d_chunk_probs)
+    return fail(e, SF_EINVAL, "null pointer argument");
+  if (n_buf < 1) return fail(e, SF_ESHAPE, "n_buf must be positive");
+  StepPlan pl;
+  AudioIn ain{d_audio, n_buf, h_audio_start, h_audio_end, {}};
+  for (int id = 0; id < s->n; ++id) {
+    if (s->finished[id]) continue;
+    const int64_t a0 = h_audio_start[id], end = h_audio_end[id];
+    if (a0 < 0 || end < a0 || end - a0 > n_buf)
+      return fail(e, SF_ESHAPE, "stream " + std::to_string(id) + ": audio range outside its buffer row");
+    const int64_t c0 = s->c0[id];
+    const int lc = c0 > 0 ? 1 : 0;
+    const int64_t m0 = 8 * (c0 - lc);
+    const int64_t need = 8 * (c0 + s->p.chunk_len + s->p.right_context);   // mel frames of chunk + look-ahead
+    const int64_t m1 = std::min<int64_t>(need, end / 160);
+    // a window is ready once its last frame's samples have arrived (last
+    // frame centred at 160 (need - 1), reaching 256 samples past it), or at
+    // the end of the stream's audio
+    const bool ready = h_final[id] ? m1 > 8 * c0 : end >= 160 * need + 96;
+    if (!ready) continue;
+    if (a0 > std::max<int64_t>(0, 160 * m0 - 257))
+      return fail(e, SF_ESHAPE, "stream " + std::to_string(id) + ": buffer starts after the window's first samples");
+    const int64_t W = m1 - m0;
+    const int n_new = (int)(enc_frames(W) - lc);
+    int cl, npop;
+    plan_sizes(s, id, n_new, cl, npop);
+    pl.sid.push_back(id);
+    pl.lc.push_back(lc);
+    pl.n_new.push_back(n_new);
+    pl.cl.push_back(cl);
+    pl.npop.push_back(npop);
+    pl.m0.push_back(0);   // window-local features
+    pl.W.push_back(W);
+    ain.m0.push_back(m0);
+  }
+  if (h_n_out)
+    for (int id = 0; id < s->n; ++id) h_n_out[id] = 0;
+  if (pl.sid.empty()) return SF_OK;   // no stream has a full window yet
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  cudaError_t ce = e->cfg.precision == SF_BF16 ? stream_step_impl<bf16>(s, nullptr, 0, pl, d_chunk_probs, st, &ain)
+                                               : stream_step_impl<float>(s, nullptr, 0, pl, d_chunk_probs, st, &ain);
+  if (ce != cudaSuccess) return cuda_fail(e, ce, "sf_stream_step_audio");
+  for (size_t i = 0; i < pl.sid.size(); ++i) {
+    const int id = pl.sid[i];
+    if (h_n_out) h_n_out[id] = pl.cl[i];
+    if (h_final[id] && s->c0[id] + pl.cl[i] >= enc_frames(h_audio_end[id] / 160)) s->finished[id] = 1;
+  }
   commit_sizes(s, pl);
   return SF_OK;
 }

@@ -39,17 +39,20 @@ __global__ void __launch_bounds__(256) mel_frames_kernel(const float* __restrict
 
   const int b = blockIdx.y;
   const int blk = blockIdx.x;
-  const int t0 = blk * MEL_FB;
+  const int t0 = blk * MEL_FB;                    // first column of this tile
   const int64_t len = args.len[b];
-  const int L = (int)(len / 160);
-  const float* x = audio + (int64_t)b * n_max;
+  const bool win_mode = args.f0 != nullptr;
+  const int64_t fb = win_mode ? args.f0[b] : 0;   // absolute frame of column 0
+  const int64_t a0 = win_mode ? args.a0[b] : 0;   // absolute sample of buffer column 0
+  const int L = win_mode ? args.nf[b] : (int)(len / 160);
+  const float* x = audio + (int64_t)(win_mode ? args.row[b] : b) * n_max - a0;   // indexed by absolute sample
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
   for (int i = tid; i < 128; i += 256) tw256[i] = tab->tw256[i];
   for (int i = tid; i < 257; i += 256) tw512[i] = tab->tw512[i];   // slot 257 is padding
   for (int i = tid; i < 512; i += 256) win[i] = tab->win[i];
-  // span sample i <-> original sample n = 160*t0 - 256 + i
-  const int64_t n0 = (int64_t)160 * t0 - 256;
+  // span sample i <-> absolute sample n = 160*(fb + t0) - 256 + i
+  const int64_t n0 = (int64_t)160 * (fb + t0) - 256;
   for (int i = tid; i < MEL_SPAN; i += 256) {
     int64_t n = n0 + i;
     float v = 0.f;
@@ -129,7 +132,7 @@ __global__ void __launch_bounds__(256) mel_frames_kernel(const float* __restrict
   for (int i = tid; i < 128 * MEL_FB; i += 256) {
     int m = i / MEL_FB, f = i % MEL_FB;
     int t = t0 + f;
-    if (t < T_cols) mel[((int64_t)b * 128 + m) * T_cols + t] = tile[m][f];
+    if (t < T_cols) mel[((int64_t)(win_mode ? args.row[b] : b) * 128 + m) * T_cols + t] = tile[m][f];
   }
   // per-bin statistics of the valid frames of this tile, shifted by the
   // tile's first value so that a constant bin gives an exact mean
@@ -157,7 +160,7 @@ __global__ void __launch_bounds__(256) mel_normalize_kernel(float* __restrict__ 
                                                             const MelArgs args, int T_cols, int n_blk) {
   SF_PDL_ENTRY();
   const int m = blockIdx.x, b = blockIdx.y;
-  const int L = (int)(args.len[b] / 160);
+  const int L = args.nf ? args.nf[b] : (int)(args.len[b] / 160);
   __shared__ float s_mu, s_inv;
   __shared__ double sn[256], smean[256], sm2[256];
   // Chan's pairwise merge of the per-tile (count, mean, M2): each thread
@@ -196,7 +199,7 @@ __global__ void __launch_bounds__(256) mel_normalize_kernel(float* __restrict__ 
   }
   __syncthreads();
   const float mu = s_mu, inv = s_inv;
-  float* row = mel + ((int64_t)b * 128 + m) * T_cols;
+  float* row = mel + ((int64_t)(args.row ? args.row[b] : b) * 128 + m) * T_cols;
   for (int t = threadIdx.x; t < T_cols; t += blockDim.x) row[t] = (t < L) ? (row[t] - mu) * inv : 0.f;
 }
 
@@ -219,6 +222,21 @@ cudaError_t launch_mel(const float* audio, int B, int64_t n_max, const MelArgs& 
   }
   attr_set = true;
   CK_LAUNCH(launch_k(mel_frames_kernel, dim3(dim3(n_blk, B)), dim3(256), smem, st, audio, n_max, args, tab, mel, part, T_cols, n_blk));
+  CK_LAUNCH(launch_k(mel_normalize_kernel, dim3(dim3(128, B)), dim3(256), 0, st, mel, part, args, T_cols, n_blk));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mel_windows(const float* audio, int B, int64_t n_buf, const MelArgs& args, const MelTables* tab,
+                               float* mel, float* part, int T_cols, cudaStream_t st) {
+  const int n_blk = (T_cols + MEL_FB - 1) / MEL_FB;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = frontend_init_attributes();
+    if (e != cudaSuccess) return e;
+  }
+  attr_set = true;
+  CK_LAUNCH(launch_k(mel_frames_kernel, dim3(dim3(n_blk, B)), dim3(256), MEL_SMEM, st, audio, n_buf, args, tab, mel, part,
+                     T_cols, n_blk));
   CK_LAUNCH(launch_k(mel_normalize_kernel, dim3(dim3(128, B)), dim3(256), 0, st, mel, part, args, T_cols, n_blk));
   return cudaGetLastError();
 }

@@ -19,10 +19,22 @@ struct MelTables {
 
 struct MelArgs {
   const int64_t* len;            // device [B] clip lengths in samples
+  // window mode (all null for whole clips): clip b is frames f0[b] ..
+  // f0[b] + nf[b] - 1 of the audio in buffer row row[b], whose column 0 is
+  // sample a0[b]; len[b] samples have arrived (zeros beyond); statistics and
+  // normalisation over the window's nf[b] frames; features go to row row[b]
+  // of the output
+  const int64_t* f0 = nullptr;
+  const int64_t* a0 = nullptr;
+  const int* nf = nullptr;
+  const int* row = nullptr;
 };
 
 cudaError_t launch_mel(const float* audio, int B, int64_t n_max, const MelArgs& args, const MelTables* tab,
                        float* mel, float* part, cudaStream_t st);
+// Window mode: T_cols window columns per clip, buffer rows of n_buf samples.
+cudaError_t launch_mel_windows(const float* audio, int B, int64_t n_buf, const MelArgs& args, const MelTables* tab,
+                               float* mel, float* part, int T_cols, cudaStream_t st);
 size_t mel_part_floats(int B, int64_t n_max);
 cudaError_t frontend_init_attributes();
 void build_mel_tables(MelTables* t);   // host
