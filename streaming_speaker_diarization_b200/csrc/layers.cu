@@ -135,18 +135,18 @@ template <> struct Vec2<bf16> {
 
 // Each thread: two channels x DW_ROWS consecutive rows; the DW_ROWS + K - 1
 // input rows they need are loaded once into registers (32-row blocks keep
-// the halo re-read at K - 1 rows per 32 and the weight loads amortised).
+// the halo re-read at K - 1 rows per 32 and the weight loads amortised;
+// 8-row blocks give short inputs more CTAs).
 // Taps outside the output row's sequence read as zero.  Swish: exact expf and
 // division for f32 outputs; for bf16 outputs the hardware exp2 and an
 // approximate reciprocal (relative error ~1e-7, far inside bf16 rounding).
-constexpr int DW_ROWS = 32;
 constexpr int DW_KMAX = 9;
 template <typename T>
 __device__ __forceinline__ float dw_swish(float a) {
   if (sizeof(T) == 2) return a * __fdividef(1.f, 1.f + __expf(-a));
   return a / (1.f + expf(-a));
 }
-template <typename T>
+template <typename T, int DW_ROWS>
 __global__ void __launch_bounds__(128) dwconv1d_kernel(const T* __restrict__ in, T* __restrict__ out,
                                                        const float* __restrict__ w, const float* __restrict__ bias,
                                                        int M, int D, int K, const SeqTable* __restrict__ seq) {
@@ -212,8 +212,15 @@ cudaError_t launch_dwconv1d(const T* in, T* out, const float* w, const float* b,
                             const SeqTable* seq, cudaStream_t st) {
   if (M <= 0) return cudaSuccess;
   if (K > DW_KMAX || (D % 2)) return cudaErrorInvalidValue;
-  dim3 grid((M + DW_ROWS - 1) / DW_ROWS, (D / 2 + 127) / 128);
-  CK_LAUNCH(launch_k(dwconv1d_kernel<T>, dim3(grid), dim3(128), 0, st, in, out, w, b, M, D, K, seq));
+  // 32-row blocks when there are enough of them to fill the GPU (streaming
+  // batches); 8-row blocks for short inputs (one clip), where parallelism wins
+  if (M >= 32 * 2 * 148) {
+    dim3 grid((M + 31) / 32, (D / 2 + 127) / 128);
+    CK_LAUNCH(launch_k(dwconv1d_kernel<T, 32>, dim3(grid), dim3(128), 0, st, in, out, w, b, M, D, K, seq));
+  } else {
+    dim3 grid((M + 7) / 8, (D / 2 + 127) / 128);
+    CK_LAUNCH(launch_k(dwconv1d_kernel<T, 8>, dim3(grid), dim3(128), 0, st, in, out, w, b, M, D, K, seq));
+  }
   return cudaGetLastError();
 }
 
