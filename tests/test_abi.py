@@ -52,3 +52,19 @@ def test_create_without_device_fails_cleanly(lib_path):
     from synth import TINY, make_weights, weights_blob
     with pytest.raises(b.SFError):
         b.sf_create(weights_blob(make_weights(TINY)), b.default_config(n_conformer=2, n_transformer=2))
+
+
+def test_header_is_plain_c(tmp_path):
+    """include/sf.h compiles as strict C99 and as C++17 (no torch or CUDA
+    types in the boundary)."""
+    import shutil
+    src = tmp_path / "use_sf.c"
+    src.write_text('#include "sf.h"\nint main(void) { sf_config c; sf_seg_params p;\n'
+                   '  return sf_default_config(&c) + sf_default_seg_params(&p); }\n')
+    inc = os.path.join(ROOT, "include")
+    for cc, std, lang in (("gcc", "-std=c99", "c"), ("g++", "-std=c++17", "c++")):
+        if shutil.which(cc) is None:
+            pytest.skip(f"{cc} not available")
+        r = subprocess.run([cc, std, "-Wall", "-Wextra", "-pedantic", "-Werror", "-x", lang, "-I", inc, "-c", str(src),
+                            "-o", str(tmp_path / f"o_{lang}.o")], capture_output=True, text=True)
+        assert r.returncode == 0, r.stderr
