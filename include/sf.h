@@ -358,8 +358,8 @@ enum {
                             kernel */
   SF_OPT_GEMM_PAIR_BN = 4, /* tile width of the CTA-pair kernel: 0 (default) chosen per shape,
                               or 128, 192, 256 */
-  SF_OPT_ATTN_PATH = 5    /* bf16 relative-position attention: 1 (default) tcgen05/TMEM/TMA
-                             kernel, 0 mma.sync kernel */
+  SF_OPT_ATTN_PATH = 5    /* bf16 attention (relative-position and Transformer): 1 (default)
+                             tcgen05/TMEM/TMA kernels, 0 mma.sync kernels */
 };
 SF_API sf_status sf_set_option(sf_engine* e, int option, int value);
 
@@ -398,6 +398,19 @@ SF_API sf_status sf_gemm_bf16(sf_engine* e, const void* d_A, int lda, const void
 SF_API sf_status sf_attention_relpos(sf_engine* e, const void* d_qkv, const void* d_ptab, int R, const float* d_u,
                                      const float* d_v, const int* h_seq_len, int n, void* d_ctx, int path,
                                      void* cuda_stream);
+
+/* The Transformer encoder's self-attention alone (bf16 engines), for tests
+ * and kernel benchmarks ("Streaming Sortformer Diarizer" model card: 18-layer
+ * Transformer, d_model 192, 8 heads of 24):
+ *   d_qkv bf16 [M x 576]  rows of the n packed sequences (h_seq_len[i] rows
+ *                         each), columns q | k | v, head h at columns
+ *                         24h .. 24h + 23 of each part
+ *   d_ctx bf16 [M x 192] (out)  softmax_j(q_i . k_j / sqrt(24)) v_j
+ * Sequence lengths in [1, the engine's longest sequence]; path 1 = tcgen05
+ * kernel, 0 = mma.sync.  Pointers 16-byte aligned.  Uses the engine's
+ * descriptor block (ordered on `cuda_stream` with its other calls). */
+SF_API sf_status sf_attention_mha(sf_engine* e, const void* d_qkv, const int* h_seq_len, int n, void* d_ctx, int path,
+                                  void* cuda_stream);
 
 /* ---------------------------------------------------------------- profiling */
 

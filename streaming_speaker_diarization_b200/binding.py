@@ -58,7 +58,7 @@ EXPORTED = ["sf_default_config", "sf_create", "sf_create_from_file", "sf_destroy
             "sf_stream_window", "sf_stream_step", "sf_stream_get_state", "sf_stream_set_state",
             "sf_stream_update", "sf_select_topk", "sf_profile_enable", "sf_profile_read", "sf_mel_noalloc",
             "sf_check", "sf_gemm_bf16", "sf_set_option", "sf_attention_relpos", "sf_default_seg_params",
-            "sf_segments", "sf_stream_step_audio"]
+            "sf_segments", "sf_stream_step_audio", "sf_attention_mha"]
 
 
 class SFError(RuntimeError):
@@ -102,6 +102,7 @@ def _load():
         "sf_default_seg_params": ([P(sf_seg_params)], I),
         "sf_segments": ([VP, VP, I, VP, I, P(sf_seg_params), I, VP, VP, VP], I),
         "sf_stream_step_audio": ([VP, VP, I64, VP, VP, VP, VP, VP, VP], I),
+        "sf_attention_mha": ([VP, VP, VP, I, VP, I, VP], I),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -310,6 +311,11 @@ def sf_attention_relpos(eng, qkv, ptab, R, u, v, seq_len, ctx, path=1, stream=No
     seq_len = np.ascontiguousarray(seq_len, np.int32)
     _check(lib.sf_attention_relpos(eng, _ptr(qkv), _ptr(ptab), R, _ptr(u), _ptr(v), _ptr(seq_len), len(seq_len),
                                    _ptr(ctx), path, _stream(stream)), eng)
+
+
+def sf_attention_mha(eng, qkv, seq_len, ctx, path=1, stream=None):
+    seq_len = np.ascontiguousarray(seq_len, np.int32)
+    _check(lib.sf_attention_mha(eng, _ptr(qkv), _ptr(seq_len), len(seq_len), _ptr(ctx), path, _stream(stream)), eng)
 
 
 def seg_params(**kw):

@@ -590,6 +590,19 @@ cudaError_t gemm_dispatch<bf16>(sf_engine* e, const bf16* A, int lda, const bf16
   return gemm_bf16_mma(A, lda, W, M, N, K, ep, st);
 }
 
+// Transformer MHSA: on tcgen05 in the bf16 engine unless the mma.sync kernel
+// is selected (SF_OPT_ATTN_PATH = 0).
+template <typename T>
+cudaError_t mha_attention(sf_engine* e, const T* qkv, T* ctx, const SeqTable* seq, int n_tiles, int M, cudaStream_t st) {
+  return launch_mha<T>(qkv, ctx, seq, n_tiles, M, st);
+}
+template <>
+cudaError_t mha_attention<bf16>(sf_engine* e, const bf16* qkv, bf16* ctx, const SeqTable* seq, int n_tiles, int M,
+                                cudaStream_t st) {
+  if (e->attn_path == 1) return launch_mha_tc(qkv, ctx, seq, e->att_tiles2, M, e->d_err, st);
+  return launch_mha<bf16>(qkv, ctx, seq, n_tiles, M, st);
+}
+
 // Relative-position attention: the bf16 engine runs it on tcgen05 unless the
 // mma.sync kernel is selected (SF_OPT_ATTN_PATH = 0).
 template <typename T>
@@ -855,7 +868,7 @@ cudaError_t run_encode(sf_engine* e, int M, int n_tiles, float* probs, cudaStrea
   for (int l = 0; l < c.n_transformer; ++l) {
     const TfW<T>& w = W.tf[l];
     CK(gemm_acc<T>(e, h2, E, w.wqkv, M, 3 * E, E, epi(EPI_BIAS, w.bqkv, big, 3 * E), st));
-    RUN(K_ATT_MHA, 1, 4.0 * e->att_s2 * E, (double)M * 4 * E * sizeof(T), launch_mha<T>(big, ctx, seq, n_tiles, M, st));
+    RUN(K_ATT_MHA, 1, 4.0 * e->att_s2 * E, (double)M * 4 * E * sizeof(T), mha_attention<T>(e, big, ctx, seq, n_tiles, M, st));
     CK(gemm_acc<T>(e, ctx, E, w.wo, M, E, E, epi(EPI_RESID, w.bo, x2, E, 1.f), st));
     RUN(K_LN, 1, 0, (double)M * E * (4 + sizeof(T) + (true ? 4 : 0)),
         launch_layernorm<T>(x2, w.ln1_g, w.ln1_b, M, E, true, h2, st));
@@ -1038,6 +1051,7 @@ sf_status sf_create(const void* blob, uint64_t nbytes, const sf_config* cfg, sf_
   if ((ce = gemm_init_attributes()) != cudaSuccess) return cuda_fail(e.get(), ce, "init"), SF_ECUDA;
   if ((ce = attention_init_attributes()) != cudaSuccess) return SF_ECUDA;
   if ((ce = attention_tc_init_attributes()) != cudaSuccess) return SF_ECUDA;
+  if ((ce = attention_mha_tc_init_attributes()) != cudaSuccess) return SF_ECUDA;
   if ((ce = gemm_tc_init_attributes()) != cudaSuccess) return SF_ECUDA;
   if ((ce = frontend_init_attributes()) != cudaSuccess) return SF_ECUDA;
   if ((ce = attention_init_f32_attributes(e->R)) != cudaSuccess) return SF_ECUDA;
@@ -1301,6 +1315,32 @@ sf_status sf_attention_relpos(sf_engine* e, const void* d_qkv, const void* d_pta
                                                 *std::max_element(lens.begin(), lens.end()), e->tc_scratch(), st)
                    : launch_relpos_attention<bf16>(qkv, ptab, R, d_u, d_v, ctx, &e->d_desc->seq, tiles, M, st);
   if (ce != cudaSuccess) return cuda_fail(e, ce, "sf_attention_relpos");
+  return SF_OK;
+}
+
+sf_status sf_attention_mha(sf_engine* e, const void* d_qkv, const int* h_seq_len, int n, void* d_ctx, int path,
+                           void* cuda_stream) {
+  if (check_engine(e) != SF_OK) return SF_EINVAL;
+  if (!d_qkv || !h_seq_len || !d_ctx) return fail(e, SF_EINVAL, "null pointer argument");
+  if (e->cfg.precision != SF_BF16) return fail(e, SF_ESTATE, "sf_attention_mha needs a bf16 engine");
+  if (n < 1 || n > MAX_SEQ || (path != 0 && path != 1)) return fail(e, SF_ESHAPE, "sequence count or path");
+  if ((reinterpret_cast<uintptr_t>(d_qkv) | reinterpret_cast<uintptr_t>(d_ctx)) & 15)
+    return fail(e, SF_EINVAL, "qkv and ctx must be 16-byte aligned");
+  std::vector<int> lens(h_seq_len, h_seq_len + n);
+  for (int v : lens)
+    if (v < 1 || v > e->max_seq_len) return fail(e, SF_ESHAPE, "sequence length out of range");
+  DescBlock* d = desc_begin(e);
+  int M, tiles;
+  fill_seq(d, lens, M, tiles);
+  const int tiles2 = d->seq.tile2_off[n];
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  cudaError_t ce = desc_upload(e, st);
+  const bf16* qkv = static_cast<const bf16*>(d_qkv);
+  bf16* ctx = static_cast<bf16*>(d_ctx);
+  if (ce == cudaSuccess)
+    ce = path == 1 ? launch_mha_tc(qkv, ctx, &e->d_desc->seq, tiles2, M, e->d_err, st)
+                   : launch_mha<bf16>(qkv, ctx, &e->d_desc->seq, tiles, M, st);
+  if (ce != cudaSuccess) return cuda_fail(e, ce, "sf_attention_mha");
   return SF_OK;
 }
 
