@@ -150,6 +150,7 @@ struct ProfRec {
 struct sf_engine {
   sf_config cfg{};
   int device = 0;
+  int n_sms = 148;        // streaming multiprocessors of the device
   std::string err;
   int R = 0;              // position-table half length (longest sequence)
   int max_seq_len = 0;
@@ -590,8 +591,11 @@ cudaError_t gemm_dispatch<bf16>(sf_engine* e, const bf16* A, int lda, const bf16
   return gemm_bf16_mma(A, lda, W, M, N, K, ep, st);
 }
 
-// Transformer MHSA: on tcgen05 in the bf16 engine unless the mma.sync kernel
-// is selected (SF_OPT_ATTN_PATH = 0).
+// Transformer MHSA in the bf16 engine: the tcgen05 kernel when its 128-row
+// (tile, head) units fill the SMs (streaming batches: measured 2-3 % faster
+// steps), the mma.sync kernel otherwise (one long clip: its 64-row CTAs
+// cover twice as many SMs; 0.34 vs 0.40 ms per 90 s forward); always
+// mma.sync with SF_OPT_ATTN_PATH = 0.
 template <typename T>
 cudaError_t mha_attention(sf_engine* e, const T* qkv, T* ctx, const SeqTable* seq, int n_tiles, int M, cudaStream_t st) {
   return launch_mha<T>(qkv, ctx, seq, n_tiles, M, st);
@@ -599,7 +603,8 @@ cudaError_t mha_attention(sf_engine* e, const T* qkv, T* ctx, const SeqTable* se
 template <>
 cudaError_t mha_attention<bf16>(sf_engine* e, const bf16* qkv, bf16* ctx, const SeqTable* seq, int n_tiles, int M,
                                 cudaStream_t st) {
-  if (e->attn_path == 1) return launch_mha_tc(qkv, ctx, seq, e->att_tiles2, M, e->d_err, st);
+  if (e->attn_path == 1 && e->att_tiles2 * 8 >= e->n_sms)
+    return launch_mha_tc(qkv, ctx, seq, e->att_tiles2, M, e->d_err, st);
   return launch_mha<bf16>(qkv, ctx, seq, n_tiles, M, st);
 }
 
@@ -1044,6 +1049,10 @@ sf_status sf_create(const void* blob, uint64_t nbytes, const sf_config* cfg, sf_
   std::unique_ptr<sf_engine> e(new sf_engine());
   e->cfg = *cfg;
   e->device = dev;
+  {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0) e->n_sms = n;
+  }
   e->R = (int)std::max<int64_t>(enc_frames(cfg->max_samples / 160), 188 + 188 + 340 + 40);
   e->max_seq_len = e->R;
   sf::attention_set_max_seq(e->R);
