@@ -2,12 +2,13 @@
 
     python -m streaming_speaker_diarization_b200.kbench gemm M N K [--epi E] [--path P] [--reps R]
     python -m streaming_speaker_diarization_b200.kbench attn N_SEQ LEN [--path P] [--reps R]
+    python -m streaming_speaker_diarization_b200.kbench mha N_SEQ LEN [--path P] [--reps R]
 
 `gemm` runs sf_gemm_bf16 (E: 1 f32 out, 2 bf16 out, 3 residual update, 4
 swish, 5 gated linear unit; P: SF_OPT_GEMM_PATH, 1 = tcgen05 with CTA pairs
 where faster, 2 = CTA pairs always, 3 = single CTAs, 0 = mma.sync); `attn`
-runs sf_attention_relpos on N_SEQ packed sequences of LEN rows (P: 1 tcgen05,
-0 mma.sync).  Operands are seeded random values on the device; three warm-up
+runs sf_attention_relpos and `mha` sf_attention_mha on N_SEQ packed
+sequences of LEN rows (P: 1 tcgen05, 0 mma.sync).  Operands are seeded random values on the device; three warm-up
 launches, then REPS launches queued behind a GPU sleep (so host launch
 overhead is hidden) and timed with CUDA events on the current stream.  Also
 the driver for single-kernel ncu captures (small REPS)."""
@@ -54,6 +55,11 @@ def main(argv=None):
     a.add_argument("length", type=int)
     a.add_argument("--path", type=int, default=1)
     a.add_argument("--reps", type=int, default=20)
+    m = sub.add_parser("mha")
+    m.add_argument("n_seq", type=int)
+    m.add_argument("length", type=int)
+    m.add_argument("--path", type=int, default=1)
+    m.add_argument("--reps", type=int, default=20)
     args = ap.parse_args(argv)
 
     import torch
@@ -73,6 +79,16 @@ def main(argv=None):
         ms = _time(torch, lambda: b.sf_gemm_bf16(eng, A, W, C, path=path), args.reps)
         print(f"gemm M={M} N={N} K={K} epi={args.epi} path={args.path}: {ms * 1e3:.1f} us/launch, "
               f"{2 * M * N * K / ms / 1e9:.1f} TFLOP/s")
+    elif args.op == "mha":
+        n, L = args.n_seq, args.length
+        eng = _engine(b, max(n, 8))
+        qkv = torch.randn(n * L, 576, device="cuda", generator=gen).to(torch.bfloat16)
+        ctx = torch.empty(n * L, 192, device="cuda", dtype=torch.bfloat16)
+        lens = np.full(n, L, np.int32)
+        ms = _time(torch, lambda: b.sf_attention_mha(eng, qkv, lens, ctx, path=args.path), args.reps)
+        flops = 2 * 2 * n * L * L * 192
+        print(f"mha n={n} L={L} path={args.path}: {ms * 1e3:.1f} us/launch, {flops / ms / 1e9:.1f} TFLOP/s "
+              f"(2 x 2 x L^2 x 192 per sequence)")
     else:
         n, L = args.n_seq, args.length
         eng = _engine(b, max(n, 8))
