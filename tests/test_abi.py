@@ -68,3 +68,17 @@ def test_header_is_plain_c(tmp_path):
         r = subprocess.run([cc, std, "-Wall", "-Wextra", "-pedantic", "-Werror", "-x", lang, "-I", inc, "-c", str(src),
                             "-o", str(tmp_path / f"o_{lang}.o")], capture_output=True, text=True)
         assert r.returncode == 0, r.stderr
+
+
+def test_host_only_entries_work_without_a_device(lib_path):
+    """Defaults and status strings are host functions: usable on a machine
+    without a GPU."""
+    from streaming_speaker_diarization_b200 import binding as b
+    p = b.seg_params()
+    assert (p.onset, p.offset, p.pad_onset, p.pad_offset, p.min_duration_on, p.min_duration_off) == \
+        (0.5, 0.5, 0.0, 0.0, 0.0, 0.0)
+    q = b.seg_params(onset=0.7, min_duration_off=0.2)
+    assert abs(q.onset - 0.7) < 1e-7 and q.min_duration_off == 0.2 and q.offset == 0.5
+    c = b.default_config()
+    assert c.sample_rate == 16000 and c.n_conformer == 17 and c.n_transformer == 18
+    assert b.lib.sf_status_str(0)
