@@ -8,6 +8,10 @@ N(0, 0.02) from seed 0: front-end -> probabilities, all in the engine's
 kernels.  Inputs are resident in HBM when the timed region starts; L2 is
 flushed (256 MiB write) between timed steps.
 
+Also in the line: the two streaming workloads (`streaming`: Low preset 64 x
+60 s, Very high preset 16 x 600 s) and the front-end alone on 1 h of audio
+(`frontend_1h`, HBM roofline).
+
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 Multi-GPU (torchrun, one process per GPU): the path has no exchange step, so
@@ -192,6 +196,50 @@ def streaming_bench(b, torch, eng_blob, rank, world, local):
     return out
 
 
+def frontend_bench(b, torch, blob, steps, warmup):
+    """Front-end alone (preemphasis, centred STFT, power, Slaney mel, log,
+    per-bin normalisation) on 1 h of audio in one sf_mel call: 57.6M samples
+    -> 128 x 360,001 features.  Audio resident on the device, CUDA events per
+    call on the launching stream; the 230 MB input and 184 MB output exceed
+    L2, which is also flushed between calls.  Roofline: HBM, algorithmic
+    bytes = 4 B per sample in + 128 x 4 B per feature column out."""
+    from synth.audio import hour_of_audio
+    x = hour_of_audio()
+    n = len(x)
+    T = 1 + n // 160
+    eng = b.sf_create(blob, b.default_config(max_batch=1, max_samples=n))
+    try:
+        audio = torch.from_numpy(x[None]).cuda()
+        mel = torch.empty((1, 128, T), device="cuda")
+        lens = np.array([n], np.int64)
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+        st = torch.cuda.current_stream()
+        for _ in range(warmup):
+            b.sf_mel(eng, audio, lens, mel)
+        b.sf_check(eng)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        torch.cuda.synchronize()
+        for i in range(steps):
+            flush.zero_()
+            ev[i][0].record(st)
+            b.sf_mel(eng, audio, lens, mel)
+            ev[i][1].record(st)
+        torch.cuda.synchronize()
+        b.sf_check(eng)
+    finally:
+        b.sf_destroy(eng)
+    ms = [a.elapsed_time(c) for a, c in ev]
+    med = float(np.median(ms))
+    alg = 4.0 * n + 4.0 * 128 * T
+    pk, kind = peaks()
+    gbs = alg / (med / 1000.0) / 1e9
+    return {"workload": "front-end only, 1 h of audio (60 x 60 s clips joined), 57.6M samples -> 128 x 360,001",
+            "value": 3600.0 / (med / 1000.0), "unit": UNIT, "ms_p50": med, "ms_p95": float(np.percentile(ms, 95)),
+            "calls": steps,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / pk["hbm_gbs"], "bytes_per_call": alg, "peak_kind": f"{kind} copy"}}
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return 0
@@ -230,6 +278,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--pdl", type=int, default=0, help="programmatic dependent launch between kernels (0/1)")
     ap.add_argument("--no-streaming", action="store_true", help="skip the streaming workloads")
+    ap.add_argument("--no-frontend", action="store_true", help="skip the 1 h front-end-only run")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
@@ -345,6 +394,8 @@ def main():
     b.sf_destroy(eng)
     if not args.no_streaming:
         line["streaming"] = streaming_bench(b, torch, weights_blob(w), rank, world, local)
+    if not args.no_frontend:
+        line["frontend_1h"] = frontend_bench(b, torch, weights_blob(w), max(args.steps, 5), max(args.warmup, 3))
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(audio_np)
     if rank == 0:

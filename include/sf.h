@@ -137,8 +137,12 @@ SF_API sf_status sf_default_config(sf_config* cfg);
  * precision, BatchNorm is folded into the depthwise conv, the relative
  * position projections are precomputed for every distance up to the longest
  * sequence the configuration allows, and the workspace is allocated.  The
- * blob may be freed after the call.  Synchronises.  Errors: SF_EINVAL,
- * SF_EFORMAT (missing/mis-shaped tensor), SF_EDEVICE, SF_ENOMEM. */
+ * blob may be freed after the call.  Synchronises.  max_samples may reach
+ * 4 h (230,400,000) in bf16; an fp32 engine keeps one attention score row
+ * per warp in shared memory, which bounds its sequences to 14,000 encoder
+ * frames (max_samples <= 17,920,159, about 18.7 min).  Errors: SF_EINVAL,
+ * SF_ESHAPE (fp32 with a longer max_samples), SF_EFORMAT (missing/mis-shaped
+ * tensor), SF_EDEVICE, SF_ENOMEM. */
 SF_API sf_status sf_create(const void* h_blob, uint64_t nbytes, const sf_config* cfg, sf_engine** out);
 SF_API sf_status sf_create_from_file(const char* path, const sf_config* cfg, sf_engine** out);
 SF_API sf_status sf_destroy(sf_engine* e);

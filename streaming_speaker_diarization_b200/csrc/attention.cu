@@ -14,6 +14,7 @@
 // a per-warp shared tile and is read back along the i - j diagonal.  Online
 // softmax in fp32 (exp2 with the scale folded in), P.V from registers.
 // fp32 path: one warp per query row (used by the fp32 engine mode).
+#include <mutex>
 #include "common.cuh"
 #include "layers.h"
 
@@ -382,7 +383,6 @@ __global__ void __launch_bounds__(256) attn_bf16_kernel(const bf16* __restrict__
 }
 
 // ---------------------------------------------------------------- launchers
-static int g_att_s_cap = 0;
 
 template <>
 cudaError_t launch_relpos_attention<float>(const float* qkv, const float* ptab, int R, const float* u, const float* v,
@@ -404,9 +404,10 @@ cudaError_t launch_relpos_attention<bf16>(const bf16* qkv, const bf16* ptab, int
 }
 
 template <>
-cudaError_t launch_mha<float>(const float* qkv, float* ctx, const SeqTable* seq, int n_tiles, int M, cudaStream_t st) {
+cudaError_t launch_mha<float>(const float* qkv, float* ctx, const SeqTable* seq, int n_tiles, int M, int R,
+                              cudaStream_t st) {
   if (M <= 0) return cudaSuccess;
-  const int s_cap = g_att_s_cap;
+  const int s_cap = R;   // no sequence is longer than R rows
   const size_t smem = (size_t)4 * (s_cap + 128) * 4;
   CK_LAUNCH(launch_k(attn_f32_kernel<24, false>, dim3(dim3((M + 3) / 4, 8)), dim3(128), smem, st, qkv, 192, nullptr, 0, nullptr, nullptr, ctx, seq,
                                                                       M, s_cap));
@@ -414,21 +415,32 @@ cudaError_t launch_mha<float>(const float* qkv, float* ctx, const SeqTable* seq,
 }
 
 template <>
-cudaError_t launch_mha<bf16>(const bf16* qkv, bf16* ctx, const SeqTable* seq, int n_tiles, int M, cudaStream_t st) {
+cudaError_t launch_mha<bf16>(const bf16* qkv, bf16* ctx, const SeqTable* seq, int n_tiles, int M, int /*R*/,
+                             cudaStream_t st) {
   if (M <= 0) return cudaSuccess;
   CK_LAUNCH(launch_k(attn_bf16_kernel<24, 32, false>, dim3(dim3(n_tiles, 8)), dim3(256), AttCfg<24, 32, false>::SMEM, st, 
       qkv, 192, nullptr, 0, nullptr, nullptr, ctx, seq));
   return cudaGetLastError();
 }
 
-void attention_set_max_seq(int s) { g_att_s_cap = s; }
-
 // fp32 path: one score row of up to R floats per warp (4 warps per CTA).
-cudaError_t attention_init_f32_attributes(int R) {
+// The shared-memory limit is a per-kernel attribute of the process, so it
+// only ever grows: an engine made for shorter sequences never lowers what
+// an earlier engine's launches need.
+int attention_f32_max_seq() { return 14000; }   // 4 x (14000 + 128) floats = 221 KB
+
+cudaError_t attention_reserve_f32(int R) {
+  static std::mutex mu;
+  static int reserved = 0;
+  if (R < 1 || R > attention_f32_max_seq()) return cudaErrorInvalidValue;
+  std::lock_guard<std::mutex> lock(mu);
+  if (R <= reserved) return cudaSuccess;
   const int smem = 4 * (R + 128) * 4;
   cudaError_t e = cudaFuncSetAttribute(attn_f32_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(attn_f32_kernel<24, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(attn_f32_kernel<24, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess) reserved = R;
+  return e;
 }
 
 cudaError_t attention_init_attributes() {

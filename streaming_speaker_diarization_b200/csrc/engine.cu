@@ -598,14 +598,14 @@ cudaError_t gemm_dispatch<bf16>(sf_engine* e, const bf16* A, int lda, const bf16
 // mma.sync with SF_OPT_ATTN_PATH = 0.
 template <typename T>
 cudaError_t mha_attention(sf_engine* e, const T* qkv, T* ctx, const SeqTable* seq, int n_tiles, int M, cudaStream_t st) {
-  return launch_mha<T>(qkv, ctx, seq, n_tiles, M, st);
+  return launch_mha<T>(qkv, ctx, seq, n_tiles, M, e->R, st);
 }
 template <>
 cudaError_t mha_attention<bf16>(sf_engine* e, const bf16* qkv, bf16* ctx, const SeqTable* seq, int n_tiles, int M,
                                 cudaStream_t st) {
   if (e->attn_path == 1 && e->att_tiles2 * 8 >= e->n_sms)
     return launch_mha_tc(qkv, ctx, seq, e->att_tiles2, M, e->d_err, st);
-  return launch_mha<bf16>(qkv, ctx, seq, n_tiles, M, st);
+  return launch_mha<bf16>(qkv, ctx, seq, n_tiles, M, e->R, st);
 }
 
 // Relative-position attention: the bf16 engine runs it on tcgen05 unless the
@@ -1055,7 +1055,7 @@ sf_status sf_create(const void* blob, uint64_t nbytes, const sf_config* cfg, sf_
   }
   e->R = (int)std::max<int64_t>(enc_frames(cfg->max_samples / 160), 188 + 188 + 340 + 40);
   e->max_seq_len = e->R;
-  sf::attention_set_max_seq(e->R);
+  if (cfg->precision == SF_FP32 && e->R > attention_f32_max_seq()) return SF_ESHAPE;
   cudaError_t ce;
   if ((ce = gemm_init_attributes()) != cudaSuccess) return cuda_fail(e.get(), ce, "init"), SF_ECUDA;
   if ((ce = attention_init_attributes()) != cudaSuccess) return SF_ECUDA;
@@ -1063,7 +1063,7 @@ sf_status sf_create(const void* blob, uint64_t nbytes, const sf_config* cfg, sf_
   if ((ce = attention_mha_tc_init_attributes()) != cudaSuccess) return SF_ECUDA;
   if ((ce = gemm_tc_init_attributes()) != cudaSuccess) return SF_ECUDA;
   if ((ce = frontend_init_attributes()) != cudaSuccess) return SF_ECUDA;
-  if ((ce = attention_init_f32_attributes(e->R)) != cudaSuccess) return SF_ECUDA;
+  if (cfg->precision == SF_FP32 && (ce = attention_reserve_f32(e->R)) != cudaSuccess) return SF_ECUDA;
   g_ws_gen = &e->ws_gen;
   std::unordered_map<std::string, TensorRef> m;
   std::string err;
@@ -1348,7 +1348,7 @@ sf_status sf_attention_mha(sf_engine* e, const void* d_qkv, const int* h_seq_len
   bf16* ctx = static_cast<bf16*>(d_ctx);
   if (ce == cudaSuccess)
     ce = path == 1 ? launch_mha_tc(qkv, ctx, &e->d_desc->seq, tiles2, M, e->d_err, st)
-                   : launch_mha<bf16>(qkv, ctx, &e->d_desc->seq, tiles, M, st);
+                   : launch_mha<bf16>(qkv, ctx, &e->d_desc->seq, tiles, M, e->max_seq_len, st);
   if (ce != cudaSuccess) return cuda_fail(e, ce, "sf_attention_mha");
   return SF_OK;
 }

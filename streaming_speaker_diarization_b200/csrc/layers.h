@@ -97,8 +97,11 @@ cudaError_t launch_to_f32(const T* in, float* out, int64_t n, cudaStream_t st);
 // d_dst (null = identity) gives the output row block of each sequence.
 cudaError_t launch_extract_rows(const float* packed, const SeqTable* seq, const int* d_first, const int* d_count,
                                 const int* d_dst, int n_seq, float* out, int t_max, cudaStream_t st);
-void attention_set_max_seq(int s);
-cudaError_t attention_init_f32_attributes(int R);
+// fp32 attention: sequences up to attention_f32_max_seq() rows (one score
+// row per warp in shared memory); attention_reserve_f32(R) raises the
+// kernels' shared-memory limit to cover R rows (never lowers it).
+int attention_f32_max_seq();
+cudaError_t attention_reserve_f32(int R);
 
 // ------------------------------------------------------- post-processing
 struct SegArgs {
@@ -120,9 +123,10 @@ cudaError_t launch_segments(const float* probs, int stride_t, const int* d_n_fra
 template <typename T>
 cudaError_t launch_relpos_attention(const T* qkv, const T* ptab, int R, const float* u, const float* v, T* ctx,
                                     const SeqTable* seq, int n_tiles, int M, cudaStream_t st);
-// Plain MHSA (d 192, 8 heads of 24), qkv act [M x 576] -> ctx act [M x 192].
+// Plain MHSA (d 192, 8 heads of 24), qkv act [M x 576] -> ctx act [M x 192];
+// R bounds the sequence lengths (used by the fp32 kernel's score rows).
 template <typename T>
-cudaError_t launch_mha(const T* qkv, T* ctx, const SeqTable* seq, int n_tiles, int M, cudaStream_t st);
+cudaError_t launch_mha(const T* qkv, T* ctx, const SeqTable* seq, int n_tiles, int M, int R, cudaStream_t st);
 cudaError_t attention_init_attributes();
 // bf16 relative-position MHSA on tcgen05 (one CTA per 128 query rows x head
 // x key split; n_tiles2 = 128-row tiles of the sequence table, max_len the

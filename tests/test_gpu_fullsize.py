@@ -88,3 +88,32 @@ def test_very_high_preset_16_streams_first_step(weights):
         assert ref.shape == (340, 4)
         err = np.max(np.abs(got[i][:340] - ref))
         assert err <= 2e-2, (i, err)
+
+
+def test_offline_batch_32_clips(weights):
+    """The variable-length batch: 32 clips of 5-120 s (seeded), padded to the
+    longest, in one offline call of the full model (bf16).  Output lengths
+    are 1 + (L - 1) // 8, padded rows are zero, and the shortest, a middle
+    and the longest clip match the oracle run on that clip alone (2e-2)."""
+    audio, lens, _ = clip_for_config(4)
+    B, n_max = audio.shape
+    eng = make_engine(weights, 1, 17, 18, max_batch=32, max_samples=int(n_max))
+    try:
+        Tp = int(O.encoder_frames(n_max // 160))
+        probs = torch.full((B, Tp, 4), float("nan"), device="cuda")
+        out_len = b.sf_forward_offline(eng, to_dev(audio), lens, probs)
+        b.sf_check(eng)
+    finally:
+        b.sf_destroy(eng)
+    got = probs.cpu().numpy()
+    T = np.array([int(O.encoder_frames(int(n) // 160)) for n in lens])
+    assert np.array_equal(np.asarray(out_len), T)
+    for i in range(B):
+        assert np.all(got[i, T[i]:] == 0), i
+        assert np.all(np.isfinite(got[i])) and got[i].min() >= 0 and got[i].max() <= 1, i
+    order = np.argsort(lens)
+    for i in (int(order[0]), int(order[B // 2]), int(order[-1])):
+        ref, tp = O.forward_offline(audio[i:i + 1, :lens[i]], lens[i:i + 1], weights)
+        assert tp[0] == T[i]
+        err = np.max(np.abs(got[i, :T[i]] - ref[0]))
+        assert err <= 2e-2, (i, err)

@@ -209,6 +209,58 @@ def test_offline_bf16_full_xavier_sampled_frames():
         b.sf_destroy(eng)
 
 
+def test_mel_one_hour():
+    """Front-end on 1 h of audio in one call (57.6M samples, 360,001 STFT
+    columns, 360,000 valid frames; the front-end throughput workload): every
+    feature against the oracle's front-end on the same hour (1e-3)."""
+    from synth.audio import hour_of_audio
+    x = hour_of_audio()
+    n = len(x)
+    eng = make_engine(tiny_weights(), 1, 2, 2, max_batch=1, max_samples=n)
+    try:
+        got, ml = gpu_mel(eng, x[None], np.array([n]))
+        b.sf_check(eng)
+    finally:
+        b.sf_destroy(eng)
+    ref, L = O.mel_features(x[None], np.array([n]))
+    assert int(ml[0]) == int(L[0]) == 360_000 and got.shape == ref.shape == (1, 128, 360_001)
+    assert np.all(got[0, :, 360_000] == 0)
+    err = np.max(np.abs(got - ref))
+    assert err <= 1e-3, err
+
+
+def test_fp32_engines_of_different_lengths_coexist():
+    """Two fp32 engines in one process: one for clips up to 120 s, then one
+    for clips up to 10 s.  The first still runs a 75 s clip (938 encoder
+    frames: longer attention rows than any sequence of the second engine)
+    after the second was made; probabilities within 1e-4."""
+    w = tiny_weights(xavier=True)
+    e1 = make_engine(w, 0, 2, 2, max_batch=1)
+    e2 = make_engine(w, 0, 2, 2, max_batch=1, max_samples=160_000)
+    try:
+        audio, lens, _ = synth_batch(91, [75.0])
+        T = int(O.encoder_frames(audio.shape[1] // 160))
+        probs = torch.zeros((1, T, 4), device="cuda")
+        b.sf_forward_offline(e1, to_dev(audio), lens, probs)
+        b.sf_check(e1)
+        ref, tp = O.forward_offline(audio, lens, w)
+        assert tp[0] == T == 938
+        assert np.max(np.abs(probs.cpu().numpy()[0] - ref[0])) <= 1e-4
+    finally:
+        b.sf_destroy(e2)
+        b.sf_destroy(e1)
+
+
+def test_fp32_engine_length_bound():
+    """fp32 attention keeps a score row per warp in shared memory: 14,000
+    encoder frames at most (max_samples 17,920,159); one sample more is
+    rejected at creation."""
+    w = tiny_weights()
+    with pytest.raises(b.SFError, match="SF_ESHAPE"):
+        make_engine(w, 0, 2, 2, max_batch=1, max_samples=17_920_160)
+    b.sf_destroy(make_engine(w, 0, 2, 2, max_batch=1, max_samples=17_920_159))
+
+
 def test_bad_arguments_rejected(eng_fp32):
     audio = to_dev(np.zeros((1, 1000), np.float32))
     probs = torch.zeros((1, 10, 4), device="cuda")
