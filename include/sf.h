@@ -30,7 +30,11 @@
  *  - An engine or stream object must not be used from two host threads at
  *    once, and calls on one engine must be ordered: issue them on one CUDA
  *    stream (or order the streams yourself), because every call reuses the
- *    engine's workspace and descriptor block.
+ *    engine's workspace and descriptor block.  Different engines may be
+ *    driven from different host threads (e.g. one engine and one thread
+ *    per GPU); the GEMM kernel selection (SF_OPT_GEMM_PATH,
+ *    SF_OPT_GEMM_PAIR_BN) is then shared by the process, so give those
+ *    engines the same values.
  */
 #ifndef SF_H_
 #define SF_H_

@@ -100,9 +100,9 @@ __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.lau
     if (_le != cudaSuccess) return _le; \
   } while (0)
 
-// Launch mode of the calling engine (set at each API entry): 0 = plain
-// stream order, 1 = programmatic dependent launch.
-extern int g_launch_pdl;
+// Launch mode of the calling engine (set at each API entry, per host
+// thread): 0 = plain stream order, 1 = programmatic dependent launch.
+extern thread_local int g_launch_pdl;
 
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,

@@ -31,13 +31,15 @@
 
 using namespace sf;
 
+// Per-call context is per host thread, so that engines driven from
+// different threads (e.g. one per GPU) do not see each other's calls.
 namespace sf {
-int g_launch_pdl = 0;
+thread_local int g_launch_pdl = 0;
 }
 
 // Source line of the first CUDA call that failed in the current API call
 // (reported by sf_last_error).
-static int g_fail_line = 0;
+static thread_local int g_fail_line = 0;
 #define CK(x)                                   \
   do {                                          \
     cudaError_t _e = (x);                       \
@@ -274,7 +276,7 @@ struct Scope {
     CK(call);                                            \
   } while (0)
 
-uint64_t* g_ws_gen = nullptr;   // generation counter of the engine whose buffers ensure() grows
+thread_local uint64_t* g_ws_gen = nullptr;   // generation counter of the engine whose buffers ensure() grows
 
 cudaError_t ensure(Buf& b, size_t bytes) {
   if (bytes <= b.bytes) return cudaSuccess;
