@@ -366,8 +366,13 @@ enum {
                             kernel */
   SF_OPT_GEMM_PAIR_BN = 4, /* tile width of the CTA-pair kernel: 0 (default) chosen per shape,
                               or 128, 192, 256 */
-  SF_OPT_ATTN_PATH = 5    /* bf16 attention (relative-position and Transformer): 1 (default)
+  SF_OPT_ATTN_PATH = 5,   /* bf16 attention (relative-position and Transformer): 1 (default)
                              tcgen05/TMEM/TMA kernels, 0 mma.sync kernels */
+  SF_OPT_MEL_PATH = 6     /* log-mel front-end (sf_mel, the offline forward, the audio-in
+                             step): 0 (default) FFT through shared memory and one
+                             normalisation CTA per (clip, bin); 1 FFT in registers with warp
+                             shuffles, then separate statistics and normalisation passes over
+                             all SMs */
 };
 SF_API sf_status sf_set_option(sf_engine* e, int option, int value);
 

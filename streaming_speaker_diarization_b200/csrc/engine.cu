@@ -168,6 +168,7 @@ struct sf_engine {
                           // 3 = never; 0 = mma.sync
   int pair_bn = 0;        // CTA-pair tile width (0 = planned)
   int attn_path = 1;      // bf16 relative-position attention: 1 = tcgen05, 0 = mma.sync
+  int mel_path = 0;       // front-end: 0 = shared-memory FFT, 1 = register FFT + all-SM normalisation
   float* d_split_ws = nullptr;   // split-K partial tiles of the tcgen05 GEMM
   int* d_split_cnt = nullptr;    // their per-tile arrival counters (kept at zero between launches)
   TcScratch tc_scratch() const { return TcScratch{d_err, d_split_ws, SPLIT_WS_BYTES, d_split_cnt, SPLIT_CNT}; }
@@ -682,7 +683,8 @@ cudaError_t run_graph(sf_engine* e, std::string key, cudaStream_t st, F&& enqueu
   if (!e->use_graphs) return enqueue(st);
   key += e->prof ? "|p" + std::to_string(e->prof_mask) : "|n";
   key += e->use_pdl ? "|pdl" : "";
-  key += "|g" + std::to_string(e->gemm_path) + "." + std::to_string(e->pair_bn) + "|a" + std::to_string(e->attn_path);
+  key += "|g" + std::to_string(e->gemm_path) + "." + std::to_string(e->pair_bn) + "|a" + std::to_string(e->attn_path) +
+         "|m" + std::to_string(e->mel_path);
   auto it = e->graphs.find(key);
   if (it != e->graphs.end() && it->second.gen != e->ws_gen) {
     cudaGraphExecDestroy(it->second.exec);
@@ -943,8 +945,9 @@ cudaError_t offline_impl(sf_engine* e, const float* d_audio, const std::vector<i
   return run_graph(e, key, st, [&](cudaStream_t st) -> cudaError_t {
     CK(desc_upload(e, st));
     MelArgs ma{e->d_desc->len};
-    RUN(K_MEL, 2, 0, (double)B * n_max * 4 + (double)B * 128 * T_cols * 4,
-        launch_mel(d_audio, B, n_max, ma, e->d_mel_tab, static_cast<float*>(e->mel.p), static_cast<float*>(e->part.p), st));
+    RUN(K_MEL, e->mel_path ? 3 : 2, 0, (double)B * n_max * 4 + (double)B * 128 * T_cols * 4,
+        launch_mel(d_audio, B, n_max, ma, e->d_mel_tab, static_cast<float*>(e->mel.p), static_cast<float*>(e->part.p), st,
+                   e->mel_path));
     CK(run_pre_encode<T>(e, static_cast<float*>(e->mel.p), T_cols, B, L_max, static_cast<T*>(e->emb.p), T3, st));
     StateBufs none{};
     none.D = e->cfg.d_model;
@@ -1156,8 +1159,8 @@ sf_status sf_mel(sf_engine* e, const float* d_audio, const int64_t* h_len, int B
   if (ce == cudaSuccess) ce = desc_upload(e, st);
   MelArgs ma{e->d_desc->len};
   if (ce == cudaSuccess) {
-    Scope sc(e, K_MEL, 2, 0, (double)B * n_max * 4 + (double)B * 128 * (1 + n_max / 160) * 4, st);
-    ce = launch_mel(d_audio, B, n_max, ma, e->d_mel_tab, d_mel, static_cast<float*>(e->part.p), st);
+    Scope sc(e, K_MEL, e->mel_path ? 3 : 2, 0, (double)B * n_max * 4 + (double)B * 128 * (1 + n_max / 160) * 4, st);
+    ce = launch_mel(d_audio, B, n_max, ma, e->d_mel_tab, d_mel, static_cast<float*>(e->part.p), st, e->mel_path);
   }
   if (ce != cudaSuccess) return cuda_fail(e, ce, "sf_mel");
   if (h_mel_len)
@@ -1396,6 +1399,10 @@ sf_status sf_set_option(sf_engine* e, int option, int value) {
       if (value != 0 && value != 1) return fail(e, SF_EINVAL, "attention path must be 0 or 1");
       e->attn_path = value;
       break;
+    case SF_OPT_MEL_PATH:
+      if (value != 0 && value != 1) return fail(e, SF_EINVAL, "front-end path must be 0 or 1");
+      e->mel_path = value;
+      break;
     case SF_OPT_GEMM_PAIR_BN:
       if (value != 0 && value != 128 && value != 192 && value != 256)
         return fail(e, SF_EINVAL, "pair tile width must be 0, 128, 192 or 256");
@@ -1567,7 +1574,7 @@ cudaError_t stream_step_impl(sf_stream* s, const float* d_feats, int64_t t_buf, 
       d->win_nf[i] = (int)pl.W[i];
     }
     CK(ensure(e->mel, (size_t)s->n * 128 * W_max * 4));   // rows by stream id, as the pre-encode reads them
-    CK(ensure(e->part, (size_t)n * ((W_max + 31) / 32) * 128 * 4 * 4));
+    CK(ensure(e->part, ((size_t)n * ((W_max + 31) / 32) * 128 * 4 + (size_t)n * 128 * 2) * 4));
     d_feats = static_cast<const float*>(e->mel.p);
     t_buf = W_max;
   }
@@ -1592,9 +1599,9 @@ cudaError_t stream_step_impl(sf_stream* s, const float* d_feats, int64_t t_buf, 
       ma.a0 = e->d_desc->win_a0;
       ma.nf = e->d_desc->win_nf;
       ma.row = e->d_desc->buf;
-      RUN(K_MEL, 2, 0, (double)n * W_max * (160 * 4 + 128 * 4),
+      RUN(K_MEL, e->mel_path ? 3 : 2, 0, (double)n * W_max * (160 * 4 + 128 * 4),
           launch_mel_windows(ain->audio, n, ain->n_buf, ma, e->d_mel_tab, static_cast<float*>(e->mel.p),
-                             static_cast<float*>(e->part.p), (int)W_max, st));
+                             static_cast<float*>(e->part.p), (int)W_max, st, e->mel_path));
     }
     CK(run_pre_encode<T>(e, d_feats, t_buf, n, W_max, static_cast<T*>(e->emb.p), T3, st));
     RUN(K_ASSEMBLE, 1, 0, (double)M * e->cfg.d_model * (4 + sizeof(T)),
