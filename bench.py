@@ -137,7 +137,7 @@ STREAM_WORKLOADS = [
 ]
 
 
-def streaming_bench(b, torch, eng_blob, rank, world, local):
+def streaming_bench(b, torch, eng_blob, rank, world, local, mel_path=0):
     """Streaming throughput: front-end over each stream's clip, then every
     step of every stream (pre_encode on the new window, encoder on
     [cache | FIFO | chunk], state update) until all streams finish.  A first
@@ -152,6 +152,7 @@ def streaming_bench(b, torch, eng_blob, rank, world, local):
         audio_np, lens, _ = clip_for_config(idx)
         audio_np, lens = np.ascontiguousarray(audio_np[lo:hi]), lens[lo:hi]
         eng = b.sf_create(eng_blob, b.default_config(max_batch=max(n, 1), max_samples=int(audio_np.shape[1])))
+        b.sf_set_option(eng, b.SF_OPT_MEL_PATH, mel_path)
         audio = torch.from_numpy(audio_np).cuda()
         T = 1 + audio_np.shape[1] // 160
         mel = torch.empty((n, 128, T), device="cuda")
@@ -196,7 +197,7 @@ def streaming_bench(b, torch, eng_blob, rank, world, local):
     return out
 
 
-def frontend_bench(b, torch, blob, steps, warmup):
+def frontend_bench(b, torch, blob, steps, warmup, mel_path=0):
     """Front-end alone (preemphasis, centred STFT, power, Slaney mel, log,
     per-bin normalisation) on 1 h of audio in one sf_mel call: 57.6M samples
     -> 128 x 360,001 features.  Audio resident on the device, CUDA events per
@@ -208,6 +209,7 @@ def frontend_bench(b, torch, blob, steps, warmup):
     n = len(x)
     T = 1 + n // 160
     eng = b.sf_create(blob, b.default_config(max_batch=1, max_samples=n))
+    b.sf_set_option(eng, b.SF_OPT_MEL_PATH, mel_path)
     try:
         audio = torch.from_numpy(x[None]).cuda()
         mel = torch.empty((1, 128, T), device="cuda")
@@ -235,7 +237,7 @@ def frontend_bench(b, torch, blob, steps, warmup):
     gbs = alg / (med / 1000.0) / 1e9
     return {"workload": "front-end only, 1 h of audio (60 x 60 s clips joined), 57.6M samples -> 128 x 360,001",
             "value": 3600.0 / (med / 1000.0), "unit": UNIT, "ms_p50": med, "ms_p95": float(np.percentile(ms, 95)),
-            "calls": steps,
+            "calls": steps, "mel_path": mel_path,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs / pk["hbm_gbs"], "bytes_per_call": alg, "peak_kind": f"{kind} copy"}}
 
@@ -279,6 +281,7 @@ def main():
     ap.add_argument("--pdl", type=int, default=0, help="programmatic dependent launch between kernels (0/1)")
     ap.add_argument("--no-streaming", action="store_true", help="skip the streaming workloads")
     ap.add_argument("--no-frontend", action="store_true", help="skip the 1 h front-end-only run")
+    ap.add_argument("--mel-path", type=int, default=0, choices=[0, 1], help="front-end implementation (SF_OPT_MEL_PATH)")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
@@ -299,6 +302,7 @@ def main():
     w = make_weights(FULL, seed=0)
     eng = b.sf_create(weights_blob(w), b.default_config(max_batch=1))
     b.sf_set_option(eng, b.SF_OPT_PDL, args.pdl)
+    b.sf_set_option(eng, b.SF_OPT_MEL_PATH, args.mel_path)
     st = torch.cuda.current_stream()
     audio = torch.from_numpy(audio_np).cuda()
     probs = torch.zeros((1, 1125, 4), device="cuda")
@@ -393,9 +397,10 @@ def main():
             "kernels": kernels}
     b.sf_destroy(eng)
     if not args.no_streaming:
-        line["streaming"] = streaming_bench(b, torch, weights_blob(w), rank, world, local)
+        line["streaming"] = streaming_bench(b, torch, weights_blob(w), rank, world, local, args.mel_path)
     if not args.no_frontend:
-        line["frontend_1h"] = frontend_bench(b, torch, weights_blob(w), max(args.steps, 5), max(args.warmup, 3))
+        line["frontend_1h"] = frontend_bench(b, torch, weights_blob(w), max(args.steps, 5), max(args.warmup, 3),
+                                             args.mel_path)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(audio_np)
     if rank == 0:
