@@ -1,0 +1,43 @@
+"""CPU checks of bench.py's host logic: the clock-sample summary, the guard
+that drops the stored DRAM traffic once the GEMM sources change, the peak
+denominators, and the reference arm's non-zero ranks exiting without work."""
+import argparse
+import os
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+
+def test_clock_summary_reports_median_and_active_reasons():
+    lines = [
+        "0, 1965, 1965, 600.1, 0x0, Not Active, Not Active, Not Active, Not Active",
+        "0, 1800, 1965, 990.5, 0x4, Not Active, Not Active, Not Active, Active",
+        "0, 1700, 1965, 1001.0, 0x4, Not Active, Not Active, Not Active, Active",
+        "garbage line",
+        "0, [N/A], 1965, 0, 0x0, Not Active, Not Active, Not Active, Not Active",
+    ]
+    c = bench.parse_clocks(lines)
+    assert c["sm_mhz"] == 1800.0 and c["sm_max_mhz"] == 1965.0 and c["samples"] == 3
+    assert c["reasons"] == ["sw_power_cap"]
+    c = bench.parse_clocks(["0, 1500, 1965, 700, 0x8, Active, Not Active, Active, Not Active"])
+    assert c["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"]
+    assert bench.parse_clocks([])["sm_mhz"] is None
+
+
+def test_traffic_dropped_when_gemm_sources_differ(monkeypatch):
+    monkeypatch.setitem(bench.GEMM_TRAFFIC, "sources_sha256", "0" * 64)
+    assert bench.gemm_traffic_per_launch() is None
+
+
+def test_peaks_are_positive():
+    pk, kind = bench.peaks()
+    assert kind in ("measured", "fallback")
+    assert pk["hbm_gbs"] > 0 and pk["bf16_tflops"] > 0 and pk["bf16_tflops_sustained"] > 0
+
+
+def test_reference_arm_other_ranks_do_no_work():
+    args = argparse.Namespace(gpus=2, steps=1, warmup=3, impl="reference")
+    assert bench.run_reference(args, 1, 2) == 0
