@@ -3,12 +3,14 @@
     python -m streaming_speaker_diarization_b200.kbench gemm M N K [--epi E] [--path P] [--reps R]
     python -m streaming_speaker_diarization_b200.kbench attn N_SEQ LEN [--path P] [--reps R]
     python -m streaming_speaker_diarization_b200.kbench mha N_SEQ LEN [--path P] [--reps R]
+    python -m streaming_speaker_diarization_b200.kbench mel SECONDS [--clips B] [--path P] [--reps R]
 
 `gemm` runs sf_gemm_bf16 (E: 1 f32 out, 2 bf16 out, 3 residual update, 4
 swish, 5 gated linear unit; P: SF_OPT_GEMM_PATH, 1 = tcgen05 with CTA pairs
 where faster, 2 = CTA pairs always, 3 = single CTAs, 0 = mma.sync); `attn`
 runs sf_attention_relpos and `mha` sf_attention_mha on N_SEQ packed
-sequences of LEN rows (P: 1 tcgen05, 0 mma.sync).  Operands are seeded random values on the device; three warm-up
+sequences of LEN rows (P: 1 tcgen05, 0 mma.sync); `mel` runs sf_mel on B
+clips of SECONDS of audio each (P: SF_OPT_MEL_PATH).  Operands are seeded random values on the device; three warm-up
 launches, then REPS launches queued behind a GPU sleep (so host launch
 overhead is hidden) and timed with CUDA events on the current stream.  Also
 the driver for single-kernel ncu captures (small REPS)."""
@@ -60,6 +62,11 @@ def main(argv=None):
     m.add_argument("length", type=int)
     m.add_argument("--path", type=int, default=1)
     m.add_argument("--reps", type=int, default=20)
+    f = sub.add_parser("mel")
+    f.add_argument("seconds", type=float)
+    f.add_argument("--clips", type=int, default=1)
+    f.add_argument("--path", type=int, default=0)
+    f.add_argument("--reps", type=int, default=10)
     args = ap.parse_args(argv)
 
     import torch
@@ -79,6 +86,22 @@ def main(argv=None):
         ms = _time(torch, lambda: b.sf_gemm_bf16(eng, A, W, C, path=path), args.reps)
         print(f"gemm M={M} N={N} K={K} epi={args.epi} path={args.path}: {ms * 1e3:.1f} us/launch, "
               f"{2 * M * N * K / ms / 1e9:.1f} TFLOP/s")
+    elif args.op == "mel":
+        n = int(args.seconds * 16000)
+        B = args.clips
+        from synth import TINY, make_weights, weights_blob
+        cfg = b.default_config(n_conformer=TINY.n_conformer, n_transformer=TINY.n_transformer, precision=1,
+                               max_batch=B, max_samples=n)
+        eng = b.sf_create(weights_blob(make_weights(TINY, seed=0)), cfg)
+        b.sf_set_option(eng, b.SF_OPT_MEL_PATH, args.path)
+        audio = 0.1 * torch.randn(B, n, device="cuda", generator=gen)
+        T = 1 + n // 160
+        mel = torch.empty(B, 128, T, device="cuda")
+        lens = np.full(B, n, np.int64)
+        ms = _time(torch, lambda: b.sf_mel(eng, audio, lens, mel), args.reps)
+        alg = B * (4.0 * n + 4.0 * 128 * T)
+        print(f"mel B={B} x {args.seconds:g} s path={args.path}: {ms * 1e3:.1f} us/call, "
+              f"{B * args.seconds / (ms / 1e3):.0f} audio-s/s, {alg / (ms / 1e3) / 1e9:.1f} GB/s algorithmic")
     elif args.op == "mha":
         n, L = args.n_seq, args.length
         eng = _engine(b, max(n, 8))
