@@ -251,6 +251,55 @@ def frontend_bench(b, torch, blob, steps, warmup, mel_path=0):
                          "frac": gbs / pk["hbm_gbs"], "bytes_per_call": alg, "peak_kind": f"{kind} copy"}}
 
 
+def oracle_subsets(w):
+    """The oracle (fp64 numpy) on declared subsets of every workload, each
+    timed once on this machine's host cores: the 90 s clip complete, the
+    front-end on 1 h complete, 2 Low-preset streams x their first 20 steps,
+    1 Very-high-preset stream x 3 steps, and the first 4 clips of the
+    variable-length batch."""
+    import oracle as O
+    from synth import clip_for_config
+    from synth.audio import hour_of_audio
+    out = []
+
+    def rec(name, sample, audio_s, dt, **kw):
+        out.append(dict({"workload": name, "sample": sample, "value": audio_s / dt, "unit": UNIT, "seconds": dt},
+                        **kw))
+
+    a, ln, _ = clip_for_config(1)
+    t0 = time.perf_counter()
+    O.forward_offline(a, ln, w)
+    rec("offline 90 s clip", "complete", 90.0, time.perf_counter() - t0)
+
+    x = hour_of_audio()
+    t0 = time.perf_counter()
+    O.mel_features(x[None], np.array([len(x)]))
+    rec("front-end only, 1 h of audio", "complete", len(x) / 16000.0, time.perf_counter() - t0)
+    del x
+
+    for idx, name, preset, n_streams, n_steps in ((2, "Low preset, 64 x 60 s", "low", 2, 20),
+                                                   (3, "Very high preset, 16 x 600 s", "very_high", 1, 3)):
+        a, ln, _ = clip_for_config(idx, n_clips=n_streams)
+        pre = O.PRESETS[preset]
+        feats, L = O.mel_features(a, ln)
+        t0 = time.perf_counter()
+        frames = 0
+        for i in range(n_streams):
+            st = O.StreamState()
+            for _ in range(n_steps):
+                frames += len(O.stream_step(st, feats[i], int(L[i]), w, pre))
+        dt = time.perf_counter() - t0
+        rec(name, f"{n_streams} stream(s) x first {n_steps} steps (front-end untimed)", frames * 0.08, dt,
+            stream_steps_per_s=n_streams * n_steps / dt)
+
+    a, ln, _ = clip_for_config(4, n_clips=4)
+    t0 = time.perf_counter()
+    O.forward_offline(a, ln, w)
+    rec("variable-length batch, 32 clips of 5-120 s", "first 4 clips", float(ln.sum()) / 16000.0,
+        time.perf_counter() - t0)
+    return out
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return 0
@@ -276,6 +325,8 @@ def run_reference(args, rank, world):
             "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
                              "sample": "each step: first 10 s of the 90 s workload clip, full model, fp64 numpy"},
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    if getattr(args, "oracle_subsets", False):
+        line["subsets"] = oracle_subsets(w)
     print(json.dumps(line), flush=True)
     return 0
 
@@ -291,6 +342,8 @@ def main():
     ap.add_argument("--no-streaming", action="store_true", help="skip the streaming workloads")
     ap.add_argument("--no-frontend", action="store_true", help="skip the 1 h front-end-only run")
     ap.add_argument("--mel-path", type=int, default=0, choices=[0, 1], help="front-end implementation (SF_OPT_MEL_PATH)")
+    ap.add_argument("--oracle-subsets", action="store_true",
+                    help="with --impl reference: also time the oracle on declared subsets of every workload")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
