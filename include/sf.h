@@ -368,11 +368,15 @@ enum {
                               or 128, 192, 256 */
   SF_OPT_ATTN_PATH = 5,   /* bf16 attention (relative-position and Transformer): 1 (default)
                              tcgen05/TMEM/TMA kernels, 0 mma.sync kernels */
-  SF_OPT_MEL_PATH = 6     /* log-mel front-end (sf_mel, the offline forward, the audio-in
+  SF_OPT_MEL_PATH = 6,    /* log-mel front-end (sf_mel, the offline forward, the audio-in
                              step): 0 (default) FFT through shared memory and one
                              normalisation CTA per (clip, bin); 1 FFT in registers with warp
                              shuffles, then separate statistics and normalisation passes over
                              all SMs */
+  SF_OPT_SUB_PATH = 7     /* ConvSubsampling's first two stages: 0 (default) the 3x3 s2 conv
+                             and the first depthwise conv as two kernels through a
+                             [T/2][64][256] tensor in memory; 1 one kernel that computes the
+                             first conv's outputs on chip (same result to the bit) */
 };
 SF_API sf_status sf_set_option(sf_engine* e, int option, int value);
 

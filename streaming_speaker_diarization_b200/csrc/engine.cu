@@ -169,6 +169,7 @@ struct sf_engine {
   int pair_bn = 0;        // CTA-pair tile width (0 = planned)
   int attn_path = 1;      // bf16 relative-position attention: 1 = tcgen05, 0 = mma.sync
   int mel_path = 0;       // front-end: 0 = shared-memory FFT, 1 = register FFT + all-SM normalisation
+  int sub_path = 0;       // subsampling: 0 = conv1 and depthwise kernels, 1 = conv1 fused into the first depthwise
   float* d_split_ws = nullptr;   // split-K partial tiles of the tcgen05 GEMM
   int* d_split_cnt = nullptr;    // their per-tile arrival counters (kept at zero between launches)
   TcScratch tc_scratch() const { return TcScratch{d_err, d_split_ws, SPLIT_WS_BYTES, d_split_cnt, SPLIT_CNT}; }
@@ -684,7 +685,7 @@ cudaError_t run_graph(sf_engine* e, std::string key, cudaStream_t st, F&& enqueu
   key += e->prof ? "|p" + std::to_string(e->prof_mask) : "|n";
   key += e->use_pdl ? "|pdl" : "";
   key += "|g" + std::to_string(e->gemm_path) + "." + std::to_string(e->pair_bn) + "|a" + std::to_string(e->attn_path) +
-         "|m" + std::to_string(e->mel_path);
+         "|m" + std::to_string(e->mel_path) + "|s" + std::to_string(e->sub_path);
   auto it = e->graphs.find(key);
   if (it != e->graphs.end() && it->second.gen != e->ws_gen) {
     cudaGraphExecDestroy(it->second.exec);
@@ -789,7 +790,7 @@ void fill_seq(DescBlock* d, const std::vector<int>& lens, int& M, int& tiles) {
 // Workspace of run_pre_encode (call before any capture).
 cudaError_t prep_pre_encode(sf_engine* e, int n_win, int64_t W_max, size_t a) {
   const int T1 = (int)half_len(W_max), T2 = (int)half_len(T1), T3 = (int)half_len(T2);
-  CK(ensure(e->sub1, (size_t)n_win * T1 * 64 * 256 * a));
+  if (e->sub_path == 0) CK(ensure(e->sub1, (size_t)n_win * T1 * 64 * 256 * a));   // path 1 keeps stage 1 on chip
   CK(ensure(e->sub2a, (size_t)n_win * T2 * 32 * 256 * a));
   CK(ensure(e->sub2b, (size_t)n_win * T2 * 32 * 256 * a));
   CK(ensure(e->sub3a, (size_t)n_win * T3 * 16 * 256 * a));
@@ -809,10 +810,17 @@ cudaError_t run_pre_encode(sf_engine* e, const float* feats, int64_t t_buf, int 
   T* s2b = static_cast<T*>(e->sub2b.p);
   T* s3a = static_cast<T*>(e->sub3a.p);
   T* s3b = static_cast<T*>(e->sub3b.p);
-  RUN(K_CONV1, 1, 18.0 * 256 * 64 * T1 * n_win, (double)n_win * W_max * 128 * 4 + (double)n_win * T1 * 64 * 256 * sizeof(T),
-      launch_conv1<T>(feats, t_buf, pa, n_win, W.c1_w, W.c1_b, s1, T1, st));
-  RUN(K_DW2D, 1, 18.0 * 256 * 32 * T2 * n_win, (double)n_win * (T1 * 64 + T2 * 32) * 256 * sizeof(T),
-      launch_dwconv3x3s2<T>(s1, T1, 64, s2a, T2, 32, pa, n_win, 1, W.dw_w[0], W.dw_b[0], st));
+  if (e->sub_path == 1) {
+    RUN(K_CONV1, 1, 18.0 * 256 * (64 * T1 + 32 * T2) * n_win,
+        (double)n_win * W_max * 128 * 4 + (double)n_win * T2 * 32 * 256 * sizeof(T),
+        launch_conv1_dw<T>(feats, t_buf, pa, n_win, W.c1_w, W.c1_b, W.dw_w[0], W.dw_b[0], s2a, T2, st));
+  } else {
+    RUN(K_CONV1, 1, 18.0 * 256 * 64 * T1 * n_win,
+        (double)n_win * W_max * 128 * 4 + (double)n_win * T1 * 64 * 256 * sizeof(T),
+        launch_conv1<T>(feats, t_buf, pa, n_win, W.c1_w, W.c1_b, s1, T1, st));
+    RUN(K_DW2D, 1, 18.0 * 256 * 32 * T2 * n_win, (double)n_win * (T1 * 64 + T2 * 32) * 256 * sizeof(T),
+        launch_dwconv3x3s2<T>(s1, T1, 64, s2a, T2, 32, pa, n_win, 1, W.dw_w[0], W.dw_b[0], st));
+  }
   CK(gemm_acc<T>(e, s2a, 256, W.pw_w[0], n_win * T2 * 32, 256, 256, epi(EPI_BIAS_RELU, W.pw_b[0], s2b, 256), st));
   RUN(K_DW2D, 1, 18.0 * 256 * 16 * T3 * n_win, (double)n_win * (T2 * 32 + T3 * 16) * 256 * sizeof(T),
       launch_dwconv3x3s2<T>(s2b, T2, 32, s3a, T3, 16, pa, n_win, 2, W.dw_w[1], W.dw_b[1], st));
@@ -1402,6 +1410,10 @@ sf_status sf_set_option(sf_engine* e, int option, int value) {
     case SF_OPT_MEL_PATH:
       if (value != 0 && value != 1) return fail(e, SF_EINVAL, "front-end path must be 0 or 1");
       e->mel_path = value;
+      break;
+    case SF_OPT_SUB_PATH:
+      if (value != 0 && value != 1) return fail(e, SF_EINVAL, "subsampling path must be 0 or 1");
+      e->sub_path = value;
       break;
     case SF_OPT_GEMM_PAIR_BN:
       if (value != 0 && value != 128 && value != 192 && value != 256)

@@ -73,6 +73,12 @@ cudaError_t launch_conv1(const float* feats, int64_t t_buf, const PreArgs& a, in
 template <typename T>
 cudaError_t launch_dwconv3x3s2(const T* in, int Tin_max, int Fin, T* out, int Tout_max, int Fout, const PreArgs& a,
                                int n_win, int stage, const float* w, const float* b, cudaStream_t st);
+// conv1 (w1, b1) and the first depthwise stage (w2, b2) in one pass: out
+// [n_win][T2max][32][256], equal to launch_conv1 followed by
+// launch_dwconv3x3s2(stage 1) without the stage-1 tensor.
+template <typename T>
+cudaError_t launch_conv1_dw(const float* feats, int64_t t_buf, const PreArgs& a, int n_win, const float* w1,
+                            const float* b1, const float* w2, const float* b2, T* out, int T2max, cudaStream_t st);
 
 // ------------------------------------------------------- norms / elementwise
 // x (f32, M x D) -> optional in-place LN(x) (f32) and/or h = act(LN(x)).

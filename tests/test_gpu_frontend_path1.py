@@ -5,7 +5,7 @@ clip, ragged batch, minimum length, silence and a pure tone, the offline
 forward, the audio-in streaming step (window mode) and one hour in one call.
 Log-mel features within 1e-3, probabilities within 1e-4 (fp32 engine).
 
-These run only with SF_TEST_MEL_PATH1=1 in the environment: the default
+These run only with SF_TEST_NEW_PATHS=1 in the environment: the default
 engine keeps path 0 until this path has been measured."""
 import os
 
@@ -18,8 +18,8 @@ from synth import clip_for_config, synth_batch, synth_clip
 from _helpers import make_engine, tiny_weights, to_dev
 
 pytestmark = [pytest.mark.gpu,
-              pytest.mark.skipif(os.environ.get("SF_TEST_MEL_PATH1") != "1",
-                                 reason="front-end path 1 is tested with SF_TEST_MEL_PATH1=1")]
+              pytest.mark.skipif(os.environ.get("SF_TEST_NEW_PATHS") != "1",
+                                 reason="kernel paths not yet default run with SF_TEST_NEW_PATHS=1")]
 torch = pytest.importorskip("torch")
 if not torch.cuda.is_available():
     pytest.skip("no CUDA device", allow_module_level=True)
