@@ -570,17 +570,6 @@ template <> Weights<float>& weights<float>(sf_engine* e) { return e->wf; }
 template <> Weights<bf16>& weights<bf16>(sf_engine* e) { return e->wb; }
 
 template <typename T>
-cudaError_t gemm(const T* A, int lda, const T* W, int M, int N, int K, const Epi& ep, cudaStream_t st);
-template <>
-cudaError_t gemm<float>(const float* A, int lda, const float* W, int M, int N, int K, const Epi& ep, cudaStream_t st) {
-  return gemm_f32(A, lda, W, M, N, K, ep, st);
-}
-template <>
-cudaError_t gemm<bf16>(const bf16* A, int lda, const bf16* W, int M, int N, int K, const Epi& ep, cudaStream_t st) {
-  return gemm_bf16_mma(A, lda, W, M, N, K, ep, st);
-}
-
-template <typename T>
 cudaError_t gemm_dispatch(sf_engine* e, const T* A, int lda, const T* W, int M, int N, int K, const Epi& ep,
                           cudaStream_t st);
 template <>
