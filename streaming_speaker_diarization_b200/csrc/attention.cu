@@ -386,7 +386,7 @@ __global__ void __launch_bounds__(256) attn_bf16_kernel(const bf16* __restrict__
 
 template <>
 cudaError_t launch_relpos_attention<float>(const float* qkv, const float* ptab, int R, const float* u, const float* v,
-                                           float* ctx, const SeqTable* seq, int n_tiles, int M, cudaStream_t st) {
+                                           float* ctx, const SeqTable* seq, int /*n_tiles*/, int M, cudaStream_t st) {
   if (M <= 0) return cudaSuccess;
   const int s_cap = R;   // no sequence is longer than the position table
   const size_t smem = (size_t)4 * (s_cap + 128) * 4;
@@ -404,7 +404,7 @@ cudaError_t launch_relpos_attention<bf16>(const bf16* qkv, const bf16* ptab, int
 }
 
 template <>
-cudaError_t launch_mha<float>(const float* qkv, float* ctx, const SeqTable* seq, int n_tiles, int M, int R,
+cudaError_t launch_mha<float>(const float* qkv, float* ctx, const SeqTable* seq, int /*n_tiles*/, int M, int R,
                               cudaStream_t st) {
   if (M <= 0) return cudaSuccess;
   const int s_cap = R;   // no sequence is longer than R rows
