@@ -387,6 +387,14 @@ SF_API sf_status sf_set_option(sf_engine* e, int option, int value);
  * device-side index check skipped an access, SF_OK otherwise. */
 SF_API sf_status sf_check(sf_engine* e, void* cuda_stream);
 
+/* Failure-detection self-test: enqueue one kernel that waits, through the
+ * bounded device wait every tcgen05 kernel uses, on a barrier that nothing
+ * completes.  The wait gives up after its clock budget (about 2 s), records
+ * the timeout in the engine's error word and returns; the next sf_check
+ * returns SF_ETIMEOUT (and clears the word), and the engine and the CUDA
+ * context remain usable.  Errors: SF_EINVAL, SF_ECUDA (launch). */
+SF_API sf_status sf_selftest_wait(sf_engine* e, void* cuda_stream);
+
 /* The engine's dense projection alone, for tests and kernel benchmarks:
  *   d_C [M x N] (out) = d_A bf16 [M x K] (row stride lda) .
  *       d_W bf16 [N x K]^T + d_bias f32 [N] (may be NULL)

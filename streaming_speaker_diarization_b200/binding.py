@@ -59,7 +59,7 @@ EXPORTED = ["sf_default_config", "sf_create", "sf_create_from_file", "sf_destroy
             "sf_stream_window", "sf_stream_step", "sf_stream_get_state", "sf_stream_set_state",
             "sf_stream_update", "sf_select_topk", "sf_profile_enable", "sf_profile_read", "sf_mel_noalloc",
             "sf_check", "sf_gemm_bf16", "sf_set_option", "sf_attention_relpos", "sf_default_seg_params",
-            "sf_segments", "sf_stream_step_audio", "sf_attention_mha"]
+            "sf_segments", "sf_stream_step_audio", "sf_attention_mha", "sf_selftest_wait"]
 
 
 class SFError(RuntimeError):
@@ -97,6 +97,7 @@ def _load():
         "sf_profile_read": ([VP, P(sf_kernel_stat), I, P(I), I], I),
         "sf_mel_noalloc": ([VP, VP, I, I64, VP, VP, VP], I),
         "sf_check": ([VP, VP], I),
+        "sf_selftest_wait": ([VP, VP], I),
         "sf_set_option": ([VP, I, I], I),
         "sf_gemm_bf16": ([VP, VP, I, VP, I, I, I, VP, VP, I, VP], I),
         "sf_attention_relpos": ([VP, VP, VP, I, VP, VP, VP, I, VP, I, VP], I),
@@ -299,6 +300,12 @@ def sf_profile_read(eng, reset=True):
 
 def sf_check(eng, stream=None):
     _check(lib.sf_check(eng, _stream(stream)), eng)
+
+
+def sf_selftest_wait(eng, stream=None):
+    """Enqueue the failure-detection self-test (a bounded device wait that
+    runs out after about 2 s); the next sf_check raises SF_ETIMEOUT."""
+    _check(lib.sf_selftest_wait(eng, _stream(stream)), eng)
 
 
 def sf_gemm_bf16(eng, A, W, C, bias=None, path=1, stream=None):

@@ -1283,6 +1283,13 @@ sf_status sf_check(sf_engine* e, void* cuda_stream) {
   return SF_OK;
 }
 
+sf_status sf_selftest_wait(sf_engine* e, void* cuda_stream) {
+  if (check_engine(e) != SF_OK) return SF_EINVAL;
+  cudaError_t ce = launch_selftest_wait(e->d_err, static_cast<cudaStream_t>(cuda_stream));
+  if (ce != cudaSuccess) return cuda_fail(e, ce, "sf_selftest_wait");
+  return SF_OK;
+}
+
 sf_status sf_gemm_bf16(sf_engine* e, const void* d_A, int lda, const void* d_W, int M, int N, int K,
                        const float* d_bias, void* d_C, int path, void* cuda_stream) {
   if (check_engine(e) != SF_OK) return SF_EINVAL;

@@ -109,6 +109,10 @@ cudaError_t launch_extract_rows(const float* packed, const SeqTable* seq, const 
 int attention_f32_max_seq();
 cudaError_t attention_reserve_f32(int R);
 
+// One CTA waits on an mbarrier nothing arrives on, through the tcgen05
+// kernels' bounded wait; when it gives up, ERR_TIMEOUT goes to *err.
+cudaError_t launch_selftest_wait(int* err, cudaStream_t st);
+
 // ------------------------------------------------------- post-processing
 struct SegArgs {
   float onset, offset;      // activity thresholds (onset >= offset)
