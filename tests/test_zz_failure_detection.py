@@ -2,8 +2,8 @@
 tcgen05 kernel uses, run on a barrier nothing completes, gives up after its
 clock budget; the host reads SF_ETIMEOUT from sf_check, the error word is
 cleared, and the same engine then runs a forward that matches the oracle.
-Collected after the parity files on purpose: it makes a device wait run out
-on purpose, so it runs once they have finished."""
+Collected after the parity files: it makes a device wait run out, so it
+runs once they have finished."""
 import time
 
 import numpy as np
