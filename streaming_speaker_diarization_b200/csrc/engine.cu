@@ -204,12 +204,14 @@ struct sf_engine {
     std::vector<cudaEvent_t> events;
   };
   std::unordered_map<std::string, GraphEntry> graphs;
+  uint64_t stream_serial = 0;   // last serial handed to a stream
   // workspace (grow-only)
   Buf mel, part, audio, sub1, sub2a, sub2b, sub3a, sub3b, emb, x, h, big, ctx, x2, h2, probs, out;
 };
 
 struct sf_stream {
   sf_engine* e = nullptr;
+  uint64_t serial = 0;    // identifies the stream's graphs (a host address may be reused after destroy)
   sf_preset p{};
   int n = 0;
   StateBufs sb{};
@@ -662,6 +664,21 @@ void destroy_graphs(sf_engine* e) {
   }
   e->graphs.clear();
 }
+
+// Graphs whose key starts with `prefix` (e.g. every graph of one stream).
+void destroy_graphs_with_prefix(sf_engine* e, const std::string& prefix) {
+  for (auto it = e->graphs.begin(); it != e->graphs.end();) {
+    if (it->first.compare(0, prefix.size(), prefix) == 0) {
+      if (it->second.exec) cudaGraphExecDestroy(it->second.exec);
+      for (cudaEvent_t ev : it->second.events) cudaEventDestroy(ev);
+      it = e->graphs.erase(it);
+    } else {
+      ++it;
+    }
+  }
+}
+
+std::string stream_graph_prefix(const sf_stream* s) { return "st|" + std::to_string(s->serial) + "|"; }
 
 // Runs `enqueue` (which must only enqueue work on `st`: no allocation, no
 // synchronisation) through a CUDA graph cached under `key`: captured on
@@ -1592,7 +1609,7 @@ cudaError_t stream_step_impl(sf_stream* s, const float* d_feats, int64_t t_buf, 
   CK(ensure(e->emb, (size_t)n * T3 * e->cfg.d_model * sizeof(T)));
   CK(ensure_encode_ws(e, M));
   CK(prep_pre_encode(e, n, W_max, sizeof(T)));
-  std::string key = "st|" + std::to_string(reinterpret_cast<uintptr_t>(s)) + "|" + std::to_string(n) + "|" +
+  std::string key = stream_graph_prefix(s) + std::to_string(n) + "|" +
                     std::to_string(M) + "|" + std::to_string(tiles) + "|" + std::to_string(e->att_tiles2) + "|" +
                     std::to_string(W_max) + "|" +
                     std::to_string(t_buf) + "|" + std::to_string(reinterpret_cast<uintptr_t>(d_feats)) + "|" +
@@ -1642,6 +1659,7 @@ sf_status sf_stream_create(sf_engine* e, const sf_preset* p, int n_streams, sf_s
   if (p->spkcache_len + p->fifo_len + p->chunk_len > CAND_MAX) return fail(e, SF_ESHAPE, "preset too large for compression");
   std::unique_ptr<sf_stream> s(new sf_stream());
   s->e = e;
+  s->serial = ++e->stream_serial;
   s->p = *p;
   s->n = n_streams;
   const int D = e->cfg.d_model;
@@ -1683,6 +1701,7 @@ sf_status sf_stream_create(sf_engine* e, const sf_preset* p, int n_streams, sf_s
 sf_status sf_stream_destroy(sf_stream* s) {
   if (!s) return SF_EINVAL;
   cudaDeviceSynchronize();
+  if (s->e) destroy_graphs_with_prefix(s->e, stream_graph_prefix(s));   // they hold this stream's buffers
   if (s->alloc) cudaFree(s->alloc);
   delete s;
   return SF_OK;
