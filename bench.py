@@ -74,10 +74,12 @@ def peaks():
 
 
 class Clocks:
-    """nvidia-smi sampling during the timed region."""
+    """nvidia-smi sampling during the timed region; the raw samples go to
+    `out_dir` (default: the system temporary directory)."""
 
-    def __init__(self, idx):
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{idx}.csv")
+    def __init__(self, idx, out_dir=None):
+        import tempfile
+        self.path = os.path.join(out_dir or tempfile.gettempdir(), f"sf_bench_clocks_rank{idx}.csv")
         os.makedirs(os.path.dirname(self.path), exist_ok=True)
         q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -345,6 +347,7 @@ def main():
     ap.add_argument("--mel-path", type=int, default=0, choices=[0, 1], help="front-end implementation (SF_OPT_MEL_PATH)")
     ap.add_argument("--sub-path", type=int, default=0, choices=[0, 1],
                     help="subsampling conv1 + first depthwise implementation (SF_OPT_SUB_PATH)")
+    ap.add_argument("--clocks-dir", default=None, help="where to keep the raw nvidia-smi clock samples")
     ap.add_argument("--oracle-subsets", action="store_true",
                     help="with --impl reference: also time the oracle on declared subsets of every workload")
     args = ap.parse_args()
@@ -387,7 +390,7 @@ def main():
     # timed region: per-step CUDA events on the launching stream, L2 flushed between steps
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     barrier()
-    clk = Clocks(local)
+    clk = Clocks(local, args.clocks_dir)
     for i in range(args.steps):
         flush.zero_()
         ev[i][0].record(st)
