@@ -149,6 +149,9 @@ SF_API sf_status sf_default_config(sf_config* cfg);
  * tensor), SF_EDEVICE, SF_ENOMEM. */
 SF_API sf_status sf_create(const void* h_blob, uint64_t nbytes, const sf_config* cfg, sf_engine** out);
 SF_API sf_status sf_create_from_file(const char* path, const sf_config* cfg, sf_engine** out);
+/* Synchronises the device and frees the engine.  Streams still alive are
+ * detached: sf_stream_destroy still frees them (and sf_stream_reset and
+ * sf_stream_window still work), every other call on them returns SF_EINVAL. */
 SF_API sf_status sf_destroy(sf_engine* e);
 SF_API sf_status sf_get_metadata(const sf_engine* e, sf_config* out);
 /* Message of the last error on this engine (never NULL; "" if none). */
@@ -233,6 +236,8 @@ SF_API sf_status sf_forward_offline_host(sf_engine* e, const float* h_audio, con
 /* A batch of n_streams independent streams sharing one preset; all state
  * (cache, FIFO, predictions, silence mean) lives on the device. */
 SF_API sf_status sf_stream_create(sf_engine* e, const sf_preset* p, int n_streams, sf_stream** out);
+/* Synchronises the device, frees the stream's state and the engine's CUDA
+ * graphs that were captured for it. */
 SF_API sf_status sf_stream_destroy(sf_stream* s);
 
 /* Restore the empty state of the listed streams (h_ids NULL = all). */

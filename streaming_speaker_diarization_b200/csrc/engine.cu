@@ -205,6 +205,7 @@ struct sf_engine {
   };
   std::unordered_map<std::string, GraphEntry> graphs;
   uint64_t stream_serial = 0;   // last serial handed to a stream
+  std::vector<sf_stream*> streams;   // live streams (detached when the engine goes first)
   // workspace (grow-only)
   Buf mel, part, audio, sub1, sub2a, sub2b, sub3a, sub3b, emb, x, h, big, ctx, x2, h2, probs, out;
 };
@@ -1133,6 +1134,7 @@ sf_status sf_create_from_file(const char* path, const sf_config* cfg, sf_engine*
 sf_status sf_destroy(sf_engine* e) {
   if (!e) return SF_EINVAL;
   cudaDeviceSynchronize();
+  for (sf_stream* s : e->streams) s->e = nullptr;   // they can still be destroyed, not stepped
   destroy_graphs(e);
   for (Buf* b : {&e->mel, &e->part, &e->audio, &e->sub1, &e->sub2a, &e->sub2b, &e->sub3a, &e->sub3b, &e->emb, &e->x,
                  &e->h, &e->big, &e->ctx, &e->x2, &e->h2, &e->probs, &e->out})
@@ -1694,6 +1696,7 @@ sf_status sf_stream_create(sf_engine* e, const sf_preset* p, int n_streams, sf_s
     cudaFree(s->alloc);
     return fail(e, SF_ECUDA, "stream state init");
   }
+  e->streams.push_back(s.get());
   *out = s.release();
   return SF_OK;
 }
@@ -1701,7 +1704,11 @@ sf_status sf_stream_create(sf_engine* e, const sf_preset* p, int n_streams, sf_s
 sf_status sf_stream_destroy(sf_stream* s) {
   if (!s) return SF_EINVAL;
   cudaDeviceSynchronize();
-  if (s->e) destroy_graphs_with_prefix(s->e, stream_graph_prefix(s));   // they hold this stream's buffers
+  if (s->e) {
+    destroy_graphs_with_prefix(s->e, stream_graph_prefix(s));   // they hold this stream's buffers
+    auto& v = s->e->streams;
+    v.erase(std::remove(v.begin(), v.end(), s), v.end());
+  }
   if (s->alloc) cudaFree(s->alloc);
   delete s;
   return SF_OK;
@@ -1889,7 +1896,7 @@ sf_status sf_stream_step_audio(sf_stream* s, const float* d_audio, int64_t n_buf
 }
 
 sf_status sf_stream_get_state(sf_stream* s, int id, sf_state_view* v, void* cuda_stream) {
-  if (!s || !v || id < 0 || id >= s->n) return SF_EINVAL;
+  if (!s || !v || id < 0 || id >= s->n || !s->e) return SF_EINVAL;
   sf_engine* e = s->e;
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
   const size_t a = act_size(e);
@@ -1917,7 +1924,7 @@ sf_status sf_stream_get_state(sf_stream* s, int id, sf_state_view* v, void* cuda
 }
 
 sf_status sf_stream_set_state(sf_stream* s, int id, const sf_state_view* v, void* cuda_stream) {
-  if (!s || !v || id < 0 || id >= s->n) return SF_EINVAL;
+  if (!s || !v || id < 0 || id >= s->n || !s->e) return SF_EINVAL;
   sf_engine* e = s->e;
   if (v->n_cache < 0 || v->n_cache > s->sb.cap_c || v->n_fifo < 0 || v->n_fifo > s->p.fifo_len || v->next_frame < 0 ||
       v->sil_count < 0)

@@ -135,3 +135,24 @@ def test_engine_still_works_after_the_rejections(setup):
     b.sf_check(eng)
     ref, _ = O.forward_offline(audio, lens, w)
     assert np.max(np.abs(probs.cpu().numpy() - ref)) <= 2e-2
+
+
+def test_stream_outliving_its_engine():
+    """The engine destroyed first: its stream is detached; stepping it or
+    reading its state returns SF_EINVAL, resetting and destroying it work."""
+    eng = make_engine(tiny_weights(), 1, 2, 2, max_batch=1)
+    p = b.sf_preset(6, 7, 188, 144, 188)
+    h = ctypes.c_void_p()
+    assert b.lib.sf_stream_create(eng, ctypes.byref(p), 1, ctypes.byref(h)) == 0
+    st = h.value
+    b.sf_destroy(eng)
+    mel = torch.zeros((1, 128, 201), device="cuda")
+    cp = torch.zeros((1, 6, 4), device="cuda")
+    start, end = np.zeros(1, np.int64), np.array([200], np.int64)
+    n_out = np.zeros(1, np.int32)
+    assert b.lib.sf_stream_step(st, mel.data_ptr(), 201, start.ctypes.data, end.ctypes.data, cp.data_ptr(),
+                                n_out.ctypes.data, _st()) == SF_EINVAL
+    v = b.sf_state_view()
+    assert b.lib.sf_stream_get_state(st, 0, ctypes.byref(v), _st()) == SF_EINVAL
+    assert b.lib.sf_stream_reset(st, None, 0) == 0
+    assert b.lib.sf_stream_destroy(st) == 0
