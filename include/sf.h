@@ -372,7 +372,10 @@ enum {
   SF_OPT_GEMM_PAIR_BN = 4, /* tile width of the CTA-pair kernel: 0 (default) chosen per shape,
                               or 128, 192, 256 */
   SF_OPT_ATTN_PATH = 5,   /* bf16 attention (relative-position and Transformer): 1 (default)
-                             tcgen05/TMEM/TMA kernels, 0 mma.sync kernels */
+                             tcgen05/TMEM/TMA kernels (the Transformer's on mma.sync when
+                             its units do not fill the SMs), 0 mma.sync kernels, 2 as 1
+                             with that mma.sync fallback splitting each CTA's keys over
+                             four warp groups instead of two */
   SF_OPT_MEL_PATH = 6,    /* log-mel front-end (sf_mel, the offline forward, the audio-in
                              step): 0 (default) FFT through shared memory and one
                              normalisation CTA per (clip, bin); 1 FFT in registers with warp
@@ -437,7 +440,8 @@ SF_API sf_status sf_attention_relpos(sf_engine* e, const void* d_qkv, const void
  *                         24h .. 24h + 23 of each part
  *   d_ctx bf16 [M x 192] (out)  softmax_j(q_i . k_j / sqrt(24)) v_j
  * Sequence lengths in [1, the engine's longest sequence]; path 1 = tcgen05
- * kernel, 0 = mma.sync.  Pointers 16-byte aligned.  Uses the engine's
+ * kernel, 0 = mma.sync (two key groups per CTA), 2 = mma.sync with four key
+ * groups per CTA.  Pointers 16-byte aligned.  Uses the engine's
  * descriptor block (ordered on `cuda_stream` with its other calls). */
 SF_API sf_status sf_attention_mha(sf_engine* e, const void* d_qkv, const int* h_seq_len, int n, void* d_ctx, int path,
                                   void* cuda_stream);

@@ -146,7 +146,8 @@ __device__ __forceinline__ void load_rows_async(bf16* dst, const bf16* src, int6
   }
 }
 
-template <int HD, int HDP, bool REL>
+// NG warp groups of 4 warps: group g takes key tiles g, g + NG, g + 2 NG, ...
+template <int HD, int HDP, bool REL, int NG = 2>
 struct AttCfg {
   static constexpr int LDS = HDP + 8;
   static constexpr int TILE = 64 * LDS;                       // bf16 elements
@@ -154,24 +155,25 @@ struct AttCfg {
   // Q (+Qv) once; per warp group, K, V and the 128-row relative slice
   // double-buffered; per warp a 16 x 80 fp32 tile of relative scores
   static constexpr int BUF = 2 * TILE + (REL ? 2 * TILE : 0);
-  static constexpr int SMEM = (NQ * TILE + 2 * 2 * BUF) * 2 + (REL ? 8 * 16 * 80 * 4 : 0);
-  static constexpr int MERGE_FLOATS = 128 * (4 + 4 * (HDP / 8));   // group 1's (m, l, O) handed to group 0
+  static constexpr int SMEM = (NQ * TILE + NG * 2 * BUF) * 2 + (REL ? 4 * NG * 16 * 80 * 4 : 0);
+  static constexpr int MERGE_FLOATS = 128 * (4 + 4 * (HDP / 8));   // a group's (m, l, O) handed to group 0
   static_assert(MERGE_FLOATS * 4 <= 2 * BUF * 2, "merge area fits in one group's buffers");
+  static_assert(NG >= 2 && NG <= 8, "2 to 8 warp groups");
 };
 
-template <int HD, int HDP, bool REL>
-__global__ void __launch_bounds__(256) attn_bf16_kernel(const bf16* __restrict__ qkv, int D,
+template <int HD, int HDP, bool REL, int NG = 2>
+__global__ void __launch_bounds__(128 * NG) attn_bf16_kernel(const bf16* __restrict__ qkv, int D,
                                                         const bf16* __restrict__ ptab, int R,
                                                         const float* __restrict__ u, const float* __restrict__ vb,
                                                         bf16* __restrict__ ctx, const SeqTable* __restrict__ seq) {
   SF_PDL_ENTRY();
-  using C = AttCfg<HD, HDP, REL>;
+  using C = AttCfg<HD, HDP, REL, NG>;
   constexpr int LDS = C::LDS;
   extern __shared__ float4 att_smem4[];
   bf16* sQu = reinterpret_cast<bf16*>(att_smem4);
   bf16* sQv = sQu + (REL ? C::TILE : 0);
   bf16* sBuf0 = sQu + C::NQ * C::TILE;                        // per group: 2 x [K | V | P(128 rows, REL)]
-  float* sBD = reinterpret_cast<float*>(sBuf0 + 2 * 2 * C::BUF);
+  float* sBD = reinterpret_cast<float*>(sBuf0 + NG * 2 * C::BUF);
 
   const int g_tile = blockIdx.x, h = blockIdx.y;
   const int s = seq_of_tile(seq, g_tile);
@@ -206,7 +208,7 @@ __global__ void __launch_bounds__(256) attn_bf16_kernel(const bf16* __restrict__
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
   const float sl2 = 1.4426950408889634f / sqrtf((float)HD);
 
-  // group `grp` takes key tiles grp, grp + 2, ...; each group double-buffers its own tiles
+  // group `grp` takes key tiles grp, grp + NG, ...; each group double-buffers its own tiles
   auto prefetch = [&](int j0, int buf) {
     bf16* k_ = sBuf + buf * C::BUF;
     load_rows_async<HD, HDP, LDS>(k_, Kg, ld, j0, 64, 0, S, gtid, 128);
@@ -220,10 +222,10 @@ __global__ void __launch_bounds__(256) attn_bf16_kernel(const bf16* __restrict__
   if (grp * 64 < S) prefetch(grp * 64, 0);
   else cp_async_commit_();
   for (int k = 0;; ++k) {
-    const int j0 = (grp + 2 * k) * 64;
+    const int j0 = (grp + NG * k) * 64;
     if (j0 >= S) break;
     // tile k+1 of this group streams in while tile k is used
-    if (j0 + 128 < S) prefetch(j0 + 128, (k + 1) & 1);
+    if (j0 + NG * 64 < S) prefetch(j0 + NG * 64, (k + 1) & 1);
     else cp_async_commit_();
     cp_async_wait_<1>();
     group_sync();
@@ -339,11 +341,12 @@ __global__ void __launch_bounds__(256) attn_bf16_kernel(const bf16* __restrict__
   l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
   l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
   l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-  // group 1 hands its running max, sum and unnormalised output to group 0
-  // (same query rows, same lane layout) through its own, now idle, buffers
-  float* mg = reinterpret_cast<float*>(sBuf0 + 2 * C::BUF) + gtid * (4 + 4 * NO);
+  // groups 1 .. NG-1 hand their running max, sum and unnormalised output to
+  // group 0 (same query rows, same lane layout) through their own, now idle,
+  // buffers; group 0 merges them in group order
   __syncthreads();
-  if (grp == 1) {
+  if (grp > 0) {
+    float* mg = reinterpret_cast<float*>(sBuf0 + grp * 2 * C::BUF) + gtid * (4 + 4 * NO);
     mg[0] = m0; mg[1] = m1; mg[2] = l0; mg[3] = l1;
 #pragma unroll
     for (int n = 0; n < NO; ++n)
@@ -351,8 +354,10 @@ __global__ void __launch_bounds__(256) attn_bf16_kernel(const bf16* __restrict__
       for (int e = 0; e < 4; ++e) mg[4 + 4 * n + e] = o[n][e];
   }
   __syncthreads();
-  if (grp == 1) return;
-  {
+  if (grp > 0) return;
+#pragma unroll 1
+  for (int g2 = 1; g2 < NG; ++g2) {
+    const float* mg = reinterpret_cast<const float*>(sBuf0 + g2 * 2 * C::BUF) + gtid * (4 + 4 * NO);
     const float mb0 = mg[0], mb1 = mg[1], lb0 = mg[2], lb1 = mg[3];
     const float n0 = fmaxf(m0, mb0), n1 = fmaxf(m1, mb1);   // m0/m1 are finite: group 0 saw key 0
     const float ca0 = exp2f(m0 - n0), cb0 = exp2f(mb0 - n0), ca1 = exp2f(m1 - n1), cb1 = exp2f(mb1 - n1);
@@ -365,6 +370,8 @@ __global__ void __launch_bounds__(256) attn_bf16_kernel(const bf16* __restrict__
       o[n][2] = o[n][2] * ca1 + mg[4 + 4 * n + 2] * cb1;
       o[n][3] = o[n][3] * ca1 + mg[4 + 4 * n + 3] * cb1;
     }
+    m0 = n0;
+    m1 = n1;
   }
   const float inv0 = 1.f / l0, inv1 = 1.f / l1;
   const int r0 = i0 + wq * 16 + g, r1 = r0 + 8;
@@ -423,6 +430,16 @@ cudaError_t launch_mha<bf16>(const bf16* qkv, bf16* ctx, const SeqTable* seq, in
   return cudaGetLastError();
 }
 
+// Transformer MHSA with four warp groups (512 threads) splitting each CTA's
+// keys four ways instead of two: a shorter per-CTA chain for one long
+// sequence, where the 64-row CTAs are about one wave.
+cudaError_t launch_mha_bf16_4g(const bf16* qkv, bf16* ctx, const SeqTable* seq, int n_tiles, int M, cudaStream_t st) {
+  if (M <= 0) return cudaSuccess;
+  CK_LAUNCH(launch_k(attn_bf16_kernel<24, 32, false, 4>, dim3(dim3(n_tiles, 8)), dim3(512),
+                     AttCfg<24, 32, false, 4>::SMEM, st, qkv, 192, nullptr, 0, nullptr, nullptr, ctx, seq));
+  return cudaGetLastError();
+}
+
 // fp32 path: one score row of up to R floats per warp (4 warps per CTA).
 // The shared-memory limit is a per-kernel attribute of the process, so it
 // only ever grows: an engine made for shorter sequences never lowers what
@@ -447,8 +464,11 @@ cudaError_t attention_init_attributes() {
   cudaError_t e = cudaFuncSetAttribute(attn_bf16_kernel<64, 64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        AttCfg<64, 64, true>::SMEM);
   if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(attn_bf16_kernel<24, 32, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              AttCfg<24, 32, false>::SMEM);
+  e = cudaFuncSetAttribute(attn_bf16_kernel<24, 32, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           AttCfg<24, 32, false>::SMEM);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(attn_bf16_kernel<24, 32, false, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              AttCfg<24, 32, false, 4>::SMEM);
 }
 
 }  // namespace sf

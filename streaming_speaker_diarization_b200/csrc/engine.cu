@@ -599,8 +599,9 @@ cudaError_t mha_attention(sf_engine* e, const T* qkv, T* ctx, const SeqTable* se
 template <>
 cudaError_t mha_attention<bf16>(sf_engine* e, const bf16* qkv, bf16* ctx, const SeqTable* seq, int n_tiles, int M,
                                 cudaStream_t st) {
-  if (e->attn_path == 1 && e->att_tiles2 * 8 >= e->n_sms)
+  if (e->attn_path >= 1 && e->att_tiles2 * 8 >= e->n_sms)
     return launch_mha_tc(qkv, ctx, seq, e->att_tiles2, M, e->d_err, st);
+  if (e->attn_path == 2) return launch_mha_bf16_4g(qkv, ctx, seq, n_tiles, M, st);
   return launch_mha<bf16>(qkv, ctx, seq, n_tiles, M, e->R, st);
 }
 
@@ -614,7 +615,7 @@ cudaError_t relpos_attention(sf_engine* e, const T* qkv, const T* ptab, const fl
 template <>
 cudaError_t relpos_attention<bf16>(sf_engine* e, const bf16* qkv, const bf16* ptab, const float* pu, const float* pv,
                                    bf16* ctx, const SeqTable* seq, int n_tiles, int M, cudaStream_t st) {
-  if (e->attn_path == 1)
+  if (e->attn_path >= 1)
     return launch_relpos_attention_tc(qkv, ptab, e->R, pu, pv, ctx, seq, e->att_tiles2, M, e->att_max_len,
                                       e->tc_scratch(), st);
   return launch_relpos_attention<bf16>(qkv, ptab, e->R, pu, pv, ctx, seq, n_tiles, M, st);
@@ -1360,7 +1361,7 @@ sf_status sf_attention_mha(sf_engine* e, const void* d_qkv, const int* h_seq_len
   if (check_engine(e) != SF_OK) return SF_EINVAL;
   if (!d_qkv || !h_seq_len || !d_ctx) return fail(e, SF_EINVAL, "null pointer argument");
   if (e->cfg.precision != SF_BF16) return fail(e, SF_ESTATE, "sf_attention_mha needs a bf16 engine");
-  if (n < 1 || n > MAX_SEQ || (path != 0 && path != 1)) return fail(e, SF_ESHAPE, "sequence count or path");
+  if (n < 1 || n > MAX_SEQ || path < 0 || path > 2) return fail(e, SF_ESHAPE, "sequence count or path");
   if ((reinterpret_cast<uintptr_t>(d_qkv) | reinterpret_cast<uintptr_t>(d_ctx)) & 15)
     return fail(e, SF_EINVAL, "qkv and ctx must be 16-byte aligned");
   std::vector<int> lens(h_seq_len, h_seq_len + n);
@@ -1375,8 +1376,9 @@ sf_status sf_attention_mha(sf_engine* e, const void* d_qkv, const int* h_seq_len
   const bf16* qkv = static_cast<const bf16*>(d_qkv);
   bf16* ctx = static_cast<bf16*>(d_ctx);
   if (ce == cudaSuccess)
-    ce = path == 1 ? launch_mha_tc(qkv, ctx, &e->d_desc->seq, tiles2, M, e->d_err, st)
-                   : launch_mha<bf16>(qkv, ctx, &e->d_desc->seq, tiles, M, e->max_seq_len, st);
+    ce = path == 1   ? launch_mha_tc(qkv, ctx, &e->d_desc->seq, tiles2, M, e->d_err, st)
+         : path == 2 ? launch_mha_bf16_4g(qkv, ctx, &e->d_desc->seq, tiles, M, st)
+                     : launch_mha<bf16>(qkv, ctx, &e->d_desc->seq, tiles, M, e->max_seq_len, st);
   if (ce != cudaSuccess) return cuda_fail(e, ce, "sf_attention_mha");
   return SF_OK;
 }
@@ -1419,7 +1421,7 @@ sf_status sf_set_option(sf_engine* e, int option, int value) {
       e->gemm_path = value;
       break;
     case SF_OPT_ATTN_PATH:
-      if (value != 0 && value != 1) return fail(e, SF_EINVAL, "attention path must be 0 or 1");
+      if (value < 0 || value > 2) return fail(e, SF_EINVAL, "attention path must be 0, 1 or 2");
       e->attn_path = value;
       break;
     case SF_OPT_MEL_PATH:

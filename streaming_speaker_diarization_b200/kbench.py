@@ -9,7 +9,8 @@
 swish, 5 gated linear unit; P: SF_OPT_GEMM_PATH, 1 = tcgen05 with CTA pairs
 where faster, 2 = CTA pairs always, 3 = single CTAs, 0 = mma.sync); `attn`
 runs sf_attention_relpos and `mha` sf_attention_mha on N_SEQ packed
-sequences of LEN rows (P: 1 tcgen05, 0 mma.sync); `mel` runs sf_mel on B
+sequences of LEN rows (P: 1 tcgen05, 0 mma.sync; `mha` also 2, mma.sync
+with four key groups per CTA); `mel` runs sf_mel on B
 clips of SECONDS of audio each (P: SF_OPT_MEL_PATH).  Operands are seeded random values on the device; three warm-up
 launches, then REPS launches queued behind a GPU sleep (so host launch
 overhead is hidden) and timed with CUDA events on the current stream.  Also

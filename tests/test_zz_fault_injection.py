@@ -92,7 +92,7 @@ def test_bad_presets(setup, preset, n, code):
 def test_unknown_options_and_values(setup):
     _, eng = setup
     assert b.lib.sf_set_option(eng, 99, 1) == SF_EINVAL
-    for opt, bad in ((b.SF_OPT_GEMM_PATH, 4), (b.SF_OPT_ATTN_PATH, 2), (b.SF_OPT_GEMM_PAIR_BN, 64),
+    for opt, bad in ((b.SF_OPT_GEMM_PATH, 4), (b.SF_OPT_ATTN_PATH, 3), (b.SF_OPT_GEMM_PAIR_BN, 64),
                      (b.SF_OPT_MEL_PATH, 2), (b.SF_OPT_SUB_PATH, -1)):
         assert b.lib.sf_set_option(eng, opt, bad) == SF_EINVAL
 
