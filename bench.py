@@ -148,7 +148,7 @@ STREAM_WORKLOADS = [
 ]
 
 
-def streaming_bench(b, torch, eng_blob, rank, world, local, mel_path=0, sub_path=0):
+def streaming_bench(b, torch, eng_blob, rank, world, local, mel_path=0, sub_path=0, attn_path=1):
     """Streaming throughput: front-end over each stream's clip, then every
     step of every stream (pre_encode on the new window, encoder on
     [cache | FIFO | chunk], state update) until all streams finish.  A first
@@ -165,6 +165,7 @@ def streaming_bench(b, torch, eng_blob, rank, world, local, mel_path=0, sub_path
         eng = b.sf_create(eng_blob, b.default_config(max_batch=max(n, 1), max_samples=int(audio_np.shape[1])))
         b.sf_set_option(eng, b.SF_OPT_MEL_PATH, mel_path)
         b.sf_set_option(eng, b.SF_OPT_SUB_PATH, sub_path)
+        b.sf_set_option(eng, b.SF_OPT_ATTN_PATH, attn_path)
         audio = torch.from_numpy(audio_np).cuda()
         T = 1 + audio_np.shape[1] // 160
         mel = torch.empty((n, 128, T), device="cuda")
@@ -345,6 +346,7 @@ def main():
     ap.add_argument("--no-streaming", action="store_true", help="skip the streaming workloads")
     ap.add_argument("--no-frontend", action="store_true", help="skip the 1 h front-end-only run")
     ap.add_argument("--mel-path", type=int, default=0, choices=[0, 1], help="front-end implementation (SF_OPT_MEL_PATH)")
+    ap.add_argument("--attn-path", type=int, default=1, choices=[0, 1, 2], help="attention kernels (SF_OPT_ATTN_PATH)")
     ap.add_argument("--sub-path", type=int, default=0, choices=[0, 1],
                     help="subsampling conv1 + first depthwise implementation (SF_OPT_SUB_PATH)")
     ap.add_argument("--clocks-dir", default=None, help="where to keep the raw nvidia-smi clock samples")
@@ -372,6 +374,7 @@ def main():
     b.sf_set_option(eng, b.SF_OPT_PDL, args.pdl)
     b.sf_set_option(eng, b.SF_OPT_MEL_PATH, args.mel_path)
     b.sf_set_option(eng, b.SF_OPT_SUB_PATH, args.sub_path)
+    b.sf_set_option(eng, b.SF_OPT_ATTN_PATH, args.attn_path)
     st = torch.cuda.current_stream()
     audio = torch.from_numpy(audio_np).cuda()
     probs = torch.zeros((1, 1125, 4), device="cuda")
@@ -458,7 +461,8 @@ def main():
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": dict(CONFIG, parallelism=f"replicas x{world}", mel_path=args.mel_path, sub_path=args.sub_path),
+            "config": dict(CONFIG, parallelism=f"replicas x{world}", mel_path=args.mel_path, sub_path=args.sub_path,
+                           attn_path=args.attn_path),
             "roofline": roof, "clocks": clocks, "gpu_launches": launches,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(audio_np.nbytes),
                     "d2h_bytes_per_step": int(h_probs.numel() * 4)},
@@ -467,7 +471,7 @@ def main():
     b.sf_destroy(eng)
     if not args.no_streaming:
         line["streaming"] = streaming_bench(b, torch, weights_blob(w), rank, world, local, args.mel_path,
-                                            args.sub_path)
+                                            args.sub_path, args.attn_path)
     if not args.no_frontend:
         line["frontend_1h"] = frontend_bench(b, torch, weights_blob(w), max(args.steps, 5), max(args.warmup, 3),
                                              args.mel_path)
