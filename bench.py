@@ -256,11 +256,11 @@ def frontend_bench(b, torch, blob, steps, warmup, mel_path=0):
 
 
 def oracle_subsets(w):
-    """The oracle (fp64 numpy) on declared subsets of every workload, each
-    timed once on this machine's host cores: the 90 s clip complete, the
-    front-end on 1 h complete, 2 Low-preset streams x their first 20 steps,
-    1 Very-high-preset stream x 3 steps, and the first 4 clips of the
-    variable-length batch."""
+    """The oracle (numpy, fp64 unless stated) on declared subsets of every
+    workload, each timed once on this machine's host cores: the 90 s clip
+    complete (fp64, then fp32), the front-end on 1 h complete, 2 Low-preset
+    streams x their first 20 steps, 1 Very-high-preset stream x 3 steps, and
+    the first 4 clips of the variable-length batch."""
     import oracle as O
     from synth import clip_for_config
     from synth.audio import hour_of_audio
@@ -274,6 +274,9 @@ def oracle_subsets(w):
     t0 = time.perf_counter()
     O.forward_offline(a, ln, w)
     rec("offline 90 s clip", "complete", 90.0, time.perf_counter() - t0)
+    t0 = time.perf_counter()
+    O.forward_offline(a, ln, w, dt=np.float32)
+    rec("offline 90 s clip, oracle in fp32", "complete", 90.0, time.perf_counter() - t0)
 
     x = hour_of_audio()
     t0 = time.perf_counter()
