@@ -1,5 +1,7 @@
 """Pins for the oracle's encoder layers: closed forms, brute force, and an
 independent re-derivation of the relative-position shift."""
+import math
+
 import numpy as np
 import pytest
 import scipy.signal
@@ -205,3 +207,147 @@ def test_parameter_count_matches_117m():
     # "Speaker diarization model (117M params)"; ~470 MB fp32 export
     assert 116.5e6 < total < 118.5e6
     assert abs(total * 4 / 1e6 - 470) < 5
+
+
+# --------------------------------------------------------------------------
+# Transformer layer and macaron FFN with non-zero weights.  The model is the
+# "Streaming Sortformer Diarizer" page's Pipeline: an 18-layer Transformer of
+# width 192 with 8 heads (head size 24) after Linear 512->192; post-LN with a
+# ReLU FFN 192->768->192 (the workload's "post-LN Transformer layers").
+
+def _tf_weights(seed=21, e=192, ff=768, scale=0.15):
+    """Non-zero weights for one Transformer layer, strong enough that every
+    softmax row is far from uniform (score spread of several units)."""
+    rng = np.random.default_rng(seed)
+    p = "tf.layers.0."
+    w = {}
+    for q in ("q", "k", "v", "o"):
+        w[p + f"att.{q}.weight"] = rng.standard_normal((e, e)) * scale
+        w[p + f"att.{q}.bias"] = rng.standard_normal(e) * scale
+    w[p + "ff.linear1.weight"] = rng.standard_normal((ff, e)) * (1 / np.sqrt(e))
+    w[p + "ff.linear1.bias"] = rng.standard_normal(ff) * 0.1
+    w[p + "ff.linear2.weight"] = rng.standard_normal((e, ff)) * (1 / np.sqrt(ff))
+    w[p + "ff.linear2.bias"] = rng.standard_normal(e) * 0.1
+    for ln in ("ln1", "ln2"):
+        w[p + f"{ln}.weight"] = 1 + 0.2 * rng.standard_normal(e)
+        w[p + f"{ln}.bias"] = 0.2 * rng.standard_normal(e)
+    return w, p
+
+
+def _loop_linear(x, Wm, b):
+    return [[sum(row[c] * Wm[o][c] for c in range(len(row))) + b[o] for o in range(len(b))] for row in x]
+
+
+def _brute_mha(x, w, p, H, scale_dim=None, head_cols=None):
+    """Pure-loop multi-head attention: head h uses feature columns
+    head_cols(h, c) (default h * dk + c), scores divided by sqrt(scale_dim)
+    (default the head size).  The two options only exist so the pins below
+    can show that a wrong scale or head split would be caught."""
+    S, e = len(x), len(x[0])
+    dk = e // H
+    scale_dim = dk if scale_dim is None else scale_dim
+    col = head_cols or (lambda h, c: h * dk + c)
+    q = _loop_linear(x, w[p + "q.weight"], w[p + "q.bias"])
+    k = _loop_linear(x, w[p + "k.weight"], w[p + "k.bias"])
+    v = _loop_linear(x, w[p + "v.weight"], w[p + "v.bias"])
+    ctx = [[0.0] * e for _ in range(S)]
+    for h in range(H):
+        for i in range(S):
+            s = [sum(q[i][col(h, c)] * k[j][col(h, c)] for c in range(dk)) / math.sqrt(scale_dim) for j in range(S)]
+            mx = max(s)
+            ex = [math.exp(t - mx) for t in s]
+            z = sum(ex)
+            for j in range(S):
+                for c in range(dk):
+                    ctx[i][col(h, c)] += ex[j] / z * v[j][col(h, c)]
+    return np.array(_loop_linear(ctx, w[p + "o.weight"], w[p + "o.bias"]))
+
+
+def _loop_layer_norm(row, g, b, eps=1e-5):
+    n = len(row)
+    mu = sum(row) / n
+    var = sum((t - mu) ** 2 for t in row) / n
+    return [(row[c] - mu) / math.sqrt(var + eps) * g[c] + b[c] for c in range(n)]
+
+
+@pytest.mark.parametrize("S", [1, 3, 8])
+def test_transformer_mha_vs_brute_force(S):
+    w, p = _tf_weights()
+    x = np.random.default_rng(30 + S).standard_normal((S, 192))
+    out = M._mha(x, w, p + "att.", 8, np.float64)
+    ref = _brute_mha(x.tolist(), w, p + "att.", 8)
+    assert np.max(np.abs(out - ref)) < 1e-10
+    if S > 1:
+        # planted mistakes the comparison must see: scale 1/sqrt(192) instead
+        # of 1/sqrt(24), and heads taken as interleaved columns c * H + h
+        wrong_scale = _brute_mha(x.tolist(), w, p + "att.", 8, scale_dim=192)
+        wrong_split = _brute_mha(x.tolist(), w, p + "att.", 8, head_cols=lambda h, c: c * 8 + h)
+        assert np.max(np.abs(out - wrong_scale)) > 1e-2
+        assert np.max(np.abs(out - wrong_split)) > 1e-2
+
+
+def test_transformer_mha_is_rel_pos_mhsa_without_positions():
+    """With linear_pos, pos_bias_u and pos_bias_v zero, the conformer's
+    relative-position attention (pinned against brute force above) is plain
+    scaled dot-product attention: the Transformer's MHA must equal it."""
+    w, p = _tf_weights(seed=5)
+    q = "enc.layers.0."
+    wr = {}
+    for a, b in (("q", "q"), ("k", "k"), ("v", "v"), ("out", "o")):
+        wr[q + f"att.linear_{a}.weight"] = w[p + f"att.{b}.weight"]
+        wr[q + f"att.linear_{a}.bias"] = w[p + f"att.{b}.bias"]
+    wr[q + "att.linear_pos.weight"] = np.zeros((192, 192))
+    wr[q + "att.pos_bias_u"] = np.zeros((8, 24))
+    wr[q + "att.pos_bias_v"] = np.zeros((8, 24))
+    x = np.random.default_rng(6).standard_normal((11, 192))
+    out = M._mha(x, w, p + "att.", 8, np.float64)
+    ref = M.rel_pos_mhsa(x, wr, q, 8)
+    assert np.max(np.abs(out - ref)) < 1e-12
+    _, probs = M.rel_pos_mhsa(x, wr, q, 8, return_probs=True)
+    assert min(float(a.max()) for a in probs) > 0.3     # attention far from uniform (1/11)
+
+
+@pytest.mark.parametrize("S", [1, 4])
+def test_transformer_layer_vs_loop_post_ln(S):
+    """Post-LN order written out with loops: y = LN1(x + MHA(x)),
+    out = LN2(y + W2 relu(W1 y + b1) + b2)."""
+    w, p = _tf_weights(seed=9)
+    x = np.random.default_rng(40 + S).standard_normal((S, 192))
+    out = M.transformer_layer(x, w, 0)
+    a = _brute_mha(x.tolist(), w, p + "att.", 8)
+    y = [_loop_layer_norm([x[i][c] + a[i][c] for c in range(192)], w[p + "ln1.weight"], w[p + "ln1.bias"])
+         for i in range(S)]
+    h = [[max(t, 0.0) for t in row] for row in _loop_linear(y, w[p + "ff.linear1.weight"], w[p + "ff.linear1.bias"])]
+    f = _loop_linear(h, w[p + "ff.linear2.weight"], w[p + "ff.linear2.bias"])
+    ref = np.array([_loop_layer_norm([y[i][c] + f[i][c] for c in range(192)], w[p + "ln2.weight"], w[p + "ln2.bias"])
+                    for i in range(S)])
+    assert np.max(np.abs(out - ref)) < 1e-10
+    # pre-LN (LN before each sublayer) is a different layer: must not match
+    pre = x + M._mha(M.layer_norm(x, w[p + "ln1.weight"], w[p + "ln1.bias"]), w, p + "att.", 8, np.float64)
+    assert np.max(np.abs(out - pre)) > 1e-2
+
+
+def test_macaron_ffn_half_step_and_swish(tiny_weights_xavier):
+    """A conformer layer whose attention and conv module have zero weights
+    (their residual branches add their output biases, zero here) and whose
+    second FFN is zero reduces to LN(x + FFN1(LN(x)) / 2) with
+    FFN(h) = W2 swish(W1 h + b1) + b2; the FFN is written out with loops."""
+    w = dict(tiny_weights_xavier)
+    p = "enc.layers.0."
+    for k in list(w):
+        if k.startswith(p) and (".att." in k or ".conv." in k or ".ff2." in k) and not k.endswith(
+                ("ln.weight", "ln.bias", "bn.running_var", "bn.weight")):
+            w[k] = np.zeros_like(w[k])
+    rng = np.random.default_rng(13)
+    x = rng.standard_normal((3, 512))
+    out = M.conformer_layer(x, w, 0)
+    g1 = np.ones(512)
+    z1 = np.zeros(512)
+    ln_x = [_loop_layer_norm(list(r), g1, z1) for r in x]
+    h = _loop_linear(ln_x, w[p + "ff1.linear1.weight"], w[p + "ff1.linear1.bias"])
+    h = [[t / (1 + math.exp(-t)) for t in row] for row in h]
+    f = _loop_linear(h, w[p + "ff1.linear2.weight"], w[p + "ff1.linear2.bias"])
+    ref = np.array([_loop_layer_norm([x[i][c] + 0.5 * f[i][c] for c in range(512)], g1, z1) for i in range(3)])
+    assert np.max(np.abs(out - ref)) < 1e-10
+    full_step = np.array([_loop_layer_norm([x[i][c] + f[i][c] for c in range(512)], g1, z1) for i in range(3)])
+    assert np.max(np.abs(out - full_step)) > 1e-2
