@@ -45,9 +45,9 @@ CONFIG = {"workload": "offline forward, 1 clip x 90 s (16 kHz, 4 speakers, 15% o
 
 
 # DRAM bytes (read + write) per projection launch of the offline forward,
-# from an ncu launch list of this workload (profiles/offline_90s_launch_list.md:
-# 815.3 MB over the 213 GEMM launches of one forward); valid only for the GEMM
-# sources it was taken with, null once they change.
+# from an ncu launch list of this workload (815.3 MB over the 213 GEMM
+# launches of one forward); valid only for the GEMM sources it was taken
+# with, null once they change.
 GEMM_TRAFFIC = {"bytes_per_launch": 815.3e6 / 213,
                 "sources_sha256": "9bad6df933c0cd329728f20224afdde012e864c83a7fc71d246a0dfde6e9963d"}
 
@@ -73,11 +73,55 @@ def peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
+# NVML clock-event reason bits (nvmlClocksEventReason*) reported in the line
+_REASON_BITS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown", 0x4: "sw_power_cap",
+                0x80: "hw_power_brake_slowdown"}
+
+
+def summarize_samples(samples):
+    """Summary of in-process clock samples [(sm_mhz, max_sm_mhz, reason_bits)]:
+    median SM clock, max clock, and every throttle reason seen active."""
+    sm = [float(a) for a, _, _ in samples]
+    reasons = set()
+    for _, _, bits in samples:
+        for bit, name in _REASON_BITS.items():
+            if bits & bit:
+                reasons.add(name)
+    return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": float(samples[-1][1]) if samples else None,
+            "reasons": sorted(reasons), "samples": len(sm)}
+
+
 class Clocks:
-    """nvidia-smi sampling during the timed region; the raw samples go to
-    `out_dir` (default: the system temporary directory)."""
+    """Clocks and throttle reasons sampled DURING a timed region.  A thread
+    polls NVML every millisecond (reading only), so regions of tens of
+    milliseconds still get samples; without NVML, nvidia-smi is sampled
+    every 200 ms (raw samples under `out_dir`, default the temporary
+    directory)."""
 
     def __init__(self, idx, out_dir=None):
+        import threading
+        self.samples, self.p = [], None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self.stop_ev = threading.Event()
+
+            def poll():
+                while not self.stop_ev.is_set():
+                    try:
+                        self.samples.append((pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM), mx,
+                                             int(pynvml.nvmlDeviceGetCurrentClocksEventReasons(h))))
+                    except Exception:
+                        pass
+                    time.sleep(0.001)
+            self.t = threading.Thread(target=poll, daemon=True)
+            self.t.start()
+            self.mode = "nvml"
+            return
+        except Exception:
+            self.mode = "nvidia-smi"
         import tempfile
         self.path = os.path.join(out_dir or tempfile.gettempdir(), f"sf_bench_clocks_rank{idx}.csv")
         os.makedirs(os.path.dirname(self.path), exist_ok=True)
@@ -92,6 +136,10 @@ class Clocks:
             self.p = None
 
     def stop(self):
+        if self.mode == "nvml":
+            self.stop_ev.set()
+            self.t.join(timeout=5)
+            return dict(summarize_samples(self.samples), source="nvml, 1 ms polling during the timed region")
         if self.p is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.p.terminate()
@@ -101,7 +149,7 @@ class Clocks:
             self.p.kill()
         self.f.close()
         with open(self.path) as f:
-            return parse_clocks(f)
+            return dict(parse_clocks(f), source="nvidia-smi, 200 ms polling during the timed region")
 
 
 def parse_clocks(lines):
@@ -140,6 +188,49 @@ def cpu_baseline(audio, seconds=30.0):
                       f"({dt:.1f} s)"}
 
 
+# Algorithmic work of the model per encoder frame of a sequence of S frames
+# (2 flops per multiply-add): conformer layer 12.06 MF of projections (FFN
+# 2 x 2 x 512 x 2048 x 2, Q/K/V/out 4 x 512^2 x 2, conv pointwise 512 x 1024
+# x 2 + 512^2 x 2) + 3 x 2 x 512 x S of attention (AC, BD, P.V);
+# Transformer layer 0.885 MF (Q/K/V/out 4 x 192^2 x 2, FFN 2 x 192 x 768 x 2)
+# + 2 x 2 x 192 x S; encoder_proj 2 x 512 x 192; head 2 x 192 x (192 + 4);
+# subsampling 16.23 MF per encoder frame it produces.  The relative-position
+# projections are weights-only (computed once when the engine is created)
+# and are not counted.
+CONF_MF, TF_MF, PROJ_HEAD_MF, SUB_MF = 12.059136e6, 0.884736e6, 0.196608e6 + 0.075264e6, 16.23e6
+
+
+def model_flops(S, new_frames, n_conf=17, n_tf=18):
+    """Flops of one encoder pass over a sequence of S frames of which
+    new_frames came out of the subsampling in this pass."""
+    per = n_conf * (CONF_MF + 3072.0 * S) + n_tf * (TF_MF + 768.0 * S) + PROJ_HEAD_MF
+    return S * per + new_frames * SUB_MF
+
+
+def stream_plan(preset, total_frames):
+    """Per step of one stream: (S, window embeddings) for a clip of
+    total_frames encoder frames under preset (chunk, right context, FIFO,
+    update period, cache).  The sizes do not depend on the data: the window
+    holds cl' = min(chunk, left) chunk frames and rc' = min(right, left - cl')
+    look-ahead frames after [cache | FIFO]; the chunk joins the FIFO, which
+    pops max(update period, overflow) frames into the cache once it is over
+    its length; the cache is compressed back to its length when it overflows."""
+    cl, rc, fl, up, cap = preset
+    n_c = n_f = c0 = 0
+    out = []
+    while c0 < total_frames:
+        c = min(cl, total_frames - c0)
+        r = min(rc, total_frames - c0 - c)
+        out.append((n_c + n_f + c + r, c + r))
+        n_f += c
+        c0 += c
+        if n_f > fl:
+            n = min(max(up, n_f - fl), n_f)
+            n_f -= n
+            n_c = min(n_c + n, cap)
+    return out
+
+
 STREAM_WORKLOADS = [
     # (name, preset chunk/right/fifo/update/cache, workload index, streams, seconds)
     ("Low preset (6/7/188/144/188, 1.04 s latency), 64 streams x 60 s, 2-4 speakers", (6, 7, 188, 144, 188), 2, 64, 60.0),
@@ -148,12 +239,16 @@ STREAM_WORKLOADS = [
 ]
 
 
-def streaming_bench(b, torch, eng_blob, rank, world, local, mel_path=0, sub_path=0, attn_path=1):
+def streaming_bench(b, torch, eng_blob, rank, world, local, mel_path=1, sub_path=1, attn_path=1, clocks_dir=None):
     """Streaming throughput: front-end over each stream's clip, then every
     step of every stream (pre_encode on the new window, encoder on
     [cache | FIFO | chunk], state update) until all streams finish.  A first
     pass captures each step shape's CUDA graph; the streams are reset and the
-    second pass is timed with CUDA events."""
+    second pass is timed with CUDA events (clocks sampled meanwhile).  A
+    third pass brackets only the state-update and selection launches with
+    events: the cache compression's microseconds per step.  The roofline is
+    the model's algorithmic flops (model_flops over every stream's steps)
+    over the timed pass."""
     from streaming_speaker_diarization_b200 import dist as sd
     from synth import clip_for_config
     out = []
@@ -192,17 +287,41 @@ def streaming_bench(b, torch, eng_blob, rank, world, local, mel_path=0, sub_path
         torch.cuda.synchronize()
         t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         steps = []
+        clk = Clocks(local, clocks_dir)
         t0.record()
         one_pass(steps)
         t1.record()
         torch.cuda.synchronize()
+        clocks = clk.stop()
         ms = t0.elapsed_time(t1)
         step_ms = [a.elapsed_time(c) for a, c in steps]
+        # compression: events around the state-update and selection launches only
+        b.sf_stream_reset(st)
+        b.sf_profile_read(eng, reset=True)
+        b.sf_profile_enable(eng, 2 * ((1 << 11) | (1 << 13)))
+        one_pass()
+        torch.cuda.synchronize()
+        upd = b.sf_profile_read(eng, reset=True)
+        b.sf_profile_enable(eng, 0)
+        upd_ms = sum(v[1] for k, v in upd.items() if k in ("state_update", "select_topk"))
         audio_s = float(lens.sum()) / 16000.0
         value = sd.throughput(audio_s, ms)
+        frames = [int(1 + (int(l) // 160 - 1) // 8) for l in lens]
+        flops = sum(model_flops(S, new) for f in frames for S, new in stream_plan(preset, f))
+        max_ms = sd.max_over_ranks(ms)
+        pk, kind = peaks()
+        tf = sd.sum_over_ranks(flops) / (max_ms / 1000.0) / 1e12
+        peak_tf = pk["bf16_tflops_sustained"] if max_ms > 1000.0 else pk["bf16_tflops"]
         out.append({"workload": name, "value": value, "unit": UNIT, "streams": n_total, "steps": len(step_ms),
-                    "ms_total": sd.max_over_ranks(ms), "step_ms_p50": float(np.median(step_ms)),
-                    "step_ms_p95": float(np.percentile(step_ms, 95))})
+                    "ms_total": max_ms, "step_ms_p50": float(np.median(step_ms)),
+                    "step_ms_p95": float(np.percentile(step_ms, 95)),
+                    "encoder_frames_per_s": sd.sum_over_ranks(sum(frames)) / (max_ms / 1000.0),
+                    "roofline": {"bound": "tensor", "kernel": "whole step (model flops)", "achieved": tf,
+                                 "peak": peak_tf, "unit": "TFLOP/s", "frac": tf / peak_tf,
+                                 "flops_total": flops,
+                                 "peak_kind": f"{kind} bf16 {'sustained' if max_ms > 1000.0 else 'burst'}"},
+                    "compression_us_per_step": 1000.0 * upd_ms / max(len(step_ms), 1),
+                    "clocks": clocks})
         b.sf_stream_destroy(st)
         b.sf_destroy(eng)
         del audio, mel
@@ -210,7 +329,7 @@ def streaming_bench(b, torch, eng_blob, rank, world, local, mel_path=0, sub_path
     return out
 
 
-def frontend_bench(b, torch, blob, steps, warmup, mel_path=0):
+def frontend_bench(b, torch, blob, steps, warmup, mel_path=1):
     """Front-end alone (preemphasis, centred STFT, power, Slaney mel, log,
     per-bin normalisation) on 1 h of audio in one sf_mel call: 57.6M samples
     -> 128 x 360,001 features.  Audio resident on the device, CUDA events per
@@ -253,6 +372,57 @@ def frontend_bench(b, torch, blob, steps, warmup, mel_path=0):
             "calls": steps, "mel_path": mel_path,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs / pk["hbm_gbs"], "bytes_per_call": alg, "peak_kind": f"{kind} copy"}}
+
+
+def batch_bench(b, torch, blob, steps, warmup, local, mel_path=1, sub_path=1, attn_path=1, clocks_dir=None):
+    """The variable-length offline batch: 32 clips of 5-120 s (seeded),
+    padded to the longest, one sf_forward_offline call per step (front-end
+    to probabilities).  Audio resident on the device, L2 flushed between
+    steps, CUDA events per step on the launching stream."""
+    from synth import clip_for_config
+    audio_np, lens, _ = clip_for_config(4)
+    B, n_max = audio_np.shape
+    eng = b.sf_create(blob, b.default_config(max_batch=B, max_samples=int(n_max)))
+    b.sf_set_option(eng, b.SF_OPT_MEL_PATH, mel_path)
+    b.sf_set_option(eng, b.SF_OPT_SUB_PATH, sub_path)
+    b.sf_set_option(eng, b.SF_OPT_ATTN_PATH, attn_path)
+    try:
+        audio = torch.from_numpy(audio_np).cuda()
+        Tp = 1 + (n_max // 160 - 1) // 8
+        probs = torch.zeros((B, Tp, 4), device="cuda")
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+        st = torch.cuda.current_stream()
+        for _ in range(warmup):
+            b.sf_forward_offline(eng, audio, lens, probs)
+        b.sf_check(eng)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        torch.cuda.synchronize()
+        clk = Clocks(local, clocks_dir)
+        for i in range(steps):
+            flush.zero_()
+            ev[i][0].record(st)
+            b.sf_forward_offline(eng, audio, lens, probs)
+            ev[i][1].record(st)
+        torch.cuda.synchronize()
+        clocks = clk.stop()
+        b.sf_check(eng)
+    finally:
+        b.sf_destroy(eng)
+    ms = [a.elapsed_time(c) for a, c in ev]
+    med = float(np.median(ms))
+    audio_s = float(lens.sum()) / 16000.0
+    frames = [int(1 + (int(l) // 160 - 1) // 8) for l in lens]
+    flops = sum(model_flops(f, f) for f in frames)
+    pk, kind = peaks()
+    tf = flops / (med / 1000.0) / 1e12
+    return {"workload": "offline variable-length batch, 32 clips of 5-120 s (seeded), padded to the longest, "
+                        "full model, bf16", "value": audio_s / (med / 1000.0), "unit": UNIT,
+            "audio_s": audio_s, "clips": B, "ms_p50": med, "ms_p95": float(np.percentile(ms, 95)), "calls": steps,
+            "encoder_frames_per_s": sum(frames) / (med / 1000.0),
+            "roofline": {"bound": "tensor", "kernel": "whole forward (model flops)", "achieved": tf,
+                         "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": tf / pk["bf16_tflops"],
+                         "flops_per_call": flops, "peak_kind": f"{kind} bf16 burst"},
+            "clocks": clocks}
 
 
 def oracle_subsets(w):
@@ -348,9 +518,10 @@ def main():
     ap.add_argument("--pdl", type=int, default=0, help="programmatic dependent launch between kernels (0/1)")
     ap.add_argument("--no-streaming", action="store_true", help="skip the streaming workloads")
     ap.add_argument("--no-frontend", action="store_true", help="skip the 1 h front-end-only run")
-    ap.add_argument("--mel-path", type=int, default=0, choices=[0, 1], help="front-end implementation (SF_OPT_MEL_PATH)")
+    ap.add_argument("--no-batch", action="store_true", help="skip the 32-clip variable-length batch")
+    ap.add_argument("--mel-path", type=int, default=1, choices=[0, 1], help="front-end implementation (SF_OPT_MEL_PATH)")
     ap.add_argument("--attn-path", type=int, default=1, choices=[0, 1, 2], help="attention kernels (SF_OPT_ATTN_PATH)")
-    ap.add_argument("--sub-path", type=int, default=0, choices=[0, 1],
+    ap.add_argument("--sub-path", type=int, default=1, choices=[0, 1],
                     help="subsampling conv1 + first depthwise implementation (SF_OPT_SUB_PATH)")
     ap.add_argument("--clocks-dir", default=None, help="where to keep the raw nvidia-smi clock samples")
     ap.add_argument("--oracle-subsets", action="store_true",
@@ -474,7 +645,10 @@ def main():
     b.sf_destroy(eng)
     if not args.no_streaming:
         line["streaming"] = streaming_bench(b, torch, weights_blob(w), rank, world, local, args.mel_path,
-                                            args.sub_path, args.attn_path)
+                                            args.sub_path, args.attn_path, args.clocks_dir)
+    if not args.no_batch and world == 1:
+        line["batch"] = batch_bench(b, torch, weights_blob(w), args.steps, max(args.warmup, 3), local, args.mel_path,
+                                    args.sub_path, args.attn_path, args.clocks_dir)
     if not args.no_frontend:
         line["frontend_1h"] = frontend_bench(b, torch, weights_blob(w), max(args.steps, 5), max(args.warmup, 3),
                                              args.mel_path)

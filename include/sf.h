@@ -28,7 +28,8 @@
  *    SF_ETIMEOUT reports that a bounded device-side wait gave up (the
  *    engine's kernels never spin without a limit).
  *  - An engine or stream object must not be used from two host threads at
- *    once, and calls on one engine must be ordered: issue them on one CUDA
+ *    once (creating or destroying a stream uses its engine), and calls on
+ *    one engine must be ordered: issue them on one CUDA
  *    stream (or order the streams yourself), because every call reuses the
  *    engine's workspace and descriptor block.  Different engines may be
  *    driven from different host threads (e.g. one engine and one thread
@@ -179,13 +180,15 @@ SF_API sf_status sf_mel(sf_engine* e, const float* d_audio, const int64_t* h_len
  * another framework's CUDA context, a real-time thread that must not block
  * in cudaMalloc/cudaFree).  Same arguments, layout and result as sf_mel, but
  * no engine is needed and nothing is allocated: the call's scratch (clip
- * lengths and per-tile statistics) is a fixed 8 MiB static device array in
- * libsf.so that every GPU loading the library keeps until exit.
+ * lengths, per-tile statistics and per-clip normalisation constants) is a
+ * fixed static device array of about 8 MiB in libsf.so that every GPU
+ * loading the library keeps until exit.
  * Limits: B <= 64 clips and B * ceil((1 + n_max/160) / 32) <= 4096 frame
  * tiles (e.g. 10 clips of 120 s); larger requests return SF_ESHAPE.
- * The first call on a device takes the array's device address and uploads
- * the FFT/window/filterbank tables with a blocking copy: make it before any
- * CUDA stream capture.  All calls share the array and it keeps the last
+ * The first call on a device (with that device current) takes the array's
+ * device address, uploads the FFT/window/filterbank tables with a blocking
+ * copy and sets the frame kernels' shared-memory attribute for the device:
+ * make it before any CUDA stream capture.  All calls share the array and it keeps the last
  * call's contents, so calls whose GPU work overlaps (on different streams or
  * threads) race and corrupt each other; order them on one stream.  No error
  * message is kept (there is no engine): the status code is the report. */
@@ -240,7 +243,10 @@ SF_API sf_status sf_stream_create(sf_engine* e, const sf_preset* p, int n_stream
  * graphs that were captured for it. */
 SF_API sf_status sf_stream_destroy(sf_stream* s);
 
-/* Restore the empty state of the listed streams (h_ids NULL = all). */
+/* Restore the empty state of the listed streams (h_ids NULL = all; else
+ * n >= 0 ids in [0, n_streams), SF_EINVAL otherwise).  Synchronises the
+ * device before and after clearing the device-side silence statistics, so
+ * it is ordered against steps on any CUDA stream. */
 SF_API sf_status sf_stream_reset(sf_stream* s, const int* h_ids, int n);
 
 /* Mel-frame window [*h_start, *h_end) the next step of stream `id` reads
@@ -372,19 +378,19 @@ enum {
   SF_OPT_GEMM_PAIR_BN = 4, /* tile width of the CTA-pair kernel: 0 (default) chosen per shape,
                               or 128, 192, 256 */
   SF_OPT_ATTN_PATH = 5,   /* bf16 attention (relative-position and Transformer): 1 (default)
-                             tcgen05/TMEM/TMA kernels (the Transformer's on mma.sync when
-                             its units do not fill the SMs), 0 mma.sync kernels, 2 as 1
-                             with that mma.sync fallback splitting each CTA's keys over
-                             four warp groups instead of two */
+                             tcgen05/TMEM/TMA kernels, whose keys are split over CTA clusters
+                             when one sequence leaves SMs idle; 0 mma.sync kernels; 2 the
+                             tcgen05 relative-position kernel with the Transformer's on
+                             mma.sync, each CTA's keys split over four warp groups */
   SF_OPT_MEL_PATH = 6,    /* log-mel front-end (sf_mel, the offline forward, the audio-in
-                             step): 0 (default) FFT through shared memory and one
-                             normalisation CTA per (clip, bin); 1 FFT in registers with warp
-                             shuffles, then separate statistics and normalisation passes over
-                             all SMs */
-  SF_OPT_SUB_PATH = 7     /* ConvSubsampling's first two stages: 0 (default) the 3x3 s2 conv
-                             and the first depthwise conv as two kernels through a
-                             [T/2][64][256] tensor in memory; 1 one kernel that computes the
-                             first conv's outputs on chip (same result to the bit) */
+                             step): 1 (default) FFT in registers with warp shuffles, then
+                             separate statistics and normalisation passes over all SMs; 0 FFT
+                             through shared memory and one normalisation CTA per (clip, bin) */
+  SF_OPT_SUB_PATH = 7     /* ConvSubsampling's first two stages: 1 (default) one kernel that
+                             computes the first conv's outputs on chip and feeds them straight
+                             into the first depthwise conv; 0 the 3x3 s2 conv and the first
+                             depthwise conv as two kernels through a [T/2][64][256] tensor in
+                             memory (same result to the bit) */
 };
 SF_API sf_status sf_set_option(sf_engine* e, int option, int value);
 

@@ -1,9 +1,9 @@
 """Kernel micro-benchmarks through the C ABI's single-op entry points.
 
-    python -m streaming_speaker_diarization_b200.kbench gemm M N K [--epi E] [--path P] [--reps R]
-    python -m streaming_speaker_diarization_b200.kbench attn N_SEQ LEN [--path P] [--reps R]
-    python -m streaming_speaker_diarization_b200.kbench mha N_SEQ LEN [--path P] [--reps R]
-    python -m streaming_speaker_diarization_b200.kbench mel SECONDS [--clips B] [--path P] [--reps R]
+    python kbench.py gemm M N K [--epi E] [--path P] [--reps R]
+    python kbench.py attn N_SEQ LEN [--path P] [--reps R]
+    python kbench.py mha N_SEQ LEN [--path P] [--reps R]
+    python kbench.py mel SECONDS [--clips B] [--path P] [--reps R]
 
 `gemm` runs sf_gemm_bf16 (E: 1 f32 out, 2 bf16 out, 3 residual update, 4
 swish, 5 gated linear unit; P: SF_OPT_GEMM_PATH, 1 = tcgen05 with CTA pairs

@@ -20,6 +20,11 @@
 // O accumulated in registers.  Shared memory ~97 KB and 256 TMEM columns, so
 // two CTAs share an SM.  Every wait is bounded: a wait that runs out raises
 // ERR_TIMEOUT, the CTA drains its own copies and frees its TMEM.
+// When the (query tile, head) units are fewer than the SMs (one long
+// sequence), each unit's key tiles are split over a cluster of 2 or 4 CTAs:
+// each CTA leaves the softmax state (O, m, l) of its key range in its own
+// shared memory and the cluster's rank 0 merges them in rank order over
+// distributed shared memory.
 #include "common.cuh"
 #include "layers.h"
 #include "tcgen05.cuh"
@@ -45,7 +50,11 @@ struct MhaTc {
   static constexpr int OFF_P = OFF_RING + MNB * STAGE;
   static constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
   static constexpr int SMEM = 1024 + OFF_BAR + 256;
+  // key split: row r's partial state O[24], m, l (+2 pad, 16-byte rows) in
+  // the P buffers once the last P.V product has completed
+  static constexpr int PSTR = MHD + 4;
   static_assert(STAGE % 1024 == 0 && OFF_P % 1024 == 0 && OFF_RING % 1024 == 0, "swizzled tiles 1024-aligned");
+  static_assert(MQ * PSTR * 4 <= 2 * P_BYTES, "partials fit in the P buffers");
 };
 
 }  // namespace
@@ -53,7 +62,8 @@ struct MhaTc {
 __global__ void __launch_bounds__(192, 2) attn_mha_tc_kernel(const __grid_constant__ CUtensorMap t_qkv,
                                                              const bf16* __restrict__ qkv, int E,
                                                              bf16* __restrict__ ctx,
-                                                             const SeqTable* __restrict__ seq, int* err) {
+                                                             const SeqTable* __restrict__ seq, int* err,
+                                                             int ks) {
   using L = MhaTc;
   extern __shared__ uint8_t mh_smem[];
   uint8_t* sm = mh_smem + ((1024 - (su32(mh_smem) & 1023)) & 1023);
@@ -75,7 +85,11 @@ __global__ void __launch_bounds__(192, 2) attn_mha_tc_kernel(const __grid_consta
   const int s = seq_of_tile2(seq, blockIdx.x);
   const int sb = seq->off[s], S = seq->off[s + 1] - sb;
   const int i0 = (blockIdx.x - seq->tile2_off[s]) * MQ;
-  const int T = (S + MK - 1) / MK;   // key tiles
+  const int T = (S + MK - 1) / MK;   // key tiles of the sequence
+  // key split: this CTA takes key tiles [t0, t0 + Tl) (blockIdx.z of ks);
+  // ring stages and barrier phases count local tiles
+  const int t0 = (int)((int64_t)T * blockIdx.z / ks);
+  const int Tl = (int)((int64_t)T * (blockIdx.z + 1) / ks) - t0;
 
   if (threadIdx.x == 0) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&t_qkv)) : "memory");
@@ -110,8 +124,8 @@ __global__ void __launch_bounds__(192, 2) attn_mha_tc_kernel(const __grid_consta
     // ---------------------------------------------------------------- loads
     if (lane == 0) {
       int t = 0;
-      for (; t < T && !*abort_flag; ++t) {
-        const int b = t % MNB, r = t / MNB, j0 = t * MK;
+      for (; t < Tl && !*abort_flag; ++t) {
+        const int b = t % MNB, r = t / MNB, j0 = (t0 + t) * MK;
         if (!mbar_wait(&kv_empty[b], (r & 1) ^ 1, abort_flag)) {
           *abort_flag = 1;
           break;
@@ -149,7 +163,7 @@ __global__ void __launch_bounds__(192, 2) attn_mha_tc_kernel(const __grid_consta
         umma_commit(&kv_empty[b]);   // K and V of tile t are no longer read
         return true;
       };
-      for (int t = 0; ok && t < T; ++t) {
+      for (int t = 0; ok && t < Tl; ++t) {
         const int b = t % MNB;
         if (!mbar_wait(&kv_full[b], (t / MNB) & 1, abort_flag)) { ok = false; break; }
         if (t > 0 && !mbar_wait(s_free, (t - 1) & 1, abort_flag)) { ok = false; break; }
@@ -160,7 +174,7 @@ __global__ void __launch_bounds__(192, 2) attn_mha_tc_kernel(const __grid_consta
         umma_commit(s_full);
         if (t > 0 && !issue_pv(t - 1)) { ok = false; break; }
       }
-      if (ok && T > 0) ok = issue_pv(T - 1);
+      if (ok && Tl > 0) ok = issue_pv(Tl - 1);
       if (!ok) *abort_flag = 1;
     }
   } else {
@@ -195,8 +209,8 @@ __global__ void __launch_bounds__(192, 2) attn_mha_tc_kernel(const __grid_consta
 #pragma unroll
     for (int d = 0; d < MHD; ++d) o[d] = 0.f;
     bool ok = true;
-    for (int t = 0; t < T; ++t) {
-      const int j0 = t * MK;
+    for (int t = 0; t < Tl; ++t) {
+      const int j0 = (t0 + t) * MK;
       if (!warp_wait(s_full, t & 1)) { ok = false; break; }
       tc_fence_after();
       float sc[MK];
@@ -223,7 +237,7 @@ __global__ void __launch_bounds__(192, 2) attn_mha_tc_kernel(const __grid_consta
           mx = fmaxf(mx, sc[c]);
         }
       }
-      const float m_new = fmaxf(m_run, mx);   // finite: key j0 < S
+      const float m_new = fmaxf(m_run, mx);   // finite: key j0 < S (every local tile starts inside S)
       const float alpha = ex2_approx(m_run - m_new);
       float ps = 0.f;
 #pragma unroll
@@ -261,9 +275,9 @@ __global__ void __launch_bounds__(192, 2) attn_mha_tc_kernel(const __grid_consta
         for (int k = 0; k < MHD; ++k) o[k] = (o[k] + __uint_as_float(v[k])) * alpha;
       }
     }
-    if (ok && T > 0) {
-      const int pb = (T - 1) & 1;
-      if (warp_wait(&pv_full[pb], ((T - 1) >> 1) & 1)) {
+    if (ok && Tl > 0) {
+      const int pb = (Tl - 1) & 1;
+      if (warp_wait(&pv_full[pb], ((Tl - 1) >> 1) & 1)) {
         tc_fence_after();
         uint32_t v[32];
         tmem_ld32(tmem + lane_base + (uint32_t)(64 + 64 * pb), v);
@@ -273,22 +287,98 @@ __global__ void __launch_bounds__(192, 2) attn_mha_tc_kernel(const __grid_consta
         ok = false;
       }
     }
-    if (!ok) {
-      *abort_flag = 1;
-    } else if (row_ok) {
-      const float inv = 1.f / l_run;
+    auto store_row = [&](const float* ov, float l) {
+      const float inv = 1.f / l;
       uint4* dst = reinterpret_cast<uint4*>(ctx + (int64_t)(sb + i) * E + h * MHD);   // 48 h bytes: 16-byte aligned
 #pragma unroll
       for (int c = 0; c < MHD / 8; ++c) {
         uint32_t w4[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          __nv_bfloat162 ho = __floats2bfloat162_rn(o[8 * c + 2 * k] * inv, o[8 * c + 2 * k + 1] * inv);
+          __nv_bfloat162 ho = __floats2bfloat162_rn(ov[8 * c + 2 * k] * inv, ov[8 * c + 2 * k + 1] * inv);
           w4[k] = *reinterpret_cast<uint32_t*>(&ho);
         }
         dst[c] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
       }
+    };
+    if (!ok) {
+      *abort_flag = 1;
+    } else if (ks == 1) {
+      if (row_ok) store_row(o, l_run);
+    } else {
+      // Key split: (O, m, l) of this CTA's key range into row r's slot of
+      // the P buffers.  The tensor cores are done reading P: this warp saw
+      // the last P.V product complete, and every softmax warp wrote its P
+      // rows before that product was issued.  A CTA with no key tiles
+      // leaves m = -inf, l = 0 (weight 0 in the merge).
+      float* mine = reinterpret_cast<float*>(sP) + r * L::PSTR;
+#pragma unroll
+      for (int d = 0; d < MHD; d += 4)
+        *reinterpret_cast<float4*>(mine + d) = make_float4(o[d], o[d + 1], o[d + 2], o[d + 3]);
+      mine[MHD] = m_run;
+      mine[MHD + 1] = l_run;
     }
+  }
+  if (ks > 1) {
+    // every thread of every CTA of the cluster meets here (also after a failed wait)
+    __syncthreads();
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+    uint32_t crank;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(crank));
+    if (crank == 0 && warp >= 2 && !*abort_flag) {
+      const int q = warp & 3, r = 32 * q + lane, i = i0 + r;
+      const uint32_t row_addr = su32(reinterpret_cast<float*>(sP) + r * L::PSTR);
+      float mz[4], lz[4];
+#pragma unroll
+      for (int zz = 0; zz < 4; ++zz) {
+        mz[zz] = -INFINITY;
+        lz[zz] = 0.f;
+        if (zz < ks) {
+          uint32_t a;
+          asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(row_addr + 4u * MHD), "r"((uint32_t)zz));
+          asm volatile("ld.shared::cluster.v2.f32 {%0, %1}, [%2];" : "=f"(mz[zz]), "=f"(lz[zz]) : "r"(a) : "memory");
+        }
+      }
+      const float m = fmaxf(fmaxf(mz[0], mz[1]), fmaxf(mz[2], mz[3]));   // finite: some rank has a key tile
+      float acc[MHD], l = 0.f;
+#pragma unroll
+      for (int d = 0; d < MHD; ++d) acc[d] = 0.f;
+#pragma unroll
+      for (int zz = 0; zz < 4; ++zz) {
+        if (zz >= ks) break;
+        const float wz = ex2_approx(mz[zz] - m);   // an empty key range has m = -inf: weight 0
+        l += wz * lz[zz];
+#pragma unroll
+        for (int d = 0; d < MHD; d += 4) {
+          uint32_t a;
+          asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(row_addr + 4u * d), "r"((uint32_t)zz));
+          float4 v4;
+          asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                       : "=f"(v4.x), "=f"(v4.y), "=f"(v4.z), "=f"(v4.w)
+                       : "r"(a)
+                       : "memory");
+          acc[d] += wz * v4.x; acc[d + 1] += wz * v4.y; acc[d + 2] += wz * v4.z; acc[d + 3] += wz * v4.w;
+        }
+      }
+      if (i < S) {
+        const float inv = 1.f / l;
+        uint4* dst = reinterpret_cast<uint4*>(ctx + (int64_t)(sb + i) * E + h * MHD);
+#pragma unroll
+        for (int c = 0; c < MHD / 8; ++c) {
+          uint32_t w4[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            __nv_bfloat162 ho = __floats2bfloat162_rn(acc[8 * c + 2 * k] * inv, acc[8 * c + 2 * k + 1] * inv);
+            w4[k] = *reinterpret_cast<uint32_t*>(&ho);
+          }
+          dst[c] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        }
+      }
+    }
+    // no CTA leaves while rank 0 may still read its shared memory
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
   }
   tc_fence_before();
   __syncthreads();
@@ -299,19 +389,75 @@ __global__ void __launch_bounds__(192, 2) attn_mha_tc_kernel(const __grid_consta
   if (threadIdx.x == 0 && *abort_flag) set_err(err, ERR_TIMEOUT);
 }
 
-cudaError_t launch_mha_tc(const bf16* qkv, bf16* ctx, const SeqTable* seq, int n_tiles2, int M, int* err,
-                          cudaStream_t st) {
+namespace {
+int g_mha_sms = 148;
+int g_mha_clusters[3] = {1, 0, 0};   // co-resident clusters of 1, 2, 4 CTAs (0: that split is off)
+}
+
+cudaError_t launch_mha_tc(const bf16* qkv, bf16* ctx, const SeqTable* seq, int n_tiles2, int M, int max_len,
+                          int* err, cudaStream_t st) {
   if (M <= 0 || n_tiles2 <= 0) return cudaSuccess;
   constexpr int E = 192;
   CUtensorMap t_qkv;
   cudaError_t r = make_bf16_map_sw128(&t_qkv, qkv, M, 3 * E, 3 * E, MK);
   if (r != cudaSuccess) return r;
-  CK_LAUNCH(launch_k(attn_mha_tc_kernel, dim3(n_tiles2, 8), dim3(192), MhaTc::SMEM, st, t_qkv, qkv, E, ctx, seq, err));
+  // fewer (query tile, head) units than the two CTAs per SM hold: split
+  // each unit's keys over a cluster of 2 or 4 CTAs (no more splits than key
+  // tiles of the longest sequence)
+  const int units = n_tiles2 * 8;
+  int ks = 1;
+  if (units < 2 * g_mha_sms) {
+    const int want = 2 * g_mha_sms / units, tmax = (max_len + MK - 1) / MK;
+    if (want >= 4 && tmax >= 4 && g_mha_clusters[2] > 0) ks = 4;
+    else if (want >= 2 && tmax >= 2 && g_mha_clusters[1] > 0) ks = 2;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(n_tiles2, 8, ks);
+  cfg.blockDim = dim3(192);
+  cfg.dynamicSmemBytes = MhaTc::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  attr[na].id = cudaLaunchAttributeClusterDimension;
+  attr[na].val.clusterDim.x = 1;
+  attr[na].val.clusterDim.y = 1;
+  attr[na].val.clusterDim.z = ks;
+  ++na;
+  if (g_launch_pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  CK_LAUNCH(cudaLaunchKernelEx(&cfg, attn_mha_tc_kernel, t_qkv, (const bf16*)qkv, E, ctx, seq, err, ks));
   return cudaGetLastError();
 }
 
 cudaError_t attention_mha_tc_init_attributes() {
-  return cudaFuncSetAttribute(attn_mha_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, MhaTc::SMEM);
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
+      n > 0)
+    g_mha_sms = n;
+  cudaError_t r = cudaFuncSetAttribute(attn_mha_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, MhaTc::SMEM);
+  if (r != cudaSuccess) return r;
+  for (int j = 1; j < 3; ++j) {   // can clusters of 2 and 4 CTAs be scheduled at all?
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1, 1, 1 << j);
+    cfg.blockDim = dim3(192);
+    cfg.dynamicSmemBytes = MhaTc::SMEM;
+    cudaLaunchAttribute a;
+    a.id = cudaLaunchAttributeClusterDimension;
+    a.val.clusterDim.x = 1;
+    a.val.clusterDim.y = 1;
+    a.val.clusterDim.z = 1 << j;
+    cfg.attrs = &a;
+    cfg.numAttrs = 1;
+    int n_cl = 0;
+    g_mha_clusters[j] = cudaOccupancyMaxActiveClusters(&n_cl, attn_mha_tc_kernel, &cfg) == cudaSuccess ? n_cl : 0;
+    cudaGetLastError();
+  }
+  return cudaSuccess;
 }
 
 }  // namespace sf

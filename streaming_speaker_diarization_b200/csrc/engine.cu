@@ -168,8 +168,8 @@ struct sf_engine {
                           // 3 = never; 0 = mma.sync
   int pair_bn = 0;        // CTA-pair tile width (0 = planned)
   int attn_path = 1;      // bf16 relative-position attention: 1 = tcgen05, 0 = mma.sync
-  int mel_path = 0;       // front-end: 0 = shared-memory FFT, 1 = register FFT + all-SM normalisation
-  int sub_path = 0;       // subsampling: 0 = conv1 and depthwise kernels, 1 = conv1 fused into the first depthwise
+  int mel_path = MEL_DEFAULT_PATH;   // front-end: 1 = register FFT + all-SM normalisation, 0 = shared-memory FFT
+  int sub_path = 1;       // subsampling: 1 = conv1 fused into the first depthwise, 0 = conv1 and depthwise kernels
   float* d_split_ws = nullptr;   // split-K partial tiles of the tcgen05 GEMM
   int* d_split_cnt = nullptr;    // their per-tile arrival counters (kept at zero between launches)
   TcScratch tc_scratch() const { return TcScratch{d_err, d_split_ws, SPLIT_WS_BYTES, d_split_cnt, SPLIT_CNT}; }
@@ -587,11 +587,10 @@ cudaError_t gemm_dispatch<bf16>(sf_engine* e, const bf16* A, int lda, const bf16
   return gemm_bf16_mma(A, lda, W, M, N, K, ep, st);
 }
 
-// Transformer MHSA in the bf16 engine: the tcgen05 kernel when its 128-row
-// (tile, head) units fill the SMs (streaming batches: measured 2-3 % faster
-// steps), the mma.sync kernel otherwise (one long clip: its 64-row CTAs
-// cover twice as many SMs; 0.34 vs 0.40 ms per 90 s forward); always
-// mma.sync with SF_OPT_ATTN_PATH = 0.
+// Transformer MHSA in the bf16 engine: the tcgen05 kernel (SF_OPT_ATTN_PATH
+// 1, the default), which splits each (query tile, head) unit's keys over a
+// CTA cluster when the units alone leave SMs idle (one long clip); the
+// mma.sync kernels with two (path 0) or four (path 2) key groups per CTA.
 template <typename T>
 cudaError_t mha_attention(sf_engine* e, const T* qkv, T* ctx, const SeqTable* seq, int n_tiles, int M, cudaStream_t st) {
   return launch_mha<T>(qkv, ctx, seq, n_tiles, M, e->R, st);
@@ -599,8 +598,7 @@ cudaError_t mha_attention(sf_engine* e, const T* qkv, T* ctx, const SeqTable* se
 template <>
 cudaError_t mha_attention<bf16>(sf_engine* e, const bf16* qkv, bf16* ctx, const SeqTable* seq, int n_tiles, int M,
                                 cudaStream_t st) {
-  if (e->attn_path >= 1 && e->att_tiles2 * 8 >= e->n_sms)
-    return launch_mha_tc(qkv, ctx, seq, e->att_tiles2, M, e->d_err, st);
+  if (e->attn_path == 1) return launch_mha_tc(qkv, ctx, seq, e->att_tiles2, M, e->att_max_len, e->d_err, st);
   if (e->attn_path == 2) return launch_mha_bf16_4g(qkv, ctx, seq, n_tiles, M, st);
   return launch_mha<bf16>(qkv, ctx, seq, n_tiles, M, e->R, st);
 }
@@ -1376,7 +1374,8 @@ sf_status sf_attention_mha(sf_engine* e, const void* d_qkv, const int* h_seq_len
   const bf16* qkv = static_cast<const bf16*>(d_qkv);
   bf16* ctx = static_cast<bf16*>(d_ctx);
   if (ce == cudaSuccess)
-    ce = path == 1   ? launch_mha_tc(qkv, ctx, &e->d_desc->seq, tiles2, M, e->d_err, st)
+    ce = path == 1   ? launch_mha_tc(qkv, ctx, &e->d_desc->seq, tiles2, M, *std::max_element(lens.begin(), lens.end()),
+                                     e->d_err, st)
          : path == 2 ? launch_mha_bf16_4g(qkv, ctx, &e->d_desc->seq, tiles, M, st)
                      : launch_mha<bf16>(qkv, ctx, &e->d_desc->seq, tiles, M, e->max_seq_len, st);
   if (ce != cudaSuccess) return cuda_fail(e, ce, "sf_attention_mha");
@@ -1718,20 +1717,27 @@ sf_status sf_stream_destroy(sf_stream* s) {
 
 sf_status sf_stream_reset(sf_stream* s, const int* ids, int n) {
   if (!s) return SF_EINVAL;
+  if (ids && n < 0) return fail(s->e, SF_EINVAL, "negative id count");
   std::vector<int> list;
   if (ids) list.assign(ids, ids + n);
   else for (int i = 0; i < s->n; ++i) list.push_back(i);
   for (int id : list)
     if (id < 0 || id >= s->n) return fail(s->e, SF_EINVAL, "stream id out of range");
+  // A step still running on any caller stream reads and writes the silence
+  // statistics: wait for it, clear them, and wait for the clear, so that the
+  // next step (on any stream) starts from the cleared state.
+  if (cudaDeviceSynchronize() != cudaSuccess) return fail(s->e, SF_ECUDA, "reset: device");
   for (int id : list) {
     s->n_c[id] = s->n_f[id] = 0;
     s->cur_c[id] = s->cur_f[id] = 0;
     s->finished[id] = 0;
     s->c0[id] = 0;
     // the silence mean restarts from zero; cache/FIFO contents are dead once sizes are 0
-    cudaMemset(s->sb.sil_mean + (size_t)id * s->sb.D, 0, (size_t)s->sb.D * 4);
-    cudaMemset(s->sb.sil_count + id, 0, sizeof(int));
+    if (cudaMemset(s->sb.sil_mean + (size_t)id * s->sb.D, 0, (size_t)s->sb.D * 4) != cudaSuccess ||
+        cudaMemset(s->sb.sil_count + id, 0, sizeof(int)) != cudaSuccess)
+      return fail(s->e, SF_ECUDA, "reset: clear");
   }
+  if (cudaDeviceSynchronize() != cudaSuccess) return fail(s->e, SF_ECUDA, "reset: device");
   return SF_OK;
 }
 

@@ -499,13 +499,11 @@ namespace {
 // (mean, 1 / (std + eps)) the B * 128 * 2 floats after them.
 cudaError_t enqueue_mel(const float* audio, int B, int64_t n_buf, const MelArgs& args, const MelTables* tab,
                         float* mel, float* part, int T_cols, int path, cudaStream_t st) {
+  // The >48 KB dynamic shared-memory attribute of the frame kernels is a
+  // per-device setting made by frontend_init_attributes() with the device
+  // current: by sf_create for an engine's device, and by sf_mel_noalloc's
+  // one-time set-up for each device it runs on.
   const int n_blk = (T_cols + MEL_FB - 1) / MEL_FB;
-  static bool attr_set = false;   // first use outside an engine (sf_mel_noalloc)
-  if (!attr_set) {
-    cudaError_t e = frontend_init_attributes();
-    if (e != cudaSuccess) return e;
-  }
-  attr_set = true;
   if (path == 1) {
     float* stats = part + (size_t)B * n_blk * 128 * 4;
     CK_LAUNCH(launch_k(mel_frames_reg_kernel, dim3(dim3(n_blk, B)), dim3(256), MEL_REG_SMEM, st, audio, n_buf, args,

@@ -14,7 +14,10 @@
 // budget: a wait that runs out sets ERR_TIMEOUT in the engine's error word,
 // raises a CTA-wide abort flag, the producer waits (bounded) for its own
 // loads in flight, and TMEM is released before the CTA exits.
-// No cluster multicast is used anywhere.
+// No TMA or bulk load uses cluster multicast: every CTA loads its own
+// operand tiles.  The CTA-pair kernel's tcgen05.commit carries the
+// .multicast::cluster qualifier only to signal the "stage free" mbarriers
+// of both CTAs of the pair on this GPU.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 

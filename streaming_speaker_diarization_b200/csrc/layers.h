@@ -150,10 +150,12 @@ cudaError_t launch_relpos_attention_tc(const bf16* qkv, const bf16* ptab, int R,
                                        const TcScratch& sc, cudaStream_t st);
 cudaError_t attention_tc_init_attributes();
 // bf16 Transformer MHSA (d 192, 8 heads of 24) on tcgen05: one CTA per 128
-// query rows x head (n_tiles2 = 128-row tiles); err gets ERR_TIMEOUT if a
-// bounded wait gives up.
-cudaError_t launch_mha_tc(const bf16* qkv, bf16* ctx, const SeqTable* seq, int n_tiles2, int M, int* err,
-                          cudaStream_t st);
+// query rows x head x key split (n_tiles2 = 128-row tiles, max_len the
+// longest sequence); with fewer units than two per SM each unit's keys are
+// split over a cluster of 2 or 4 CTAs merged in shared memory; err gets
+// ERR_TIMEOUT if a bounded wait gives up.
+cudaError_t launch_mha_tc(const bf16* qkv, bf16* ctx, const SeqTable* seq, int n_tiles2, int M, int max_len,
+                          int* err, cudaStream_t st);
 cudaError_t attention_mha_tc_init_attributes();
 
 }  // namespace sf

@@ -37,7 +37,10 @@ constexpr int NOALLOC_MAX_CLIPS = 64;
 // of 120 s (376 tiles each) or one clip of 21.8 minutes.
 constexpr int NOALLOC_MAX_TILES = 4096;
 constexpr int LEN_FLOATS = NOALLOC_MAX_CLIPS * 2;                 // int64 lengths stored first
-constexpr size_t SCRATCH_FLOATS = LEN_FLOATS + (size_t)NOALLOC_MAX_TILES * 128 * 4;   // 8.0 MiB
+// per-tile partial statistics (4 floats per tile and bin), then the per-clip
+// (mean, 1 / (std + eps)) of each bin that front-end path 1 writes after them
+constexpr size_t PART_FLOATS = (size_t)NOALLOC_MAX_TILES * 128 * 4 + (size_t)NOALLOC_MAX_CLIPS * 128 * 2;
+constexpr size_t SCRATCH_FLOATS = LEN_FLOATS + PART_FLOATS;         // 8.06 MiB
 
 static __device__ __align__(256) float g_mel_scratch[SCRATCH_FLOATS];
 static __device__ __align__(256) sf::MelTables g_mel_noalloc_tables;
@@ -64,6 +67,8 @@ sf_status setup_device(int dev, DeviceSlot** out) {
     sf::MelTables host;
     sf::build_mel_tables(&host);
     if (cudaMemcpyToSymbol(g_mel_noalloc_tables, &host, sizeof(host)) != cudaSuccess) return SF_ECUDA;
+    // per-device: the frame kernels need more than 48 KB of dynamic shared memory
+    if (sf::frontend_init_attributes() != cudaSuccess) return SF_ECUDA;
     s.ready = true;
   }
   *out = &s;
@@ -78,6 +83,7 @@ extern "C" SF_API sf_status sf_mel_noalloc(const float* d_audio, const int64_t* 
   if (B < 1 || B > NOALLOC_MAX_CLIPS || n_max < 1600) return SF_ESHAPE;
   const int64_t tiles_per_clip = (1 + n_max / 160 + 31) / 32;
   if (tiles_per_clip * B > NOALLOC_MAX_TILES) return SF_ESHAPE;
+  if (sf::mel_part_floats(B, n_max) > PART_FLOATS) return SF_ESHAPE;
   for (int b = 0; b < B; ++b)
     if (h_len[b] < 1600 || h_len[b] > n_max) return SF_EINVAL;
   int dev = 0;
@@ -92,7 +98,9 @@ extern "C" SF_API sf_status sf_mel_noalloc(const float* d_audio, const int64_t* 
   if (cudaMemcpyAsync(d_len, h_len, (size_t)B * sizeof(int64_t), cudaMemcpyHostToDevice, st) != cudaSuccess)
     return SF_ECUDA;
   sf::MelArgs args{d_len};
-  if (sf::launch_mel(d_audio, B, n_max, args, slot->tables, d_mel, d_part, st) != cudaSuccess) return SF_ECUDA;
+  // the engine's default front-end path, so the result equals sf_mel's to the bit
+  if (sf::launch_mel(d_audio, B, n_max, args, slot->tables, d_mel, d_part, st, sf::MEL_DEFAULT_PATH) != cudaSuccess)
+    return SF_ECUDA;
   if (h_mel_len)
     for (int b = 0; b < B; ++b) h_mel_len[b] = h_len[b] / 160;
   return SF_OK;

@@ -41,3 +41,41 @@ def test_peaks_are_positive():
 def test_reference_arm_other_ranks_do_no_work():
     args = argparse.Namespace(gpus=2, steps=1, warmup=3, impl="reference")
     assert bench.run_reference(args, 1, 2) == 0
+
+
+def test_in_process_clock_summary():
+    s = bench.summarize_samples([(1965, 1965, 0), (1900, 1965, 0x4), (1800, 1965, 0x4 | 0x8)])
+    assert s["sm_mhz"] == 1900.0 and s["sm_max_mhz"] == 1965.0 and s["samples"] == 3
+    assert s["reasons"] == ["hw_slowdown", "sw_power_cap"]
+    assert bench.summarize_samples([])["sm_mhz"] is None
+
+
+def test_stream_plan_matches_the_oracle_bookkeeping():
+    """The host-side size plan used for the streaming roofline must follow
+    the oracle's FIFO/cache rules (data-independent sizes)."""
+    import numpy as np
+    import oracle as O
+    from synth import make_weights, TINY, synth_clip
+    pre = O.PRESETS["low"]
+    w = make_weights(TINY, seed=0)
+    a, _ = synth_clip(7, 12.0, 2)
+    f, L = O.mel_features(a[None], np.array([len(a)]))
+    L = int(L[0])
+    total = 1 + (L - 1) // 8
+    plan = bench.stream_plan((pre.chunk_len, pre.right_context, pre.fifo_len, pre.update_period, pre.spkcache_len),
+                             total)
+    st, taps = O.StreamState(), []
+    while st.c0 < total:
+        O.stream_step(st, f[0], L, w, pre, taps=taps)
+    assert len(plan) == len(taps)
+    for (S, new), t in zip(plan, taps):
+        assert S == len(t["P"]) and new == len(t["new"])
+
+
+def test_stream_plan_low_preset_sizes():
+    plan = bench.stream_plan((6, 7, 188, 144, 188), 750)
+    assert len(plan) == 125
+    assert plan[31] == (199, 13) and plan[56] == (249, 13) and plan[-1] == (362, 6)
+    assert bench.stream_plan((340, 40, 40, 300, 188), 7500)[1] == (608, 380)
+    # one full-size offline clip: 1125 encoder frames, ~351 GFLOP
+    assert abs(bench.model_flops(1125, 1125) / 1e9 - 350.7) < 0.1

@@ -84,3 +84,21 @@ def test_mha_streaming_batch(eng):
     for s in (0, 40, 63):
         assert np.max(np.abs(got[322 * s:322 * (s + 1)] - ref[s])) <= 1.5e-2, s
     assert np.max(np.abs(got - _run(eng, qkv, lens, 0))) <= 2e-2
+
+
+@pytest.mark.parametrize("lens", [[1125], [1, 65, 700, 3], [129, 1500]])
+def test_mha_key_split(eng, lens):
+    """Few (query tile, head) units: the tcgen05 kernel splits each unit's
+    keys over a cluster of CTAs (4 for one 1125-frame clip) and merges them;
+    sequences shorter than the split leave some CTAs without key tiles.
+    Against float64, bitwise repeatable, and close to the mma.sync kernel."""
+    qkv = _inputs(5, lens)
+    got = _run(eng, qkv, lens, 1)
+    assert np.isfinite(got).all()
+    ref = _reference(qkv, lens, range(len(lens)))
+    offs = np.concatenate([[0], np.cumsum(lens)])
+    for s in range(len(lens)):
+        err = np.max(np.abs(got[offs[s]:offs[s + 1]] - ref[s]))
+        assert err <= 1.5e-2, (lens[s], err)
+    assert np.array_equal(got, _run(eng, qkv, lens, 1))
+    assert np.max(np.abs(got - _run(eng, qkv, lens, 0))) <= 2e-2

@@ -1,14 +1,11 @@
-"""GPU parity of the second front-end implementation (SF_OPT_MEL_PATH = 1:
-FFT in registers with warp shuffles, separate statistics and normalisation
-passes) against the oracle, on the cases the default path is tested on:
-clip, ragged batch, minimum length, silence and a pure tone, the offline
-forward, the audio-in streaming step (window mode) and one hour in one call.
-Log-mel features within 1e-3, probabilities within 1e-4 (fp32 engine).
-
-These run only with SF_TEST_NEW_PATHS=1 in the environment: the default
-engine keeps path 0 until this path has been measured."""
-import os
-
+"""GPU parity of the alternative front-end implementation (SF_OPT_MEL_PATH
+= 0: radix-2 FFT through shared memory, one normalisation CTA per (clip,
+bin)) against the oracle, on the cases the default path (1: FFT in
+registers with warp shuffles, separate statistics and normalisation passes
+over all SMs) is tested on elsewhere: clip, ragged batch, minimum length,
+silence and a pure tone, the offline forward, the audio-in streaming step
+(window mode) and one hour in one call.  Log-mel features within 1e-3,
+probabilities within 1e-4 (fp32 engine)."""
 import numpy as np
 import pytest
 
@@ -17,9 +14,8 @@ from oracle.streaming import stream_run_audio
 from synth import clip_for_config, synth_batch, synth_clip
 from _helpers import make_engine, tiny_weights, to_dev
 
-pytestmark = [pytest.mark.gpu,
-              pytest.mark.skipif(os.environ.get("SF_TEST_NEW_PATHS") != "1",
-                                 reason="kernel paths not yet default run with SF_TEST_NEW_PATHS=1")]
+pytestmark = pytest.mark.gpu
+ALT_PATH = 0
 torch = pytest.importorskip("torch")
 if not torch.cuda.is_available():
     pytest.skip("no CUDA device", allow_module_level=True)
@@ -28,7 +24,7 @@ from streaming_speaker_diarization_b200 import binding as b  # noqa: E402
 
 def _engine(w, **kw):
     e = make_engine(w, 0, 2, 2, **kw)
-    b.sf_set_option(e, b.SF_OPT_MEL_PATH, 1)
+    b.sf_set_option(e, b.SF_OPT_MEL_PATH, ALT_PATH)
     return e
 
 
@@ -48,7 +44,7 @@ def gpu_mel(e, audio, lens):
 
 
 @pytest.mark.parametrize("case", ["cfg0", "ragged", "short", "silence_tone"])
-def test_mel_path1_parity(eng, case):
+def test_mel_alt_path_parity(eng, case):
     if case == "cfg0":
         audio, lens, _ = clip_for_config(0)
     elif case == "ragged":
@@ -70,7 +66,7 @@ def test_mel_path1_parity(eng, case):
         assert np.all(got[i, :, l:] == 0)
 
 
-def test_offline_forward_path1(eng):
+def test_offline_forward_alt_path(eng):
     w = tiny_weights(xavier=True)
     audio, lens, _ = synth_batch(83, [6.0, 2.2])
     Tp = int(O.encoder_frames(audio.shape[1] // 160))
@@ -81,7 +77,7 @@ def test_offline_forward_path1(eng):
     assert np.max(np.abs(probs.cpu().numpy() - ref)) <= 1e-4
 
 
-def test_audio_in_stream_path1(eng):
+def test_audio_in_stream_alt_path(eng):
     w = tiny_weights(xavier=True)
     pre = O.PRESETS["low"]
     clip = synth_clip([60, 0], 9.0, 3)[0]
@@ -111,12 +107,12 @@ def test_audio_in_stream_path1(eng):
     assert np.max(np.abs(got - ref)) <= 1e-4
 
 
-def test_mel_path1_one_hour():
+def test_mel_alt_path_one_hour():
     from synth.audio import hour_of_audio
     x = hour_of_audio()
     n = len(x)
     e = make_engine(tiny_weights(), 1, 2, 2, max_batch=1, max_samples=n)
-    b.sf_set_option(e, b.SF_OPT_MEL_PATH, 1)
+    b.sf_set_option(e, b.SF_OPT_MEL_PATH, ALT_PATH)
     try:
         got, ml = gpu_mel(e, x[None], np.array([n]))
     finally:

@@ -1,17 +1,31 @@
 """GPU parity at full size, in the launch configurations bench.py times.
 
-Full model (17 FastConformer + 18 Transformer layers), bf16, seeded N(0, 0.02)
-weights.  Streaming workloads run with all their streams batched exactly as
-in the benchmark; sampled streams are compared with the oracle run on that
-stream alone (probabilities within 2e-2).  Only steps before the first FIFO
-pop / cache compression are compared free-running: until then no step takes
-a threshold decision, so the two runs see identical state structure."""
+Full model (17 FastConformer + 18 Transformer layers), bf16, with two weight
+sets:
+
+* xavier-scaled weights (each matrix / sqrt(fan_in)): activations stay O(1)
+  through the stack and the oracle's probabilities spread over roughly
+  [0.2, 0.8], so the 2e-2 bound can fail.  These are the parity tests.
+  Each asserts that the oracle probabilities it compares against spread by
+  more than four times the bound, so that a constant output fails it.
+* the benchmark's N(0, 0.02) weights: probabilities sit within ~0.015 of
+  0.5, where a 2e-2 bound says little.  These runs check shapes, state sizes,
+  zero padding and finiteness only.
+
+Streaming workloads run with all their streams batched exactly as in the
+benchmark.  Sampled streams are teacher-forced: before a compared step the
+oracle's state for that stream (cache, FIFO, silence mean, next frame) is
+injected with sf_stream_set_state, so bf16 rounding cannot flip one of the
+FIFO/cache decisions, and that step's chunk probabilities must be within
+2e-2 of the oracle's, the stream's new FIFO/cache sizes must equal the
+oracle's, and the FIFO embeddings it pushed must be within relative L2 3e-2
+of the oracle's pre-encode embeddings."""
 import numpy as np
 import pytest
 
 import oracle as O
 from synth import clip_for_config
-from _helpers import full_weights, make_engine, to_dev
+from _helpers import full_weights, get_state, make_engine, oracle_states, set_state, to_dev
 
 pytestmark = pytest.mark.gpu
 torch = pytest.importorskip("torch")
@@ -19,85 +33,125 @@ if not torch.cuda.is_available():
     pytest.skip("no CUDA device", allow_module_level=True)
 from streaming_speaker_diarization_b200 import binding as b  # noqa: E402
 
+TOL = 2e-2          # bf16 probabilities
+EMB_TOL = 3e-2      # bf16 embeddings, relative L2
+
+
+def rel_l2(a, ref):
+    return float(np.linalg.norm(np.asarray(a, np.float64) - ref) / max(np.linalg.norm(ref), 1e-30))
+
+
+def spread_guard(ref):
+    """A constant output must fail the comparison against `ref`."""
+    assert float(ref.max() - ref.min()) > 4 * TOL, (float(ref.min()), float(ref.max()))
+
 
 @pytest.fixture(scope="module")
-def weights():
+def weights_x():
+    return full_weights(xavier=True)
+
+
+@pytest.fixture(scope="module")
+def weights_std():
     return full_weights()
 
 
-def _run_steps(eng, preset, audio, lens, n_steps):
+def _gpu_mel(eng, audio, lens):
     n = audio.shape[0]
-    T = 1 + audio.shape[1] // 160
-    mel = torch.empty((n, 128, T), device="cuda")
+    mel = torch.empty((n, 128, 1 + audio.shape[1] // 160), device="cuda")
     ml = b.sf_mel(eng, to_dev(audio), lens, mel)
-    st = b.sf_stream_create(eng, preset, n)
-    cp = torch.zeros((n, preset[0], 4), device="cuda")
-    outs = [[] for _ in range(n)]
+    return mel, ml
+
+
+def _teacher_forced(eng, pre, audio, lens, w, compare, n_steps):
+    """Run every stream of the batch for n_steps steps; for stream i and each
+    step k in compare[i], inject the oracle's state before step k and compare
+    the step's outputs with the oracle's.  Returns the number of compared
+    (stream, step) pairs and, per stream, the oracle chunk probabilities."""
+    n = audio.shape[0]
+    mel, ml = _gpu_mel(eng, audio, lens)
+    ref = {}
+    for i, steps in compare.items():
+        f, L = O.mel_features(audio[i:i + 1, :lens[i]], lens[i:i + 1])
+        ref[i] = oracle_states(w, f[0], int(L[0]), pre, max(steps) + 1)
+    tup = (pre.chunk_len, pre.right_context, pre.fifo_len, pre.update_period, pre.spkcache_len)
+    st = b.sf_stream_create(eng, tup, n)
+    cp = torch.zeros((n, pre.chunk_len, 4), device="cuda")
+    done, seen = 0, {i: [] for i in compare}
     try:
-        for _ in range(n_steps):
+        for k in range(n_steps):
+            for i, steps in compare.items():
+                if k in steps:
+                    set_state(eng, st, i, ref[i][0][k], 1)
             n_out = b.sf_stream_step(eng, st, mel, np.zeros(n, np.int64), ml, cp)
-            c = cp.cpu().numpy()
-            for i in range(n):
-                outs[i].append(c[i, :n_out[i]])
+            got = cp.cpu().numpy()
+            for i, steps in compare.items():
+                if k not in steps:
+                    continue
+                states, taps = ref[i]
+                t = taps[k]
+                exp = t["P"][t["n_c"] + t["n_f"]:][:t["n_chunk"]]
+                assert n_out[i] == len(exp), (i, k)
+                err = float(np.max(np.abs(got[i, :n_out[i]] - exp)))
+                assert err <= TOL, (i, k, err)
+                seen[i].append(exp)
+                g = get_state(eng, st, i, 1, pre.spkcache_len, pre.fifo_len + pre.chunk_len)
+                nxt = states[k + 1]
+                assert (g["n_c"], g["n_f"], g["c0"]) == (len(nxt.cache_emb), len(nxt.fifo_emb), nxt.c0), (i, k)
+                m = min(len(exp), g["n_f"])          # the chunk frames pushed this step (still in the FIFO)
+                if m:
+                    e = rel_l2(g["fifo_emb"][g["n_f"] - m:], nxt.fifo_emb[len(nxt.fifo_emb) - m:])
+                    assert e <= EMB_TOL, (i, k, e)
+                done += 1
         b.sf_check(eng)
-        sizes = []
-        for i in (0, n - 1):
-            v = b.sf_state_view()
-            b.sf_stream_get_state(eng, st, i, v)
-            sizes.append((v.n_cache, v.n_fifo, v.next_frame))
     finally:
         b.sf_stream_destroy(st)
-    return [np.concatenate(o) for o in outs], ml, sizes
+    return done, {i: np.concatenate(v) for i, v in seen.items()}
 
 
-def test_low_preset_64_streams_first_12_steps(weights):
-    """Low preset, 64 streams x 60 s (the benchmark's streaming workload)."""
+def test_low_preset_64_streams_teacher_forced(weights_x):
+    """Low preset, 64 streams x 60 s (the benchmark's streaming workload),
+    steady-state steps included: stream 0 through its first FIFO pop (step
+    31), the first cache compression (step 55) and the steps after it;
+    stream 63 early."""
     pre = O.PRESETS["low"]
     audio, lens, _ = clip_for_config(2)
-    eng = make_engine(weights, 1, 17, 18, max_batch=64)
+    eng = make_engine(weights_x, 1, 17, 18, max_batch=64)
     try:
-        got, ml, sizes = _run_steps(eng, (6, 7, 188, 144, 188), audio, lens, 12)
+        compare = {0: [0, 11, 30, 31, 32, 44, 54, 55, 56, 57], 63: [0, 6, 11]}
+        done, seen = _teacher_forced(eng, pre, audio, lens, weights_x, compare, 58)
     finally:
         b.sf_destroy(eng)
-    assert sizes[0] == (0, 72, 72) and sizes[1] == (0, 72, 72)
-    for i in (0, 17, 63):
-        f, L = O.mel_features(audio[i:i + 1, :lens[i]], lens[i:i + 1])
-        st = O.StreamState()
-        ref = np.concatenate([O.stream_step(st, f[0], int(L[0]), weights, pre) for _ in range(12)])
-        assert got[i].shape == ref.shape == (72, 4)
-        err = np.max(np.abs(got[i] - ref))
-        assert err <= 2e-2, (i, err)
+    assert done == 13
+    for i in compare:
+        spread_guard(seen[i])
 
 
-def test_very_high_preset_16_streams_first_step(weights):
-    """Very high preset, 16 streams x 600 s: the first step (S = 380 frames,
-    chunk 340 emitted) of sampled streams, then the state sizes after a
-    second step (pop of 300 frames into a compressed 188-frame cache)."""
+def test_very_high_preset_16_streams_teacher_forced(weights_x):
+    """Very high preset, 16 streams x 600 s: S = 380 on the first step, then
+    a pop of 300 frames into a compressed 188-frame cache, then the
+    full-size step S = 188 + 40 + 380 = 608."""
     pre = O.PRESETS["very_high"]
     audio, lens, _ = clip_for_config(3)
-    eng = make_engine(weights, 1, 17, 18, max_batch=16, max_samples=int(audio.shape[1]))
+    eng = make_engine(weights_x, 1, 17, 18, max_batch=16, max_samples=int(audio.shape[1]))
     try:
-        got, ml, sizes = _run_steps(eng, (340, 40, 40, 300, 188), audio, lens, 2)
+        compare = {0: [0, 1, 2], 15: [1, 2]}
+        done, seen = _teacher_forced(eng, pre, audio, lens, weights_x, compare, 3)
     finally:
         b.sf_destroy(eng)
-    assert sizes[0] == sizes[1] == (188, 40, 680)   # step 2 popped 340 of 380 FIFO frames; cache compressed to 188
-    for i in (0, 15):
-        f, L = O.mel_features(audio[i:i + 1, :lens[i]], lens[i:i + 1])
-        st = O.StreamState()
-        ref = O.stream_step(st, f[0], int(L[0]), weights, pre)
-        assert ref.shape == (340, 4)
-        err = np.max(np.abs(got[i][:340] - ref))
-        assert err <= 2e-2, (i, err)
+    assert done == 5
+    for i in compare:
+        spread_guard(seen[i])
 
 
-def test_offline_batch_32_clips(weights):
+def test_offline_batch_32_clips(weights_x):
     """The variable-length batch: 32 clips of 5-120 s (seeded), padded to the
     longest, in one offline call of the full model (bf16).  Output lengths
     are 1 + (L - 1) // 8, padded rows are zero, and the shortest, a middle
     and the longest clip match the oracle run on that clip alone (2e-2)."""
     audio, lens, _ = clip_for_config(4)
     B, n_max = audio.shape
-    eng = make_engine(weights, 1, 17, 18, max_batch=32, max_samples=int(n_max))
+    eng = make_engine(weights_x, 1, 17, 18, max_batch=32, max_samples=int(n_max))
     try:
         Tp = int(O.encoder_frames(n_max // 160))
         probs = torch.full((B, Tp, 4), float("nan"), device="cuda")
@@ -113,7 +167,60 @@ def test_offline_batch_32_clips(weights):
         assert np.all(np.isfinite(got[i])) and got[i].min() >= 0 and got[i].max() <= 1, i
     order = np.argsort(lens)
     for i in (int(order[0]), int(order[B // 2]), int(order[-1])):
-        ref, tp = O.forward_offline(audio[i:i + 1, :lens[i]], lens[i:i + 1], weights)
+        ref, tp = O.forward_offline(audio[i:i + 1, :lens[i]], lens[i:i + 1], weights_x)
         assert tp[0] == T[i]
+        spread_guard(ref[0])
         err = np.max(np.abs(got[i, :T[i]] - ref[0]))
-        assert err <= 2e-2, (i, err)
+        assert err <= TOL, (i, err)
+
+
+# ---------------------------------------------------------------- shape checks
+# The benchmark's own N(0, 0.02) weights in the same launch shapes: sizes,
+# padding and finiteness (the probabilities sit at 0.5 +- 0.015 there).
+
+def test_low_preset_benchmark_weights_shapes(weights_std):
+    audio, lens, _ = clip_for_config(2)
+    n = audio.shape[0]
+    eng = make_engine(weights_std, 1, 17, 18, max_batch=64)
+    try:
+        mel, ml = _gpu_mel(eng, audio, lens)
+        st = b.sf_stream_create(eng, (6, 7, 188, 144, 188), n)
+        cp = torch.zeros((n, 6, 4), device="cuda")
+        try:
+            for k in range(57):
+                n_out = b.sf_stream_step(eng, st, mel, np.zeros(n, np.int64), ml, cp)
+                assert np.all(n_out == 6), k
+                c = cp.cpu().numpy()
+                assert np.all(np.isfinite(c)) and c.min() >= 0 and c.max() <= 1, k
+            b.sf_check(eng)
+            for i in (0, 63):
+                g = get_state(eng, st, i, 1, 188, 194)
+                # 57 steps x 6 frames: pop of 144 at step 31 and 55, compression at 55
+                assert (g["n_c"], g["n_f"], g["c0"]) == (188, 54, 342), (i, g["n_c"], g["n_f"], g["c0"])
+        finally:
+            b.sf_stream_destroy(st)
+    finally:
+        b.sf_destroy(eng)
+
+
+def test_very_high_benchmark_weights_shapes(weights_std):
+    audio, lens, _ = clip_for_config(3)
+    n = audio.shape[0]
+    eng = make_engine(weights_std, 1, 17, 18, max_batch=16, max_samples=int(audio.shape[1]))
+    try:
+        mel, ml = _gpu_mel(eng, audio, lens)
+        st = b.sf_stream_create(eng, (340, 40, 40, 300, 188), n)
+        cp = torch.zeros((n, 340, 4), device="cuda")
+        try:
+            for k in range(2):
+                n_out = b.sf_stream_step(eng, st, mel, np.zeros(n, np.int64), ml, cp)
+                assert np.all(n_out == 340), k
+                assert torch.isfinite(cp).all()
+            b.sf_check(eng)
+            for i in (0, 15):
+                g = get_state(eng, st, i, 1, 188, 380)
+                assert (g["n_c"], g["n_f"], g["c0"]) == (188, 40, 680)
+        finally:
+            b.sf_stream_destroy(st)
+    finally:
+        b.sf_destroy(eng)

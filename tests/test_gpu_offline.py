@@ -172,20 +172,29 @@ def test_offline_host_entry_matches_device_entry(eng_fp32_x):
 
 
 def test_offline_bf16_full_cfg1():
-    """Full model (17 + 18 layers) bf16 on the 90 s workload: probabilities
-    within 2e-2 of the fp64 oracle on all 1125 frames."""
-    w = full_weights()
-    eng = make_engine(w, 1, 17, 18, max_batch=1)
-    try:
-        audio, lens, _ = clip_for_config(1)
-        probs = torch.zeros((1, 1125, 4), device="cuda")
-        b.sf_forward_offline(eng, to_dev(audio), lens, probs)
-        torch.cuda.synchronize()
-        ref, tp = O.forward_offline(audio, lens, w)
-        err = np.max(np.abs(probs.cpu().numpy() - ref))
-        assert tp[0] == 1125 and err <= 2e-2, err
-    finally:
-        b.sf_destroy(eng)
+    """Full model (17 + 18 layers) bf16 on the 90 s workload clip, in the
+    benchmark's launch shape: with xavier-scaled weights (probabilities
+    spread over ~[0.2, 0.8], so a constant output fails) all 1125 frames
+    within 2e-2 of the fp64 oracle; with the benchmark's N(0, 0.02) weights
+    (probabilities at 0.5 +- 0.015) a shape and range check only."""
+    audio, lens, _ = clip_for_config(1)
+    for xavier in (True, False):
+        w = full_weights(xavier=xavier)
+        eng = make_engine(w, 1, 17, 18, max_batch=1)
+        try:
+            probs = torch.full((1, 1125, 4), float("nan"), device="cuda")
+            b.sf_forward_offline(eng, to_dev(audio), lens, probs)
+            b.sf_check(eng)
+            got = probs.cpu().numpy()
+        finally:
+            b.sf_destroy(eng)
+        assert np.all(np.isfinite(got)) and got.min() >= 0 and got.max() <= 1
+        if xavier:
+            ref, tp = O.forward_offline(audio, lens, w)
+            assert tp[0] == 1125
+            assert float(ref.max() - ref.min()) > 0.08     # 4 x the bound
+            err = np.max(np.abs(got - ref))
+            assert err <= 2e-2, err
 
 
 def test_offline_bf16_full_xavier_sampled_frames():

@@ -11,7 +11,8 @@ import pytest
 import oracle as O
 from oracle import streaming as OS
 from synth import synth_batch, synth_clip
-from _helpers import act_dtype, bf16_round, make_engine, tiny_weights, to_dev
+from _helpers import (act_dtype, bf16_round, get_state, make_engine, oracle_states as _oracle_states, set_state,
+                      tiny_weights, to_dev)
 
 pytestmark = pytest.mark.gpu
 torch = pytest.importorskip("torch")
@@ -41,40 +42,6 @@ def eng16():
     b.sf_destroy(e)
 
 
-def set_state(eng, st, sid, ost, precision):
-    dt = act_dtype(precision)
-    keep = []
-
-    def dev(a, d=None):
-        t = to_dev(a if len(a) else np.zeros((1,) + a.shape[1:]), d)
-        keep.append(t)
-        return t.data_ptr()
-    v = b.sf_state_view()
-    v.n_cache, v.n_fifo, v.next_frame = len(ost.cache_emb), len(ost.fifo_emb), ost.c0
-    v.finished, v.sil_count = 0, ost.sil_count
-    v.d_cache_emb, v.d_cache_preds = dev(ost.cache_emb, dt), dev(ost.cache_preds)
-    v.d_fifo_emb, v.d_fifo_preds = dev(ost.fifo_emb, dt), dev(ost.fifo_preds)
-    v.d_sil_mean = dev(ost.sil_mean)
-    b.sf_stream_set_state(eng, st, sid, v)
-    torch.cuda.synchronize()
-
-
-def get_state(eng, st, sid, precision, cap_c, cap_f):
-    dt = act_dtype(precision)
-    t = dict(ce=torch.zeros((cap_c, 512), device="cuda", dtype=dt), cp=torch.zeros((cap_c, 4), device="cuda"),
-             fe=torch.zeros((cap_f, 512), device="cuda", dtype=dt), fp=torch.zeros((cap_f, 4), device="cuda"),
-             sm=torch.zeros(512, device="cuda"))
-    v = b.sf_state_view()
-    v.d_cache_emb, v.d_cache_preds = t["ce"].data_ptr(), t["cp"].data_ptr()
-    v.d_fifo_emb, v.d_fifo_preds, v.d_sil_mean = t["fe"].data_ptr(), t["fp"].data_ptr(), t["sm"].data_ptr()
-    b.sf_stream_get_state(eng, st, sid, v)
-    nc, nf = v.n_cache, v.n_fifo
-    return dict(n_c=nc, n_f=nf, c0=v.next_frame, finished=v.finished, sil_count=v.sil_count,
-                cache_emb=t["ce"][:nc].float().cpu().numpy(), cache_preds=t["cp"][:nc].cpu().numpy(),
-                fifo_emb=t["fe"][:nf].float().cpu().numpy(), fifo_preds=t["fp"][:nf].cpu().numpy(),
-                sil_mean=t["sm"].cpu().numpy())
-
-
 @pytest.mark.parametrize("seed", range(6))
 def test_select_topk_bit_exact(eng32, seed):
     rng = np.random.default_rng(seed)
@@ -95,15 +62,6 @@ def test_select_topk_bit_exact(eng32, seed):
         for s in range(4):
             ref += [-1 - s] * (k - len(sel[s]))
         assert list(got[i]) == ref
-
-
-def _oracle_states(w, feats, L, preset, upto):
-    st = O.StreamState()
-    states, taps = [], []
-    while st.c0 < 1 + (L - 1) // 8 and len(states) < upto:
-        states.append(st.copy())
-        O.stream_step(st, feats, L, w, preset, taps=taps)
-    return states, taps
 
 
 @pytest.mark.parametrize("precision", [0, 1])

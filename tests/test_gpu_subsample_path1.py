@@ -3,12 +3,8 @@ s2 conv's outputs computed on chip and fed straight into the first
 depthwise conv).  It sums every output's taps in the order of the two-kernel
 path and rounds the stage-1 values the same way, so pre_encode embeddings,
 offline probabilities and streaming steps must equal path 0 to the bit;
-the embeddings are also checked against the oracle.
-
-These run only with SF_TEST_NEW_PATHS=1 in the environment: the default
-engine keeps path 0 until this path has been measured."""
-import os
-
+the embeddings are also checked against the oracle.  Path 1 is the default;
+path 0 stays selectable and is the bitwise reference here."""
 import numpy as np
 import pytest
 
@@ -16,9 +12,7 @@ import oracle as O
 from synth import clip_for_config, synth_batch
 from _helpers import act_dtype, make_engine, tiny_weights, to_dev
 
-pytestmark = [pytest.mark.gpu,
-              pytest.mark.skipif(os.environ.get("SF_TEST_NEW_PATHS") != "1",
-                                 reason="kernel paths not yet default run with SF_TEST_NEW_PATHS=1")]
+pytestmark = pytest.mark.gpu
 torch = pytest.importorskip("torch")
 if not torch.cuda.is_available():
     pytest.skip("no CUDA device", allow_module_level=True)
