@@ -386,6 +386,10 @@ enum {
                              step): 1 (default) FFT in registers with warp shuffles, then
                              separate statistics and normalisation passes over all SMs; 0 FFT
                              through shared memory and one normalisation CTA per (clip, bin) */
+  SF_OPT_LN_FUSE = 8,     /* bf16 engines: 1 (default) LayerNorm fused into the epilogue of the
+                             residual projection before it wherever the projection's 64-column
+                             tiles of a 128-row block fit one CTA cluster and all row blocks
+                             one wave; 0 separate LayerNorm kernels */
   SF_OPT_SUB_PATH = 7     /* ConvSubsampling's first two stages: 1 (default) one kernel that
                              computes the first conv's outputs on chip and feeds them straight
                              into the first depthwise conv; 0 the 3x3 s2 conv and the first
@@ -420,6 +424,23 @@ SF_API sf_status sf_selftest_wait(sf_engine* e, void* cuda_stream);
  * Requires N % 16 == 0, K % 64 == 0, lda % 8 == 0, 16-byte aligned A/W. */
 SF_API sf_status sf_gemm_bf16(sf_engine* e, const void* d_A, int lda, const void* d_W, int M, int N, int K,
                               const float* d_bias, void* d_C, int path, void* cuda_stream);
+
+/* The engine's residual projection with the LayerNorm that follows it fused
+ * into the epilogue (bf16 engines), for tests and kernel benchmarks; the
+ * conformer and Transformer layers' "x = x + f(x); h = LN(x)" steps
+ * ("Streaming Sortformer Diarizer", Pipeline: FastConformer and post-LN
+ * Transformer layers):
+ *   x_new = d_x f32 [M x N] + alpha (d_A bf16 [M x K] . d_W bf16 [N x K]^T
+ *           + d_bias f32 [N] (may be NULL))
+ *   xnorm 0: d_x <- x_new,     d_h bf16 [M x N] <- LN(x_new)
+ *   xnorm 1: d_x <- LN(x_new), d_h <- LN2(LN(x_new)) with d_g2/d_b2, else LN(x_new)
+ * LN(v) = (v - mean) / sqrt(var + 1e-5) * g + b over each row (biased
+ * variance), g/b f32 [N].  Requires N a multiple of 64 up to 512 and every
+ * 128-row block's cluster of N/64 CTAs co-resident (SF_ESHAPE otherwise),
+ * K % 64 == 0, lda % 8 == 0, 16-byte aligned A/W/x, 8-byte aligned h. */
+SF_API sf_status sf_gemm_bf16_ln(sf_engine* e, const void* d_A, int lda, const void* d_W, int M, int N, int K,
+                                 const float* d_bias, float alpha, float* d_x, const float* d_g, const float* d_b,
+                                 const float* d_g2, const float* d_b2, int xnorm, void* d_h, void* cuda_stream);
 
 /* The engine's relative-position self-attention alone (bf16 engines), for
  * tests and kernel benchmarks ("Streaming Sortformer Diarizer" model card,

@@ -4,6 +4,8 @@
     python kbench.py attn N_SEQ LEN [--path P] [--reps R]
     python kbench.py mha N_SEQ LEN [--path P] [--reps R]
     python kbench.py mel SECONDS [--clips B] [--path P] [--reps R]
+    python kbench.py ln M N K [--xnorm X] [--double] [--reps R]
+    python kbench.py stream N_STREAMS STEPS [--preset C R F U S]
 
 `gemm` runs sf_gemm_bf16 (E: 1 f32 out, 2 bf16 out, 3 residual update, 4
 swish, 5 gated linear unit; P: SF_OPT_GEMM_PATH, 1 = tcgen05 with CTA pairs
@@ -11,7 +13,13 @@ where faster, 2 = CTA pairs always, 3 = single CTAs, 0 = mma.sync); `attn`
 runs sf_attention_relpos and `mha` sf_attention_mha on N_SEQ packed
 sequences of LEN rows (P: 1 tcgen05, 0 mma.sync; `mha` also 2, mma.sync
 with four key groups per CTA); `mel` runs sf_mel on B
-clips of SECONDS of audio each (P: SF_OPT_MEL_PATH).  Operands are seeded random values on the device; three warm-up
+clips of SECONDS of audio each (P: SF_OPT_MEL_PATH); `ln` runs
+sf_gemm_bf16_ln, the residual projection with the LayerNorm after it fused
+into the epilogue (X: 1 = the residual stream receives the normalised row;
+--double: a second LayerNorm into the bf16 output); `stream` runs STEPS
+streaming steps of N_STREAMS streams (a 2 + 2-layer bf16 engine, random
+normalised features, default the Low preset 6/7/188/144/188): the state
+update and cache compression kernels at full state sizes.  Operands are seeded random values on the device; three warm-up
 launches, then REPS launches queued behind a GPU sleep (so host launch
 overhead is hidden) and timed with CUDA events on the current stream.  Also
 the driver for single-kernel ncu captures (small REPS)."""
@@ -66,8 +74,19 @@ def main(argv=None):
     f = sub.add_parser("mel")
     f.add_argument("seconds", type=float)
     f.add_argument("--clips", type=int, default=1)
-    f.add_argument("--path", type=int, default=0)
+    f.add_argument("--path", type=int, default=1)
     f.add_argument("--reps", type=int, default=10)
+    n = sub.add_parser("ln")
+    n.add_argument("M", type=int)
+    n.add_argument("N", type=int)
+    n.add_argument("K", type=int)
+    n.add_argument("--xnorm", type=int, default=0)
+    n.add_argument("--double", action="store_true")
+    n.add_argument("--reps", type=int, default=20)
+    t = sub.add_parser("stream")
+    t.add_argument("n_streams", type=int)
+    t.add_argument("steps", type=int)
+    t.add_argument("--preset", type=int, nargs=5, default=[6, 7, 188, 144, 188])
     args = ap.parse_args(argv)
 
     import torch
@@ -87,6 +106,38 @@ def main(argv=None):
         ms = _time(torch, lambda: b.sf_gemm_bf16(eng, A, W, C, path=path), args.reps)
         print(f"gemm M={M} N={N} K={K} epi={args.epi} path={args.path}: {ms * 1e3:.1f} us/launch, "
               f"{2 * M * N * K / ms / 1e9:.1f} TFLOP/s")
+    elif args.op == "ln":
+        eng = _engine(b, 8)
+        M, N, K = args.M, args.N, args.K
+        A = (torch.randn(M, K, device="cuda", generator=gen) / K ** 0.5).to(torch.bfloat16)
+        W = torch.randn(N, K, device="cuda", generator=gen).to(torch.bfloat16)
+        x = torch.randn(M, N, device="cuda", generator=gen)
+        h = torch.empty(M, N, device="cuda", dtype=torch.bfloat16)
+        g, bb = torch.ones(N, device="cuda"), torch.zeros(N, device="cuda")
+        two = args.double
+        ms = _time(torch, lambda: b.sf_gemm_bf16_ln(eng, A, W, x, g, bb, h, alpha=0.5, xnorm=1 if two else args.xnorm,
+                                                     g2=g if two else None, b2=bb if two else None), args.reps)
+        print(f"gemm+ln M={M} N={N} K={K} xnorm={args.xnorm} double={two}: {ms * 1e3:.1f} us/launch, "
+              f"{2 * M * N * K / ms / 1e9:.1f} TFLOP/s")
+    elif args.op == "stream":
+        n, pre = args.n_streams, tuple(args.preset)
+        eng = _engine(b, n)
+        T = 8 * (pre[0] * args.steps + pre[1]) + 8
+        feats = torch.randn(n, 128, T, device="cuda", generator=gen)
+        st = b.sf_stream_create(eng, pre, n)
+        cp = torch.zeros(n, pre[0], 4, device="cuda")
+        zero, end = np.zeros(n, np.int64), np.full(n, T, np.int64)
+        for _ in range(3):   # capture the step graphs
+            b.sf_stream_step(eng, st, feats, zero, end, cp)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        b.sf_stream_reset(st)
+        e0.record()
+        for _ in range(args.steps):
+            b.sf_stream_step(eng, st, feats, zero, end, cp)
+        e1.record()
+        torch.cuda.synchronize()
+        b.sf_stream_destroy(st)
+        print(f"stream n={n} preset={pre}: {args.steps} steps, {e0.elapsed_time(e1) / args.steps * 1e3:.1f} us/step")
     elif args.op == "mel":
         n = int(args.seconds * 16000)
         B = args.clips

@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(HERE, "libsf.so")
 SF_FP32, SF_BF16 = 0, 1
 SF_OPT_GRAPHS, SF_OPT_PDL, SF_OPT_GEMM_PATH, SF_OPT_GEMM_PAIR_BN, SF_OPT_ATTN_PATH, SF_OPT_MEL_PATH = 1, 2, 3, 4, 5, 6
 SF_OPT_SUB_PATH = 7
+SF_OPT_LN_FUSE = 8
 STATUS = {0: "SF_OK", 1: "SF_EINVAL", 2: "SF_ESHAPE", 3: "SF_ENOMEM", 4: "SF_ECUDA", 5: "SF_ESTATE",
           6: "SF_ETIMEOUT", 7: "SF_EDEVICE", 8: "SF_EFORMAT"}
 
@@ -59,7 +60,7 @@ EXPORTED = ["sf_default_config", "sf_create", "sf_create_from_file", "sf_destroy
             "sf_stream_window", "sf_stream_step", "sf_stream_get_state", "sf_stream_set_state",
             "sf_stream_update", "sf_select_topk", "sf_profile_enable", "sf_profile_read", "sf_mel_noalloc",
             "sf_check", "sf_gemm_bf16", "sf_set_option", "sf_attention_relpos", "sf_default_seg_params",
-            "sf_segments", "sf_stream_step_audio", "sf_attention_mha", "sf_selftest_wait"]
+            "sf_segments", "sf_stream_step_audio", "sf_attention_mha", "sf_selftest_wait", "sf_gemm_bf16_ln"]
 
 
 class SFError(RuntimeError):
@@ -100,6 +101,7 @@ def _load():
         "sf_selftest_wait": ([VP, VP], I),
         "sf_set_option": ([VP, I, I], I),
         "sf_gemm_bf16": ([VP, VP, I, VP, I, I, I, VP, VP, I, VP], I),
+        "sf_gemm_bf16_ln": ([VP, VP, I, VP, I, I, I, VP, ctypes.c_float, VP, VP, VP, VP, VP, I, VP, VP], I),
         "sf_attention_relpos": ([VP, VP, VP, I, VP, VP, VP, I, VP, I, VP], I),
         "sf_default_seg_params": ([P(sf_seg_params)], I),
         "sf_segments": ([VP, VP, I, VP, I, P(sf_seg_params), I, VP, VP, VP], I),
@@ -313,6 +315,15 @@ def sf_gemm_bf16(eng, A, W, C, bias=None, path=1, stream=None):
     N = W.shape[0]
     _check(lib.sf_gemm_bf16(eng, _ptr(A), A.stride(0), _ptr(W), M, N, K, _ptr(bias), _ptr(C), path,
                             _stream(stream)), eng)
+
+
+def sf_gemm_bf16_ln(eng, A, W, x, g, b, h, bias=None, alpha=1.0, xnorm=0, g2=None, b2=None, stream=None):
+    """Residual projection + LayerNorm in one launch: see sf.h."""
+    M, K = A.shape
+    N = W.shape[0]
+    _check(lib.sf_gemm_bf16_ln(eng, _ptr(A), A.stride(0), _ptr(W), M, N, K, _ptr(bias), ctypes.c_float(alpha),
+                               _ptr(x), _ptr(g), _ptr(b), _ptr(g2), _ptr(b2), int(xnorm), _ptr(h), _stream(stream)),
+           eng)
 
 
 def sf_attention_relpos(eng, qkv, ptab, R, u, v, seq_len, ctx, path=1, stream=None):

@@ -170,6 +170,7 @@ struct sf_engine {
   int attn_path = 1;      // bf16 relative-position attention: 1 = tcgen05, 0 = mma.sync
   int mel_path = MEL_DEFAULT_PATH;   // front-end: 1 = register FFT + all-SM normalisation, 0 = shared-memory FFT
   int sub_path = 1;       // subsampling: 1 = conv1 fused into the first depthwise, 0 = conv1 and depthwise kernels
+  int ln_fuse = 1;        // bf16: LayerNorm fused into the residual projections' epilogue where it fits
   float* d_split_ws = nullptr;   // split-K partial tiles of the tcgen05 GEMM
   int* d_split_cnt = nullptr;    // their per-tile arrival counters (kept at zero between launches)
   TcScratch tc_scratch() const { return TcScratch{d_err, d_split_ws, SPLIT_WS_BYTES, d_split_cnt, SPLIT_CNT}; }
@@ -639,6 +640,37 @@ Epi epi(int kind, const float* bias, void* out, int ldo, float alpha = 1.f) {
   return e;
 }
 
+// Residual projection followed by LayerNorm over each row of the f32
+// residual stream x [M x N]: x_new = x + alpha (A W^T + bias); then with
+// xnorm = 0: x <- x_new, h <- act(LN(x_new)); with xnorm = 1: x <- LN(x_new)
+// and h <- act(LN2(x)) when g2 is given, else act(x).  One launch (the
+// LayerNorm in the GEMM's epilogue, exchanged across the row block's CTA
+// cluster) in bf16 engines where the shape allows it, else the projection
+// and a LayerNorm kernel.
+template <typename T>
+cudaError_t resid_ln(sf_engine* e, const T* A, int lda, const T* W, int M, int N, int K, const float* bias,
+                     float alpha, float* x, const float* g, const float* b, bool xnorm, T* h, cudaStream_t st,
+                     const float* g2 = nullptr, const float* b2 = nullptr) {
+  if (sizeof(T) == 2 && e->ln_fuse && e->gemm_path >= 1 && gemm_ln_fusable(M, N, K)) {
+    Epi ep = epi(EPI_RESID_LN, bias, x, N, alpha);
+    ep.ln_g = g;
+    ep.ln_b = b;
+    ep.ln_g2 = g2;
+    ep.ln_b2 = b2;
+    ep.ln_h = h;
+    ep.ldh = N;
+    ep.ln_xnorm = xnorm ? 1 : 0;
+    const double a = sizeof(T);
+    RUN(K_GEMM, 1, 2.0 * M * N * K, ((double)M * K + (double)N * K) * a + (double)M * N * (8.0 + a),
+        gemm_dispatch<T>(e, A, lda, W, M, N, K, ep, st));
+    return cudaSuccess;
+  }
+  CK(gemm_acc<T>(e, A, lda, W, M, N, K, epi(EPI_RESID, bias, x, N, alpha), st));
+  RUN(K_LN, 1, 0, (double)M * N * (4 + sizeof(T) + (xnorm ? 4 : 0)),
+      launch_layernorm<T>(x, g, b, M, N, xnorm, h, st, g2, b2));
+  return cudaSuccess;
+}
+
 // ------------------------------------------------------------ descriptors
 DescBlock* desc_begin(sf_engine* e) {
   if (e->desc_pending) {
@@ -691,7 +723,7 @@ cudaError_t run_graph(sf_engine* e, std::string key, cudaStream_t st, F&& enqueu
   key += e->prof ? "|p" + std::to_string(e->prof_mask) : "|n";
   key += e->use_pdl ? "|pdl" : "";
   key += "|g" + std::to_string(e->gemm_path) + "." + std::to_string(e->pair_bn) + "|a" + std::to_string(e->attn_path) +
-         "|m" + std::to_string(e->mel_path) + "|s" + std::to_string(e->sub_path);
+         "|m" + std::to_string(e->mel_path) + "|s" + std::to_string(e->sub_path) + "|n" + std::to_string(e->ln_fuse);
   auto it = e->graphs.find(key);
   if (it != e->graphs.end() && it->second.gen != e->ws_gen) {
     cudaGraphExecDestroy(it->second.exec);
@@ -855,30 +887,20 @@ cudaError_t run_encode(sf_engine* e, int M, int n_tiles, float* probs, cudaStrea
     if (l == 0)   // later layers get this LN fused into the previous layer's final LN
       RUN(K_LN, 1, 0, (double)M * D * (4 + sizeof(T)), launch_layernorm<T>(x, w.ff1_g, w.ff1_b, M, D, false, h, st));
     CK(gemm_acc<T>(e, h, D, w.ff1_w1, M, DFF, D, epi(EPI_BIAS_SWISH, w.ff1_b1, big, DFF), st));
-    CK(gemm_acc<T>(e, big, DFF, w.ff1_w2, M, D, DFF, epi(EPI_RESID, w.ff1_b2, x, D, 0.5f), st));
-    RUN(K_LN, 1, 0, (double)M * D * (4 + sizeof(T)),
-        launch_layernorm<T>(x, w.att_g, w.att_b, M, D, false, h, st));
+    CK(resid_ln<T>(e, big, DFF, w.ff1_w2, M, D, DFF, w.ff1_b2, 0.5f, x, w.att_g, w.att_b, false, h, st));
     CK(gemm_acc<T>(e, h, D, w.wqkv, M, 3 * D, D, epi(EPI_BIAS, w.bqkv, big, 3 * D), st));
     RUN(K_ATT_REL, 1, 6.0 * e->att_s2 * D, (double)M * 4 * D * sizeof(T),
         relpos_attention<T>(e, big, w.ptab, w.pu, w.pv, ctx, seq, n_tiles, M, st));
-    CK(gemm_acc<T>(e, ctx, D, w.wo, M, D, D, epi(EPI_RESID, w.bo, x, D, 1.f), st));
-    RUN(K_LN, 1, 0, (double)M * D * (4 + sizeof(T)),
-        launch_layernorm<T>(x, w.conv_g, w.conv_b, M, D, false, h, st));
+    CK(resid_ln<T>(e, ctx, D, w.wo, M, D, D, w.bo, 1.f, x, w.conv_g, w.conv_b, false, h, st));
     CK(gemm_acc<T>(e, h, D, w.pw1, M, 2 * D, D, epi(EPI_BIAS_GLU, w.pw1_b, ctx, D), st));
     RUN(K_DW1D, 1, 2.0 * M * D * c.conv_kernel, (double)M * D * 2 * sizeof(T),
         launch_dwconv1d<T>(ctx, h, w.dw_w, w.dw_b, M, D, c.conv_kernel, seq, st));
-    CK(gemm_acc<T>(e, h, D, w.pw2, M, D, D, epi(EPI_RESID, w.pw2_b, x, D, 1.f), st));
-    RUN(K_LN, 1, 0, (double)M * D * (4 + sizeof(T)),
-        launch_layernorm<T>(x, w.ff2_g, w.ff2_b, M, D, false, h, st));
+    CK(resid_ln<T>(e, h, D, w.pw2, M, D, D, w.pw2_b, 1.f, x, w.ff2_g, w.ff2_b, false, h, st));
     CK(gemm_acc<T>(e, h, D, w.ff2_w1, M, DFF, D, epi(EPI_BIAS_SWISH, w.ff2_b1, big, DFF), st));
-    CK(gemm_acc<T>(e, big, DFF, w.ff2_w2, M, D, DFF, epi(EPI_RESID, w.ff2_b2, x, D, 0.5f), st));
-    if (l + 1 < c.n_conformer) {   // layer-final LN, then the next layer's FFN1 LN, in one pass
-      const ConfW<T>& wn = W.conf[l + 1];
-      RUN(K_LN, 1, 0, (double)M * D * (4 + 4 + sizeof(T)),
-          launch_layernorm<T>(x, w.out_g, w.out_b, M, D, true, h, st, wn.ff1_g, wn.ff1_b));
-    } else {
-      RUN(K_LN, 1, 0, (double)M * D * (4 + 4 + sizeof(T)), launch_layernorm<T>(x, w.out_g, w.out_b, M, D, true, h, st));
-    }
+    // layer-final LN (x <- LN(x)), then the next layer's FFN1 LN into h
+    const bool next = l + 1 < c.n_conformer;
+    CK(resid_ln<T>(e, big, DFF, w.ff2_w2, M, D, DFF, w.ff2_b2, 0.5f, x, w.out_g, w.out_b, true, h, st,
+                   next ? W.conf[l + 1].ff1_g : nullptr, next ? W.conf[l + 1].ff1_b : nullptr));
   }
   float* x2 = static_cast<float*>(e->x2.p);
   T* h2 = static_cast<T*>(e->h2.p);
@@ -892,13 +914,9 @@ cudaError_t run_encode(sf_engine* e, int M, int n_tiles, float* probs, cudaStrea
     const TfW<T>& w = W.tf[l];
     CK(gemm_acc<T>(e, h2, E, w.wqkv, M, 3 * E, E, epi(EPI_BIAS, w.bqkv, big, 3 * E), st));
     RUN(K_ATT_MHA, 1, 4.0 * e->att_s2 * E, (double)M * 4 * E * sizeof(T), mha_attention<T>(e, big, ctx, seq, n_tiles, M, st));
-    CK(gemm_acc<T>(e, ctx, E, w.wo, M, E, E, epi(EPI_RESID, w.bo, x2, E, 1.f), st));
-    RUN(K_LN, 1, 0, (double)M * E * (4 + sizeof(T) + (true ? 4 : 0)),
-        launch_layernorm<T>(x2, w.ln1_g, w.ln1_b, M, E, true, h2, st));
+    CK(resid_ln<T>(e, ctx, E, w.wo, M, E, E, w.bo, 1.f, x2, w.ln1_g, w.ln1_b, true, h2, st));
     CK(gemm_acc<T>(e, h2, E, w.w1, M, c.tf_ff, E, epi(EPI_BIAS_RELU, w.b1, big, c.tf_ff), st));
-    CK(gemm_acc<T>(e, big, c.tf_ff, w.w2, M, E, c.tf_ff, epi(EPI_RESID, w.b2, x2, E, 1.f), st));
-    RUN(K_LN, 1, 0, (double)M * E * (4 + sizeof(T) + (true ? 4 : 0)),
-        launch_layernorm<T>(x2, w.ln2_g, w.ln2_b, M, E, true, h2, st));
+    CK(resid_ln<T>(e, big, c.tf_ff, w.w2, M, E, c.tf_ff, w.b2, 1.f, x2, w.ln2_g, w.ln2_b, true, h2, st));
   }
   CK(gemm_acc<T>(e, h2, E, W.head_w1, M, E, E, epi(EPI_BIAS_RELU, W.head_b1, ctx, E), st));
   RUN(K_HEAD, 1, 2.0 * M * E * 4, (double)M * (E * sizeof(T) + 16), launch_head_out<T>(ctx, W.head_w2, W.head_b2, probs, M, E, st));
@@ -1325,6 +1343,31 @@ sf_status sf_gemm_bf16(sf_engine* e, const void* d_A, int lda, const void* d_W, 
   return SF_OK;
 }
 
+sf_status sf_gemm_bf16_ln(sf_engine* e, const void* d_A, int lda, const void* d_W, int M, int N, int K,
+                          const float* d_bias, float alpha, float* d_x, const float* d_g, const float* d_b,
+                          const float* d_g2, const float* d_b2, int xnorm, void* d_h, void* cuda_stream) {
+  if (check_engine(e) != SF_OK) return SF_EINVAL;
+  if (!d_A || !d_W || !d_x || !d_g || !d_b || !d_h || (d_g2 && !d_b2)) return fail(e, SF_EINVAL, "null pointer argument");
+  if (d_g2 && !xnorm) return fail(e, SF_EINVAL, "a second LayerNorm needs xnorm = 1");
+  if (e->cfg.precision != SF_BF16) return fail(e, SF_ESTATE, "sf_gemm_bf16_ln needs a bf16 engine");
+  if (M < 1 || K < 64 || K % 64 || lda < K || lda % 8 || !gemm_ln_fusable(M, N, K))
+    return fail(e, SF_ESHAPE, "sf_gemm_bf16_ln: N a multiple of 64 up to 512, one wave of row blocks, K % 64 == 0");
+  if ((reinterpret_cast<uintptr_t>(d_x) & 15) || (reinterpret_cast<uintptr_t>(d_h) & 7))
+    return fail(e, SF_EINVAL, "x must be 16-byte and h 8-byte aligned");
+  Epi ep = epi(EPI_RESID_LN, d_bias, d_x, N, alpha);
+  ep.ln_g = d_g;
+  ep.ln_b = d_b;
+  ep.ln_g2 = d_g2;
+  ep.ln_b2 = d_b2;
+  ep.ln_h = d_h;
+  ep.ldh = N;
+  ep.ln_xnorm = xnorm ? 1 : 0;
+  cudaError_t ce = gemm_bf16_tc(static_cast<const bf16*>(d_A), lda, static_cast<const bf16*>(d_W), M, N, K, ep,
+                                e->tc_scratch(), static_cast<cudaStream_t>(cuda_stream));
+  if (ce != cudaSuccess) return cuda_fail(e, ce, "sf_gemm_bf16_ln");
+  return SF_OK;
+}
+
 sf_status sf_attention_relpos(sf_engine* e, const void* d_qkv, const void* d_ptab, int R, const float* d_u,
                               const float* d_v, const int* h_seq_len, int n, void* d_ctx, int path,
                               void* cuda_stream) {
@@ -1430,6 +1473,10 @@ sf_status sf_set_option(sf_engine* e, int option, int value) {
     case SF_OPT_SUB_PATH:
       if (value != 0 && value != 1) return fail(e, SF_EINVAL, "subsampling path must be 0 or 1");
       e->sub_path = value;
+      break;
+    case SF_OPT_LN_FUSE:
+      if (value != 0 && value != 1) return fail(e, SF_EINVAL, "LayerNorm fusion must be 0 or 1");
+      e->ln_fuse = value;
       break;
     case SF_OPT_GEMM_PAIR_BN:
       if (value != 0 && value != 128 && value != 192 && value != 256)

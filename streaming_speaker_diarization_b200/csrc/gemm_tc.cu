@@ -40,7 +40,8 @@ struct TcCfg {
   static constexpr int A_BYTES = TC_BM * TC_BK * 2;
   static constexpr int B_BYTES = BN * TC_BK * 2;
   static constexpr int SMEM = 1024 + STAGES * (A_BYTES + B_BYTES) + 256;
-  static_assert(STAGES * (A_BYTES + B_BYTES) >= 4 * 32 * 68 * 4, "epilogue staging reuses the pipeline buffers");
+  static_assert(STAGES * (A_BYTES + B_BYTES) >= 4 * 32 * 68 * 4 + 2 * 128 * 8,
+                "epilogue staging (and the LayerNorm statistics) reuse the pipeline buffers");
 };
 
 // Epilogue of one warp's 32 rows: per CW-column chunk (CW = 64 or 32), the
@@ -174,6 +175,170 @@ __device__ __forceinline__ void reduce_tile(const Epi& e, const float* base, int
   }
 }
 
+__device__ __forceinline__ void cluster_arrive_wait() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Row statistics of the whole output row from the cluster's partials: rank
+// j of the cluster holds (mean, M2) of columns [64 j, 64 j + 64) of local
+// row r in its `stat` array.  Chan's pairwise merge of equal-count parts:
+// mean = average of the means, M2 = sum(M2_j) + 64 sum((mean_j - mean)^2).
+__device__ __forceinline__ void ln_row_stats(const float2* stat, int r, int ncl, int ncols, float& mean,
+                                             float& rstd) {
+  const uint32_t a0 = su32(stat + r);
+  float mj[8], m2j[8];
+  float s = 0.f;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    mj[j] = 0.f;
+    m2j[j] = 0.f;
+    if (j < ncl) {
+      uint32_t a;
+      asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(a0), "r"((uint32_t)j));
+      asm volatile("ld.shared::cluster.v2.f32 {%0, %1}, [%2];" : "=f"(mj[j]), "=f"(m2j[j]) : "r"(a) : "memory");
+      s += mj[j];
+    }
+  }
+  mean = s / (float)ncl;
+  float m2 = 0.f;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    if (j < ncl) {
+      const float d = mj[j] - mean;
+      m2 += m2j[j] + 64.f * d * d;
+    }
+  }
+  rstd = 1.0f / sqrtf(m2 / (float)ncols + 1e-5f);
+}
+
+// (mean, M2) of the 64 staged columns of this thread's row (thread = row).
+__device__ __forceinline__ float2 ln_tile_stats(const float* row) {
+  float s = 0.f;
+#pragma unroll
+  for (int j = 0; j < 64; j += 4) {
+    const float4 v = *reinterpret_cast<const float4*>(row + j);
+    s += (v.x + v.y) + (v.z + v.w);
+  }
+  const float mean = s * (1.f / 64.f);
+  float m2 = 0.f;
+#pragma unroll
+  for (int j = 0; j < 64; j += 4) {
+    const float4 v = *reinterpret_cast<const float4*>(row + j);
+    float d = v.x - mean; m2 = fmaf(d, d, m2);
+    d = v.y - mean; m2 = fmaf(d, d, m2);
+    d = v.z - mean; m2 = fmaf(d, d, m2);
+    d = v.w - mean; m2 = fmaf(d, d, m2);
+  }
+  return make_float2(mean, m2);
+}
+
+// EPI_RESID_LN epilogue of one warp's 32 rows of a 128 x 64 tile whose CTA
+// is rank n0 / 64 of a cluster spanning the row block's N / 64 tiles.
+// x_new = x + alpha (acc + b) is staged in shared memory; each thread (one
+// row) takes (mean, M2) of its 64 columns; after a cluster barrier every CTA
+// merges the partials of all ranks for its rows and normalises its own
+// columns; a second LayerNorm, if any, repeats the exchange on the first
+// one's output.  Every epilogue thread passes the same cluster barriers
+// (n_cluster_barriers(e) of them) whether or not its CTA's accumulator is
+// valid (`ok`), so no CTA of the cluster waits for ever; the last barrier
+// keeps each CTA's statistics alive until its peers have read them.
+__device__ __forceinline__ int n_cluster_barriers(const Epi& e) { return e.ln_g2 ? 3 : 2; }
+
+__device__ __forceinline__ void resid_ln_epilogue(const Epi& e, uint32_t tmem, float* stage, float2* st1, float2* st2,
+                                                  int M, int N, int m0, int n0, int q, int lane, bool ok) {
+  constexpr int LD = 68;
+  const int l4 = lane & 15, rh = lane >> 4;
+  const int c = n0 + 4 * l4;
+  const int ncl = N / 64;
+  if (ok) {
+    uint32_t v[64];
+    tmem_ld64(tmem + ((uint32_t)(32 * q) << 16), v);
+#pragma unroll
+    for (int j = 0; j < 64; j += 4)
+      *reinterpret_cast<float4*>(stage + lane * LD + j) =
+          make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]), __uint_as_float(v[j + 2]),
+                      __uint_as_float(v[j + 3]));
+  }
+  __syncwarp();
+  if (ok) {   // x_new = x + alpha (acc + b) into the staged tile
+    float4 bv = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (e.bias) bv = *reinterpret_cast<const float4*>(e.bias + c);
+#pragma unroll 1
+    for (int i0 = 0; i0 < 16; i0 += 8) {
+      float4 xv[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int row = m0 + 32 * q + 2 * (i0 + i) + rh;
+        xv[i] = row < M ? *reinterpret_cast<const float4*>(epi_f32_ptr(e, row, c)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float* sp = stage + (2 * (i0 + i) + rh) * LD + 4 * l4;
+        const float4 t = *reinterpret_cast<const float4*>(sp);
+        float4 x = xv[i];
+        x.x += e.alpha * (t.x + bv.x); x.y += e.alpha * (t.y + bv.y);
+        x.z += e.alpha * (t.z + bv.z); x.w += e.alpha * (t.w + bv.w);
+        *reinterpret_cast<float4*>(sp) = x;
+      }
+    }
+  }
+  __syncwarp();
+  st1[32 * q + lane] = ok ? ln_tile_stats(stage + lane * LD) : make_float2(0.f, 0.f);
+  cluster_arrive_wait();
+  float mean, rstd;
+  ln_row_stats(st1, 32 * q + lane, ncl, N, mean, rstd);
+  const bool two = e.ln_g2 != nullptr;
+  {
+    const float4 g = *reinterpret_cast<const float4*>(e.ln_g + c);
+    const float4 bb = *reinterpret_cast<const float4*>(e.ln_b + c);
+#pragma unroll 4
+    for (int i = 0; i < 16; ++i) {
+      const int rr = 2 * i + rh, row = m0 + 32 * q + rr;
+      const float mu = __shfl_sync(0xffffffffu, mean, rr), rs = __shfl_sync(0xffffffffu, rstd, rr);
+      float* sp = stage + rr * LD + 4 * l4;
+      const float4 v = *reinterpret_cast<const float4*>(sp);
+      float4 y;
+      y.x = (v.x - mu) * rs * g.x + bb.x; y.y = (v.y - mu) * rs * g.y + bb.y;
+      y.z = (v.z - mu) * rs * g.z + bb.z; y.w = (v.w - mu) * rs * g.w + bb.w;
+      if (ok && row < M) {
+        *reinterpret_cast<float4*>(epi_f32_ptr(e, row, c)) = e.ln_xnorm ? y : v;
+        if (!two) {
+          __nv_bfloat162 a = __floats2bfloat162_rn(y.x, y.y), b2 = __floats2bfloat162_rn(y.z, y.w);
+          uint2 pk;
+          pk.x = *reinterpret_cast<uint32_t*>(&a);
+          pk.y = *reinterpret_cast<uint32_t*>(&b2);
+          *reinterpret_cast<uint2*>(reinterpret_cast<bf16*>(e.ln_h) + (int64_t)row * e.ldh + c) = pk;
+        }
+      }
+      if (two) *reinterpret_cast<float4*>(sp) = y;
+    }
+  }
+  if (two) {
+    __syncwarp();
+    st2[32 * q + lane] = ok ? ln_tile_stats(stage + lane * LD) : make_float2(0.f, 0.f);
+    cluster_arrive_wait();
+    ln_row_stats(st2, 32 * q + lane, ncl, N, mean, rstd);
+    const float4 g = *reinterpret_cast<const float4*>(e.ln_g2 + c);
+    const float4 bb = *reinterpret_cast<const float4*>(e.ln_b2 + c);
+#pragma unroll 4
+    for (int i = 0; i < 16; ++i) {
+      const int rr = 2 * i + rh, row = m0 + 32 * q + rr;
+      const float mu = __shfl_sync(0xffffffffu, mean, rr), rs = __shfl_sync(0xffffffffu, rstd, rr);
+      const float4 v = *reinterpret_cast<const float4*>(stage + rr * LD + 4 * l4);
+      if (ok && row < M) {
+        __nv_bfloat162 a = __floats2bfloat162_rn((v.x - mu) * rs * g.x + bb.x, (v.y - mu) * rs * g.y + bb.y);
+        __nv_bfloat162 b2 = __floats2bfloat162_rn((v.z - mu) * rs * g.z + bb.z, (v.w - mu) * rs * g.w + bb.w);
+        uint2 pk;
+        pk.x = *reinterpret_cast<uint32_t*>(&a);
+        pk.y = *reinterpret_cast<uint32_t*>(&b2);
+        *reinterpret_cast<uint2*>(reinterpret_cast<bf16*>(e.ln_h) + (int64_t)row * e.ldh + c) = pk;
+      }
+    }
+  }
+  cluster_arrive_wait();   // peers have read this CTA's statistics
+}
+
 template <int BN, int STAGES>
 __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__ CUtensorMap ta,
                                                          const __grid_constant__ CUtensorMap tb, int M, int N, int K,
@@ -265,6 +430,15 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
       umma_commit(accf);   // arrives once every MMA issued above has completed
       pdl_trigger();
     }
+  } else if (e.kind == EPI_RESID_LN) {
+    const int q = warp & 3;
+    float* stage = reinterpret_cast<float*>(sm) + q * (32 * 68);
+    float2* st1 = reinterpret_cast<float2*>(reinterpret_cast<float*>(sm) + 4 * 32 * 68);
+    prefetch_resid(e, M, N, m0 + 32 * q, 32, n0, BN, lane);
+    const bool ok = mbar_wait(accf, 0, abort_flag) && !*abort_flag;
+    if (!ok) *abort_flag = 1;
+    tc_fence_after();
+    resid_ln_epilogue(e, tmem, stage, st1, st1 + 128, M, N, m0, n0, q, lane, ok);
   } else {
     // Epilogue: per 64-column chunk, each warp copies its 32 x 64 accumulator
     // block from TMEM to a padded shared tile (thread = row), then writes it
@@ -315,6 +489,10 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
     } else {
       *abort_flag = 1;
     }
+  }
+  if (e.kind == EPI_RESID_LN && warp < 2) {   // the epilogue warps' cluster barriers, for the whole CTA
+    __syncwarp();
+    for (int i = 0; i < n_cluster_barriers(e); ++i) cluster_arrive_wait();
   }
   tc_fence_before();
   __syncthreads();
@@ -768,6 +946,40 @@ cudaError_t launch_tc(const bf16* A, int lda, const bf16* W, int M, int N, int K
 }
 
 int g_num_sms = 148;
+int g_ln_clusters[9] = {};   // co-resident clusters of n CTAs of gemm_tc_kernel<64, 8> (0: unusable)
+
+// EPI_RESID_LN: 128 x 64 tiles, one cluster of N / 64 CTAs per row block.
+cudaError_t launch_tc_ln(const bf16* A, int lda, const bf16* W, int M, int N, int K, const Epi& e,
+                         const TcScratch& sc, cudaStream_t st) {
+  constexpr int BN = 64, STAGES = 8;
+  CUtensorMap ta, tb;
+  cudaError_t r = make_map(&ta, A, M, K, lda, TC_BM);
+  if (r != cudaSuccess) return r;
+  r = make_map(&tb, W, N, K, K, BN);
+  if (r != cudaSuccess) return r;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(N / BN, (M + TC_BM - 1) / TC_BM, 1);
+  cfg.blockDim = dim3(192);
+  cfg.dynamicSmemBytes = TcCfg<BN, STAGES>::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  attr[na].id = cudaLaunchAttributeClusterDimension;
+  attr[na].val.clusterDim.x = N / BN;
+  attr[na].val.clusterDim.y = 1;
+  attr[na].val.clusterDim.z = 1;
+  ++na;
+  if (g_launch_pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  CK_LAUNCH(cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, STAGES>, ta, tb, M, N, K, e, sc.err, (float*)nullptr,
+                               (int*)nullptr));
+  return cudaGetLastError();
+}
 
 template <int BN, int STAGES>
 cudaError_t launch_tcp(const bf16* A, int lda, const bf16* W, int M, int N, int K, const Epi& e, const TcScratch& sc,
@@ -868,12 +1080,24 @@ void gemm_tc_plan(int M, int N, int K, const TcScratch& sc, int* bn_out, int* s_
   *s_out = bs;
 }
 
+bool gemm_ln_fusable(int M, int N, int K) {
+  if (M <= 0 || K % 8 || N % 64 || N / 64 > 8) return false;
+  return (M + TC_BM - 1) / TC_BM <= g_ln_clusters[N / 64];
+}
+
 cudaError_t gemm_bf16_tc(const bf16* A, int lda, const bf16* W, int M, int N, int K, const Epi& e,
                          const TcScratch& sc, cudaStream_t st) {
   if (M <= 0) return cudaSuccess;
   if (N % 16 || K % 8) return cudaErrorInvalidValue;
   cudaError_t r = get_encoder();
   if (r != cudaSuccess) return r;
+  if (e.kind == EPI_RESID_LN) {
+    if (!gemm_ln_fusable(M, N, K) || !e.ln_g || !e.ln_b || !e.ln_h || (e.ln_g2 && (!e.ln_b2 || !e.ln_xnorm)) ||
+        e.rpg || (reinterpret_cast<uintptr_t>(e.out) & 15) || (reinterpret_cast<uintptr_t>(e.ln_h) & 7) ||
+        e.ldo % 4 || e.ldh % 4)
+      return cudaErrorInvalidValue;
+    return launch_tc_ln(A, lda, W, M, N, K, e, sc, st);
+  }
   int bn, sp;
   gemm_tc_plan(M, N, K, sc, &bn, &sp);
   // more tiles than SMs: the persistent kernel overlaps each tile's epilogue
@@ -931,7 +1155,24 @@ cudaError_t gemm_tc_init_attributes() {
     r = cudaFuncSetAttribute(gemm_tc_kernel<128, 6>, cudaFuncAttributeMaxDynamicSharedMemorySize, TcCfg<128, 6>::SMEM);
   if (r == cudaSuccess)
     r = cudaFuncSetAttribute(gemm_tc_kernel<64, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, TcCfg<64, 8>::SMEM);
-  return r;
+  if (r != cudaSuccess) return r;
+  for (int n = 1; n <= 8; ++n) {   // clusters of n CTAs for the LayerNorm-fused epilogue
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(n, 1, 1);
+    cfg.blockDim = dim3(192);
+    cfg.dynamicSmemBytes = TcCfg<64, 8>::SMEM;
+    cudaLaunchAttribute a;
+    a.id = cudaLaunchAttributeClusterDimension;
+    a.val.clusterDim.x = n;
+    a.val.clusterDim.y = 1;
+    a.val.clusterDim.z = 1;
+    cfg.attrs = &a;
+    cfg.numAttrs = 1;
+    int n_cl = 0;
+    g_ln_clusters[n] = cudaOccupancyMaxActiveClusters(&n_cl, gemm_tc_kernel<64, 8>, &cfg) == cudaSuccess ? n_cl : 0;
+    cudaGetLastError();
+  }
+  return cudaSuccess;
 }
 
 }  // namespace sf

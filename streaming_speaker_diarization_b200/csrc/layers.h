@@ -17,6 +17,11 @@ enum EpiKind : int {
   EPI_RESID = 4,       // out(f32) += alpha * (acc + b)
   EPI_F32 = 5,         // out(f32) = acc + b
   EPI_F32_AND_T = 6,   // out(f32) = acc + b and out2(act) = acc + b
+  EPI_RESID_LN = 7,    // x_new = out(f32) + alpha * (acc + b), then LayerNorm over each full row:
+                       //   ln_xnorm 0: out <- x_new,     ln_h <- act(LN(x_new))
+                       //   ln_xnorm 1: out <- LN(x_new), ln_h <- act(LN2(LN(x_new))) with ln_g2,
+                       //               else act(LN(x_new))
+                       // (bf16 tcgen05 path only; the N tiles of a row block form a CTA cluster)
 };
 
 struct Epi {
@@ -29,6 +34,15 @@ struct Epi {
   int ldo2;
   int rpg;             // row remap: 0 = identity, else row r -> (r / rpg) * gstride + r % rpg
   int64_t gstride;
+  // EPI_RESID_LN: LayerNorm weights (length N), optional second LayerNorm,
+  // the act output [M x ldh] and whether out receives the normalised row
+  const float* ln_g;
+  const float* ln_b;
+  const float* ln_g2;
+  const float* ln_b2;
+  void* ln_h;
+  int ldh;
+  int ln_xnorm;
 };
 
 cudaError_t gemm_f32(const float* A, int lda, const float* W, int M, int N, int K, const Epi& e, cudaStream_t st);
@@ -59,6 +73,10 @@ extern int g_gemm_pairs;
 // Pair tile width forced for those GEMMs (128, 192 or 256); 0 = planned.
 extern int g_gemm_pair_bn;
 void gemm_tc_plan(int M, int N, int K, const TcScratch& sc, int* bn, int* splits);
+// Whether an EPI_RESID_LN GEMM of this shape runs fused: N a multiple of 64
+// with at most 8 tiles of 64 (one cluster per 128-row block) and every
+// cluster co-resident (one wave); otherwise use EPI_RESID and a LayerNorm.
+bool gemm_ln_fusable(int M, int N, int K);
 
 // --------------------------------------------------------- subsampling
 struct PreArgs {        // device arrays, one entry per window

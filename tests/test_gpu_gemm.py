@@ -164,3 +164,82 @@ def _check_fused(eng, M, N, K, path):
     b.sf_check(eng)
     got = C.float().cpu().numpy()
     assert np.all(np.abs(got - ref) <= np.abs(ref) * tol_rel + tol_abs)
+
+
+# --------------------------------------------------------------------------
+# Residual projection with the LayerNorm fused into the epilogue (the
+# conformer's "x += f(x); h = LN(x)" steps and the Transformer's post-LN),
+# against float64 of the same bf16 operands: x to fp32 accumulation
+# accuracy, h (bf16) to one bf16 rounding (2^-8 relative) plus that.
+
+def _ln64(v, g, b):
+    mu = v.mean(1, keepdims=True)
+    var = ((v - mu) ** 2).mean(1, keepdims=True)
+    return (v - mu) / np.sqrt(var + 1e-5) * g + b
+
+
+LN_SHAPES = [(1125, 512, 512, 0.5, 0, False), (1125, 512, 2048, 0.5, 1, True), (1125, 512, 512, 1.0, 0, False),
+             (1125, 192, 192, 1.0, 1, False), (1125, 192, 768, 1.0, 1, False), (1, 512, 64, 1.0, 0, False),
+             (130, 192, 128, 0.5, 1, True), (1000, 64, 256, 1.0, 0, False), (513, 320, 192, 1.0, 1, False)]
+
+
+@pytest.mark.parametrize("M,N,K,alpha,xnorm,two", LN_SHAPES)
+def test_gemm_resid_layernorm_fused(eng, M, N, K, alpha, xnorm, two):
+    g = torch.Generator().manual_seed(M + 3 * N + 5 * K)
+    A = (torch.randn(M, K, generator=g) / np.sqrt(K)).to(torch.bfloat16)
+    W = torch.randn(N, K, generator=g).to(torch.bfloat16)
+    bias = torch.randn(N, generator=g)
+    x0 = torch.randn(M, N, generator=g) * 2 + 0.3
+    lg, lb = 1 + 0.3 * torch.randn(N, generator=g), 0.2 * torch.randn(N, generator=g)
+    lg2, lb2 = 1 + 0.3 * torch.randn(N, generator=g), 0.2 * torch.randn(N, generator=g)
+    x = x0.cuda().contiguous()
+    h = torch.full((M, N), float("nan"), device="cuda", dtype=torch.bfloat16)
+    b.sf_gemm_bf16_ln(eng, A.cuda(), W.cuda(), x, lg.cuda(), lb.cuda(), h, bias=bias.cuda(), alpha=alpha, xnorm=xnorm,
+                      g2=lg2.cuda() if two else None, b2=lb2.cuda() if two else None)
+    b.sf_check(eng)
+    d = lambda t: t.double().numpy()  # noqa: E731
+    xn = d(x0) + alpha * (d(A) @ d(W).T + d(bias))
+    y = _ln64(xn, d(lg), d(lb))
+    x_ref = y if xnorm else xn
+    h_ref = _ln64(y, d(lg2), d(lb2)) if two else y
+    gx, gh = x.cpu().numpy(), h.float().cpu().numpy()
+    assert np.max(np.abs(gx - x_ref)) <= 2e-4 * max(1.0, np.sqrt(K / 512)) * (2 if xnorm else 4)
+    assert np.max(np.abs(gh - h_ref) / (np.abs(h_ref) + 1e-2)) <= 1e-2
+    assert np.max(np.abs(gh - h_ref)) <= 3e-2
+
+
+def test_gemm_resid_layernorm_rejects_unfusable(eng):
+    A = torch.zeros((10, 64), dtype=torch.bfloat16, device="cuda")
+    W = torch.zeros((576, 64), dtype=torch.bfloat16, device="cuda")     # 9 tiles of 64: more than a cluster
+    x = torch.zeros((10, 576), device="cuda")
+    h = torch.zeros((10, 576), dtype=torch.bfloat16, device="cuda")
+    one = torch.ones(576, device="cuda")
+    with pytest.raises(b.SFError, match="SF_ESHAPE"):
+        b.sf_gemm_bf16_ln(eng, A, W, x, one, one, h)
+
+
+def test_offline_forward_with_and_without_layernorm_fusion():
+    """The bf16 offline forward with the fused residual LayerNorms equals the
+    unfused engine to bf16 accuracy and the oracle within 2e-2 (xavier
+    weights, so the probabilities spread over ~[0.45, 0.8])."""
+    import oracle as O
+    from synth import synth_batch
+    from _helpers import to_dev
+    w = tiny_weights(xavier=True)
+    e = make_engine(w, 1, 2, 2, max_batch=4)
+    try:
+        audio, lens, _ = synth_batch(85, [9.0, 4.1])
+        Tp = int(O.encoder_frames(audio.shape[1] // 160))
+        outs = []
+        for fuse in (1, 0):
+            b.sf_set_option(e, b.SF_OPT_LN_FUSE, fuse)
+            p = torch.zeros((2, Tp, 4), device="cuda")
+            b.sf_forward_offline(e, to_dev(audio), lens, p)
+            b.sf_check(e)
+            outs.append(p.cpu().numpy())
+    finally:
+        b.sf_destroy(e)
+    ref, tp = O.forward_offline(audio, lens, w)
+    for i in range(2):
+        assert np.max(np.abs(outs[0][i, :tp[i]] - ref[i, :tp[i]])) <= 2e-2
+    assert np.max(np.abs(outs[0] - outs[1])) <= 1e-2
