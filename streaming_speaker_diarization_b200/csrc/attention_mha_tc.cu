@@ -176,6 +176,7 @@ __global__ void __launch_bounds__(192, 2) attn_mha_tc_kernel(const __grid_consta
       }
       if (ok && Tl > 0) ok = issue_pv(Tl - 1);
       if (!ok) *abort_flag = 1;
+      pdl_trigger();   // the next kernel may launch and set up; it waits for this grid's memory
     }
   } else {
     // -------------------------------------------------------------- softmax
@@ -403,13 +404,14 @@ cudaError_t launch_mha_tc(const bf16* qkv, bf16* ctx, const SeqTable* seq, int n
   if (r != cudaSuccess) return r;
   // fewer (query tile, head) units than the two CTAs per SM hold: split
   // each unit's keys over a cluster of 2 or 4 CTAs (no more splits than key
-  // tiles of the longest sequence)
+  // tiles of the longest sequence), but only as far as every cluster is
+  // co-resident (one wave: a second wave would double the time)
   const int units = n_tiles2 * 8;
   int ks = 1;
   if (units < 2 * g_mha_sms) {
     const int want = 2 * g_mha_sms / units, tmax = (max_len + MK - 1) / MK;
-    if (want >= 4 && tmax >= 4 && g_mha_clusters[2] > 0) ks = 4;
-    else if (want >= 2 && tmax >= 2 && g_mha_clusters[1] > 0) ks = 2;
+    if (want >= 4 && tmax >= 4 && units <= g_mha_clusters[2]) ks = 4;
+    else if (want >= 2 && tmax >= 2 && units <= g_mha_clusters[1]) ks = 2;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(n_tiles2, 8, ks);

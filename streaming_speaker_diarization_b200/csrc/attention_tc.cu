@@ -216,6 +216,7 @@ __global__ void __launch_bounds__(192, 1) attn_relpos_tc_kernel(const __grid_con
       }
       if (ok) ok = issue_pv(Tl - 1);
       if (!ok) *abort_flag = 1;
+      pdl_trigger();   // the next kernel may launch and set up; it waits for this grid's memory
     }
   } else {
     // -------------------------------------------------------------- softmax
@@ -481,13 +482,14 @@ cudaError_t launch_relpos_attention_tc(const bf16* qkv, const bf16* ptab, int R,
   if (r != cudaSuccess) return r;
   // fewer (query tile, head) units than SMs: split each unit's keys over a
   // cluster of 2 or 4 CTAs (no more splits than key tiles of the longest
-  // sequence), merged in the cluster's shared memory
+  // sequence, and only while every cluster is co-resident), merged in the
+  // cluster's shared memory
   const int units = n_tiles2 * 8;
   int ks = 1;
   if (units < g_att_sms) {
     const int want = g_att_sms / units, tmax = (max_len + AK - 1) / AK;
-    if (want >= 4 && tmax >= 4 && g_att_clusters[2] > 0) ks = 4;
-    else if (want >= 2 && tmax >= 2 && g_att_clusters[1] > 0) ks = 2;
+    if (want >= 4 && tmax >= 4 && units <= g_att_clusters[2]) ks = 4;
+    else if (want >= 2 && tmax >= 2 && units <= g_att_clusters[1]) ks = 2;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(n_tiles2, 8, ks);

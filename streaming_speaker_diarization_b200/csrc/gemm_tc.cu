@@ -188,18 +188,20 @@ __device__ __forceinline__ void ln_row_stats(const float2* stat, int r, int ncl,
                                              float& rstd) {
   const uint32_t a0 = su32(stat + r);
   float mj[8], m2j[8];
-  float s = 0.f;
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
+  for (int j = 0; j < 8; ++j) {   // all loads issued before any result is used
     mj[j] = 0.f;
     m2j[j] = 0.f;
     if (j < ncl) {
       uint32_t a;
       asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(a0), "r"((uint32_t)j));
       asm volatile("ld.shared::cluster.v2.f32 {%0, %1}, [%2];" : "=f"(mj[j]), "=f"(m2j[j]) : "r"(a) : "memory");
-      s += mj[j];
     }
   }
+  float s = 0.f;
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    if (j < ncl) s += mj[j];
   mean = s / (float)ncl;
   float m2 = 0.f;
 #pragma unroll
@@ -385,13 +387,23 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // set-up above overlaps the previous kernel; global memory only from here
-  SF_PDL_ENTRY();
+  // Set-up above overlaps the previous kernel (programmatic dependent
+  // launch).  The weights do not depend on it either: the producer issues
+  // the first ring's weight tiles before waiting for the previous kernel's
+  // memory; everything else touches global memory only after the wait.
+  if (warp != 0) SF_PDL_ENTRY();
 
   if (warp == 0) {
     if (lane == 0) {
-      int issued = 0;
-      for (int kb = 0; kb < KB; ++kb) {
+      const int pre = KB < STAGES ? KB : STAGES;   // stages whose empty barrier is free from the start
+      for (int kb = 0; kb < pre; ++kb) {
+        mbar_expect_tx(&full[kb], C::A_BYTES + C::B_BYTES);
+        tma_load_2d(sB + kb * C::B_BYTES, &tb, &full[kb], (kb0 + kb) * TC_BK, n0);
+      }
+      pdl_wait();
+      for (int kb = 0; kb < pre; ++kb) tma_load_2d(sA + kb * C::A_BYTES, &ta, &full[kb], (kb0 + kb) * TC_BK, m0);
+      int issued = pre;
+      for (int kb = pre; kb < KB; ++kb) {
         const int s = kb % STAGES, r = kb / STAGES;
         if (!mbar_wait(&empty[s], (r & 1) ^ 1, abort_flag)) {
           *abort_flag = 1;
@@ -949,9 +961,10 @@ int g_num_sms = 148;
 int g_ln_clusters[9] = {};   // co-resident clusters of n CTAs of gemm_tc_kernel<64, 8> (0: unusable)
 
 // EPI_RESID_LN: 128 x 64 tiles, one cluster of N / 64 CTAs per row block.
-cudaError_t launch_tc_ln(const bf16* A, int lda, const bf16* W, int M, int N, int K, const Epi& e,
-                         const TcScratch& sc, cudaStream_t st) {
-  constexpr int BN = 64, STAGES = 8;
+template <int STAGES>
+cudaError_t launch_tc_ln_s(const bf16* A, int lda, const bf16* W, int M, int N, int K, const Epi& e,
+                           const TcScratch& sc, cudaStream_t st) {
+  constexpr int BN = 64;
   CUtensorMap ta, tb;
   cudaError_t r = make_map(&ta, A, M, K, lda, TC_BM);
   if (r != cudaSuccess) return r;
@@ -979,6 +992,16 @@ cudaError_t launch_tc_ln(const bf16* A, int lda, const bf16* W, int M, int N, in
   CK_LAUNCH(cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, STAGES>, ta, tb, M, N, K, e, sc.err, (float*)nullptr,
                                (int*)nullptr));
   return cudaGetLastError();
+}
+
+// With programmatic dependent launch the single-wave GEMMs run with half
+// the operand ring (96 KB of shared memory), so that a CTA of the next
+// kernel fits on the same SM and starts its set-up and weight loads while
+// this one finishes.
+cudaError_t launch_tc_ln(const bf16* A, int lda, const bf16* W, int M, int N, int K, const Epi& e,
+                         const TcScratch& sc, cudaStream_t st) {
+  if (g_launch_pdl) return launch_tc_ln_s<4>(A, lda, W, M, N, K, e, sc, st);
+  return launch_tc_ln_s<8>(A, lda, W, M, N, K, e, sc, st);
 }
 
 template <int BN, int STAGES>
@@ -1116,6 +1139,13 @@ cudaError_t gemm_bf16_tc(const bf16* A, int lda, const bf16* W, int M, int N, in
     if (N >= 256) return launch_tcp<256, 3>(A, lda, W, M, N, K, e, sc, st);
     return launch_tcp<128, 4>(A, lda, W, M, N, K, e, sc, st);
   }
+  if (g_launch_pdl) {   // lean rings: two CTAs per SM (see launch_tc_ln)
+    switch (bn) {
+      case 256: return launch_tc<256, 4>(A, lda, W, M, N, K, sp, e, sc, st);
+      case 128: return launch_tc<128, 3>(A, lda, W, M, N, K, sp, e, sc, st);
+      default: return launch_tc<64, 4>(A, lda, W, M, N, K, sp, e, sc, st);
+    }
+  }
   switch (bn) {
     case 256: return launch_tc<256, 4>(A, lda, W, M, N, K, sp, e, sc, st);
     case 128: return launch_tc<128, 6>(A, lda, W, M, N, K, sp, e, sc, st);
@@ -1155,6 +1185,10 @@ cudaError_t gemm_tc_init_attributes() {
     r = cudaFuncSetAttribute(gemm_tc_kernel<128, 6>, cudaFuncAttributeMaxDynamicSharedMemorySize, TcCfg<128, 6>::SMEM);
   if (r == cudaSuccess)
     r = cudaFuncSetAttribute(gemm_tc_kernel<64, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, TcCfg<64, 8>::SMEM);
+  if (r == cudaSuccess)
+    r = cudaFuncSetAttribute(gemm_tc_kernel<128, 3>, cudaFuncAttributeMaxDynamicSharedMemorySize, TcCfg<128, 3>::SMEM);
+  if (r == cudaSuccess)
+    r = cudaFuncSetAttribute(gemm_tc_kernel<64, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, TcCfg<64, 4>::SMEM);
   if (r != cudaSuccess) return r;
   for (int n = 1; n <= 8; ++n) {   // clusters of n CTAs for the LayerNorm-fused epilogue
     cudaLaunchConfig_t cfg = {};

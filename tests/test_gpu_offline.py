@@ -278,3 +278,27 @@ def test_bad_arguments_rejected(eng_fp32):
     audio = to_dev(np.zeros((1, 4000), np.float32))
     with pytest.raises(b.SFError, match="SF_EINVAL"):
         b.sf_forward_offline(eng_fp32, audio, np.array([4001]), probs)       # length > buffer
+
+
+def test_offline_forward_programmatic_launch_is_bitwise_equal():
+    """With programmatic dependent launch (SF_OPT_PDL = 1) each GEMM loads
+    its first weight tiles before waiting for the previous kernel, and the
+    single-wave GEMMs run with half the operand ring so that two CTAs fit on
+    an SM; the arithmetic is unchanged, so the bf16 forward is bitwise equal
+    to the one with plain stream ordering (full model, 90 s clip)."""
+    w = full_weights(xavier=True)
+    eng = make_engine(w, 1, 17, 18, max_batch=1)
+    try:
+        audio, lens, _ = clip_for_config(1)
+        outs = []
+        for pdl in (0, 1, 0, 1):
+            b.sf_set_option(eng, b.SF_OPT_PDL, pdl)
+            probs = torch.full((1, 1125, 4), float("nan"), device="cuda")
+            b.sf_forward_offline(eng, to_dev(audio), lens, probs)
+            b.sf_check(eng)
+            outs.append(probs.cpu().numpy())
+    finally:
+        b.sf_destroy(eng)
+    assert np.all(np.isfinite(outs[1]))
+    for o in outs[1:]:
+        assert np.array_equal(o, outs[0])
