@@ -390,6 +390,11 @@ enum {
                              residual projection before it wherever the projection's 64-column
                              tiles of a 128-row block fit one CTA cluster and all row blocks
                              one wave; 0 separate LayerNorm kernels */
+  SF_OPT_TF_FUSE = 9,     /* bf16 engines, Transformer layers: 1 (default) everything after each
+                             layer's attention (output projection, LN1, FFN, LN2 and the next
+                             layer's Q|K|V projection) in one kernel per layer, a cluster of four
+                             CTAs per 128-row block, when one wave of clusters covers the rows; 2
+                             that kernel for any number of rows; 0 separate projections */
   SF_OPT_SUB_PATH = 7     /* ConvSubsampling's first two stages: 1 (default) one kernel that
                              computes the first conv's outputs on chip and feeds them straight
                              into the first depthwise conv; 0 the 3x3 s2 conv and the first
@@ -493,7 +498,7 @@ typedef struct {
  * the kernel classes whose bit is set in `mask` (bit k = the k-th class in
  * the order mel, conv1, dwconv3x3s2, gemm, attention_relpos, attention_mha,
  * layernorm, dwconv1d, head_out, assemble, extract, state_update, to_f32,
- * select_topk); enable = 0 stops recording. */
+ * select_topk, tf_layer); enable = 0 stops recording. */
 SF_API sf_status sf_profile_enable(sf_engine* e, int enable);
 /* Synchronise on the recorded events and report one entry per kernel class
  * with at least one launch since the last reset (at most `max` entries,

@@ -20,6 +20,7 @@ SF_FP32, SF_BF16 = 0, 1
 SF_OPT_GRAPHS, SF_OPT_PDL, SF_OPT_GEMM_PATH, SF_OPT_GEMM_PAIR_BN, SF_OPT_ATTN_PATH, SF_OPT_MEL_PATH = 1, 2, 3, 4, 5, 6
 SF_OPT_SUB_PATH = 7
 SF_OPT_LN_FUSE = 8
+SF_OPT_TF_FUSE = 9
 STATUS = {0: "SF_OK", 1: "SF_EINVAL", 2: "SF_ESHAPE", 3: "SF_ENOMEM", 4: "SF_ECUDA", 5: "SF_ESTATE",
           6: "SF_ETIMEOUT", 7: "SF_EDEVICE", 8: "SF_EFORMAT"}
 

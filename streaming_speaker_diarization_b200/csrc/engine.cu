@@ -138,11 +138,11 @@ constexpr size_t SPLIT_WS_BYTES = (size_t)40 << 20;
 constexpr int SPLIT_CNT = 1 << 16;
 enum KClass : int {
   K_MEL = 0, K_CONV1, K_DW2D, K_GEMM, K_ATT_REL, K_ATT_MHA, K_LN, K_DW1D, K_HEAD, K_ASSEMBLE, K_EXTRACT,
-  K_UPDATE, K_TOF32, K_SELECT, K_COUNT
+  K_UPDATE, K_TOF32, K_SELECT, K_TFL, K_COUNT
 };
 const char* const KNAMES[K_COUNT] = {"mel", "conv1", "dwconv3x3s2", "gemm", "attention_relpos", "attention_mha",
                                      "layernorm", "dwconv1d", "head_out", "assemble", "extract", "state_update",
-                                     "to_f32", "select_topk"};
+                                     "to_f32", "select_topk", "tf_layer"};
 struct ProfRec {
   int cls;
   cudaEvent_t a, b;
@@ -171,6 +171,8 @@ struct sf_engine {
   int mel_path = MEL_DEFAULT_PATH;   // front-end: 1 = register FFT + all-SM normalisation, 0 = shared-memory FFT
   int sub_path = 1;       // subsampling: 1 = conv1 fused into the first depthwise, 0 = conv1 and depthwise kernels
   int ln_fuse = 1;        // bf16: LayerNorm fused into the residual projections' epilogue where it fits
+  int tf_fuse = 1;        // bf16 Transformer layers after the attention: 1 fused where one wave covers the rows,
+                          // 2 fused always, 0 separate projections and LayerNorms
   float* d_split_ws = nullptr;   // split-K partial tiles of the tcgen05 GEMM
   int* d_split_cnt = nullptr;    // their per-tile arrival counters (kept at zero between launches)
   TcScratch tc_scratch() const { return TcScratch{d_err, d_split_ws, SPLIT_WS_BYTES, d_split_cnt, SPLIT_CNT}; }
@@ -723,7 +725,7 @@ cudaError_t run_graph(sf_engine* e, std::string key, cudaStream_t st, F&& enqueu
   key += e->prof ? "|p" + std::to_string(e->prof_mask) : "|n";
   key += e->use_pdl ? "|pdl" : "";
   key += "|g" + std::to_string(e->gemm_path) + "." + std::to_string(e->pair_bn) + "|a" + std::to_string(e->attn_path) +
-         "|m" + std::to_string(e->mel_path) + "|s" + std::to_string(e->sub_path) + "|n" + std::to_string(e->ln_fuse);
+         "|m" + std::to_string(e->mel_path) + "|s" + std::to_string(e->sub_path) + "|n" + std::to_string(e->ln_fuse) + "|t" + std::to_string(e->tf_fuse);
   auto it = e->graphs.find(key);
   if (it != e->graphs.end() && it->second.gen != e->ws_gen) {
     cudaGraphExecDestroy(it->second.exec);
@@ -910,6 +912,28 @@ cudaError_t run_encode(sf_engine* e, int M, int n_tiles, float* probs, cudaStrea
     ep.ldo2 = E;
     CK(gemm_acc<T>(e, h, D, W.proj_w, M, E, D, ep, st));
   }
+  if (sizeof(T) == 2 && e->gemm_path >= 1 && c.n_transformer > 0 && E == 192 && c.tf_ff == 768 &&
+      (e->tf_fuse == 2 || (e->tf_fuse == 1 && M <= tf_layer_max_rows()))) {
+    // fused layers: layer 0's Q|K|V projection, then per layer the attention
+    // and one kernel for the rest of the layer and the next layer's Q|K|V
+    auto tfw = [&](int l) {
+      const TfW<T>& w = W.tf[l];
+      return TfLayerW{reinterpret_cast<const bf16*>(w.wqkv), reinterpret_cast<const bf16*>(w.wo),
+                      reinterpret_cast<const bf16*>(w.w1), reinterpret_cast<const bf16*>(w.w2), w.bqkv, w.bo,
+                      w.ln1_g, w.ln1_b, w.b1, w.b2, w.ln2_g, w.ln2_b};
+    };
+    CK(gemm_acc<T>(e, h2, E, W.tf[0].wqkv, M, 3 * E, E, epi(EPI_BIAS, W.tf[0].bqkv, big, 3 * E), st));
+    for (int l = 0; l < c.n_transformer; ++l) {
+      const bool next = l + 1 < c.n_transformer;
+      RUN(K_ATT_MHA, 1, 4.0 * e->att_s2 * E, (double)M * 4 * E * sizeof(T),
+          mha_attention<T>(e, big, ctx, seq, n_tiles, M, st));
+      const TfLayerW cur = tfw(l), nxt = next ? tfw(l + 1) : TfLayerW{};
+      RUN(K_TFL, 1, 2.0 * M * E * (E + 2.0 * c.tf_ff + (next ? 3.0 * E : 0.0)),
+          (double)M * (E * sizeof(T) + 8.0 * E + (next ? 3.0 * E : E) * sizeof(T)),
+          launch_tf_layer(reinterpret_cast<const bf16*>(ctx), cur, next ? &nxt : nullptr, x2,
+                          reinterpret_cast<bf16*>(big), reinterpret_cast<bf16*>(h2), M, e->d_err, st));
+    }
+  } else {
   for (int l = 0; l < c.n_transformer; ++l) {
     const TfW<T>& w = W.tf[l];
     CK(gemm_acc<T>(e, h2, E, w.wqkv, M, 3 * E, E, epi(EPI_BIAS, w.bqkv, big, 3 * E), st));
@@ -917,6 +941,7 @@ cudaError_t run_encode(sf_engine* e, int M, int n_tiles, float* probs, cudaStrea
     CK(resid_ln<T>(e, ctx, E, w.wo, M, E, E, w.bo, 1.f, x2, w.ln1_g, w.ln1_b, true, h2, st));
     CK(gemm_acc<T>(e, h2, E, w.w1, M, c.tf_ff, E, epi(EPI_BIAS_RELU, w.b1, big, c.tf_ff), st));
     CK(resid_ln<T>(e, big, c.tf_ff, w.w2, M, E, c.tf_ff, w.b2, 1.f, x2, w.ln2_g, w.ln2_b, true, h2, st));
+  }
   }
   CK(gemm_acc<T>(e, h2, E, W.head_w1, M, E, E, epi(EPI_BIAS_RELU, W.head_b1, ctx, E), st));
   RUN(K_HEAD, 1, 2.0 * M * E * 4, (double)M * (E * sizeof(T) + 16), launch_head_out<T>(ctx, W.head_w2, W.head_b2, probs, M, E, st));
@@ -1100,6 +1125,7 @@ sf_status sf_create(const void* blob, uint64_t nbytes, const sf_config* cfg, sf_
   if ((ce = attention_mha_tc_init_attributes()) != cudaSuccess) return SF_ECUDA;
   if ((ce = gemm_tc_init_attributes()) != cudaSuccess) return SF_ECUDA;
   if ((ce = frontend_init_attributes()) != cudaSuccess) return SF_ECUDA;
+  if ((ce = tf_layer_init_attributes()) != cudaSuccess) return SF_ECUDA;
   if (cfg->precision == SF_FP32 && (ce = attention_reserve_f32(e->R)) != cudaSuccess) return SF_ECUDA;
   g_ws_gen = &e->ws_gen;
   std::unordered_map<std::string, TensorRef> m;
@@ -1477,6 +1503,10 @@ sf_status sf_set_option(sf_engine* e, int option, int value) {
     case SF_OPT_LN_FUSE:
       if (value != 0 && value != 1) return fail(e, SF_EINVAL, "LayerNorm fusion must be 0 or 1");
       e->ln_fuse = value;
+      break;
+    case SF_OPT_TF_FUSE:
+      if (value < 0 || value > 2) return fail(e, SF_EINVAL, "Transformer layer fusion must be 0, 1 or 2");
+      e->tf_fuse = value;
       break;
     case SF_OPT_GEMM_PAIR_BN:
       if (value != 0 && value != 128 && value != 192 && value != 256)

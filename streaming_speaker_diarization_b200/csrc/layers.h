@@ -176,4 +176,26 @@ cudaError_t launch_mha_tc(const bf16* qkv, bf16* ctx, const SeqTable* seq, int n
                           int* err, cudaStream_t st);
 cudaError_t attention_mha_tc_init_attributes();
 
+// ------------------------------------------------- fused Transformer layer
+// One post-LN Transformer layer after its attention (d 192, FFN 768 ReLU):
+// x <- LN1(x + ctx Wo^T + bo); x <- LN2(x + relu(x W1^T + b1) W2^T + b2);
+// then qkv <- x Wqkv'^T + bqkv' of the next layer (next given) or h <- bf16(x).
+// One cluster of four CTAs per 128-row block (tcgen05 products, LayerNorm
+// statistics and FFN partial sums exchanged in distributed shared memory).
+struct TfLayerW {
+  const bf16 *wqkv, *wo, *w1, *w2;   // [576 x 192], [192 x 192], [768 x 192], [192 x 768]
+  const float *bqkv, *bo, *ln1_g, *ln1_b, *b1, *b2, *ln2_g, *ln2_b;
+};
+struct TfLayerArgs {
+  float* x;
+  const float *bo, *ln1_g, *ln1_b, *b1, *b2, *ln2_g, *ln2_b, *bq;
+  bf16* qkv;
+  bf16* h;
+};
+cudaError_t launch_tf_layer(const bf16* ctx, const TfLayerW& w, const TfLayerW* next, float* x, bf16* qkv, bf16* h,
+                            int M, int* err, cudaStream_t st);
+// Rows the fused layer covers in one wave (co-resident clusters x 128).
+int tf_layer_max_rows();
+cudaError_t tf_layer_init_attributes();
+
 }  // namespace sf

@@ -302,3 +302,35 @@ def test_offline_forward_programmatic_launch_is_bitwise_equal():
     assert np.all(np.isfinite(outs[1]))
     for o in outs[1:]:
         assert np.array_equal(o, outs[0])
+
+
+@pytest.mark.parametrize("lens_s,force", [([9.0, 4.1, 0.3], 1), ([60.0] * 6 + [41.3, 7.7], 2)])
+def test_fused_transformer_layer_vs_unfused_and_oracle(lens_s, force):
+    """The Transformer layers with everything after the attention in one
+    kernel (cluster of four CTAs per 128-row block) against the separate
+    projections and LayerNorms (same bf16 operands: within 1e-2) and against
+    the oracle (2e-2), on a ragged batch whose 128-row blocks straddle
+    sequences; the second case has 5,112 rows (more clusters than one wave,
+    SF_OPT_TF_FUSE = 2)."""
+    w = tiny_weights(xavier=True)
+    audio, lens, _ = synth_batch(87, lens_s)
+    B = len(lens_s)
+    eng = make_engine(w, 1, 2, 2, max_batch=B)
+    try:
+        Tp = int(O.encoder_frames(audio.shape[1] // 160))
+        outs = []
+        for fuse in (force, 0):
+            b.sf_set_option(eng, b.SF_OPT_TF_FUSE, fuse)
+            p = torch.full((B, Tp, 4), float("nan"), device="cuda")
+            b.sf_forward_offline(eng, to_dev(audio), lens, p)
+            b.sf_check(eng)
+            outs.append(p.cpu().numpy())
+    finally:
+        b.sf_destroy(eng)
+    T = np.array([int(O.encoder_frames(int(n) // 160)) for n in lens])
+    for i in range(B):
+        assert np.all(outs[0][i, T[i]:] == 0)
+    assert np.max(np.abs(outs[0] - outs[1])) <= 1e-2
+    for i in (0, B - 1):
+        ref, tp = O.forward_offline(audio[i:i + 1, :lens[i]], lens[i:i + 1], w)
+        assert np.max(np.abs(outs[0][i, :T[i]] - ref[0])) <= 2e-2, i
