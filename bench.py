@@ -239,7 +239,17 @@ STREAM_WORKLOADS = [
 ]
 
 
-def streaming_bench(b, torch, eng_blob, rank, world, local, mel_path=1, sub_path=1, attn_path=1, clocks_dir=None):
+def set_options(b, eng, args):
+    """The kernel-selection options of the command line on one engine."""
+    b.sf_set_option(eng, b.SF_OPT_PDL, args.pdl)
+    b.sf_set_option(eng, b.SF_OPT_MEL_PATH, args.mel_path)
+    b.sf_set_option(eng, b.SF_OPT_SUB_PATH, args.sub_path)
+    b.sf_set_option(eng, b.SF_OPT_ATTN_PATH, args.attn_path)
+    b.sf_set_option(eng, b.SF_OPT_TF_FUSE, args.tf_fuse)
+    b.sf_set_option(eng, b.SF_OPT_LN_FUSE, args.ln_fuse)
+
+
+def streaming_bench(b, torch, eng_blob, rank, world, local, args, clocks_dir=None):
     """Streaming throughput: front-end over each stream's clip, then every
     step of every stream (pre_encode on the new window, encoder on
     [cache | FIFO | chunk], state update) until all streams finish.  A first
@@ -258,9 +268,7 @@ def streaming_bench(b, torch, eng_blob, rank, world, local, mel_path=1, sub_path
         audio_np, lens, _ = clip_for_config(idx)
         audio_np, lens = np.ascontiguousarray(audio_np[lo:hi]), lens[lo:hi]
         eng = b.sf_create(eng_blob, b.default_config(max_batch=max(n, 1), max_samples=int(audio_np.shape[1])))
-        b.sf_set_option(eng, b.SF_OPT_MEL_PATH, mel_path)
-        b.sf_set_option(eng, b.SF_OPT_SUB_PATH, sub_path)
-        b.sf_set_option(eng, b.SF_OPT_ATTN_PATH, attn_path)
+        set_options(b, eng, args)
         audio = torch.from_numpy(audio_np).cuda()
         T = 1 + audio_np.shape[1] // 160
         mel = torch.empty((n, 128, T), device="cuda")
@@ -374,7 +382,7 @@ def frontend_bench(b, torch, blob, steps, warmup, mel_path=1):
                          "frac": gbs / pk["hbm_gbs"], "bytes_per_call": alg, "peak_kind": f"{kind} copy"}}
 
 
-def batch_bench(b, torch, blob, steps, warmup, local, mel_path=1, sub_path=1, attn_path=1, clocks_dir=None):
+def batch_bench(b, torch, blob, steps, warmup, local, args, clocks_dir=None):
     """The variable-length offline batch: 32 clips of 5-120 s (seeded),
     padded to the longest, one sf_forward_offline call per step (front-end
     to probabilities).  Audio resident on the device, L2 flushed between
@@ -383,9 +391,7 @@ def batch_bench(b, torch, blob, steps, warmup, local, mel_path=1, sub_path=1, at
     audio_np, lens, _ = clip_for_config(4)
     B, n_max = audio_np.shape
     eng = b.sf_create(blob, b.default_config(max_batch=B, max_samples=int(n_max)))
-    b.sf_set_option(eng, b.SF_OPT_MEL_PATH, mel_path)
-    b.sf_set_option(eng, b.SF_OPT_SUB_PATH, sub_path)
-    b.sf_set_option(eng, b.SF_OPT_ATTN_PATH, attn_path)
+    set_options(b, eng, args)
     try:
         audio = torch.from_numpy(audio_np).cuda()
         Tp = 1 + (n_max // 160 - 1) // 8
@@ -515,14 +521,17 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--pdl", type=int, default=0, help="programmatic dependent launch between kernels (0/1)")
+    ap.add_argument("--pdl", type=int, default=1, help="programmatic dependent launch between kernels (0/1)")
     ap.add_argument("--no-streaming", action="store_true", help="skip the streaming workloads")
     ap.add_argument("--no-frontend", action="store_true", help="skip the 1 h front-end-only run")
     ap.add_argument("--no-batch", action="store_true", help="skip the 32-clip variable-length batch")
     ap.add_argument("--mel-path", type=int, default=1, choices=[0, 1], help="front-end implementation (SF_OPT_MEL_PATH)")
-    ap.add_argument("--attn-path", type=int, default=1, choices=[0, 1, 2], help="attention kernels (SF_OPT_ATTN_PATH)")
+    ap.add_argument("--attn-path", type=int, default=1, choices=[0, 1], help="attention kernels (SF_OPT_ATTN_PATH)")
     ap.add_argument("--sub-path", type=int, default=1, choices=[0, 1],
                     help="subsampling conv1 + first depthwise implementation (SF_OPT_SUB_PATH)")
+    ap.add_argument("--tf-fuse", type=int, default=1, choices=[0, 1, 2],
+                    help="fused Transformer layers (SF_OPT_TF_FUSE: 1 where one wave covers the rows, 2 always)")
+    ap.add_argument("--ln-fuse", type=int, default=1, choices=[0, 1], help="LayerNorm in the residual epilogue")
     ap.add_argument("--clocks-dir", default=None, help="where to keep the raw nvidia-smi clock samples")
     ap.add_argument("--oracle-subsets", action="store_true",
                     help="with --impl reference: also time the oracle on declared subsets of every workload")
@@ -545,10 +554,7 @@ def main():
     audio_np, lens, _ = clip_for_config(1)
     w = make_weights(FULL, seed=0)
     eng = b.sf_create(weights_blob(w), b.default_config(max_batch=1))
-    b.sf_set_option(eng, b.SF_OPT_PDL, args.pdl)
-    b.sf_set_option(eng, b.SF_OPT_MEL_PATH, args.mel_path)
-    b.sf_set_option(eng, b.SF_OPT_SUB_PATH, args.sub_path)
-    b.sf_set_option(eng, b.SF_OPT_ATTN_PATH, args.attn_path)
+    set_options(b, eng, args)
     st = torch.cuda.current_stream()
     audio = torch.from_numpy(audio_np).cuda()
     probs = torch.zeros((1, 1125, 4), device="cuda")
@@ -636,7 +642,7 @@ def main():
             "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": dict(CONFIG, parallelism=f"replicas x{world}", mel_path=args.mel_path, sub_path=args.sub_path,
-                           attn_path=args.attn_path),
+                           attn_path=args.attn_path, tf_fuse=args.tf_fuse, ln_fuse=args.ln_fuse, pdl=args.pdl),
             "roofline": roof, "clocks": clocks, "gpu_launches": launches,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(audio_np.nbytes),
                     "d2h_bytes_per_step": int(h_probs.numel() * 4)},
@@ -644,11 +650,10 @@ def main():
             "kernels": kernels}
     b.sf_destroy(eng)
     if not args.no_streaming:
-        line["streaming"] = streaming_bench(b, torch, weights_blob(w), rank, world, local, args.mel_path,
-                                            args.sub_path, args.attn_path, args.clocks_dir)
+        line["streaming"] = streaming_bench(b, torch, weights_blob(w), rank, world, local, args, args.clocks_dir)
     if not args.no_batch and world == 1:
-        line["batch"] = batch_bench(b, torch, weights_blob(w), args.steps, max(args.warmup, 3), local, args.mel_path,
-                                    args.sub_path, args.attn_path, args.clocks_dir)
+        line["batch"] = batch_bench(b, torch, weights_blob(w), args.steps, max(args.warmup, 3), local, args,
+                                    args.clocks_dir)
     if not args.no_frontend:
         line["frontend_1h"] = frontend_bench(b, torch, weights_blob(w), max(args.steps, 5), max(args.warmup, 3),
                                              args.mel_path)

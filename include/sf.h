@@ -369,7 +369,10 @@ SF_API sf_status sf_segments(sf_engine* e, const float* d_probs, int stride_t, c
 enum {
   SF_OPT_GRAPHS = 1,     /* 1 (default): capture each call shape once as a CUDA graph and
                             replay it; 0: launch kernel by kernel */
-  SF_OPT_PDL = 2,        /* 1: programmatic dependent launch between kernels; 0 (default) */
+  SF_OPT_PDL = 2,        /* 1 (default): programmatic dependent launch between kernels (each
+                            kernel may start its set-up and weight loads while its predecessor
+                            finishes; single-wave GEMMs then use half the operand ring so two
+                            CTAs share an SM); 0 plain stream order (same results to the bit) */
   SF_OPT_GEMM_PATH = 3,  /* bf16 projections on the tcgen05/TMEM/TMA kernels: 1 (default) with
                             multi-wave projections of K >= 1024 and width >= 256 on CTA
                             pairs (tcgen05 cta_group::2, 256-row tiles), 2 every multi-wave
@@ -379,9 +382,7 @@ enum {
                               or 128, 192, 256 */
   SF_OPT_ATTN_PATH = 5,   /* bf16 attention (relative-position and Transformer): 1 (default)
                              tcgen05/TMEM/TMA kernels, whose keys are split over CTA clusters
-                             when one sequence leaves SMs idle; 0 mma.sync kernels; 2 the
-                             tcgen05 relative-position kernel with the Transformer's on
-                             mma.sync, each CTA's keys split over four warp groups */
+                             when one sequence leaves SMs idle; 0 mma.sync kernels */
   SF_OPT_MEL_PATH = 6,    /* log-mel front-end (sf_mel, the offline forward, the audio-in
                              step): 1 (default) FFT in registers with warp shuffles, then
                              separate statistics and normalisation passes over all SMs; 0 FFT
@@ -472,8 +473,8 @@ SF_API sf_status sf_attention_relpos(sf_engine* e, const void* d_qkv, const void
  *                         24h .. 24h + 23 of each part
  *   d_ctx bf16 [M x 192] (out)  softmax_j(q_i . k_j / sqrt(24)) v_j
  * Sequence lengths in [1, the engine's longest sequence]; path 1 = tcgen05
- * kernel, 0 = mma.sync (two key groups per CTA), 2 = mma.sync with four key
- * groups per CTA.  Pointers 16-byte aligned.  Uses the engine's
+ * kernel (keys split over CTA clusters when the (query tile, head) units
+ * leave SMs idle), 0 = mma.sync.  Pointers 16-byte aligned.  Uses the engine's
  * descriptor block (ordered on `cuda_stream` with its other calls). */
 SF_API sf_status sf_attention_mha(sf_engine* e, const void* d_qkv, const int* h_seq_len, int n, void* d_ctx, int path,
                                   void* cuda_stream);

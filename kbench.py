@@ -11,8 +11,7 @@
 swish, 5 gated linear unit; P: SF_OPT_GEMM_PATH, 1 = tcgen05 with CTA pairs
 where faster, 2 = CTA pairs always, 3 = single CTAs, 0 = mma.sync); `attn`
 runs sf_attention_relpos and `mha` sf_attention_mha on N_SEQ packed
-sequences of LEN rows (P: 1 tcgen05, 0 mma.sync; `mha` also 2, mma.sync
-with four key groups per CTA); `mel` runs sf_mel on B
+sequences of LEN rows (P: 1 tcgen05, 0 mma.sync); `mel` runs sf_mel on B
 clips of SECONDS of audio each (P: SF_OPT_MEL_PATH); `ln` runs
 sf_gemm_bf16_ln, the residual projection with the LayerNorm after it fused
 into the epilogue (X: 1 = the residual stream receives the normalised row;

@@ -430,16 +430,6 @@ cudaError_t launch_mha<bf16>(const bf16* qkv, bf16* ctx, const SeqTable* seq, in
   return cudaGetLastError();
 }
 
-// Transformer MHSA with four warp groups (512 threads) splitting each CTA's
-// keys four ways instead of two: a shorter per-CTA chain for one long
-// sequence, where the 64-row CTAs are about one wave.
-cudaError_t launch_mha_bf16_4g(const bf16* qkv, bf16* ctx, const SeqTable* seq, int n_tiles, int M, cudaStream_t st) {
-  if (M <= 0) return cudaSuccess;
-  CK_LAUNCH(launch_k(attn_bf16_kernel<24, 32, false, 4>, dim3(dim3(n_tiles, 8)), dim3(512),
-                     AttCfg<24, 32, false, 4>::SMEM, st, qkv, 192, nullptr, 0, nullptr, nullptr, ctx, seq));
-  return cudaGetLastError();
-}
-
 // fp32 path: one score row of up to R floats per warp (4 warps per CTA).
 // The shared-memory limit is a per-kernel attribute of the process, so it
 // only ever grows: an engine made for shorter sequences never lowers what
@@ -464,11 +454,8 @@ cudaError_t attention_init_attributes() {
   cudaError_t e = cudaFuncSetAttribute(attn_bf16_kernel<64, 64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        AttCfg<64, 64, true>::SMEM);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(attn_bf16_kernel<24, 32, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           AttCfg<24, 32, false>::SMEM);
-  if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(attn_bf16_kernel<24, 32, false, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              AttCfg<24, 32, false, 4>::SMEM);
+  return cudaFuncSetAttribute(attn_bf16_kernel<24, 32, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              AttCfg<24, 32, false>::SMEM);
 }
 
 }  // namespace sf

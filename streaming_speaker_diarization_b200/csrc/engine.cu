@@ -193,7 +193,7 @@ struct sf_engine {
   double ms_acc[K_COUNT] = {};   // event time already read back (graph replays)
   // CUDA graphs: one per launch shape, replayed; invalidated when the workspace moves
   bool use_graphs = true;
-  int use_pdl = 0;
+  int use_pdl = 1;         // programmatic dependent launch (measured 4.5 % faster offline; bitwise equal)
   bool capturing = false;
   cudaStream_t cap_stream = nullptr;     // graphs are captured here, launched on the caller's stream
   std::vector<cudaEvent_t> cap_events;   // events created for the graph being captured
@@ -593,7 +593,7 @@ cudaError_t gemm_dispatch<bf16>(sf_engine* e, const bf16* A, int lda, const bf16
 // Transformer MHSA in the bf16 engine: the tcgen05 kernel (SF_OPT_ATTN_PATH
 // 1, the default), which splits each (query tile, head) unit's keys over a
 // CTA cluster when the units alone leave SMs idle (one long clip); the
-// mma.sync kernels with two (path 0) or four (path 2) key groups per CTA.
+// mma.sync kernel (path 0).
 template <typename T>
 cudaError_t mha_attention(sf_engine* e, const T* qkv, T* ctx, const SeqTable* seq, int n_tiles, int M, cudaStream_t st) {
   return launch_mha<T>(qkv, ctx, seq, n_tiles, M, e->R, st);
@@ -602,7 +602,6 @@ template <>
 cudaError_t mha_attention<bf16>(sf_engine* e, const bf16* qkv, bf16* ctx, const SeqTable* seq, int n_tiles, int M,
                                 cudaStream_t st) {
   if (e->attn_path == 1) return launch_mha_tc(qkv, ctx, seq, e->att_tiles2, M, e->att_max_len, e->d_err, st);
-  if (e->attn_path == 2) return launch_mha_bf16_4g(qkv, ctx, seq, n_tiles, M, st);
   return launch_mha<bf16>(qkv, ctx, seq, n_tiles, M, e->R, st);
 }
 
@@ -616,7 +615,7 @@ cudaError_t relpos_attention(sf_engine* e, const T* qkv, const T* ptab, const fl
 template <>
 cudaError_t relpos_attention<bf16>(sf_engine* e, const bf16* qkv, const bf16* ptab, const float* pu, const float* pv,
                                    bf16* ctx, const SeqTable* seq, int n_tiles, int M, cudaStream_t st) {
-  if (e->attn_path >= 1)
+  if (e->attn_path == 1)
     return launch_relpos_attention_tc(qkv, ptab, e->R, pu, pv, ctx, seq, e->att_tiles2, M, e->att_max_len,
                                       e->tc_scratch(), st);
   return launch_relpos_attention<bf16>(qkv, ptab, e->R, pu, pv, ctx, seq, n_tiles, M, st);
@@ -1428,7 +1427,7 @@ sf_status sf_attention_mha(sf_engine* e, const void* d_qkv, const int* h_seq_len
   if (check_engine(e) != SF_OK) return SF_EINVAL;
   if (!d_qkv || !h_seq_len || !d_ctx) return fail(e, SF_EINVAL, "null pointer argument");
   if (e->cfg.precision != SF_BF16) return fail(e, SF_ESTATE, "sf_attention_mha needs a bf16 engine");
-  if (n < 1 || n > MAX_SEQ || path < 0 || path > 2) return fail(e, SF_ESHAPE, "sequence count or path");
+  if (n < 1 || n > MAX_SEQ || path < 0 || path > 1) return fail(e, SF_ESHAPE, "sequence count or path");
   if ((reinterpret_cast<uintptr_t>(d_qkv) | reinterpret_cast<uintptr_t>(d_ctx)) & 15)
     return fail(e, SF_EINVAL, "qkv and ctx must be 16-byte aligned");
   std::vector<int> lens(h_seq_len, h_seq_len + n);
@@ -1445,7 +1444,6 @@ sf_status sf_attention_mha(sf_engine* e, const void* d_qkv, const int* h_seq_len
   if (ce == cudaSuccess)
     ce = path == 1   ? launch_mha_tc(qkv, ctx, &e->d_desc->seq, tiles2, M, *std::max_element(lens.begin(), lens.end()),
                                      e->d_err, st)
-         : path == 2 ? launch_mha_bf16_4g(qkv, ctx, &e->d_desc->seq, tiles, M, st)
                      : launch_mha<bf16>(qkv, ctx, &e->d_desc->seq, tiles, M, e->max_seq_len, st);
   if (ce != cudaSuccess) return cuda_fail(e, ce, "sf_attention_mha");
   return SF_OK;
@@ -1489,7 +1487,7 @@ sf_status sf_set_option(sf_engine* e, int option, int value) {
       e->gemm_path = value;
       break;
     case SF_OPT_ATTN_PATH:
-      if (value < 0 || value > 2) return fail(e, SF_EINVAL, "attention path must be 0, 1 or 2");
+      if (value != 0 && value != 1) return fail(e, SF_EINVAL, "attention path must be 0 or 1");
       e->attn_path = value;
       break;
     case SF_OPT_MEL_PATH:

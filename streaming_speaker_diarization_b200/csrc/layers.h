@@ -156,8 +156,6 @@ cudaError_t launch_relpos_attention(const T* qkv, const T* ptab, int R, const fl
 template <typename T>
 cudaError_t launch_mha(const T* qkv, T* ctx, const SeqTable* seq, int n_tiles, int M, int R, cudaStream_t st);
 cudaError_t attention_init_attributes();
-// The bf16 Transformer MHSA with four key groups per CTA (512 threads).
-cudaError_t launch_mha_bf16_4g(const bf16* qkv, bf16* ctx, const SeqTable* seq, int n_tiles, int M, cudaStream_t st);
 // bf16 relative-position MHSA on tcgen05 (one CTA per 128 query rows x head
 // x key split; n_tiles2 = 128-row tiles of the sequence table, max_len the
 // longest sequence); with fewer (tile, head) units than SMs each unit's keys

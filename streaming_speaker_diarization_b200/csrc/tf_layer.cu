@@ -49,7 +49,9 @@ struct TlSmem {
   static constexpr int OFF_H = OFF_Y + TL_KB * KB_A;
   static constexpr int OFF_RING = OFF_H + TL_KB * KB_A;
   static constexpr int OFF_ST = OFF_RING + TL_RING * STAGE;   // 2 x 128 float2 statistics
-  static constexpr int OFF_BAR = OFF_ST + 2 * TL_R * 8;
+  static constexpr int OFF_PAR = OFF_ST + 2 * TL_R * 8;      // this rank's biases and LayerNorm weights
+  static constexpr int N_PAR = 5 * TL_EJ + TL_FJ + TL_QJ;     // bo, ln1 g/b, b1, b2, ln2 g/b, bq
+  static constexpr int OFF_BAR = OFF_PAR + N_PAR * 4;
   static constexpr int SMEM = 1024 + OFF_BAR + 256;
   static_assert(SMEM <= 232448, "shared memory per CTA");
   static_assert(TL_E * TL_R * 4 == 2 * TL_KB * KB_A, "F2 partial staging (f32 [192][128]) fills CTX and H");
@@ -295,30 +297,56 @@ __global__ void __launch_bounds__(192, 1) tf_layer_kernel(
     const int q = warp & 3, r = 32 * q + lane, row = m0 + r;
     const bool valid = row < M;
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+    // this rank's slices of the biases and LayerNorm weights, once, into
+    // shared memory (read there by every epilogue below)
+    float* par = reinterpret_cast<float*>(sm + L::OFF_PAR);
+    float* p_bo = par;
+    float* p_g1 = p_bo + TL_EJ;
+    float* p_be1 = p_g1 + TL_EJ;
+    float* p_b2 = p_be1 + TL_EJ;
+    float* p_g2 = p_b2 + TL_EJ;
+    float* p_be2 = p_g2 + TL_EJ;
+    float* p_b1 = p_be2 + TL_EJ;   // TL_FJ
+    float* p_bq = p_b1 + TL_FJ;    // TL_QJ
+    {
+      const int t = threadIdx.x - 64;   // 0 .. 127
+      for (int i = t; i < TL_EJ; i += 128) {
+        p_bo[i] = a.bo[TL_EJ * j + i];
+        p_g1[i] = a.ln1_g[TL_EJ * j + i];
+        p_be1[i] = a.ln1_b[TL_EJ * j + i];
+        p_b2[i] = a.b2[TL_EJ * j + i];
+        p_g2[i] = a.ln2_g[TL_EJ * j + i];
+        p_be2[i] = a.ln2_b[TL_EJ * j + i];
+      }
+      for (int i = t; i < TL_FJ; i += 128) p_b1[i] = a.b1[TL_FJ * j + i];
+      if (has_next)
+        for (int i = t; i < TL_QJ; i += 128) p_bq[i] = a.bq[TL_QJ * j + i];
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+    }
     pdl_wait();   // x and the outputs belong to the previous kernels' stream order
     auto wait_all = [&](uint64_t* bar) -> bool {
       return __all_sync(0xffffffffu, mbar_wait(bar, 0, abort_flag)) && !*abort_flag;
     };
     float y1[TL_EJ];
     // --- E1: O projection + bias + residual, LN1
+    float v[TL_EJ];
+    {   // the residual row is loaded while the O product is computed
+      const float* xr = a.x + (int64_t)row * TL_E + TL_EJ * j;
+#pragma unroll
+      for (int c = 0; c < TL_EJ; c += 4) {
+        const float4 xv = valid ? *reinterpret_cast<const float4*>(xr + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+        v[c] = xv.x; v[c + 1] = xv.y; v[c + 2] = xv.z; v[c + 3] = xv.w;
+      }
+    }
     bool ok = wait_all(o_done);
     {
-      float v[TL_EJ];
       if (ok) {
         tc_fence_after();
         uint32_t u[48];
         tmem_ld32(tmem + lane_base + TM_O, u);
         tmem_ld16(tmem + lane_base + TM_O + 32, u + 32);
-        const float* xr = a.x + (int64_t)row * TL_E + TL_EJ * j;
 #pragma unroll
-        for (int c = 0; c < TL_EJ; c += 4) {
-          const float4 xv = valid ? *reinterpret_cast<const float4*>(xr + c) : make_float4(0.f, 0.f, 0.f, 0.f);
-          const float4 bv = *reinterpret_cast<const float4*>(a.bo + TL_EJ * j + c);
-          v[c] = xv.x + (__uint_as_float(u[c]) + bv.x);
-          v[c + 1] = xv.y + (__uint_as_float(u[c + 1]) + bv.y);
-          v[c + 2] = xv.z + (__uint_as_float(u[c + 2]) + bv.z);
-          v[c + 3] = xv.w + (__uint_as_float(u[c + 3]) + bv.w);
-        }
+        for (int c = 0; c < TL_EJ; ++c) v[c] += __uint_as_float(u[c]) + p_bo[c];
       } else {
 #pragma unroll
         for (int c = 0; c < TL_EJ; ++c) v[c] = 0.f;
@@ -328,14 +356,7 @@ __global__ void __launch_bounds__(192, 1) tf_layer_kernel(
       float mean, rstd;
       tl_row_stats(st1, r, mean, rstd);
 #pragma unroll
-      for (int c = 0; c < TL_EJ; c += 4) {
-        const float4 g = *reinterpret_cast<const float4*>(a.ln1_g + TL_EJ * j + c);
-        const float4 bb = *reinterpret_cast<const float4*>(a.ln1_b + TL_EJ * j + c);
-        y1[c] = (v[c] - mean) * rstd * g.x + bb.x;
-        y1[c + 1] = (v[c + 1] - mean) * rstd * g.y + bb.y;
-        y1[c + 2] = (v[c + 2] - mean) * rstd * g.z + bb.z;
-        y1[c + 3] = (v[c + 3] - mean) * rstd * g.w + bb.w;
-      }
+      for (int c = 0; c < TL_EJ; ++c) y1[c] = (v[c] - mean) * rstd * p_g1[c] + p_be1[c];
       if (!valid || !ok) {
 #pragma unroll
         for (int c = 0; c < TL_EJ; ++c) y1[c] = 0.f;   // rows past M feed zeros to the products
@@ -355,8 +376,8 @@ __global__ void __launch_bounds__(192, 1) tf_layer_kernel(
 #pragma unroll
         for (int g = 0; g < 8; ++g) {
           const int col = c0 + 8 * g;
-          const float4 b0 = *reinterpret_cast<const float4*>(a.b1 + TL_FJ * j + col);
-          const float4 b1 = *reinterpret_cast<const float4*>(a.b1 + TL_FJ * j + col + 4);
+          const float4 b0 = *reinterpret_cast<const float4*>(p_b1 + col);
+          const float4 b1 = *reinterpret_cast<const float4*>(p_b1 + col + 4);
           float h[8] = {__uint_as_float(u[8 * g]) + b0.x,     __uint_as_float(u[8 * g + 1]) + b0.y,
                         __uint_as_float(u[8 * g + 2]) + b0.z, __uint_as_float(u[8 * g + 3]) + b0.w,
                         __uint_as_float(u[8 * g + 4]) + b1.x, __uint_as_float(u[8 * g + 5]) + b1.y,
@@ -393,30 +414,24 @@ __global__ void __launch_bounds__(192, 1) tf_layer_kernel(
     }
     cl_sync();   // C
     {
-      float v[TL_EJ];
 #pragma unroll
       for (int c = 0; c < TL_EJ; ++c) v[c] = 0.f;
       if (ok) {
 #pragma unroll 1
-        for (int rk = 0; rk < TL_C; ++rk) {   // fixed rank order: the sum does not depend on timing
-          float t[TL_EJ];
+        for (int rk = 0; rk < TL_C; rk += 2) {   // fixed rank order: the sum does not depend on timing
+          float t0[TL_EJ], t1[TL_EJ];
 #pragma unroll
-          for (int c = 0; c < TL_EJ; ++c) {   // all of a rank's loads in flight before the sum
+          for (int c = 0; c < TL_EJ; ++c) {   // two ranks' loads in flight before the sums
             const int col = TL_EJ * j + c;
-            const float* p = (col < 96 ? pst_lo + col * TL_R : pst_hi + (col - 96) * TL_R) + r;
-            t[c] = ld_cluster_f32(cl_map(su32(p), (uint32_t)rk));
+            const uint32_t p = su32((col < 96 ? pst_lo + col * TL_R : pst_hi + (col - 96) * TL_R) + r);
+            t0[c] = ld_cluster_f32(cl_map(p, (uint32_t)rk));
+            t1[c] = ld_cluster_f32(cl_map(p, (uint32_t)rk + 1));
           }
 #pragma unroll
-          for (int c = 0; c < TL_EJ; ++c) v[c] += t[c];
+          for (int c = 0; c < TL_EJ; ++c) v[c] = (v[c] + t0[c]) + t1[c];
         }
 #pragma unroll
-        for (int c = 0; c < TL_EJ; c += 4) {
-          const float4 bv = *reinterpret_cast<const float4*>(a.b2 + TL_EJ * j + c);
-          v[c] = y1[c] + (v[c] + bv.x);
-          v[c + 1] = y1[c + 1] + (v[c + 1] + bv.y);
-          v[c + 2] = y1[c + 2] + (v[c + 2] + bv.z);
-          v[c + 3] = y1[c + 3] + (v[c + 3] + bv.w);
-        }
+        for (int c = 0; c < TL_EJ; ++c) v[c] = y1[c] + (v[c] + p_b2[c]);
       }
       st2[r] = tl_local_stats(v);
       cl_sync();   // D
@@ -424,14 +439,7 @@ __global__ void __launch_bounds__(192, 1) tf_layer_kernel(
       tl_row_stats(st2, r, mean, rstd);
       float y2[TL_EJ];
 #pragma unroll
-      for (int c = 0; c < TL_EJ; c += 4) {
-        const float4 g = *reinterpret_cast<const float4*>(a.ln2_g + TL_EJ * j + c);
-        const float4 bb = *reinterpret_cast<const float4*>(a.ln2_b + TL_EJ * j + c);
-        y2[c] = (v[c] - mean) * rstd * g.x + bb.x;
-        y2[c + 1] = (v[c + 1] - mean) * rstd * g.y + bb.y;
-        y2[c + 2] = (v[c + 2] - mean) * rstd * g.z + bb.z;
-        y2[c + 3] = (v[c + 3] - mean) * rstd * g.w + bb.w;
-      }
+      for (int c = 0; c < TL_EJ; ++c) y2[c] = (v[c] - mean) * rstd * p_g2[c] + p_be2[c];
       if (ok && valid) {
         float* xr = a.x + (int64_t)row * TL_E + TL_EJ * j;
 #pragma unroll
@@ -458,7 +466,7 @@ __global__ void __launch_bounds__(192, 1) tf_layer_kernel(
     if (has_next && ok && wait_all(q_done)) {
       tc_fence_after();
       bf16* qr = a.qkv + (int64_t)row * (3 * TL_E) + TL_QJ * j;
-      const float* bq = a.bq + TL_QJ * j;
+      const float* bq = p_bq;
       auto store16 = [&](const uint32_t* uu, int c0) {
         float f[16];
 #pragma unroll
