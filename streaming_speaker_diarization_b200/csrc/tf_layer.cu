@@ -50,7 +50,7 @@ struct TlSmem {
   static constexpr int OFF_RING = OFF_H + TL_KB * KB_A;
   static constexpr int OFF_ST = OFF_RING + TL_RING * STAGE;   // 2 x 128 float2 statistics
   static constexpr int OFF_PAR = OFF_ST + 2 * TL_R * 8;      // this rank's biases and LayerNorm weights
-  static constexpr int N_PAR = 5 * TL_EJ + TL_FJ + TL_QJ;     // bo, ln1 g/b, b1, b2, ln2 g/b, bq
+  static constexpr int N_PAR = 6 * TL_EJ + TL_FJ + TL_QJ;     // bo, ln1 g/b, b2, ln2 g/b (48 each), b1, bq
   static constexpr int OFF_BAR = OFF_PAR + N_PAR * 4;
   static constexpr int SMEM = 1024 + OFF_BAR + 256;
   static_assert(SMEM <= 232448, "shared memory per CTA");
@@ -308,6 +308,7 @@ __global__ void __launch_bounds__(192, 1) tf_layer_kernel(
     float* p_be2 = p_g2 + TL_EJ;
     float* p_b1 = p_be2 + TL_EJ;   // TL_FJ
     float* p_bq = p_b1 + TL_FJ;    // TL_QJ
+    static_assert(6 * TL_EJ + TL_FJ + TL_QJ == L::N_PAR, "parameter block layout");
     {
       const int t = threadIdx.x - 64;   // 0 .. 127
       for (int i = t; i < TL_EJ; i += 128) {
