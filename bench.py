@@ -45,11 +45,11 @@ CONFIG = {"workload": "offline forward, 1 clip x 90 s (16 kHz, 4 speakers, 15% o
 
 
 # DRAM bytes (read + write) per projection launch of the offline forward,
-# from an ncu launch list of this workload (815.3 MB over the 213 GEMM
-# launches of one forward); valid only for the GEMM sources it was taken
-# with, null once they change.
-GEMM_TRAFFIC = {"bytes_per_launch": 815.3e6 / 213,
-                "sources_sha256": "9bad6df933c0cd329728f20224afdde012e864c83a7fc71d246a0dfde6e9963d"}
+# from an ncu launch list of this workload (710.3 MB over the 142 GEMM
+# launches of one forward, the residual + LayerNorm epilogues included);
+# valid only for the GEMM sources it was taken with, null once they change.
+GEMM_TRAFFIC = {"bytes_per_launch": 710.3e6 / 142,
+                "sources_sha256": "96c1fc973e1294bf7a9863b128ac0a4ee3da73af5337d5fd12e044258253cf78"}
 
 
 def gemm_traffic_per_launch():
