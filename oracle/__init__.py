@@ -4,7 +4,7 @@ TEST INFRASTRUCTURE ONLY.  This package is the plain, slow, obviously correct
 statement of what the engine computes, written from the pages (the
 "Streaming Sortformer Diarizer" model description, the NeMo Speaker
 Diarization API and the Transformers "Nemotron 3 Diarization" streaming
-notes).  Only the tests, the smoke check and the benchmark's CPU-baseline leg
+notes), and of the Nemotron-3 variant's offline forward (``nemotron``).  Only the tests, the smoke check and the benchmark's CPU-baseline leg
 may import it; the engine never does, and this package imports nothing from
 the engine.  It shares no code with the CUDA path: only the seeded input
 generators in ``synth`` feed both.
@@ -27,3 +27,5 @@ from .model import (encoder_frames, subsample, rel_pos_table, rel_pos_mhsa, conf
 from .streaming import (Preset, PRESETS, StreamState, compress_scores, select_topk,  # noqa: F401
                         compress_cache, stream_step, stream_run, state_update)
 from .postprocess import SegParams, binarize, speaker_segments, segments  # noqa: F401
+from .nemotron import (stack_frames, rope, rope_mha, nem_layer, nem_head, nem_encode,  # noqa: F401
+                       nem_forward_offline)

@@ -7,3 +7,4 @@ the CUDA path consume what it produces, each with its own implementation.
 """
 from .weights import ModelDims, TINY, FULL, manifest, make_weights, weights_blob  # noqa: F401
 from .audio import synth_clip, synth_batch, clip_for_config  # noqa: F401
+from .nemotron_weights import NemDims, NEM_FULL, NEM_TINY, nem_manifest, make_nem_weights  # noqa: F401
