@@ -506,6 +506,59 @@ SF_API sf_status sf_profile_enable(sf_engine* e, int enable);
  * count in *n_out).  reset = 1 clears the counters afterwards. */
 SF_API sf_status sf_profile_read(sf_engine* e, sf_kernel_stat* out, int max, int* n_out, int reset);
 
+/* ------------------------------------------------ Nemotron-3 variant (offline) */
+
+/* The Nemotron-3 diarization model's offline forward ("Enable
+ * Nemotron-3-Diarization on MLX, CUDA, XNNPACK, and Vulkan", model
+ * description: 16 kHz mono audio, 128-bin mel stacked to 80 ms encoder
+ * frames, a 31-layer Transformer with rotary position embedding, a Conv1D
+ * upsampling head giving up to 8 speakers' activity every 10 ms;
+ * Transformers "Nemotron 3 Diarization": logits (1, frames, 8), one frame
+ * every 10 ms).  The pages give no widths; this engine implements the
+ * readings d_model 512 in 8 heads of 64, FFN 2048 (swish), pre-LN layers and
+ * a final LayerNorm, frame-major stacking of 8 normalised mel frames into a
+ * Linear 1024 -> 512, rotate-half RoPE from each clip's start (base 10000),
+ * and a transposed conv with kernel = stride = 8 (512 -> 8 speakers) and a
+ * sigmoid as the head.  bf16 weights and activations, fp32 accumulation and
+ * residual stream.  Streaming (the arrival-order speaker cache) is not
+ * implemented here. */
+typedef struct sf_nem_engine sf_nem_engine;
+typedef struct {
+  int n_layers;          /* Transformer layers (31; any count >= 1)                  */
+  int d_model;           /* must be 512                                              */
+  int ff;                /* must be 2048                                             */
+  int n_spk;             /* must be 8                                                */
+  int max_batch;         /* clips per call, 1 .. 512                                 */
+  int64_t max_samples;   /* longest clip, 1,600 .. 230,400,000 samples               */
+} sf_nem_config;
+SF_API sf_status sf_nem_default_config(sf_nem_config* out);
+/* Weights: the SFW1 container with tensors nem.stack.weight [512 x 1024],
+ * nem.stack.bias [512], per layer l nem.layers.l.{ln1,ln2}.{weight,bias}
+ * [512], .att.{q,k,v,o}.weight [512 x 512] and .bias [512],
+ * .ff.linear1.weight [2048 x 512], .ff.linear1.bias [2048],
+ * .ff.linear2.weight [512 x 2048], .ff.linear2.bias [512], then
+ * nem.final_ln.{weight,bias} [512], nem.head.weight [512 x 8 x 8]
+ * (in channel, speaker, tap), nem.head.bias [8].  Copies and converts the
+ * weights, allocates the workspace for max_batch clips of max_samples and
+ * synchronises.  Errors: SF_EINVAL (configuration), SF_EDEVICE (not an
+ * sm_100 device), SF_EFORMAT, SF_ENOMEM, SF_ECUDA. */
+SF_API sf_status sf_nem_create(const void* h_blob, uint64_t nbytes, const sf_nem_config* cfg, sf_nem_engine** out);
+/* Synchronises the device and frees the engine. */
+SF_API sf_status sf_nem_destroy(sf_nem_engine* e);
+/* Offline forward of B clips:
+ *   d_audio   f32 [B x n_max]  16 kHz mono, clip b's first h_len[b] samples valid
+ *   h_len     i64 [B]  each in [1600, n_max]
+ *   d_probs   f32 [B x (n_max / 160) x 8] (out)  speaker activity every 10 ms;
+ *             frames at or past a clip's h_len / 160 are written as 0
+ *   h_out_len i64 [B] (out, may be NULL)  h_len / 160
+ * Synchronises on cuda_stream (reads the device error word).  Errors:
+ * SF_EINVAL, SF_ESHAPE (B or n_max beyond the configuration), SF_EDEVICE
+ * (another device is current), SF_ETIMEOUT (a bounded device wait gave up),
+ * SF_ECUDA. */
+SF_API sf_status sf_nem_forward_offline(sf_nem_engine* e, const float* d_audio, const int64_t* h_len, int B,
+                                        int64_t n_max, float* d_probs, int64_t* h_out_len, void* cuda_stream);
+SF_API const char* sf_nem_last_error(const sf_nem_engine* e);
+
 #ifdef __cplusplus
 }
 #endif

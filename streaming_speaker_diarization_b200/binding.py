@@ -50,6 +50,11 @@ class sf_seg_params(ctypes.Structure):
                 ("min_duration_off", ctypes.c_double)]
 
 
+class sf_nem_config(ctypes.Structure):
+    _fields_ = [("n_layers", ctypes.c_int), ("d_model", ctypes.c_int), ("ff", ctypes.c_int), ("n_spk", ctypes.c_int),
+                ("max_batch", ctypes.c_int), ("max_samples", ctypes.c_int64)]
+
+
 class sf_kernel_stat(ctypes.Structure):
     _fields_ = [("name", ctypes.c_char * 32), ("launches", ctypes.c_int64), ("ms", ctypes.c_double),
                 ("flops", ctypes.c_double), ("bytes", ctypes.c_double)]
@@ -61,7 +66,8 @@ EXPORTED = ["sf_default_config", "sf_create", "sf_create_from_file", "sf_destroy
             "sf_stream_window", "sf_stream_step", "sf_stream_get_state", "sf_stream_set_state",
             "sf_stream_update", "sf_select_topk", "sf_profile_enable", "sf_profile_read", "sf_mel_noalloc",
             "sf_check", "sf_gemm_bf16", "sf_set_option", "sf_attention_relpos", "sf_default_seg_params",
-            "sf_segments", "sf_stream_step_audio", "sf_attention_mha", "sf_selftest_wait", "sf_gemm_bf16_ln"]
+            "sf_segments", "sf_stream_step_audio", "sf_attention_mha", "sf_selftest_wait", "sf_gemm_bf16_ln", "sf_nem_default_config", "sf_nem_create",
+            "sf_nem_destroy", "sf_nem_forward_offline", "sf_nem_last_error"]
 
 
 class SFError(RuntimeError):
@@ -108,6 +114,11 @@ def _load():
         "sf_segments": ([VP, VP, I, VP, I, P(sf_seg_params), I, VP, VP, VP], I),
         "sf_stream_step_audio": ([VP, VP, I64, VP, VP, VP, VP, VP, VP], I),
         "sf_attention_mha": ([VP, VP, VP, I, VP, I, VP], I),
+        "sf_nem_default_config": ([P(sf_nem_config)], I),
+        "sf_nem_create": ([VP, ctypes.c_uint64, P(sf_nem_config), P(VP)], I),
+        "sf_nem_destroy": ([VP], I),
+        "sf_nem_forward_offline": ([VP, VP, VP, I, I64, VP, VP, VP], I),
+        "sf_nem_last_error": ([VP], ctypes.c_char_p),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -361,3 +372,37 @@ def sf_segments(eng, probs, n_frames, params=None, max_seg=256, stream=None):
 
 def sf_set_option(eng, option, value):
     _check(lib.sf_set_option(eng, option, value), eng)
+
+
+# ---------------------------------------------------------- Nemotron-3 variant
+
+def nem_default_config(**kw):
+    c = sf_nem_config()
+    _check(lib.sf_nem_default_config(ctypes.byref(c)))
+    for k, v in kw.items():
+        setattr(c, k, v)
+    return c
+
+
+def sf_nem_create(blob, cfg):
+    out = ctypes.c_void_p()
+    rc = lib.sf_nem_create(blob, len(blob), ctypes.byref(cfg), ctypes.byref(out))
+    if rc != 0:
+        raise SFError(f"{STATUS.get(rc, rc)}: sf_nem_create")
+    return out
+
+
+def sf_nem_destroy(eng):
+    _check(lib.sf_nem_destroy(eng))
+
+
+def sf_nem_forward_offline(eng, audio, lengths, probs, stream=None):
+    """audio: device f32 [B, n_max]; probs: device f32 [B, n_max // 160, 8]."""
+    lengths = np.ascontiguousarray(lengths, np.int64)
+    out_len = np.zeros_like(lengths)
+    B, N = audio.shape
+    rc = lib.sf_nem_forward_offline(eng, _ptr(audio), _ptr(lengths), B, N, _ptr(probs), _ptr(out_len),
+                                    _stream(stream))
+    if rc != 0:
+        raise SFError(f"{STATUS.get(rc, rc)}: {lib.sf_nem_last_error(eng).decode()}")
+    return out_len

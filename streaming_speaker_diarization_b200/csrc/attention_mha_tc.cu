@@ -35,8 +35,7 @@ namespace {
 
 constexpr int MQ = 128;     // query rows per CTA
 constexpr int MK = 64;      // keys per tile
-constexpr int MHD = 24;     // head dim
-constexpr int MHP = 64;     // head dim as carried (zero-padded in Q)
+constexpr int MHP = 64;     // head dim as carried (zero-padded in Q when the head is narrower)
 constexpr int MNB = 3;      // K / V ring stages
 
 struct MhaTc {
@@ -50,15 +49,17 @@ struct MhaTc {
   static constexpr int OFF_P = OFF_RING + MNB * STAGE;
   static constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
   static constexpr int SMEM = 1024 + OFF_BAR + 256;
-  // key split: row r's partial state O[24], m, l (+2 pad, 16-byte rows) in
-  // the P buffers once the last P.V product has completed
-  static constexpr int PSTR = MHD + 4;
   static_assert(STAGE % 1024 == 0 && OFF_P % 1024 == 0 && OFF_RING % 1024 == 0, "swizzled tiles 1024-aligned");
-  static_assert(MQ * PSTR * 4 <= 2 * P_BYTES, "partials fit in the P buffers");
+  // key split: row r's partial state O[head dim], m, l (+2 pad, 16-byte
+  // rows) goes to the K/V ring once the last P.V product has completed
+  static_assert(MQ * (MHP + 4) * 4 <= MNB * STAGE, "partials fit in the ring");
 };
 
 }  // namespace
 
+// MHD: the head dimension (24 for the Sortformer Transformer, 64 for the
+// Nemotron-3 variant); E = 8 x MHD is a runtime argument.
+template <int MHD>
 __global__ void __launch_bounds__(192, 2) attn_mha_tc_kernel(const __grid_constant__ CUtensorMap t_qkv,
                                                              const bf16* __restrict__ qkv, int E,
                                                              bf16* __restrict__ ctx,
@@ -194,7 +195,7 @@ __global__ void __launch_bounds__(192, 2) attn_mha_tc_kernel(const __grid_consta
 #pragma unroll
       for (int c = 0; c < MHP / 8; ++c) {
         uint4 v = make_uint4(0, 0, 0, 0);
-        if (row_ok && c < MHD / 8) {   // 24 dims = three 16-byte chunks, 16-byte aligned (48 h bytes)
+        if (row_ok && c < MHD / 8) {   // 24 or 64 dims = 3 or 8 16-byte chunks, 16-byte aligned
           v = *reinterpret_cast<const uint4*>(qrow + 8 * c);
         }
         *reinterpret_cast<uint4*>(sQ + sw128_off(r, c)) = v;
@@ -204,7 +205,9 @@ __global__ void __launch_bounds__(192, 2) attn_mha_tc_kernel(const __grid_consta
       if (lane == 0) mbar_arrive(q_ready);
     }
 
-    const float sl2 = 1.4426950408889634f * 0.20412414523193151f;   // log2(e) / sqrt(24)
+    static_assert(MHD == 24 || MHD == 64, "head dims of the two Transformers");
+    constexpr float inv_sqrt_hd = MHD == 64 ? 0.125f : 0.20412414523193151f;
+    const float sl2 = 1.4426950408889634f * inv_sqrt_hd;   // log2(e) / sqrt(head dim)
     float m_run = -INFINITY, l_run = 0.f;
     float o[MHD];
 #pragma unroll
@@ -270,8 +273,9 @@ __global__ void __launch_bounds__(192, 2) attn_mha_tc_kernel(const __grid_consta
         const int pb = (t - 1) & 1;
         if (!warp_wait(&pv_full[pb], ((t - 1) >> 1) & 1)) { ok = false; break; }
         tc_fence_after();
-        uint32_t v[32];
-        tmem_ld32(tmem + lane_base + (uint32_t)(64 + 64 * pb), v);   // columns 0-31: the head's 24 + 8 unused
+        uint32_t v[64];
+        if (MHD <= 32) tmem_ld32(tmem + lane_base + (uint32_t)(64 + 64 * pb), v);   // the head's columns
+        else tmem_ld64(tmem + lane_base + (uint32_t)(64 + 64 * pb), v);
 #pragma unroll
         for (int k = 0; k < MHD; ++k) o[k] = (o[k] + __uint_as_float(v[k])) * alpha;
       }
@@ -280,8 +284,9 @@ __global__ void __launch_bounds__(192, 2) attn_mha_tc_kernel(const __grid_consta
       const int pb = (Tl - 1) & 1;
       if (warp_wait(&pv_full[pb], ((Tl - 1) >> 1) & 1)) {
         tc_fence_after();
-        uint32_t v[32];
-        tmem_ld32(tmem + lane_base + (uint32_t)(64 + 64 * pb), v);
+        uint32_t v[64];
+        if (MHD <= 32) tmem_ld32(tmem + lane_base + (uint32_t)(64 + 64 * pb), v);
+        else tmem_ld64(tmem + lane_base + (uint32_t)(64 + 64 * pb), v);
 #pragma unroll
         for (int k = 0; k < MHD; ++k) o[k] += __uint_as_float(v[k]);
       } else {
@@ -290,7 +295,7 @@ __global__ void __launch_bounds__(192, 2) attn_mha_tc_kernel(const __grid_consta
     }
     auto store_row = [&](const float* ov, float l) {
       const float inv = 1.f / l;
-      uint4* dst = reinterpret_cast<uint4*>(ctx + (int64_t)(sb + i) * E + h * MHD);   // 48 h bytes: 16-byte aligned
+      uint4* dst = reinterpret_cast<uint4*>(ctx + (int64_t)(sb + i) * E + h * MHD);   // 2 x MHD h bytes: 16-byte aligned
 #pragma unroll
       for (int c = 0; c < MHD / 8; ++c) {
         uint32_t w4[4];
@@ -308,11 +313,12 @@ __global__ void __launch_bounds__(192, 2) attn_mha_tc_kernel(const __grid_consta
       if (row_ok) store_row(o, l_run);
     } else {
       // Key split: (O, m, l) of this CTA's key range into row r's slot of
-      // the P buffers.  The tensor cores are done reading P: this warp saw
-      // the last P.V product complete, and every softmax warp wrote its P
-      // rows before that product was issued.  A CTA with no key tiles
-      // leaves m = -inf, l = 0 (weight 0 in the merge).
-      float* mine = reinterpret_cast<float*>(sP) + r * L::PSTR;
+      // the K/V ring.  Every K/V tile landed and was consumed: this warp saw
+      // the last P.V product complete, which follows every product that read
+      // the ring.  A CTA with no key tiles leaves m = -inf, l = 0 (weight 0
+      // in the merge).
+      constexpr int PSTR = MHD + 4;
+      float* mine = reinterpret_cast<float*>(sRing) + r * PSTR;
 #pragma unroll
       for (int d = 0; d < MHD; d += 4)
         *reinterpret_cast<float4*>(mine + d) = make_float4(o[d], o[d + 1], o[d + 2], o[d + 3]);
@@ -329,7 +335,8 @@ __global__ void __launch_bounds__(192, 2) attn_mha_tc_kernel(const __grid_consta
     asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(crank));
     if (crank == 0 && warp >= 2 && !*abort_flag) {
       const int q = warp & 3, r = 32 * q + lane, i = i0 + r;
-      const uint32_t row_addr = su32(reinterpret_cast<float*>(sP) + r * L::PSTR);
+      constexpr int PSTR = MHD + 4;
+      const uint32_t row_addr = su32(reinterpret_cast<float*>(sRing) + r * PSTR);
       float mz[4], lz[4];
 #pragma unroll
       for (int zz = 0; zz < 4; ++zz) {
@@ -392,13 +399,13 @@ __global__ void __launch_bounds__(192, 2) attn_mha_tc_kernel(const __grid_consta
 
 namespace {
 int g_mha_sms = 148;
-int g_mha_clusters[3] = {1, 0, 0};   // co-resident clusters of 1, 2, 4 CTAs (0: that split is off)
-}
+int g_mha_clusters[2][3] = {{1, 0, 0}, {1, 0, 0}};   // [head dim 24 / 64]: co-resident clusters of 1, 2, 4 CTAs
 
-cudaError_t launch_mha_tc(const bf16* qkv, bf16* ctx, const SeqTable* seq, int n_tiles2, int M, int max_len,
-                          int* err, cudaStream_t st) {
+template <int MHD>
+cudaError_t launch_mha_tc_t(const bf16* qkv, bf16* ctx, const SeqTable* seq, int n_tiles2, int M, int max_len, int E,
+                            int* err, cudaStream_t st) {
   if (M <= 0 || n_tiles2 <= 0) return cudaSuccess;
-  constexpr int E = 192;
+  if (E != 8 * MHD) return cudaErrorInvalidValue;
   CUtensorMap t_qkv;
   cudaError_t r = make_bf16_map_sw128(&t_qkv, qkv, M, 3 * E, 3 * E, MK);
   if (r != cudaSuccess) return r;
@@ -406,12 +413,13 @@ cudaError_t launch_mha_tc(const bf16* qkv, bf16* ctx, const SeqTable* seq, int n
   // each unit's keys over a cluster of 2 or 4 CTAs (no more splits than key
   // tiles of the longest sequence), but only as far as every cluster is
   // co-resident (one wave: a second wave would double the time)
+  const int* cl = g_mha_clusters[MHD == 64 ? 1 : 0];
   const int units = n_tiles2 * 8;
   int ks = 1;
   if (units < 2 * g_mha_sms) {
     const int want = 2 * g_mha_sms / units, tmax = (max_len + MK - 1) / MK;
-    if (want >= 4 && tmax >= 4 && units <= g_mha_clusters[2]) ks = 4;
-    else if (want >= 2 && tmax >= 2 && units <= g_mha_clusters[1]) ks = 2;
+    if (want >= 4 && tmax >= 4 && units <= cl[2]) ks = 4;
+    else if (want >= 2 && tmax >= 2 && units <= cl[1]) ks = 2;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(n_tiles2, 8, ks);
@@ -432,18 +440,16 @@ cudaError_t launch_mha_tc(const bf16* qkv, bf16* ctx, const SeqTable* seq, int n
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  CK_LAUNCH(cudaLaunchKernelEx(&cfg, attn_mha_tc_kernel, t_qkv, (const bf16*)qkv, E, ctx, seq, err, ks));
+  CK_LAUNCH(cudaLaunchKernelEx(&cfg, attn_mha_tc_kernel<MHD>, t_qkv, (const bf16*)qkv, E, ctx, seq, err, ks));
   return cudaGetLastError();
 }
 
-cudaError_t attention_mha_tc_init_attributes() {
-  int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
-      n > 0)
-    g_mha_sms = n;
-  cudaError_t r = cudaFuncSetAttribute(attn_mha_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, MhaTc::SMEM);
+template <int MHD>
+cudaError_t init_mha_tc() {
+  cudaError_t r =
+      cudaFuncSetAttribute(attn_mha_tc_kernel<MHD>, cudaFuncAttributeMaxDynamicSharedMemorySize, MhaTc::SMEM);
   if (r != cudaSuccess) return r;
-  for (int j = 1; j < 3; ++j) {   // can clusters of 2 and 4 CTAs be scheduled at all?
+  for (int j = 1; j < 3; ++j) {   // can clusters of 2 and 4 CTAs be scheduled at all, and how many at once?
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(1, 1, 1 << j);
     cfg.blockDim = dim3(192);
@@ -456,10 +462,32 @@ cudaError_t attention_mha_tc_init_attributes() {
     cfg.attrs = &a;
     cfg.numAttrs = 1;
     int n_cl = 0;
-    g_mha_clusters[j] = cudaOccupancyMaxActiveClusters(&n_cl, attn_mha_tc_kernel, &cfg) == cudaSuccess ? n_cl : 0;
+    g_mha_clusters[MHD == 64 ? 1 : 0][j] =
+        cudaOccupancyMaxActiveClusters(&n_cl, attn_mha_tc_kernel<MHD>, &cfg) == cudaSuccess ? n_cl : 0;
     cudaGetLastError();
   }
   return cudaSuccess;
+}
+}  // namespace
+
+cudaError_t launch_mha_tc(const bf16* qkv, bf16* ctx, const SeqTable* seq, int n_tiles2, int M, int max_len,
+                          int* err, cudaStream_t st) {
+  return launch_mha_tc_t<24>(qkv, ctx, seq, n_tiles2, M, max_len, 192, err, st);
+}
+
+cudaError_t launch_mha_tc_hd64(const bf16* qkv, bf16* ctx, const SeqTable* seq, int n_tiles2, int M, int max_len,
+                               int E, int* err, cudaStream_t st) {
+  return launch_mha_tc_t<64>(qkv, ctx, seq, n_tiles2, M, max_len, E, err, st);
+}
+
+cudaError_t attention_mha_tc_init_attributes() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
+      n > 0)
+    g_mha_sms = n;
+  cudaError_t r = init_mha_tc<24>();
+  if (r != cudaSuccess) return r;
+  return init_mha_tc<64>();
 }
 
 }  // namespace sf

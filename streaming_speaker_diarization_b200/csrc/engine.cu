@@ -24,6 +24,7 @@
 #include <vector>
 
 #include "../../include/sf.h"
+#include "blob.h"
 #include "common.cuh"
 #include "frontend.h"
 #include "layers.h"
@@ -50,25 +51,6 @@ static thread_local int g_fail_line = 0;
   } while (0)
 
 namespace {
-
-// ------------------------------------------------------------------ utils
-uint16_t f2bf_bits(float f) {   // round to nearest even
-  uint32_t u;
-  memcpy(&u, &f, 4);
-  if ((u & 0x7f800000u) == 0x7f800000u) return (uint16_t)((u >> 16) | ((u & 0xffff) ? 0x40 : 0));
-  u += 0x7fffu + ((u >> 16) & 1u);
-  return (uint16_t)(u >> 16);
-}
-
-struct TensorRef {
-  const float* data = nullptr;
-  std::vector<uint32_t> shape;
-  size_t numel() const {
-    size_t n = 1;
-    for (auto d : shape) n *= d;
-    return n;
-  }
-};
 
 struct Buf {
   void* p = nullptr;
@@ -302,60 +284,6 @@ size_t act_size(const sf_engine* e) { return e->cfg.precision == SF_BF16 ? 2 : 4
 
 inline int64_t enc_frames(int64_t L) { return L <= 0 ? 0 : 1 + (L - 1) / 8; }
 inline int64_t half_len(int64_t l) { return 1 + (l - 1) / 2; }
-
-// ------------------------------------------------------------ blob parsing
-bool parse_blob(const void* blob, uint64_t n, std::unordered_map<std::string, TensorRef>& out, std::string& err) {
-  const uint8_t* b = static_cast<const uint8_t*>(blob);
-  if (n < 16 || memcmp(b, "SFW1", 4) != 0) { err = "weight blob: bad magic"; return false; }
-  uint32_t cnt;
-  uint64_t data_off;
-  memcpy(&cnt, b + 4, 4);
-  memcpy(&data_off, b + 8, 8);
-  size_t pos = 16;
-  for (uint32_t i = 0; i < cnt; ++i) {
-    if (pos + 2 > n) { err = "weight blob: truncated header"; return false; }
-    uint16_t nl;
-    memcpy(&nl, b + pos, 2);
-    pos += 2;
-    if (pos + nl + 1 > n) { err = "weight blob: truncated name"; return false; }
-    std::string name(reinterpret_cast<const char*>(b + pos), nl);
-    pos += nl;
-    uint8_t nd = b[pos++];
-    TensorRef t;
-    for (int d = 0; d < nd; ++d) {
-      uint32_t v;
-      if (pos + 4 > n) { err = "weight blob: truncated dims"; return false; }
-      memcpy(&v, b + pos, 4);
-      pos += 4;
-      t.shape.push_back(v);
-    }
-    uint64_t off;
-    if (pos + 8 > n) { err = "weight blob: truncated offset"; return false; }
-    memcpy(&off, b + pos, 8);
-    pos += 8;
-    if (data_off + off + t.numel() * 4 > n) { err = "weight blob: payload of " + name + " out of range"; return false; }
-    t.data = reinterpret_cast<const float*>(b + data_off + off);
-    out[name] = t;
-  }
-  return true;
-}
-
-struct Loader {
-  std::unordered_map<std::string, TensorRef>& m;
-  std::string err;
-  const float* get(const std::string& name, std::vector<uint32_t> shape) {
-    auto it = m.find(name);
-    if (it == m.end()) {
-      if (err.empty()) err = "weight blob: missing tensor " + name;
-      return nullptr;
-    }
-    if (it->second.shape != shape) {
-      if (err.empty()) err = "weight blob: tensor " + name + " has an unexpected shape";
-      return nullptr;
-    }
-    return it->second.data;
-  }
-};
 
 template <typename T> void to_act(const std::vector<float>& src, std::vector<uint8_t>& dst) {
   dst.resize(src.size() * sizeof(T));

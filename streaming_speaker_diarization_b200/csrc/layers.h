@@ -172,6 +172,9 @@ cudaError_t attention_tc_init_attributes();
 // ERR_TIMEOUT if a bounded wait gives up.
 cudaError_t launch_mha_tc(const bf16* qkv, bf16* ctx, const SeqTable* seq, int n_tiles2, int M, int max_len,
                           int* err, cudaStream_t st);
+// The same kernel with heads of 64 (8 heads, E = 512: the Nemotron-3 variant).
+cudaError_t launch_mha_tc_hd64(const bf16* qkv, bf16* ctx, const SeqTable* seq, int n_tiles2, int M, int max_len,
+                               int E, int* err, cudaStream_t st);
 cudaError_t attention_mha_tc_init_attributes();
 
 // ------------------------------------------------- fused Transformer layer
