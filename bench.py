@@ -9,8 +9,9 @@ kernels.  Inputs are resident in HBM when the timed region starts; L2 is
 flushed (256 MiB write) between timed steps.
 
 Also in the line: the two streaming workloads (`streaming`: Low preset 64 x
-60 s, Very high preset 16 x 600 s) and the front-end alone on 1 h of audio
-(`frontend_1h`, HBM roofline).
+60 s, Very high preset 16 x 600 s), the variable-length batch of 32 clips
+(`batch`), the Nemotron-3 variant on the same 90 s clip (`nemotron`) and the
+front-end alone on 1 h of audio (`frontend_1h`, HBM roofline).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -431,6 +432,57 @@ def batch_bench(b, torch, blob, steps, warmup, local, args, clocks_dir=None):
             "clocks": clocks}
 
 
+def nem_model_flops(T, n_layers=31):
+    """Flops of the Nemotron-3 variant's offline forward over one clip of T
+    encoder frames (80 ms): stacking projection 2 x 1024 x 512, per layer
+    Q|K|V + output 4 x 2 x 512^2 and FFN 2 x 2 x 512 x 2048 per frame plus
+    2 x 2 x 512 x T of attention, head 2 x 512 x 64."""
+    per = 2.0 * 1024 * 512 + n_layers * (8.0 * 512 ** 2 + 4.0 * 512 * 2048 + 2048.0 * T) + 2.0 * 512 * 64
+    return T * per
+
+
+def nemotron_bench(b, torch, steps, warmup, local, clocks_dir=None):
+    """The Nemotron-3 variant (31 RoPE Transformer layers, 8 speakers at
+    10 ms) on the same 90 s clip: offline forward per step, audio resident on
+    the device, L2 flushed between steps, CUDA events; weights N(0, 0.02)."""
+    from synth import NEM_FULL, clip_for_config, make_nem_weights, weights_blob
+    audio_np, lens, _ = clip_for_config(1)
+    eng = b.sf_nem_create(weights_blob(make_nem_weights(NEM_FULL, seed=0)), b.nem_default_config(max_batch=1))
+    try:
+        audio = torch.from_numpy(audio_np).cuda()
+        probs = torch.zeros((1, audio_np.shape[1] // 160, 8), device="cuda")
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+        st = torch.cuda.current_stream()
+        for _ in range(warmup):
+            b.sf_nem_forward_offline(eng, audio, lens, probs)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        torch.cuda.synchronize()
+        clk = Clocks(local, clocks_dir)
+        for i in range(steps):
+            flush.zero_()
+            ev[i][0].record(st)
+            b.sf_nem_forward_offline(eng, audio, lens, probs)
+            ev[i][1].record(st)
+        torch.cuda.synchronize()
+        clocks = clk.stop()
+    finally:
+        b.sf_nem_destroy(eng)
+    ms = [a.elapsed_time(c) for a, c in ev]
+    med = float(np.median(ms))
+    T = (int(lens[0]) // 160 + 7) // 8
+    flops = nem_model_flops(T)
+    pk, kind = peaks()
+    tf = flops / (med / 1000.0) / 1e12
+    return {"workload": "Nemotron-3 variant offline, 1 clip x 90 s (the headline clip), 31 RoPE Transformer layers "
+                        "d 512, 8 speakers every 10 ms, bf16", "value": 90.0 / (med / 1000.0), "unit": UNIT,
+            "ms_p50": med, "ms_p95": float(np.percentile(ms, 95)), "calls": steps,
+            "output_frames_per_s": (int(lens[0]) // 160) / (med / 1000.0),
+            "roofline": {"bound": "tensor", "kernel": "whole forward (model flops)", "achieved": tf,
+                         "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": tf / pk["bf16_tflops"],
+                         "flops_per_call": flops, "peak_kind": f"{kind} bf16 burst"},
+            "clocks": clocks}
+
+
 def oracle_subsets(w):
     """The oracle (numpy, fp64 unless stated) on declared subsets of every
     workload, each timed once on this machine's host cores: the 90 s clip
@@ -525,6 +577,7 @@ def main():
     ap.add_argument("--no-streaming", action="store_true", help="skip the streaming workloads")
     ap.add_argument("--no-frontend", action="store_true", help="skip the 1 h front-end-only run")
     ap.add_argument("--no-batch", action="store_true", help="skip the 32-clip variable-length batch")
+    ap.add_argument("--no-nemotron", action="store_true", help="skip the Nemotron-3 variant's offline forward")
     ap.add_argument("--mel-path", type=int, default=1, choices=[0, 1], help="front-end implementation (SF_OPT_MEL_PATH)")
     ap.add_argument("--attn-path", type=int, default=1, choices=[0, 1], help="attention kernels (SF_OPT_ATTN_PATH)")
     ap.add_argument("--sub-path", type=int, default=1, choices=[0, 1],
@@ -651,6 +704,8 @@ def main():
     b.sf_destroy(eng)
     if not args.no_streaming:
         line["streaming"] = streaming_bench(b, torch, weights_blob(w), rank, world, local, args, args.clocks_dir)
+    if not args.no_nemotron and world == 1:
+        line["nemotron"] = nemotron_bench(b, torch, args.steps, max(args.warmup, 3), local, args.clocks_dir)
     if not args.no_batch and world == 1:
         line["batch"] = batch_bench(b, torch, weights_blob(w), args.steps, max(args.warmup, 3), local, args,
                                     args.clocks_dir)

@@ -79,3 +79,11 @@ def test_stream_plan_low_preset_sizes():
     assert bench.stream_plan((340, 40, 40, 300, 188), 7500)[1] == (608, 380)
     # one full-size offline clip: 1125 encoder frames, ~351 GFLOP
     assert abs(bench.model_flops(1125, 1125) / 1e9 - 350.7) < 0.1
+
+
+def test_nemotron_flops_count():
+    # 90 s clip: 1125 encoder frames; per frame 2 x 1024 x 512 + 31 x (8 x 512^2
+    # + 4 x 512 x 2048 + 2048 x 1125) + 2 x 512 x 64 flops
+    per = 2 * 1024 * 512 + 31 * (8 * 512 ** 2 + 4 * 512 * 2048 + 2048 * 1125) + 2 * 512 * 64
+    assert abs(bench.nem_model_flops(1125) - 1125 * per) < 1.0
+    assert 300e9 < bench.nem_model_flops(1125) < 302e9
