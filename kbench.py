@@ -6,6 +6,7 @@
     python kbench.py mel SECONDS [--clips B] [--path P] [--reps R]
     python kbench.py ln M N K [--xnorm X] [--double] [--reps R]
     python kbench.py stream N_STREAMS STEPS [--preset C R F U S]
+    python kbench.py nem SECONDS [--clips B] [--layers L] [--reps R]
 
 `gemm` runs sf_gemm_bf16 (E: 1 f32 out, 2 bf16 out, 3 residual update, 4
 swish, 5 gated linear unit; P: SF_OPT_GEMM_PATH, 1 = tcgen05 with CTA pairs
@@ -18,7 +19,9 @@ into the epilogue (X: 1 = the residual stream receives the normalised row;
 --double: a second LayerNorm into the bf16 output); `stream` runs STEPS
 streaming steps of N_STREAMS streams (a 2 + 2-layer bf16 engine, random
 normalised features, default the Low preset 6/7/188/144/188): the state
-update and cache compression kernels at full state sizes.  Operands are seeded random values on the device; three warm-up
+update and cache compression kernels at full state sizes; `nem` runs
+sf_nem_forward_offline, the Nemotron-3 variant's offline forward (L layers,
+default all 31; weights N(0, 0.02)) on B clips of SECONDS each.  Operands are seeded random values on the device; three warm-up
 launches, then REPS launches queued behind a GPU sleep (so host launch
 overhead is hidden) and timed with CUDA events on the current stream.  Also
 the driver for single-kernel ncu captures (small REPS)."""
@@ -86,6 +89,11 @@ def main(argv=None):
     t.add_argument("n_streams", type=int)
     t.add_argument("steps", type=int)
     t.add_argument("--preset", type=int, nargs=5, default=[6, 7, 188, 144, 188])
+    v = sub.add_parser("nem")
+    v.add_argument("seconds", type=float)
+    v.add_argument("--clips", type=int, default=1)
+    v.add_argument("--layers", type=int, default=31)
+    v.add_argument("--reps", type=int, default=10)
     args = ap.parse_args(argv)
 
     import torch
@@ -137,6 +145,18 @@ def main(argv=None):
         torch.cuda.synchronize()
         b.sf_stream_destroy(st)
         print(f"stream n={n} preset={pre}: {args.steps} steps, {e0.elapsed_time(e1) / args.steps * 1e3:.1f} us/step")
+    elif args.op == "nem":
+        from synth import NemDims, make_nem_weights, weights_blob
+        B, n = args.clips, int(args.seconds * 16000)
+        eng = b.sf_nem_create(weights_blob(make_nem_weights(NemDims(n_layers=args.layers), seed=0)),
+                              b.nem_default_config(n_layers=args.layers, max_batch=B, max_samples=n))
+        audio = 0.1 * torch.randn(B, n, device="cuda", generator=gen)
+        lens = np.full(B, n, np.int64)
+        probs = torch.zeros(B, n // 160, 8, device="cuda")
+        ms = _time(torch, lambda: b.sf_nem_forward_offline(eng, audio, lens, probs), args.reps)
+        b.sf_nem_destroy(eng)
+        print(f"nem {B} x {args.seconds} s, {args.layers} layers: {ms * 1e3:.1f} us/forward, "
+              f"{B * args.seconds / ms * 1e3:.0f} audio-s/s")
     elif args.op == "mel":
         n = int(args.seconds * 16000)
         B = args.clips
