@@ -157,6 +157,7 @@ def main(argv=None):
         b.sf_nem_destroy(eng)
         print(f"nem {B} x {args.seconds} s, {args.layers} layers: {ms * 1e3:.1f} us/forward, "
               f"{B * args.seconds / ms * 1e3:.0f} audio-s/s")
+        return   # a Nemotron engine: not an sf_engine handle for the checks below
     elif args.op == "mel":
         n = int(args.seconds * 16000)
         B = args.clips
