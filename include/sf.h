@@ -443,7 +443,7 @@ SF_API sf_status sf_gemm_bf16(sf_engine* e, const void* d_A, int lda, const void
  * LN(v) = (v - mean) / sqrt(var + 1e-5) * g + b over each row (biased
  * variance), g/b f32 [N].  Requires N a multiple of 64 up to 512 and every
  * 128-row block's cluster of N/64 CTAs co-resident (SF_ESHAPE otherwise),
- * K % 64 == 0, lda % 8 == 0, 16-byte aligned A/W/x, 8-byte aligned h. */
+ * K % 64 == 0, lda % 8 == 0, 16-byte aligned A/W/x/h. */
 SF_API sf_status sf_gemm_bf16_ln(sf_engine* e, const void* d_A, int lda, const void* d_W, int M, int N, int K,
                                  const float* d_bias, float alpha, float* d_x, const float* d_g, const float* d_b,
                                  const float* d_g2, const float* d_b2, int xnorm, void* d_h, void* cuda_stream);

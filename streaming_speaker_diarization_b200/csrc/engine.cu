@@ -1649,6 +1649,23 @@ cudaError_t stream_step_impl(sf_stream* s, const float* d_feats, int64_t t_buf, 
   });
 }
 
+// Workspaces of a streaming step of n streams at its largest: window of
+// 8 (1 + chunk_len + right_context) mel frames, encoder rows per stream up to
+// the cache, the FIFO with a chunk, and the window's new frames.
+cudaError_t reserve_stream_ws(sf_engine* e, int n, const sf_preset& p) {
+  const size_t a = act_size(e);
+  const int64_t W_max = 8 * (1 + (int64_t)p.chunk_len + p.right_context);
+  const int64_t T3 = enc_frames(W_max);
+  const int64_t S_max = (int64_t)p.spkcache_len + p.fifo_len + p.chunk_len + T3;
+  g_ws_gen = &e->ws_gen;
+  CK(ensure_encode_ws(e, (int)(n * S_max)));
+  CK(ensure(e->emb, (size_t)n * T3 * e->cfg.d_model * a));
+  CK(prep_pre_encode(e, n, W_max, a));
+  CK(ensure(e->mel, (size_t)n * 128 * W_max * 4));
+  CK(ensure(e->part, ((size_t)n * ((W_max + 31) / 32) * 128 * 4 + (size_t)n * 128 * 2) * 4));
+  return cudaSuccess;
+}
+
 }  // namespace
 
 extern "C" {
@@ -1699,6 +1716,13 @@ sf_status sf_stream_create(sf_engine* e, const sf_preset* p, int n_streams, sf_s
   if (cudaMemset(s->alloc, 0, total) != cudaSuccess) {
     cudaFree(s->alloc);
     return fail(e, SF_ECUDA, "stream state init");
+  }
+  // The engine's workspaces at this preset's largest step, reserved now: a
+  // buffer that grew during the steps would move and invalidate every step
+  // graph captured before it.
+  if (reserve_stream_ws(e, n_streams, *p) != cudaSuccess) {
+    cudaFree(s->alloc);
+    return fail(e, SF_ENOMEM, "stream workspaces");
   }
   e->streams.push_back(s.get());
   *out = s.release();

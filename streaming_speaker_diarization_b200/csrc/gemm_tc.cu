@@ -20,9 +20,11 @@
 // of both CTAs of the pair on this GPU.
 #include <cuda.h>
 #include <cudaTypedefs.h>
+#include <cstring>
 
 #include "common.cuh"
 #include "epilogue.cuh"
+#include "epilogue_tma.cuh"
 #include "layers.h"
 #include "tcgen05.cuh"
 
@@ -40,8 +42,8 @@ struct TcCfg {
   static constexpr int A_BYTES = TC_BM * TC_BK * 2;
   static constexpr int B_BYTES = BN * TC_BK * 2;
   static constexpr int SMEM = 1024 + STAGES * (A_BYTES + B_BYTES) + 256;
-  static_assert(STAGES * (A_BYTES + B_BYTES) >= 4 * 32 * 68 * 4 + 2 * 128 * 8,
-                "epilogue staging (and the LayerNorm statistics) reuse the pipeline buffers");
+  static_assert(STAGES * (A_BYTES + B_BYTES) >= 4 * 32 * 68 * 4 && STAGES * (A_BYTES + B_BYTES) >= 12 * 4096 + 2 * 128 * 8,
+                "epilogue staging, TMA boxes and the LayerNorm statistics reuse the pipeline buffers");
 };
 
 // Epilogue of one warp's 32 rows: per CW-column chunk (CW = 64 or 32), the
@@ -214,138 +216,113 @@ __device__ __forceinline__ void ln_row_stats(const float2* stat, int r, int ncl,
   rstd = 1.0f / sqrtf(m2 / (float)ncols + 1e-5f);
 }
 
-// (mean, M2) of the 64 staged columns of this thread's row (thread = row).
-__device__ __forceinline__ float2 ln_tile_stats(const float* row) {
-  float s = 0.f;
-#pragma unroll
-  for (int j = 0; j < 64; j += 4) {
-    const float4 v = *reinterpret_cast<const float4*>(row + j);
-    s += (v.x + v.y) + (v.z + v.w);
-  }
-  const float mean = s * (1.f / 64.f);
-  float m2 = 0.f;
-#pragma unroll
-  for (int j = 0; j < 64; j += 4) {
-    const float4 v = *reinterpret_cast<const float4*>(row + j);
-    float d = v.x - mean; m2 = fmaf(d, d, m2);
-    d = v.y - mean; m2 = fmaf(d, d, m2);
-    d = v.z - mean; m2 = fmaf(d, d, m2);
-    d = v.w - mean; m2 = fmaf(d, d, m2);
-  }
-  return make_float2(mean, m2);
-}
-
 // EPI_RESID_LN epilogue of one warp's 32 rows of a 128 x 64 tile whose CTA
-// is rank n0 / 64 of a cluster spanning the row block's N / 64 tiles.
-// x_new = x + alpha (acc + b) is staged in shared memory; each thread (one
-// row) takes (mean, M2) of its 64 columns; after a cluster barrier every CTA
-// merges the partials of all ranks for its rows and normalises its own
-// columns; a second LayerNorm, if any, repeats the exchange on the first
-// one's output.  Every epilogue thread passes the same cluster barriers
+// is rank n0 / 64 of a cluster spanning the row block's N / 64 tiles; thread
+// = row, the tile's 64 columns in registers.  x_new = x + alpha (acc + b)
+// (x prefetched by the caller into xr); each thread takes (mean, M2) of its
+// 64 values; after a cluster barrier every CTA merges the partials of all
+// ranks for its rows and normalises its own columns; a second LayerNorm, if
+// any, repeats the exchange on the first one's output.  The f32 row and the
+// bf16 normalised row go out as three TMA box stores from `boxes` (12 KB).
+// Every epilogue thread passes the same cluster barriers
 // (n_cluster_barriers(e) of them) whether or not its CTA's accumulator is
 // valid (`ok`), so no CTA of the cluster waits for ever; the last barrier
 // keeps each CTA's statistics alive until its peers have read them.
 __device__ __forceinline__ int n_cluster_barriers(const Epi& e) { return e.ln_g2 ? 3 : 2; }
 
-__device__ __forceinline__ void resid_ln_epilogue(const Epi& e, uint32_t tmem, float* stage, float2* st1, float2* st2,
-                                                  int M, int N, int m0, int n0, int q, int lane, bool ok) {
-  constexpr int LD = 68;
-  const int l4 = lane & 15, rh = lane >> 4;
-  const int c = n0 + 4 * l4;
-  const int ncl = N / 64;
-  if (ok) {
-    uint32_t v[64];
-    tmem_ld64(tmem + ((uint32_t)(32 * q) << 16), v);
+__device__ __forceinline__ float2 row_stats64(const float* v) {
+  float s = 0.f;
 #pragma unroll
-    for (int j = 0; j < 64; j += 4)
-      *reinterpret_cast<float4*>(stage + lane * LD + j) =
-          make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]), __uint_as_float(v[j + 2]),
-                      __uint_as_float(v[j + 3]));
+  for (int k = 0; k < 64; ++k) s += v[k];
+  const float mean = s * (1.f / 64.f);
+  float m2 = 0.f;
+#pragma unroll
+  for (int k = 0; k < 64; ++k) {
+    const float d = v[k] - mean;
+    m2 = fmaf(d, d, m2);
   }
-  __syncwarp();
-  if (ok) {   // x_new = x + alpha (acc + b) into the staged tile
-    float4 bv = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (e.bias) bv = *reinterpret_cast<const float4*>(e.bias + c);
-#pragma unroll 1
-    for (int i0 = 0; i0 < 16; i0 += 8) {
-      float4 xv[8];
+  return make_float2(mean, m2);
+}
+
+// Lane-spread epilogue parameters of a 64-column LayerNorm tile (bias, and
+// the weights of one or two LayerNorms), read before the accumulator wait.
+struct LnParams {
+  float2 bias, g, b, g2, b2;
+};
+
+__device__ __forceinline__ void layer_norm64(float* v, float2 g, float2 b, float mean, float rstd) {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int row = m0 + 32 * q + 2 * (i0 + i) + rh;
-        xv[i] = row < M ? *reinterpret_cast<const float4*>(epi_f32_ptr(e, row, c)) : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
+  for (int k = 0; k < 64; ++k) v[k] = (v[k] - mean) * rstd * col64(g, k) + col64(b, k);
+}
+
+// 64 f32 values as two 32-column boxes (128-byte rows) at b and b + 4 KB
+__device__ __forceinline__ void stage_f32x64(uint32_t b, int lane, const float* v) {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        float* sp = stage + (2 * (i0 + i) + rh) * LD + 4 * l4;
-        const float4 t = *reinterpret_cast<const float4*>(sp);
-        float4 x = xv[i];
-        x.x += e.alpha * (t.x + bv.x); x.y += e.alpha * (t.y + bv.y);
-        x.z += e.alpha * (t.z + bv.z); x.w += e.alpha * (t.w + bv.w);
-        *reinterpret_cast<float4*>(sp) = x;
-      }
+  for (int h = 0; h < 2; ++h)
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const float* w = v + 32 * h + 4 * u;
+      sts128(sw128_unit(b + h * EPI_BOX_BYTES, lane, u), __float_as_uint(w[0]), __float_as_uint(w[1]),
+             __float_as_uint(w[2]), __float_as_uint(w[3]));
     }
+}
+__device__ __forceinline__ void stage_bf16x64(uint32_t b, int lane, const float* v) {
+#pragma unroll
+  for (int u = 0; u < 8; ++u)
+    sts128(sw128_unit(b, lane, u), pack_bf16(v[8 * u], v[8 * u + 1]), pack_bf16(v[8 * u + 2], v[8 * u + 3]),
+           pack_bf16(v[8 * u + 4], v[8 * u + 5]), pack_bf16(v[8 * u + 6], v[8 * u + 7]));
+}
+
+__device__ __forceinline__ void resid_ln_rows(const Epi& e, const CUtensorMap* mx, const CUtensorMap* mh,
+                                              uint32_t tmem, uint8_t* boxes, float2* st1, float2* st2, int M, int N,
+                                              int m_w, int n0, int q, int lane, bool ok, const float* xr,
+                                              const LnParams& lp) {
+  const int ncl = N / 64;
+  const uint32_t sb = su32(boxes);
+  float v[64];
+  if (ok) {
+    tmem_ld64(tmem + ((uint32_t)(32 * q) << 16), reinterpret_cast<uint32_t*>(v));
+#pragma unroll
+    for (int k = 0; k < 64; ++k) v[k] = xr[k] + e.alpha * (v[k] + col64(lp.bias, k));
+  } else {
+#pragma unroll
+    for (int k = 0; k < 64; ++k) v[k] = 0.f;
   }
-  __syncwarp();
-  st1[32 * q + lane] = ok ? ln_tile_stats(stage + lane * LD) : make_float2(0.f, 0.f);
+  st1[32 * q + lane] = ok ? row_stats64(v) : make_float2(0.f, 0.f);
   cluster_arrive_wait();
   float mean, rstd;
   ln_row_stats(st1, 32 * q + lane, ncl, N, mean, rstd);
   const bool two = e.ln_g2 != nullptr;
-  {
-    const float4 g = *reinterpret_cast<const float4*>(e.ln_g + c);
-    const float4 bb = *reinterpret_cast<const float4*>(e.ln_b + c);
-#pragma unroll 4
-    for (int i = 0; i < 16; ++i) {
-      const int rr = 2 * i + rh, row = m0 + 32 * q + rr;
-      const float mu = __shfl_sync(0xffffffffu, mean, rr), rs = __shfl_sync(0xffffffffu, rstd, rr);
-      float* sp = stage + rr * LD + 4 * l4;
-      const float4 v = *reinterpret_cast<const float4*>(sp);
-      float4 y;
-      y.x = (v.x - mu) * rs * g.x + bb.x; y.y = (v.y - mu) * rs * g.y + bb.y;
-      y.z = (v.z - mu) * rs * g.z + bb.z; y.w = (v.w - mu) * rs * g.w + bb.w;
-      if (ok && row < M) {
-        *reinterpret_cast<float4*>(epi_f32_ptr(e, row, c)) = e.ln_xnorm ? y : v;
-        if (!two) {
-          __nv_bfloat162 a = __floats2bfloat162_rn(y.x, y.y), b2 = __floats2bfloat162_rn(y.z, y.w);
-          uint2 pk;
-          pk.x = *reinterpret_cast<uint32_t*>(&a);
-          pk.y = *reinterpret_cast<uint32_t*>(&b2);
-          *reinterpret_cast<uint2*>(reinterpret_cast<bf16*>(e.ln_h) + (int64_t)row * e.ldh + c) = pk;
-        }
-      }
-      if (two) *reinterpret_cast<float4*>(sp) = y;
-    }
-  }
+  if (!e.ln_xnorm) stage_f32x64(sb, lane, v);   // out <- x_new
+  layer_norm64(v, lp.g, lp.b, mean, rstd);
+  if (e.ln_xnorm) stage_f32x64(sb, lane, v);    // out <- LN(x_new)
   if (two) {
-    __syncwarp();
-    st2[32 * q + lane] = ok ? ln_tile_stats(stage + lane * LD) : make_float2(0.f, 0.f);
+    st2[32 * q + lane] = ok ? row_stats64(v) : make_float2(0.f, 0.f);
     cluster_arrive_wait();
     ln_row_stats(st2, 32 * q + lane, ncl, N, mean, rstd);
-    const float4 g = *reinterpret_cast<const float4*>(e.ln_g2 + c);
-    const float4 bb = *reinterpret_cast<const float4*>(e.ln_b2 + c);
-#pragma unroll 4
-    for (int i = 0; i < 16; ++i) {
-      const int rr = 2 * i + rh, row = m0 + 32 * q + rr;
-      const float mu = __shfl_sync(0xffffffffu, mean, rr), rs = __shfl_sync(0xffffffffu, rstd, rr);
-      const float4 v = *reinterpret_cast<const float4*>(stage + rr * LD + 4 * l4);
-      if (ok && row < M) {
-        __nv_bfloat162 a = __floats2bfloat162_rn((v.x - mu) * rs * g.x + bb.x, (v.y - mu) * rs * g.y + bb.y);
-        __nv_bfloat162 b2 = __floats2bfloat162_rn((v.z - mu) * rs * g.z + bb.z, (v.w - mu) * rs * g.w + bb.w);
-        uint2 pk;
-        pk.x = *reinterpret_cast<uint32_t*>(&a);
-        pk.y = *reinterpret_cast<uint32_t*>(&b2);
-        *reinterpret_cast<uint2*>(reinterpret_cast<bf16*>(e.ln_h) + (int64_t)row * e.ldh + c) = pk;
-      }
-    }
+    layer_norm64(v, lp.g2, lp.b2, mean, rstd);
   }
+  stage_bf16x64(sb + 2 * EPI_BOX_BYTES, lane, v);
+  fence_async_smem();
+  __syncwarp();
+  if (lane == 0 && ok && m_w < M) {
+    tma_store_2d(mx, boxes, n0, m_w);
+    tma_store_2d(mx, boxes + EPI_BOX_BYTES, n0 + 32, m_w);
+    tma_store_2d(mh, boxes + 2 * EPI_BOX_BYTES, n0, m_w);
+    bulk_commit();
+    bulk_wait_read_all();
+  }
+  __syncwarp();
   cluster_arrive_wait();   // peers have read this CTA's statistics
 }
 
 template <int BN, int STAGES>
 __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__ CUtensorMap ta,
-                                                         const __grid_constant__ CUtensorMap tb, int M, int N, int K,
+                                                         const __grid_constant__ CUtensorMap tb,
+                                                         const __grid_constant__ CUtensorMap mo,
+                                                         const __grid_constant__ CUtensorMap mo2, int M, int N, int K,
                                                          Epi e, int* err, float* __restrict__ split_ws,
-                                                         int* __restrict__ split_cnt) {
+                                                         int* __restrict__ split_cnt, int tma_epi) {
   using C = TcCfg<BN, STAGES>;
   extern __shared__ uint8_t tc_smem[];
   uint8_t* sm = tc_smem + ((1024 - (su32(tc_smem) & 1023)) & 1023);
@@ -443,14 +420,39 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
       pdl_trigger();
     }
   } else if (e.kind == EPI_RESID_LN) {
-    const int q = warp & 3;
-    float* stage = reinterpret_cast<float*>(sm) + q * (32 * 68);
-    float2* st1 = reinterpret_cast<float2*>(reinterpret_cast<float*>(sm) + 4 * 32 * 68);
-    prefetch_resid(e, M, N, m0 + 32 * q, 32, n0, BN, lane);
-    const bool ok = mbar_wait(accf, 0, abort_flag) && !*abort_flag;
+    // thread = row: the residual row segment is read while the main loop runs
+    const int q = warp & 3, m_w = m0 + 32 * q, row = m_w + lane;
+    float2* st1 = reinterpret_cast<float2*>(sm + 4 * 3 * EPI_BOX_BYTES);
+    float xr[64];
+    load_resid32(e, row, M, n0, N, xr);
+    load_resid32(e, row, M, n0 + 32, N, xr + 32);
+    LnParams lp;
+    lp.bias = lane_param64(e.bias, n0, N, lane);
+    lp.g = lane_param64(e.ln_g, n0, N, lane);
+    lp.b = lane_param64(e.ln_b, n0, N, lane);
+    lp.g2 = lane_param64(e.ln_g2, n0, N, lane);
+    lp.b2 = lane_param64(e.ln_b2, n0, N, lane);
+    // warp-uniform: tcgen05.ld is a warp-wide instruction
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(accf, 0, abort_flag) && !*abort_flag);
     if (!ok) *abort_flag = 1;
     tc_fence_after();
-    resid_ln_epilogue(e, tmem, stage, st1, st1 + 128, M, N, m0, n0, q, lane, ok);
+    resid_ln_rows(e, &mo, &mo2, tmem, sm + q * 3 * EPI_BOX_BYTES, st1, st1 + 128, M, N, m_w, n0, q, lane, ok, xr, lp);
+  } else if (tma_epi) {
+    // thread = row, TMA box stores; the pipeline buffers are free once the
+    // accumulator is complete, so the boxes reuse them
+    const int q = warp & 3, m_w = m0 + 32 * q;
+    float xr[32];
+    float2 b2;
+    epi_prefetch<true, BN>(e, M, N, m_w, n0, 0, lane, xr, b2);
+    if (__all_sync(0xffffffffu, mbar_wait(accf, 0, abort_flag) && !*abort_flag)) {
+      tc_fence_after();
+      BoxRing ring{sm + q * 2 * EPI_BOX_BYTES, 0};
+      row_epilogue_any<BN, true>(e, &mo, &mo2, tmem + ((uint32_t)(32 * q) << 16), ring, M, N, m_w, n0, 0, 1, lane, xr,
+                                 b2);
+      ring.drain(lane);
+    } else {
+      *abort_flag = 1;
+    }
   } else {
     // Epilogue: per 64-column chunk, each warp copies its 32 x 64 accumulator
     // block from TMEM to a padded shared tile (thread = row), then writes it
@@ -528,15 +530,17 @@ template <int BN, int STAGES>
 struct TcpCfg {
   static constexpr int A_BYTES = TC_BM * TC_BK * 2;
   static constexpr int B_BYTES = BN * TC_BK * 2;
-  static constexpr int STAGE_FLOATS = 8 * 32 * 68;
+  static constexpr int STAGE_FLOATS = 8 * 2 * EPI_BOX_BYTES / 4;   // per epilogue warp two TMA boxes (or a 32 x 36 tile)
   static constexpr int SMEM = 1024 + STAGES * (A_BYTES + B_BYTES) + STAGE_FLOATS * 4 + 256;
   static_assert(SMEM <= 232448, "shared memory per CTA");
 };
 
 template <int BN, int STAGES>
 __global__ void __launch_bounds__(320, 1) gemm_tcp_kernel(const __grid_constant__ CUtensorMap ta,
-                                                          const __grid_constant__ CUtensorMap tb, int M, int N, int K,
-                                                          Epi e, int* err) {
+                                                          const __grid_constant__ CUtensorMap tb,
+                                                          const __grid_constant__ CUtensorMap mo,
+                                                          const __grid_constant__ CUtensorMap mo2, int M, int N, int K,
+                                                          Epi e, int* err, int tma_epi) {
   using C = TcpCfg<BN, STAGES>;
   extern __shared__ uint8_t tc_smem[];
   uint8_t* sm = tc_smem + ((1024 - (su32(tc_smem) & 1023)) & 1023);
@@ -638,32 +642,42 @@ __global__ void __launch_bounds__(320, 1) gemm_tcp_kernel(const __grid_constant_
     }
   } else {
     const int q = warp & 3, hc = (warp - 2) >> 2;   // TMEM lane quarter, column half
-    float* stage = stg + (warp - 2) * (32 * 68);
+    float* stage = stg + (warp - 2) * (32 * 36);
+    BoxRing ring{reinterpret_cast<uint8_t*>(stg) + (warp - 2) * 2 * EPI_BOX_BYTES, 0};
+    float xr[32];
+    float2 b2 = make_float2(0.f, 0.f);
     int i = 0;
     for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++i) {
       const int a = i & 1, u = i >> 1;
       const int m0 = (tile / tiles_n) * TC_BM, n0 = (tile % tiles_n) * BN;
-      prefetch_resid(e, M, N, m0 + 32 * q, 32, n0 + hc * BN / 2, BN / 2, lane);
-      if (!mbar_wait(&accf[a], u & 1, abort_flag) || *abort_flag) {
+      if (!tma_epi) prefetch_resid(e, M, N, m0 + 32 * q, 32, n0 + hc * BN / 2, BN / 2, lane);
+      else epi_prefetch<false, BN>(e, M, N, m0 + 32 * q, n0, hc, lane, xr, b2);
+      if (__any_sync(0xffffffffu, !mbar_wait(&accf[a], u & 1, abort_flag) || *abort_flag)) {
         *abort_flag = 1;
         break;
       }
       tc_fence_after();
       const uint32_t acc = tmem + (uint32_t)(a * BN);
-      const int cb = hc * BN / 2, ce = cb + BN / 2;
-      switch (e.kind) {
-        case EPI_BIAS: epilogue_tile<EPI_BIAS, BN>(e, acc, stage, nullptr, M, N, m0, n0, q, lane, 1, cb, ce); break;
-        case EPI_BIAS_RELU: epilogue_tile<EPI_BIAS_RELU, BN>(e, acc, stage, nullptr, M, N, m0, n0, q, lane, 1, cb, ce); break;
-        case EPI_BIAS_SWISH: epilogue_tile<EPI_BIAS_SWISH, BN>(e, acc, stage, nullptr, M, N, m0, n0, q, lane, 1, cb, ce); break;
-        case EPI_BIAS_GLU: epilogue_tile<EPI_BIAS_GLU, BN>(e, acc, stage, nullptr, M, N, m0, n0, q, lane, 1, cb, ce); break;
-        case EPI_RESID: epilogue_tile<EPI_RESID, BN>(e, acc, stage, nullptr, M, N, m0, n0, q, lane, 1, cb, ce); break;
-        case EPI_F32: epilogue_tile<EPI_F32, BN>(e, acc, stage, nullptr, M, N, m0, n0, q, lane, 1, cb, ce); break;
-        default: epilogue_tile<EPI_F32_AND_T, BN>(e, acc, stage, nullptr, M, N, m0, n0, q, lane, 1, cb, ce); break;
+      if (tma_epi) {   // chunks alternate between the two warps of a lane quarter
+        row_epilogue_any<BN, false>(e, &mo, &mo2, acc + ((uint32_t)(32 * q) << 16), ring, M, N, m0 + 32 * q, n0, hc, 2, lane,
+                             xr, b2);
+      } else {
+        const int cb = hc * BN / 2, ce = cb + BN / 2;
+        switch (e.kind) {
+          case EPI_BIAS: epilogue_tile<EPI_BIAS, BN, 32>(e, acc, stage, nullptr, M, N, m0, n0, q, lane, 1, cb, ce); break;
+          case EPI_BIAS_RELU: epilogue_tile<EPI_BIAS_RELU, BN, 32>(e, acc, stage, nullptr, M, N, m0, n0, q, lane, 1, cb, ce); break;
+          case EPI_BIAS_SWISH: epilogue_tile<EPI_BIAS_SWISH, BN, 32>(e, acc, stage, nullptr, M, N, m0, n0, q, lane, 1, cb, ce); break;
+          case EPI_BIAS_GLU: epilogue_tile<EPI_BIAS_GLU, BN, 32>(e, acc, stage, nullptr, M, N, m0, n0, q, lane, 1, cb, ce); break;
+          case EPI_RESID: epilogue_tile<EPI_RESID, BN, 32>(e, acc, stage, nullptr, M, N, m0, n0, q, lane, 1, cb, ce); break;
+          case EPI_F32: epilogue_tile<EPI_F32, BN, 32>(e, acc, stage, nullptr, M, N, m0, n0, q, lane, 1, cb, ce); break;
+          default: epilogue_tile<EPI_F32_AND_T, BN, 32>(e, acc, stage, nullptr, M, N, m0, n0, q, lane, 1, cb, ce); break;
+        }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acce[a]);   // this warp is done reading accumulator a
     }
+    ring.drain(lane);
   }
   tc_fence_before();
   __syncthreads();
@@ -746,10 +760,11 @@ constexpr int PAIR_BM = 256;
 
 template <int BN, int STAGES>
 struct Tc2Cfg {
-  static constexpr int CW = 32;        // epilogue chunk width (columns)
+  static constexpr int CW = 32;        // epilogue chunk width (columns) of the staged fallback epilogue
   static constexpr int A_BYTES = TC_BM * TC_BK * 2;
   static constexpr int B_BYTES = (BN / 2) * TC_BK * 2;
-  static constexpr int STAGE_FLOATS = 8 * 32 * (CW + 4);
+  static constexpr int STAGE_FLOATS = 8 * 2 * EPI_BOX_BYTES / 4;   // per epilogue warp two TMA boxes
+  static_assert(STAGE_FLOATS >= 8 * 32 * (CW + 4), "fallback staging fits the box buffers");
   static constexpr int SMEM = 1024 + STAGES * (A_BYTES + B_BYTES) + STAGE_FLOATS * 4 + 256;
   // TMEM columns: two accumulators, rounded up to a power of two
   static constexpr uint32_t TMEM_COLS = 2 * BN <= 256 ? 256u : 512u;
@@ -765,8 +780,9 @@ __host__ __device__ constexpr uint32_t idesc_bf16_m256(int n) {
 
 template <int BN, int STAGES>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
-    gemm_tc2_kernel(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtensorMap tb, int M, int N,
-                    int K, Epi e, int* err) {
+    gemm_tc2_kernel(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtensorMap tb,
+                    const __grid_constant__ CUtensorMap mo, const __grid_constant__ CUtensorMap mo2, int M, int N,
+                    int K, Epi e, int* err, int tma_epi) {
   using C = Tc2Cfg<BN, STAGES>;
   extern __shared__ uint8_t tc_smem[];
   uint8_t* sm = tc_smem + ((1024 - (su32(tc_smem) & 1023)) & 1023);
@@ -869,19 +885,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
   } else {
     const int q = warp & 3, hc = (warp - 2) >> 2;   // TMEM lane quarter, column half
     float* stage = stg + (warp - 2) * (32 * (C::CW + 4));
+    BoxRing ring{reinterpret_cast<uint8_t*>(stg) + (warp - 2) * 2 * EPI_BOX_BYTES, 0};
+    float xr[32];
+    float2 b2 = make_float2(0.f, 0.f);
     int i = 0;
     for (int tile = pair; tile < tiles; tile += npairs, ++i) {
       const int a = i & 1, u = i >> 1;
       const int m0 = (tile / tiles_n) * PAIR_BM + TC_BM * (int)rank, n0 = (tile % tiles_n) * BN;
-      prefetch_resid(e, M, N, m0 + 32 * q, 32, n0 + hc * BN / 2, BN / 2, lane);
-      if (!mbar_wait(&accf[a], u & 1, abort_flag) || *abort_flag) {
+      if (!tma_epi) prefetch_resid(e, M, N, m0 + 32 * q, 32, n0 + hc * BN / 2, BN / 2, lane);
+      else epi_prefetch<false, BN>(e, M, N, m0 + 32 * q, n0, hc, lane, xr, b2);
+      if (__any_sync(0xffffffffu, !mbar_wait(&accf[a], u & 1, abort_flag) || *abort_flag)) {
         *abort_flag = 1;
         break;
       }
       tc_fence_after();
       const uint32_t acc = tmem + (uint32_t)(a * BN);
       const int cb = hc * BN / 2, ce = cb + BN / 2;
-      switch (e.kind) {
+      if (tma_epi) {
+        row_epilogue_any<BN, false>(e, &mo, &mo2, acc + ((uint32_t)(32 * q) << 16), ring, M, N, m0 + 32 * q, n0, hc, 2, lane,
+                             xr, b2);
+      } else switch (e.kind) {
         case EPI_BIAS: epilogue_tile<EPI_BIAS, BN, C::CW>(e, acc, stage, nullptr, M, N, m0, n0, q, lane, 1, cb, ce); break;
         case EPI_BIAS_RELU: epilogue_tile<EPI_BIAS_RELU, BN, C::CW>(e, acc, stage, nullptr, M, N, m0, n0, q, lane, 1, cb, ce); break;
         case EPI_BIAS_SWISH: epilogue_tile<EPI_BIAS_SWISH, BN, C::CW>(e, acc, stage, nullptr, M, N, m0, n0, q, lane, 1, cb, ce); break;
@@ -894,6 +917,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(mapa_shared(su32(&acce[a]), 0));   // accumulator a drained here
     }
+    ring.drain(lane);
   }
   tc_fence_before();
   __syncthreads();
@@ -944,16 +968,57 @@ cudaError_t make_map(CUtensorMap* m, const void* base, int rows, int cols, int l
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// 2-D output tensor map for the TMA box stores of the row-per-thread
+// epilogue: 32-row boxes of box_cols elements, rows of 128 bytes (128-byte
+// swizzle) or 64 bytes (64-byte swizzle).
+bool make_out_map(CUtensorMap* m, const void* base, bool f32, int rows, int cols, int64_t ld, int box_cols) {
+  const int esz = f32 ? 4 : 2;
+  if (!base || (reinterpret_cast<uintptr_t>(base) & 15) || (ld * esz) % 16 || rows <= 0 || cols <= 0) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(ld * esz)};
+  cuuint32_t box[2] = {(cuuint32_t)box_cols, 32u};
+  cuuint32_t estr[2] = {1, 1};
+  const int row_bytes = box_cols * esz;
+  CUresult r = g_encode(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                        const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Output maps of an epilogue (row_epilogue / resid_ln_rows); false where the
+// staged epilogue has to run instead (row remap, unaligned outputs).
+bool make_epi_maps(const Epi& e, int M, int N, CUtensorMap* mo, CUtensorMap* mo2) {
+  memset(mo, 0, sizeof(*mo));
+  memset(mo2, 0, sizeof(*mo2));
+  if (e.rpg) return false;
+  switch (e.kind) {
+    case EPI_BIAS:
+    case EPI_BIAS_RELU:
+    case EPI_BIAS_SWISH: return make_out_map(mo, e.out, false, M, N, e.ldo, 64);
+    case EPI_BIAS_GLU: return make_out_map(mo, e.out, false, M, N / 2, e.ldo, 32);
+    case EPI_RESID:
+    case EPI_F32: return make_out_map(mo, e.out, true, M, N, e.ldo, 32);
+    case EPI_F32_AND_T:
+      return make_out_map(mo, e.out, true, M, N, e.ldo, 32) && make_out_map(mo2, e.out2, false, M, N, e.ldo2, 32);
+    case EPI_RESID_LN:
+      return make_out_map(mo, e.out, true, M, N, e.ldo, 32) && make_out_map(mo2, e.ln_h, false, M, N, e.ldh, 64);
+    default: return false;
+  }
+}
+
 template <int BN, int STAGES>
 cudaError_t launch_tc(const bf16* A, int lda, const bf16* W, int M, int N, int K, int splits, const Epi& e,
                       const TcScratch& sc, cudaStream_t st) {
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, mo, mo2;
   cudaError_t r = make_map(&ta, A, M, K, lda, TC_BM);
   if (r != cudaSuccess) return r;
   r = make_map(&tb, W, N, K, K, BN);
   if (r != cudaSuccess) return r;
+  const int te = (splits == 1 && make_epi_maps(e, M, N, &mo, &mo2)) ? 1 : 0;
   dim3 grid((N + BN - 1) / BN, (M + TC_BM - 1) / TC_BM, splits);
-  CK_LAUNCH(launch_k(gemm_tc_kernel<BN, STAGES>, dim3(grid), dim3(192), TcCfg<BN, STAGES>::SMEM, st, ta, tb, M, N, K, e, sc.err, sc.ws, sc.cnt));
+  CK_LAUNCH(launch_k(gemm_tc_kernel<BN, STAGES>, dim3(grid), dim3(192), TcCfg<BN, STAGES>::SMEM, st, ta, tb, mo, mo2, M,
+                     N, K, e, sc.err, sc.ws, sc.cnt, te));
   return cudaGetLastError();
 }
 
@@ -965,11 +1030,12 @@ template <int STAGES>
 cudaError_t launch_tc_ln_s(const bf16* A, int lda, const bf16* W, int M, int N, int K, const Epi& e,
                            const TcScratch& sc, cudaStream_t st) {
   constexpr int BN = 64;
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, mo, mo2;
   cudaError_t r = make_map(&ta, A, M, K, lda, TC_BM);
   if (r != cudaSuccess) return r;
   r = make_map(&tb, W, N, K, K, BN);
   if (r != cudaSuccess) return r;
+  if (!make_epi_maps(e, M, N, &mo, &mo2)) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(N / BN, (M + TC_BM - 1) / TC_BM, 1);
   cfg.blockDim = dim3(192);
@@ -989,8 +1055,8 @@ cudaError_t launch_tc_ln_s(const bf16* A, int lda, const bf16* W, int M, int N, 
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  CK_LAUNCH(cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, STAGES>, ta, tb, M, N, K, e, sc.err, (float*)nullptr,
-                               (int*)nullptr));
+  CK_LAUNCH(cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, STAGES>, ta, tb, mo, mo2, M, N, K, e, sc.err,
+                               (float*)nullptr, (int*)nullptr, 1));
   return cudaGetLastError();
 }
 
@@ -1007,15 +1073,16 @@ cudaError_t launch_tc_ln(const bf16* A, int lda, const bf16* W, int M, int N, in
 template <int BN, int STAGES>
 cudaError_t launch_tcp(const bf16* A, int lda, const bf16* W, int M, int N, int K, const Epi& e, const TcScratch& sc,
                        cudaStream_t st) {
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, mo, mo2;
   cudaError_t r = make_map(&ta, A, M, K, lda, TC_BM);
   if (r != cudaSuccess) return r;
   r = make_map(&tb, W, N, K, K, BN);
   if (r != cudaSuccess) return r;
+  const int te = make_epi_maps(e, M, N, &mo, &mo2) ? 1 : 0;
   const int tiles = ((M + TC_BM - 1) / TC_BM) * ((N + BN - 1) / BN);
   const int grid = tiles < g_num_sms ? tiles : g_num_sms;
-  CK_LAUNCH(launch_k(gemm_tcp_kernel<BN, STAGES>, dim3(grid), dim3(320), TcpCfg<BN, STAGES>::SMEM, st, ta, tb, M, N, K,
-                     e, sc.err));
+  CK_LAUNCH(launch_k(gemm_tcp_kernel<BN, STAGES>, dim3(grid), dim3(320), TcpCfg<BN, STAGES>::SMEM, st, ta, tb, mo, mo2,
+                     M, N, K, e, sc.err, te));
   return cudaGetLastError();
 }
 
@@ -1024,16 +1091,17 @@ int g_max_pairs = 0;   // co-resident CTA pairs of gemm_tc2_kernel (0: not queri
 template <int BN, int STAGES>
 cudaError_t launch_tc2(const bf16* A, int lda, const bf16* W, int M, int N, int K, const Epi& e, const TcScratch& sc,
                        cudaStream_t st) {
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, mo, mo2;
   cudaError_t r = make_map(&ta, A, M, K, lda, TC_BM);
   if (r != cudaSuccess) return r;
   r = make_map(&tb, W, N, K, K, BN / 2);
   if (r != cudaSuccess) return r;
+  const int te = make_epi_maps(e, M, N, &mo, &mo2) ? 1 : 0;
   const int tiles = ((M + PAIR_BM - 1) / PAIR_BM) * ((N + BN - 1) / BN);
   const int cap = g_max_pairs > 0 ? g_max_pairs : g_num_sms / 2;
   const int pairs = tiles < cap ? tiles : cap;
-  CK_LAUNCH(launch_k(gemm_tc2_kernel<BN, STAGES>, dim3(2 * pairs), dim3(320), Tc2Cfg<BN, STAGES>::SMEM, st, ta, tb, M,
-                     N, K, e, sc.err));
+  CK_LAUNCH(launch_k(gemm_tc2_kernel<BN, STAGES>, dim3(2 * pairs), dim3(320), Tc2Cfg<BN, STAGES>::SMEM, st, ta, tb, mo,
+                     mo2, M, N, K, e, sc.err, te));
   return cudaGetLastError();
 }
 
@@ -1116,8 +1184,8 @@ cudaError_t gemm_bf16_tc(const bf16* A, int lda, const bf16* W, int M, int N, in
   if (r != cudaSuccess) return r;
   if (e.kind == EPI_RESID_LN) {
     if (!gemm_ln_fusable(M, N, K) || !e.ln_g || !e.ln_b || !e.ln_h || (e.ln_g2 && (!e.ln_b2 || !e.ln_xnorm)) ||
-        e.rpg || (reinterpret_cast<uintptr_t>(e.out) & 15) || (reinterpret_cast<uintptr_t>(e.ln_h) & 7) ||
-        e.ldo % 4 || e.ldh % 4)
+        e.rpg || (reinterpret_cast<uintptr_t>(e.out) & 15) || (reinterpret_cast<uintptr_t>(e.ln_h) & 15) ||
+        e.ldo % 4 || e.ldh % 8)
       return cudaErrorInvalidValue;
     return launch_tc_ln(A, lda, W, M, N, K, e, sc, st);
   }
@@ -1132,8 +1200,8 @@ cudaError_t gemm_bf16_tc(const bf16* A, int lda, const bf16* W, int M, int N, in
     if (g_gemm_pairs == 2 || (g_gemm_pairs == 1 && K >= 1024 && N >= 256)) {
       switch (g_gemm_pair_bn ? g_gemm_pair_bn : gemm_pair_plan(M, N, K)) {
         case 256: return launch_tc2<256, 5>(A, lda, W, M, N, K, e, sc, st);
-        case 192: return launch_tc2<192, 6>(A, lda, W, M, N, K, e, sc, st);
-        default: return launch_tc2<128, 7>(A, lda, W, M, N, K, e, sc, st);
+        case 192: return launch_tc2<192, 5>(A, lda, W, M, N, K, e, sc, st);
+        default: return launch_tc2<128, 6>(A, lda, W, M, N, K, e, sc, st);
       }
     }
     if (N >= 256) return launch_tcp<256, 3>(A, lda, W, M, N, K, e, sc, st);
@@ -1162,9 +1230,9 @@ cudaError_t gemm_tc_init_attributes() {
     g_num_sms = n_sm;
   r = cudaFuncSetAttribute(gemm_tc2_kernel<256, 5>, cudaFuncAttributeMaxDynamicSharedMemorySize, Tc2Cfg<256, 5>::SMEM);
   if (r == cudaSuccess)
-    r = cudaFuncSetAttribute(gemm_tc2_kernel<192, 6>, cudaFuncAttributeMaxDynamicSharedMemorySize, Tc2Cfg<192, 6>::SMEM);
+    r = cudaFuncSetAttribute(gemm_tc2_kernel<192, 5>, cudaFuncAttributeMaxDynamicSharedMemorySize, Tc2Cfg<192, 5>::SMEM);
   if (r == cudaSuccess)
-    r = cudaFuncSetAttribute(gemm_tc2_kernel<128, 7>, cudaFuncAttributeMaxDynamicSharedMemorySize, Tc2Cfg<128, 7>::SMEM);
+    r = cudaFuncSetAttribute(gemm_tc2_kernel<128, 6>, cudaFuncAttributeMaxDynamicSharedMemorySize, Tc2Cfg<128, 6>::SMEM);
   if (r != cudaSuccess) return r;
   {   // every configuration holds one CTA per SM: the same number of co-resident pairs
     cudaLaunchConfig_t cfg = {};
