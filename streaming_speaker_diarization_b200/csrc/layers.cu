@@ -136,14 +136,21 @@ template <> struct Vec2<bf16> {
 // Each thread: two channels x DW_ROWS consecutive rows; the DW_ROWS + K - 1
 // input rows they need are loaded once into registers (32-row blocks keep
 // the halo re-read at K - 1 rows per 32 and the weight loads amortised;
-// 8-row blocks give short inputs more CTAs).
+// 8-row blocks give short inputs more CTAs).  The two channels are one
+// packed f32x2 FMA per tap (each lane an ordinary fused multiply-add).
 // Taps outside the output row's sequence read as zero.  Swish: exact expf and
-// division for f32 outputs; for bf16 outputs the hardware exp2 and an
-// approximate reciprocal (relative error ~1e-7, far inside bf16 rounding).
+// division for f32 outputs; for bf16 outputs sigmoid(a) = (1 + tanh(a/2)) / 2
+// with the hardware tanh approximation (absolute error about 2^-11, below
+// bf16 rounding; one special-function operation where exp and reciprocal
+// take two).
 constexpr int DW_KMAX = 9;
 template <typename T>
 __device__ __forceinline__ float dw_swish(float a) {
-  if (sizeof(T) == 2) return a * __fdividef(1.f, 1.f + __expf(-a));
+  if (sizeof(T) == 2) {
+    float t;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * a));
+    return a * fmaf(0.5f, t, 0.5f);
+  }
   return a / (1.f + expf(-a));
 }
 template <typename T, int DW_ROWS>
@@ -155,22 +162,19 @@ __global__ void __launch_bounds__(128) dwconv1d_kernel(const T* __restrict__ in,
   if (c >= D) return;
   const int r0 = blockIdx.x * DW_ROWS;
   const int pad = (K - 1) / 2;
-  float w0[DW_KMAX], w1[DW_KMAX];
+  float2 wc[DW_KMAX];
 #pragma unroll
-  for (int j = 0; j < DW_KMAX; ++j) {   // channels c, c + 1: 2K consecutive floats at c * K
-    w0[j] = j < K ? w[(int64_t)c * K + j] : 0.f;
-    w1[j] = j < K ? w[(int64_t)c * K + K + j] : 0.f;
-  }
-  const float b0 = bias[c], b1 = bias[c + 1];
-  float x0[DW_ROWS + DW_KMAX - 1], x1[DW_ROWS + DW_KMAX - 1];
+  for (int j = 0; j < DW_KMAX; ++j)   // channels c, c + 1: 2K consecutive floats at c * K
+    wc[j] = j < K ? make_float2(w[(int64_t)c * K + j], w[(int64_t)c * K + K + j]) : make_float2(0.f, 0.f);
+  const float2 bc = make_float2(bias[c], bias[c + 1]);
+  float2 xc[DW_ROWS + DW_KMAX - 1];
 #pragma unroll
   for (int i = 0; i < DW_ROWS + DW_KMAX - 1; ++i) {
     const int ri = r0 - pad + i;
-    x0[i] = x1[i] = 0.f;
+    xc[i] = make_float2(0.f, 0.f);
     if (ri >= 0 && ri < M && i < DW_ROWS + K - 1) {
       const auto v = Vec2<T>::load(in + (int64_t)ri * D + c);
-      x0[i] = Vec2<T>::lo(v);
-      x1[i] = Vec2<T>::hi(v);
+      xc[i] = make_float2(Vec2<T>::lo(v), Vec2<T>::hi(v));
     }
   }
   int s = seq_of_row(seq, r0 < M ? r0 : M - 1);
@@ -184,26 +188,19 @@ __global__ void __launch_bounds__(128) dwconv1d_kernel(const T* __restrict__ in,
       sb = seq->off[s];
       se = seq->off[s + 1];
     }
-    float a0 = b0, a1 = b1;
+    float2 a = bc;
     if (r - pad >= sb && r + pad < se) {   // interior row: every tap inside the sequence
 #pragma unroll
-      for (int j = 0; j < DW_KMAX; ++j) {
-        if (j < K) {
-          a0 = fmaf(w0[j], x0[k + j], a0);
-          a1 = fmaf(w1[j], x1[k + j], a1);
-        }
-      }
+      for (int j = 0; j < DW_KMAX; ++j)
+        if (j < K) a = __ffma2_rn(wc[j], xc[k + j], a);
     } else {
 #pragma unroll
       for (int j = 0; j < DW_KMAX; ++j) {
         const int ri = r + j - pad;
-        if (j < K && ri >= sb && ri < se) {
-          a0 = fmaf(w0[j], x0[k + j], a0);
-          a1 = fmaf(w1[j], x1[k + j], a1);
-        }
+        if (j < K && ri >= sb && ri < se) a = __ffma2_rn(wc[j], xc[k + j], a);
       }
     }
-    Vec2<T>::store(out + (int64_t)r * D + c, dw_swish<T>(a0), dw_swish<T>(a1));
+    Vec2<T>::store(out + (int64_t)r * D + c, dw_swish<T>(a.x), dw_swish<T>(a.y));
   }
 }
 
