@@ -227,29 +227,32 @@ __global__ void __launch_bounds__(192, 2) attn_mha_tc_kernel(const __grid_consta
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(s_free);   // S of tile t read out of TMEM
+      // the running maximum over the raw scores (the scale is positive), then
+      // p = 2^(s sl2 - m) with one packed FMA per two keys
+      const bool full = j0 + MK <= S;
+      if (!full) {   // last tile: keys past the sequence end get no weight
+#pragma unroll
+        for (int c = 0; c < MK; ++c)
+          if (j0 + c >= S) sc[c] = -INFINITY;
+      }
       float mx = -INFINITY;
-      if (j0 + MK <= S) {
 #pragma unroll
-        for (int c = 0; c < MK; ++c) {
-          sc[c] *= sl2;
-          mx = fmaxf(mx, sc[c]);
-        }
-      } else {   // last tile: keys past the sequence end get no weight
-#pragma unroll
-        for (int c = 0; c < MK; ++c) {
-          sc[c] = j0 + c < S ? sc[c] * sl2 : -INFINITY;
-          mx = fmaxf(mx, sc[c]);
-        }
-      }
-      const float m_new = fmaxf(m_run, mx);   // finite: key j0 < S (every local tile starts inside S)
+      for (int c = 0; c < MK; ++c) mx = fmaxf(mx, sc[c]);
+      const float m_new = fmaxf(m_run, mx * sl2);   // finite: key j0 < S (every local tile starts inside S)
       const float alpha = ex2_approx(m_run - m_new);
-      float ps = 0.f;
+      const float2 s2 = make_float2(sl2, sl2), nm2 = make_float2(-m_new, -m_new);
+      float2 ps2 = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int c = 0; c < MK; ++c) {
-        sc[c] = ex2_approx(sc[c] - m_new);
-        ps += sc[c];
+      for (int c = 0; c < MK; c += 2) {
+        const float2 x = __ffma2_rn(make_float2(sc[c], sc[c + 1]), s2, nm2);
+        float2 pe;
+        pe.x = ex2_approx(x.x);
+        pe.y = ex2_approx(x.y);
+        sc[c] = pe.x;
+        sc[c + 1] = pe.y;
+        ps2 = __fadd2_rn(ps2, pe);
       }
-      l_run = l_run * alpha + ps;
+      l_run = l_run * alpha + (ps2.x + ps2.y);
       m_run = m_new;
       // P row as bf16 into the swizzled A tile of P.V (buffer t % 2; its
       // previous tile's P.V completed before iteration t - 1 read its result)
@@ -276,8 +279,15 @@ __global__ void __launch_bounds__(192, 2) attn_mha_tc_kernel(const __grid_consta
         uint32_t v[64];
         if (MHD <= 32) tmem_ld32(tmem + lane_base + (uint32_t)(64 + 64 * pb), v);   // the head's columns
         else tmem_ld64(tmem + lane_base + (uint32_t)(64 + 64 * pb), v);
+        const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll
-        for (int k = 0; k < MHD; ++k) o[k] = (o[k] + __uint_as_float(v[k])) * alpha;
+        for (int k = 0; k < MHD; k += 2) {
+          const float2 t = __fmul2_rn(__fadd2_rn(make_float2(o[k], o[k + 1]),
+                                                 make_float2(__uint_as_float(v[k]), __uint_as_float(v[k + 1]))),
+                                      a2);
+          o[k] = t.x;
+          o[k + 1] = t.y;
+        }
       }
     }
     if (ok && Tl > 0) {

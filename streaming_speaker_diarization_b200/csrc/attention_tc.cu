@@ -292,33 +292,41 @@ __global__ void __launch_bounds__(192, 1) attn_relpos_tc_kernel(const __grid_con
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(s_free);   // AC / BD of tile t read out of TMEM
-      // key c of row r: BD column r - c + 63 = staged column lane + 63 - c
+      // key c of row r: BD column r - c + 63 = staged column lane + 63 - c.
+      // AC + BD as packed adds, the running maximum over the unscaled sums
+      // (the scale is positive), then p = 2^(s sl2 - m) as one packed FMA per
+      // two keys
+      const float* bdr = stg + lane * (BD_LD + 1) + (AK - 1);
+#pragma unroll
+      for (int c = 0; c < AK; c += 2) {
+        const float2 t = __fadd2_rn(make_float2(sc[c], sc[c + 1]), make_float2(bdr[-c], bdr[-c - 1]));
+        sc[c] = t.x;
+        sc[c + 1] = t.y;
+      }
+      const bool full = j0 + AK <= S;
+      if (!full) {   // last tile: keys past the sequence end get no weight
+#pragma unroll
+        for (int c = 0; c < AK; ++c)
+          if (j0 + c >= S) sc[c] = -INFINITY;
+      }
       float mx = -INFINITY;
-      if (j0 + AK <= S) {
 #pragma unroll
-        for (int c = 0; c < AK; ++c) {
-          const float x = (sc[c] + stg[lane * (BD_LD + 1) + (AK - 1) - c]) * sl2;
-          sc[c] = x;
-          mx = fmaxf(mx, x);
-        }
-      } else {   // last tile: keys past the sequence end get no weight
-#pragma unroll
-        for (int c = 0; c < AK; ++c) {
-          float x = (sc[c] + stg[lane * (BD_LD + 1) + (AK - 1) - c]) * sl2;
-          if (j0 + c >= S) x = -INFINITY;
-          sc[c] = x;
-          mx = fmaxf(mx, x);
-        }
-      }
-      const float m_new = fmaxf(m_run, mx);   // finite: key j0 < S
+      for (int c = 0; c < AK; ++c) mx = fmaxf(mx, sc[c]);
+      const float m_new = fmaxf(m_run, mx * sl2);   // finite: key j0 < S
       const float alpha = ex2_approx(m_run - m_new);
-      float ps = 0.f;
+      const float2 s2 = make_float2(sl2, sl2), nm2 = make_float2(-m_new, -m_new);
+      float2 ps2 = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int c = 0; c < AK; ++c) {
-        sc[c] = ex2_approx(sc[c] - m_new);
-        ps += sc[c];
+      for (int c = 0; c < AK; c += 2) {
+        const float2 x = __ffma2_rn(make_float2(sc[c], sc[c + 1]), s2, nm2);
+        float2 pe;
+        pe.x = ex2_approx(x.x);
+        pe.y = ex2_approx(x.y);
+        sc[c] = pe.x;
+        sc[c + 1] = pe.y;
+        ps2 = __fadd2_rn(ps2, pe);
       }
-      l_run = l_run * alpha + ps;
+      l_run = l_run * alpha + (ps2.x + ps2.y);
       m_run = m_new;
       // P row as bf16 into the swizzled A tile of P.V (buffer t % 2; its
       // previous tile's P.V completed before iteration t - 1 read its result)
@@ -344,8 +352,15 @@ __global__ void __launch_bounds__(192, 1) attn_relpos_tc_kernel(const __grid_con
         tc_fence_after();
         uint32_t v[AHD];
         tmem_ld64(tmem + lane_base + (uint32_t)(256 + 64 * pb), v);
+        const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll
-        for (int k = 0; k < AHD; ++k) o[k] = (o[k] + __uint_as_float(v[k])) * alpha;
+        for (int k = 0; k < AHD; k += 2) {
+          const float2 t = __fmul2_rn(__fadd2_rn(make_float2(o[k], o[k + 1]),
+                                                 make_float2(__uint_as_float(v[k]), __uint_as_float(v[k + 1]))),
+                                      a2);
+          o[k] = t.x;
+          o[k + 1] = t.y;
+        }
       }
     }
     if (ok && Tl > 0) {

@@ -27,6 +27,7 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+
 // Byte offset of element (row, col) (col in bf16 units, < 64) of a K-major
 // tile with 128-byte rows and the 128-byte swizzle (16-byte chunk index
 // XOR row % 8), as TMA writes it and tcgen05 reads it.
