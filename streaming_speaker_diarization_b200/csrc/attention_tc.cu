@@ -309,13 +309,20 @@ __global__ void __launch_bounds__(192, 1) attn_relpos_tc_kernel(const __grid_con
         for (int c = 0; c < AK; ++c)
           if (j0 + c >= S) sc[c] = -INFINITY;
       }
-      float mx = -INFINITY;
+      // row maximum and sum as 8 / 4 independent partial chains (one warp per
+      // scheduler: a single serial chain would expose every latency)
+      float mp[8];
 #pragma unroll
-      for (int c = 0; c < AK; ++c) mx = fmaxf(mx, sc[c]);
+      for (int k = 0; k < 8; ++k) mp[k] = sc[k];
+#pragma unroll
+      for (int c = 8; c < AK; ++c) mp[c & 7] = fmaxf(mp[c & 7], sc[c]);
+      const float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])), fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
       const float m_new = fmaxf(m_run, mx * sl2);   // finite: key j0 < S
       const float alpha = ex2_approx(m_run - m_new);
       const float2 s2 = make_float2(sl2, sl2), nm2 = make_float2(-m_new, -m_new);
-      float2 ps2 = make_float2(0.f, 0.f);
+      float2 ps2[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) ps2[k] = make_float2(0.f, 0.f);
 #pragma unroll
       for (int c = 0; c < AK; c += 2) {
         const float2 x = __ffma2_rn(make_float2(sc[c], sc[c + 1]), s2, nm2);
@@ -324,9 +331,10 @@ __global__ void __launch_bounds__(192, 1) attn_relpos_tc_kernel(const __grid_con
         pe.y = ex2_approx(x.y);
         sc[c] = pe.x;
         sc[c + 1] = pe.y;
-        ps2 = __fadd2_rn(ps2, pe);
+        ps2[(c >> 1) & 3] = __fadd2_rn(ps2[(c >> 1) & 3], pe);
       }
-      l_run = l_run * alpha + (ps2.x + ps2.y);
+      const float2 pt2 = __fadd2_rn(__fadd2_rn(ps2[0], ps2[1]), __fadd2_rn(ps2[2], ps2[3]));
+      l_run = l_run * alpha + (pt2.x + pt2.y);
       m_run = m_new;
       // P row as bf16 into the swizzled A tile of P.V (buffer t % 2; its
       // previous tile's P.V completed before iteration t - 1 read its result)
