@@ -187,8 +187,8 @@ SF_API sf_status sf_mel(sf_engine* e, const float* d_audio, const int64_t* h_len
  * tiles (e.g. 10 clips of 120 s); larger requests return SF_ESHAPE.
  * The first call on a device (with that device current) takes the array's
  * device address, uploads the FFT/window/filterbank tables with a blocking
- * copy and sets the frame kernels' shared-memory attribute for the device:
- * make it before any CUDA stream capture.  All calls share the array and it keeps the last
+ * copy and sets the frame kernels' shared-memory attribute for the device.
+ * All calls share the array and it keeps the last
  * call's contents, so calls whose GPU work overlaps (on different streams or
  * threads) race and corrupt each other; order them on one stream.  No error
  * message is kept (there is no engine): the status code is the report. */

@@ -16,8 +16,7 @@
 // with cudaGetSymbolAddress, once per device, with that device current, the
 // first time the entry point is called on that device; that first call also
 // uploads the (host-computed) FFT/window/filterbank tables into a second
-// static array with a blocking copy.  Make that first call before any CUDA
-// stream capture.
+// static array with a blocking copy.
 //
 // All calls share the one array and it keeps the last call's contents: two
 // calls whose GPU work overlaps (different streams, or different threads
