@@ -532,7 +532,10 @@ struct TcpCfg {
   static constexpr int B_BYTES = BN * TC_BK * 2;
   static constexpr int STAGE_FLOATS = 8 * 2 * EPI_BOX_BYTES / 4;   // per epilogue warp two TMA boxes (or a 32 x 36 tile)
   static constexpr int SMEM = 1024 + STAGES * (A_BYTES + B_BYTES) + STAGE_FLOATS * 4 + 256;
+  // two accumulators, rounded up to a power of two
+  static constexpr uint32_t TMEM_COLS = 2 * BN <= 256 ? 256u : 512u;
   static_assert(SMEM <= 232448, "shared memory per CTA");
+  static_assert((STAGES * (A_BYTES + B_BYTES)) % 1024 == 0, "box buffers stay 1024-byte aligned");
 };
 
 template <int BN, int STAGES>
@@ -576,7 +579,7 @@ __global__ void __launch_bounds__(320, 1) gemm_tcp_kernel(const __grid_constant_
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(tmem_slot)),
-                 "r"((uint32_t)(2 * BN))
+                 "r"(C::TMEM_COLS)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
@@ -683,7 +686,7 @@ __global__ void __launch_bounds__(320, 1) gemm_tcp_kernel(const __grid_constant_
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"((uint32_t)(2 * BN))
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::TMEM_COLS)
                  : "memory");
   }
   if (threadIdx.x == 0 && *abort_flag) set_err(err, ERR_TIMEOUT);
@@ -1204,6 +1207,9 @@ cudaError_t gemm_bf16_tc(const bf16* A, int lda, const bf16* W, int M, int N, in
         default: return launch_tc2<128, 6>(A, lda, W, M, N, K, e, sc, st);
       }
     }
+    // whole tiles where N allows: 192 columns for N = 192 or 576 (the
+    // d 192 Transformer), else 256 or 128
+    if (N % 256 && N % 192 == 0) return launch_tcp<192, 3>(A, lda, W, M, N, K, e, sc, st);
     if (N >= 256) return launch_tcp<256, 3>(A, lda, W, M, N, K, e, sc, st);
     return launch_tcp<128, 4>(A, lda, W, M, N, K, e, sc, st);
   }
@@ -1246,6 +1252,8 @@ cudaError_t gemm_tc_init_attributes() {
   r = cudaFuncSetAttribute(gemm_tcp_kernel<256, 3>, cudaFuncAttributeMaxDynamicSharedMemorySize, TcpCfg<256, 3>::SMEM);
   if (r == cudaSuccess)
     r = cudaFuncSetAttribute(gemm_tcp_kernel<128, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, TcpCfg<128, 4>::SMEM);
+  if (r == cudaSuccess)
+    r = cudaFuncSetAttribute(gemm_tcp_kernel<192, 3>, cudaFuncAttributeMaxDynamicSharedMemorySize, TcpCfg<192, 3>::SMEM);
   if (r != cudaSuccess) return r;
   r = cudaFuncSetAttribute(gemm_tc_kernel<256, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        TcCfg<256, 4>::SMEM);
