@@ -49,8 +49,8 @@ CONFIG = {"workload": "offline forward, 1 clip x 90 s (16 kHz, 4 speakers, 15% o
 # from an ncu launch list of this workload (710.4 MB over the 142 GEMM
 # launches of one forward, the residual + LayerNorm epilogues included);
 # valid only for the GEMM sources it was taken with, null once they change.
-GEMM_TRAFFIC = {"bytes_per_launch": 710.42e6 / 142,
-                "sources_sha256": "3ac0b2a2d3d4312db44920575299d2a2a510d19f15a894ae62288b2b2c0dd649"}
+GEMM_TRAFFIC = {"bytes_per_launch": 710.39e6 / 142,
+                "sources_sha256": "3e3d6f6e68709a918c93f54dfcce911303ec88df9e8263fabb8c681e2c4973b2"}
 
 
 def gemm_traffic_per_launch():
@@ -257,7 +257,8 @@ def streaming_bench(b, torch, eng_blob, rank, world, local, args, clocks_dir=Non
     pass captures each step shape's CUDA graph; the streams are reset and the
     second pass is timed with CUDA events (clocks sampled meanwhile).  A
     third pass brackets only the state-update and selection launches with
-    events: the cache compression's microseconds per step.  The roofline is
+    events: the cache compression's microseconds per step; a fourth brackets
+    the projection GEMMs: their class throughput in the step.  The roofline is
     the model's algorithmic flops (model_flops over every stream's steps)
     over the timed pass."""
     from streaming_speaker_diarization_b200 import dist as sd
@@ -311,6 +312,12 @@ def streaming_bench(b, torch, eng_blob, rank, world, local, args, clocks_dir=Non
         one_pass()
         torch.cuda.synchronize()
         upd = b.sf_profile_read(eng, reset=True)
+        # the projection GEMMs: events around the GEMM launches only (class 3)
+        b.sf_stream_reset(st)
+        b.sf_profile_enable(eng, 2 * (1 << 3))
+        one_pass()
+        torch.cuda.synchronize()
+        gm = b.sf_profile_read(eng, reset=True).get("gemm", (0, 0.0, 0.0, 0.0))
         b.sf_profile_enable(eng, 0)
         upd_ms = sum(v[1] for k, v in upd.items() if k in ("state_update", "select_topk"))
         audio_s = float(lens.sum()) / 16000.0
@@ -330,6 +337,11 @@ def streaming_bench(b, torch, eng_blob, rank, world, local, args, clocks_dir=Non
                                  "flops_total": flops,
                                  "peak_kind": f"{kind} bf16 {'sustained' if max_ms > 1000.0 else 'burst'}"},
                     "compression_us_per_step": 1000.0 * upd_ms / max(len(step_ms), 1),
+                    "gemm": {"launches": int(gm[0]), "ms": gm[1], "share_of_pass": gm[1] / max_ms if max_ms else None,
+                             "tflops": gm[2] / (gm[1] / 1000.0) / 1e12 if gm[1] else None,
+                             "frac": (gm[2] / (gm[1] / 1000.0) / 1e12) / pk["bf16_tflops"] if gm[1] else None,
+                             "peak_kind": f"{kind} bf16 burst",
+                             "note": "events around the GEMM launches of a separate pass (they add a few us each)"},
                     "clocks": clocks})
         b.sf_stream_destroy(st)
         b.sf_destroy(eng)
