@@ -53,6 +53,28 @@ GEMM_TRAFFIC = {"bytes_per_launch": 710.39e6 / 142,
                 "sources_sha256": "3e3d6f6e68709a918c93f54dfcce911303ec88df9e8263fabb8c681e2c4973b2"}
 
 
+# Warp instructions one sf_mel call on the 1 h workload issues (front-end
+# path 1: frame, statistics and normalisation kernels; ncu
+# smsp__inst_executed.sum, 438.2M + 4.1M + 25.0M), valid only for the
+# front-end source it was taken with.  The call is bound by instruction
+# issue (the FFT), not by HBM: its issue roofline is 148 SMs x 4 schedulers
+# x one warp instruction per clock x 1965 MHz.
+FRONTEND_INST = {"warp_inst_per_call": 467.33e6,
+                 "sources_sha256": "edb41f3764b09c48b0e44751b1cddb013dde6b4fa3aba91f82a005ee84a5d525"}
+ISSUE_PEAK = 148 * 4 * 1.965e9   # warp instructions per second
+
+
+def frontend_inst_per_call():
+    import hashlib
+    try:
+        with open(os.path.join(os.path.dirname(os.path.abspath(__file__)), "streaming_speaker_diarization_b200", "csrc",
+                               "frontend.cu"), "rb") as fh:
+            h = hashlib.sha256(fh.read()).hexdigest()
+    except OSError:
+        return None
+    return FRONTEND_INST["warp_inst_per_call"] if h == FRONTEND_INST["sources_sha256"] else None
+
+
 def gemm_traffic_per_launch():
     import hashlib
     h = hashlib.sha256()
@@ -388,11 +410,18 @@ def frontend_bench(b, torch, blob, steps, warmup, mel_path=1):
     alg = 4.0 * n + 4.0 * 128 * T
     pk, kind = peaks()
     gbs = alg / (med / 1000.0) / 1e9
+    inst = frontend_inst_per_call()
+    issue = None if inst is None else {
+        "bound": "alu", "kernel": "front-end call (warp instructions issued, FFT-dominated)",
+        "achieved": inst / (med / 1000.0), "peak": ISSUE_PEAK, "unit": "warp instructions/s",
+        "frac": inst / (med / 1000.0) / ISSUE_PEAK, "inst_per_call": inst,
+        "peak_kind": "148 SMs x 4 schedulers x 1 issue per clock x 1965 MHz"}
     return {"workload": "front-end only, 1 h of audio (60 x 60 s clips joined), 57.6M samples -> 128 x 360,001",
             "value": 3600.0 / (med / 1000.0), "unit": UNIT, "ms_p50": med, "ms_p95": float(np.percentile(ms, 95)),
             "calls": steps, "mel_path": mel_path,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                         "frac": gbs / pk["hbm_gbs"], "bytes_per_call": alg, "peak_kind": f"{kind} copy"}}
+                         "frac": gbs / pk["hbm_gbs"], "bytes_per_call": alg, "peak_kind": f"{kind} copy"},
+            "roofline_issue": issue}
 
 
 def batch_bench(b, torch, blob, steps, warmup, local, args, clocks_dir=None):
