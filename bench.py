@@ -50,7 +50,7 @@ CONFIG = {"workload": "offline forward, 1 clip x 90 s (16 kHz, 4 speakers, 15% o
 # launches of one forward, the residual + LayerNorm epilogues included);
 # valid only for the GEMM sources it was taken with, null once they change.
 GEMM_TRAFFIC = {"bytes_per_launch": 710.39e6 / 142,
-                "sources_sha256": "3e3d6f6e68709a918c93f54dfcce911303ec88df9e8263fabb8c681e2c4973b2"}
+                "sources_sha256": "5a99fd4c077623cdb9c15a9d3dac351a0b5526390688605243c2ae093c86cf2b"}
 
 
 # Warp instructions one sf_mel call on the 1 h workload issues (front-end

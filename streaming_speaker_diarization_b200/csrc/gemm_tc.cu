@@ -9,7 +9,11 @@
 //           tcgen05.mma.cta_group::1.kind::f16 (M=128, N=BN, K=16) four times
 //           per 64-wide k-block and frees each buffer with tcgen05.commit;
 //   warps 2-5 wait for the accumulator, read it with tcgen05.ld (each warp
-//           its 32-lane TMEM quarter = 32 output rows) and apply the epilogue.
+//           its 32-lane TMEM quarter = 32 output rows, thread = row) and
+//           apply the epilogue (epilogue_tma.cuh): finished row segments go
+//           into swizzled 32-row shared-memory boxes stored by TMA; split-K
+//           partials and row-remapped outputs take the staged epilogue
+//           (epilogue_tile) instead.
 // Full/empty mbarriers order the ring; every wait is bounded by a clock
 // budget: a wait that runs out sets ERR_TIMEOUT in the engine's error word,
 // raises a CTA-wide abort flag, the producer waits (bounded) for its own
@@ -454,9 +458,10 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
       *abort_flag = 1;
     }
   } else {
-    // Epilogue: per 64-column chunk, each warp copies its 32 x 64 accumulator
-    // block from TMEM to a padded shared tile (thread = row), then writes it
-    // out with lanes along the columns (one contiguous row segment per store
+    // Staged epilogue (split-K partials, row-remapped or unaligned outputs):
+    // per 64-column chunk, each warp copies its 32 x 64 accumulator block
+    // from TMEM to a padded shared tile (thread = row), then writes it out
+    // with lanes along the columns (one contiguous row segment per store
     // instruction).  The pipeline buffers are free once the accumulator is
     // complete, so the tiles reuse them.
     const int q = warp & 3;            // TMEM lane quarter this warp may access
@@ -1143,11 +1148,13 @@ int gemm_pair_plan(int M, int N, int K) {
 }
 
 // Tile width BN and split count S from a cost model of this kernel on 148
-// SMs, calibrated with per-phase timestamps on B200: per CTA ~1.4 us of
-// set-up and first-load latency, ~0.28 us per 64-wide k-block (bounded by
-// loads in flight, nearly independent of BN), and an epilogue of ~1.4 / 2.1 /
-// 3.8 us for BN = 64 / 128 / 256; a split-K partial round trip costs about
-// (BN / 64) x (1.5 + 0.9 S) us.  Splits need scratch and at most 2 waves.
+// SMs, calibrated with per-phase timestamps on B200 (with the staged
+// epilogue; the TMA-store epilogue is shorter, by about the same amount for
+// every choice): per CTA ~1.4 us of set-up and first-load latency, ~0.28 us
+// per 64-wide k-block (bounded by loads in flight, nearly independent of
+// BN), and an epilogue of ~1.4 / 2.1 / 3.8 us for BN = 64 / 128 / 256; a
+// split-K partial round trip costs about (BN / 64) x (1.5 + 0.9 S) us.
+// Splits need scratch and at most 2 waves.
 void gemm_tc_plan(int M, int N, int K, const TcScratch& sc, int* bn_out, int* s_out) {
   const int tm = (M + TC_BM - 1) / TC_BM;
   const int KB = (K + TC_BK - 1) / TC_BK;
