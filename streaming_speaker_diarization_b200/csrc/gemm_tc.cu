@@ -321,7 +321,7 @@ __device__ __forceinline__ void resid_ln_rows(const Epi& e, const CUtensorMap* m
 }
 
 template <int BN, int STAGES>
-__global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__ CUtensorMap ta,
+__global__ void __launch_bounds__(192, 2) gemm_tc_kernel(const __grid_constant__ CUtensorMap ta,
                                                          const __grid_constant__ CUtensorMap tb,
                                                          const __grid_constant__ CUtensorMap mo,
                                                          const __grid_constant__ CUtensorMap mo2, int M, int N, int K,
