@@ -264,6 +264,111 @@ __device__ __forceinline__ void epi_prefetch(const Epi& e, int M, int N, int m_w
   if (e.kind == EPI_RESID) load_resid32(e, m_w + lane, M, c, N, xr);
 }
 
+// EPI_RESID in the persistent kernels: the residual comes into the warp's
+// two box buffers as 32 x 32 f32 boxes by TMA loads through the output map
+// itself, each thread reads its row segment back from shared memory, adds
+// alpha (acc + bias) in place, and the box goes out by the TMA store.  Per
+// thread that replaces eight 16-byte global loads per chunk, each touching
+// 32 rows in a warp, by conflict-free shared-memory reads.  A tile's first
+// two chunks are requested before its accumulator wait; the buffer of chunk
+// t is reloaded with chunk t + 2 as soon as chunk t's store has read it, so
+// that load runs while chunk t + 1 is processed.  Warps whose 32 rows start
+// past M load and store nothing.
+struct ResidTma {
+  uint64_t* bar;       // the warp's two mbarriers (one per box buffer)
+  uint32_t phase;      // bit b: parity of buffer b's next load completion
+  uint32_t pending;    // bit b: a load into buffer b is not yet waited for
+};
+
+__device__ __forceinline__ void lds128(uint32_t addr, float* v) {
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3])
+               : "r"(addr)
+               : "memory");
+}
+
+// Request the residual box (columns c .., rows m_w ..) into buffer b; the
+// caller has made sure no store still reads that buffer.
+__device__ __forceinline__ void resid_tma_request(const CUtensorMap* mo, const BoxRing& ring, ResidTma& rt, int b, int c,
+                                                  int m_w, int M, int N, int lane) {
+  if (m_w >= M || c >= N) return;   // uniform over the warp
+  if (lane == 0) {
+    mbar_expect_tx(&rt.bar[b], EPI_BOX_BYTES);
+    tma_load_2d(ring.base + b * EPI_BOX_BYTES, mo, &rt.bar[b], c, m_w);
+  }
+  rt.pending |= 1u << b;
+}
+
+// Before a tile's accumulator wait: the tile's bias lines into L1, every
+// earlier store of this warp done reading its buffer, the first two
+// residual boxes requested.
+template <int BN>
+__device__ __forceinline__ void resid_tma_prologue(const Epi& e, const CUtensorMap* mo, const BoxRing& ring,
+                                                   ResidTma& rt, int M, int N, int m_w, int n0, int first, int step,
+                                                   int lane) {
+  prefetch_bias_l1(e.bias, n0, BN, N, lane);
+  if (lane == 0) bulk_wait_read_all();
+  __syncwarp();
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int j = first + t * step;
+    if (j < BN / 32) resid_tma_request(mo, ring, rt, t, n0 + j * 32, m_w, M, N, lane);
+  }
+}
+
+// The warp's chunks j = first, first + step, ... of the tile; false when a
+// residual load was not seen within the wait bound (or the kernel aborted).
+template <int BN>
+__device__ __forceinline__ bool resid_tma_rows(const Epi& e, const CUtensorMap* mo, uint32_t acc, BoxRing& ring,
+                                               ResidTma& rt, int M, int N, int m_w, int n0, int first, int step,
+                                               int lane, volatile int* abort_flag) {
+  constexpr int NCH = BN / 32;
+  int t = 0;
+#pragma unroll 1
+  for (int j = first; j < NCH; j += step, ++t) {
+    const int c = n0 + j * 32, b = t & 1;
+    const bool valid = m_w < M && c < N;
+    float v[32];
+    tmem_ld32(acc + (uint32_t)(j * 32), reinterpret_cast<uint32_t*>(v));
+    add_bias_bcast<32>(v, e.bias, c, N);
+    uint8_t* box = ring.base + b * EPI_BOX_BYTES;
+    const uint32_t sb = su32(box);
+    if (valid) {
+      if (__any_sync(0xffffffffu, !mbar_wait(&rt.bar[b], (rt.phase >> b) & 1u, abort_flag))) return false;
+      rt.phase ^= 1u << b;
+      rt.pending &= ~(1u << b);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        float x[4];
+        const uint32_t a = sw128_unit(sb, lane, u);
+        lds128(a, x);
+        sts128(a, __float_as_uint(x[0] + e.alpha * v[4 * u]), __float_as_uint(x[1] + e.alpha * v[4 * u + 1]),
+               __float_as_uint(x[2] + e.alpha * v[4 * u + 2]), __float_as_uint(x[3] + e.alpha * v[4 * u + 3]));
+      }
+    }
+    ring.store(mo, box, c, m_w, valid, lane);
+    if (j + 2 * step < NCH) {
+      if (lane == 0) bulk_wait_read_all();   // the store just issued has read the buffer
+      __syncwarp();
+      resid_tma_request(mo, ring, rt, b, n0 + (j + 2 * step) * 32, m_w, M, N, lane);
+    }
+  }
+  return true;
+}
+
+// Before the shared memory is released: loads that were requested but not
+// waited for (only after an abort) land first, within the wait bound.
+__device__ __forceinline__ void resid_tma_drain(ResidTma& rt) {
+#pragma unroll
+  for (int b = 0; b < 2; ++b) {
+    if (!(rt.pending >> b & 1u)) continue;
+    const long long t0 = clock64();
+    while (!mbar_try_wait(&rt.bar[b], (rt.phase >> b) & 1u) && clock64() - t0 < WAIT_CYCLES) {
+    }
+  }
+  rt.pending = 0;
+}
+
 // Dispatch on the epilogue kind (after epi_prefetch).
 template <int BN, bool LANE_BIAS>
 __device__ __forceinline__ void row_epilogue_any(const Epi& e, const CUtensorMap* mo, const CUtensorMap* mo2,

@@ -536,11 +536,14 @@ struct TcpCfg {
   static constexpr int A_BYTES = TC_BM * TC_BK * 2;
   static constexpr int B_BYTES = BN * TC_BK * 2;
   static constexpr int STAGE_FLOATS = 8 * 2 * EPI_BOX_BYTES / 4;   // per epilogue warp two TMA boxes (or a 32 x 36 tile)
-  static constexpr int SMEM = 1024 + STAGES * (A_BYTES + B_BYTES) + STAGE_FLOATS * 4 + 256;
+  // + barriers: STAGES full / empty, two accumulator pairs, two residual
+  // loads per epilogue warp, the TMEM slot and the abort flag
+  static constexpr int SMEM = 1024 + STAGES * (A_BYTES + B_BYTES) + STAGE_FLOATS * 4 + 512;
   // two accumulators, rounded up to a power of two
   static constexpr uint32_t TMEM_COLS = 2 * BN <= 256 ? 256u : 512u;
   static_assert(SMEM <= 232448, "shared memory per CTA");
   static_assert((STAGES * (A_BYTES + B_BYTES)) % 1024 == 0, "box buffers stay 1024-byte aligned");
+  static_assert((2 * STAGES + 4 + 16) * 8 + 8 <= 512, "barrier area");
 };
 
 template <int BN, int STAGES>
@@ -559,7 +562,8 @@ __global__ void __launch_bounds__(320, 1) gemm_tcp_kernel(const __grid_constant_
   uint64_t* empty = full + STAGES;
   uint64_t* accf = empty + STAGES;     // [2]
   uint64_t* acce = accf + 2;           // [2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce + 2);
+  uint64_t* rbar = acce + 2;           // [8][2] residual box loads of the epilogue warps
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(rbar + 16);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -578,6 +582,7 @@ __global__ void __launch_bounds__(320, 1) gemm_tcp_kernel(const __grid_constant_
       mbar_init(&accf[a], 1);
       mbar_init(&acce[a], 8);
     }
+    for (int b = 0; b < 16; ++b) mbar_init(&rbar[b], 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -652,6 +657,8 @@ __global__ void __launch_bounds__(320, 1) gemm_tcp_kernel(const __grid_constant_
     const int q = warp & 3, hc = (warp - 2) >> 2;   // TMEM lane quarter, column half
     float* stage = stg + (warp - 2) * (32 * 36);
     BoxRing ring{reinterpret_cast<uint8_t*>(stg) + (warp - 2) * 2 * EPI_BOX_BYTES, 0};
+    ResidTma rt{rbar + 2 * (warp - 2), 0u, 0u};
+    const bool resid_tma = tma_epi && e.kind == EPI_RESID;
     float xr[32];
     float2 b2 = make_float2(0.f, 0.f);
     int i = 0;
@@ -659,6 +666,7 @@ __global__ void __launch_bounds__(320, 1) gemm_tcp_kernel(const __grid_constant_
       const int a = i & 1, u = i >> 1;
       const int m0 = (tile / tiles_n) * TC_BM, n0 = (tile % tiles_n) * BN;
       if (!tma_epi) prefetch_resid(e, M, N, m0 + 32 * q, 32, n0 + hc * BN / 2, BN / 2, lane);
+      else if (resid_tma) resid_tma_prologue<BN>(e, &mo, ring, rt, M, N, m0 + 32 * q, n0, hc, 2, lane);
       else epi_prefetch<false, BN>(e, M, N, m0 + 32 * q, n0, hc, lane, xr, b2);
       if (__any_sync(0xffffffffu, !mbar_wait(&accf[a], u & 1, abort_flag) || *abort_flag)) {
         *abort_flag = 1;
@@ -666,7 +674,11 @@ __global__ void __launch_bounds__(320, 1) gemm_tcp_kernel(const __grid_constant_
       }
       tc_fence_after();
       const uint32_t acc = tmem + (uint32_t)(a * BN);
-      if (tma_epi) {   // chunks alternate between the two warps of a lane quarter
+      if (resid_tma) {
+        if (!resid_tma_rows<BN>(e, &mo, acc + ((uint32_t)(32 * q) << 16), ring, rt, M, N, m0 + 32 * q, n0, hc, 2, lane,
+                                abort_flag))
+          *abort_flag = 1;
+      } else if (tma_epi) {   // chunks alternate between the two warps of a lane quarter
         row_epilogue_any<BN, false>(e, &mo, &mo2, acc + ((uint32_t)(32 * q) << 16), ring, M, N, m0 + 32 * q, n0, hc, 2, lane,
                              xr, b2);
       } else {
@@ -685,6 +697,7 @@ __global__ void __launch_bounds__(320, 1) gemm_tcp_kernel(const __grid_constant_
       __syncwarp();
       if (lane == 0) mbar_arrive(&acce[a]);   // this warp is done reading accumulator a
     }
+    if (lane == 0) resid_tma_drain(rt);
     ring.drain(lane);
   }
   tc_fence_before();
@@ -773,7 +786,8 @@ struct Tc2Cfg {
   static constexpr int B_BYTES = (BN / 2) * TC_BK * 2;
   static constexpr int STAGE_FLOATS = 8 * 2 * EPI_BOX_BYTES / 4;   // per epilogue warp two TMA boxes
   static_assert(STAGE_FLOATS >= 8 * 32 * (CW + 4), "fallback staging fits the box buffers");
-  static constexpr int SMEM = 1024 + STAGES * (A_BYTES + B_BYTES) + STAGE_FLOATS * 4 + 256;
+  static constexpr int SMEM = 1024 + STAGES * (A_BYTES + B_BYTES) + STAGE_FLOATS * 4 + 512;
+  static_assert((2 * STAGES + 4 + 16) * 8 + 16 <= 512, "barrier area");
   // TMEM columns: two accumulators, rounded up to a power of two
   static constexpr uint32_t TMEM_COLS = 2 * BN <= 256 ? 256u : 512u;
   static_assert(SMEM <= 232448, "shared memory per CTA");
@@ -801,7 +815,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
   uint64_t* empty = full + STAGES;
   uint64_t* accf = empty + STAGES;     // [2]
   uint64_t* acce = accf + 2;           // [2], used in rank 0
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce + 2);
+  uint64_t* rbar = acce + 2;           // [8][2] residual box loads of the epilogue warps
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(rbar + 16);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* peer_abort = abort_flag + 1;   // written by the other CTA at teardown
 
@@ -823,6 +838,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
       mbar_init(&accf[a], 1);
       mbar_init(&acce[a], 16);
     }
+    for (int b = 0; b < 16; ++b) mbar_init(&rbar[b], 1);
     *abort_flag = 0;
     *peer_abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -894,6 +910,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
     const int q = warp & 3, hc = (warp - 2) >> 2;   // TMEM lane quarter, column half
     float* stage = stg + (warp - 2) * (32 * (C::CW + 4));
     BoxRing ring{reinterpret_cast<uint8_t*>(stg) + (warp - 2) * 2 * EPI_BOX_BYTES, 0};
+    ResidTma rt{rbar + 2 * (warp - 2), 0u, 0u};
+    const bool resid_tma = tma_epi && e.kind == EPI_RESID;
     float xr[32];
     float2 b2 = make_float2(0.f, 0.f);
     int i = 0;
@@ -901,6 +919,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
       const int a = i & 1, u = i >> 1;
       const int m0 = (tile / tiles_n) * PAIR_BM + TC_BM * (int)rank, n0 = (tile % tiles_n) * BN;
       if (!tma_epi) prefetch_resid(e, M, N, m0 + 32 * q, 32, n0 + hc * BN / 2, BN / 2, lane);
+      else if (resid_tma) resid_tma_prologue<BN>(e, &mo, ring, rt, M, N, m0 + 32 * q, n0, hc, 2, lane);
       else epi_prefetch<false, BN>(e, M, N, m0 + 32 * q, n0, hc, lane, xr, b2);
       if (__any_sync(0xffffffffu, !mbar_wait(&accf[a], u & 1, abort_flag) || *abort_flag)) {
         *abort_flag = 1;
@@ -909,7 +928,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
       tc_fence_after();
       const uint32_t acc = tmem + (uint32_t)(a * BN);
       const int cb = hc * BN / 2, ce = cb + BN / 2;
-      if (tma_epi) {
+      if (resid_tma) {
+        if (!resid_tma_rows<BN>(e, &mo, acc + ((uint32_t)(32 * q) << 16), ring, rt, M, N, m0 + 32 * q, n0, hc, 2, lane,
+                                abort_flag))
+          *abort_flag = 1;
+      } else if (tma_epi) {
         row_epilogue_any<BN, false>(e, &mo, &mo2, acc + ((uint32_t)(32 * q) << 16), ring, M, N, m0 + 32 * q, n0, hc, 2, lane,
                              xr, b2);
       } else switch (e.kind) {
@@ -925,6 +948,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(mapa_shared(su32(&acce[a]), 0));   // accumulator a drained here
     }
+    if (lane == 0) resid_tma_drain(rt);
     ring.drain(lane);
   }
   tc_fence_before();

@@ -104,6 +104,14 @@ def test_gemm_tc_fused_epilogues(eng, M, N, K, path):
     _check_fused(eng, M, N, K, path)
 
 
+@pytest.mark.parametrize("M,N,K", [(20608, 512, 512), (20608, 512, 2048), (20001, 512, 2048), (19030, 1536, 512)])
+def test_gemm_tc_resid_streaming_shapes(eng, M, N, K):
+    """Path 3 at the streaming step's residual projections (the persistent
+    and CTA-pair kernels, residual boxes loaded by TMA), and with ragged M
+    whose last tile leaves whole 32-row warps past M."""
+    _check_fused(eng, M, N, K, 3)
+
+
 @pytest.fixture(scope="module", params=[0, 128, 192, 256])
 def eng_pairs(request):
     """Engine on the CTA-pair GEMM path: planned tile width (0) or forced."""
