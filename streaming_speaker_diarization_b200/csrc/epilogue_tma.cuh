@@ -8,8 +8,9 @@
 // permuted by r), and one lane stores the 32-row box with
 // cp.async.bulk.tensor.  The TMA engine clips rows >= M and columns past the
 // matrix; the threads never wait for global stores.  Residual rows are read
-// into registers before the accumulator is complete, so their latency hides
-// behind the main loop.
+// before the accumulator is complete, so their latency hides behind the main
+// loop: into registers in the single-wave kernel, as TMA boxes into the box
+// buffers in the persistent kernels (resid_tma_*).
 //
 // Box buffers: each warp alternates between its buffers; before rewriting a
 // buffer, lane 0 waits until at most one earlier store group still reads
